@@ -1,0 +1,423 @@
+"""Benchmark of the GQE attention layer on B200.
+
+A step is one prefill forward of the paper's main GQE layer (16 query experts /
+8 KV heads, top-1 of 2 per group, one shared head, d_model 1024, d_head 64) over
+one batch of 8 x 2048 synthetic tokens: router -> routed/shared query
+projection -> K/V projection -> routed causal attention -> output construction
+-> output projection, all in libgqe.so kernels.
+
+Prints one JSON line: whole-job tokens/s (max over ranks of the summed
+per-step CUDA-event time), the attention kernel's roofline against the
+measured bf16 tensor peak, the end-to-end number through host buffers, the
+fp64 oracle's CPU throughput on a bounded sample, a decode sub-measurement
+(64 sequences x 32768-entry cache, % of HBM bandwidth), and the SM clocks
+sampled during the timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+For N > 1 it runs under torchrun, one independent replica per GPU (the layer's
+path has no exchange step), and reports the aggregate.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import gqe_inputs as gi  # noqa: E402
+
+WORKLOAD = "main_prefill"
+DECODE_WORKLOAD = "decode"
+METRIC = "GQE prefill tokens/s per layer"
+FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def attn_useful_flops(dims) -> float:
+    """Causal useful FLOPs of the routed + shared attention: QK^T and PV over the
+    kG+1 active query heads, keys 0..t only: 2 * 2 * d * T(T+1)/2 per head."""
+    return 2.0 * dims.d * dims.T * (dims.T + 1) * dims.B * dims.h_active
+
+
+def decode_attn_bytes(dims, L) -> float:
+    """Algorithmic bytes of the decode attention: the K and V cache read once
+    (bf16), plus the query rows and outputs."""
+    cache = 2.0 * dims.B * dims.G * L * dims.d * 2
+    q_o = 2.0 * dims.B * (dims.G * dims.k + dims.n_shared) * dims.d * 2
+    return cache + q_o
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (replicas; the only cross-rank steps are the barrier and
+# the max over ranks of the measured time)
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [s.strip() for s in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    mx = float(p[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample
+
+def cpu_baseline(seconds_budget=20.0):
+    import oracle as orc
+    cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 0) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    w = gi.WORKLOADS[WORKLOAD]
+    dims = w.dims.replace(B=1)           # one 2048-token sequence of the workload
+    x = gi.layer_input(w.dims, rows=[0])
+    Wt = gi.layer_weights(dims)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        orc.gqe_forward(x, Wt, dims, gi.router_bias(w))
+        n += 1
+        if time.perf_counter() - t0 > seconds_budget or n >= 3:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n * dims.N / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} x one sequence (T={dims.T}) of the {WORKLOAD} workload, fp64 numpy, "
+                      f"{dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------
+
+def run_reference(args):
+    """Reference arm: the fp64 oracle timed on the host cores (rank 0 only)."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle as orc
+    w = gi.WORKLOADS[WORKLOAD]
+    dims = w.dims.replace(B=1)
+    x = gi.layer_input(w.dims, rows=[0])
+    Wt = gi.layer_weights(dims)
+    for _ in range(min(args.warmup, 1)):
+        orc.gqe_forward(x, Wt, dims)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.gqe_forward(x, Wt, dims)
+    dt = time.perf_counter() - t0
+    value = args.steps * dims.N / dt
+    cores = os.cpu_count()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": f"{WORKLOAD} (one sequence per step: bounded CPU sample)",
+                                            "B": 1, "T": dims.T},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"one {dims.T}-token sequence of {WORKLOAD} per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_env()
+    import torch
+    import moe_gqa_query_b200 as gq
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    peaks = load_peaks()
+
+    # ---------------- prefill workload
+    w = gi.WORKLOADS[WORKLOAD]
+    dims = w.dims
+    Wt = gi.layer_weights(dims, seed=0)
+    layer = gq.GQELayer(dims, {k: torch.from_numpy(v.view(np.int16)) for k, v in Wt.items()},
+                        gi.router_bias(w), device=device)
+    x_host = torch.from_numpy(gi.layer_input(dims, seed=rank).view(np.int16)).view(torch.bfloat16)
+    x = x_host.to(device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    # per-call events inside every timed step (router, q-proj, kv-proj, attention, combine, out-proj)
+    seg_names = ["router", "routed_qproj", "kv_proj", "attn_prefill", "combine", "out_proj"]
+
+    def step(evs=None):
+        c = layer.cfg
+        B, T, N = dims.B, dims.T, dims.N
+        d_ = gq.make_dims(c, B=B, T=T)
+        L = gq
+        idx = layer._buf("idx", (N, c.G, c.k), torch.int32)
+        wt = layer._buf("w", (N, c.G, c.k), torch.float32)
+        q = layer._buf("q", (B, c.G, T, c.k, c.d))
+        qs = layer._buf("qs", (B, T, c.d))
+        K = layer._buf("K", (B, c.G, T, c.d))
+        V = layer._buf("V", (B, c.G, T, c.d))
+        o = layer._buf("o", (B, c.G, T, c.k, c.d))
+        os_ = layer._buf("os", (B, T, c.d))
+        h = layer._buf("h", (N, c.slots * c.d))
+        y = layer._buf("y", (B, T, c.D))
+        ws = layer._ws("ws_q", L.gqe_workspace_size(d_, L.GQE_OP_ROUTED_QPROJ))
+        rec = (lambda i: evs[i].record(stream)) if evs is not None else (lambda i: None)
+        rec(0)
+        L.gqe_router_topk(d_, x, layer.Wr, layer.bias, idx, wt, None)
+        rec(1)
+        L.gqe_routed_qproj(d_, x, layer.Wq, layer.Wsh, idx, q, qs, ws)
+        rec(2)
+        L.gqe_kv_proj(d_, x, layer.Wk, layer.Wv, K, V)
+        rec(3)
+        L.gqe_attn_prefill(d_, q, qs, K, V, o, os_, None)
+        rec(4)
+        L.gqe_combine(d_, o, os_, wt, h)
+        rec(5)
+        L.gqe_linear(h, layer.Wo, y)
+        rec(6)
+        return y
+
+    launches_per_step = 9   # router, 3 permutation kernels, routed GEMM, K/V GEMM, attention, combine, Wo GEMM
+
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    assert gq.gqe_device_error() == 0
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for s in range(args.steps):
+            flush.zero_()                       # L2 flushed between timed steps (outside the events)
+            step(events[s])
+        torch.cuda.synchronize()
+    barrier(dist, device)
+    seg_ms = np.array([[events[s][i].elapsed_time(events[s][i + 1]) for i in range(6)] for s in range(args.steps)])
+    step_ms = seg_ms.sum(axis=1)
+    local_total_ms = float(step_ms.sum())
+    total_ms = max_over_ranks(local_total_ms, dist, device)
+    tokens = world * dims.N * args.steps
+    value = tokens / (total_ms / 1e3)
+    err_code = gq.gqe_device_error()
+
+    # attention kernel roofline (tensor bound)
+    attn_ms = float(seg_ms[:, 3].mean())
+    flops = attn_useful_flops(dims)
+    achieved_tf = flops / (attn_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attn_prefill_kernel<64>", "achieved": achieved_tf,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
+                "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": None,
+                "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_ms}
+
+    # ---------------- end to end through host buffers (pinned), on the same step
+    e2e = None
+    x_pin = x_host.pin_memory()
+    y_pin = torch.empty((dims.B, dims.T, dims.D), dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        layer.forward_host(x_pin, y_pin)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 20))
+    barrier(dist, device)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        layer.forward_host(x_pin, y_pin)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    e2e = {"value": world * dims.N * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(y_pin.numel() * 2),
+           "steps": n_e2e}
+
+    # ---------------- decode sub-measurement (64 sequences x 32768-entry cache)
+    decode = None
+    if not args.no_decode:
+        dw = gi.WORKLOADS[DECODE_WORKLOAD]
+        dd, Lc = dw.dims, dw.L
+        dlayer = gq.GQELayer(dd, {k: torch.from_numpy(v.view(np.int16)) for k, v in gi.layer_weights(dd).items()},
+                             device=device)
+        gen = torch.Generator(device=device).manual_seed(1234 + rank)
+        Kc = torch.empty((dd.B, dd.G, Lc, dd.d), dtype=torch.bfloat16, device=device).normal_(generator=gen)
+        Vc = torch.empty_like(Kc).normal_(generator=gen)
+        xn = torch.from_numpy(gi.normal_bf16(rank, "xdec", (dd.B, dd.D)).view(np.int16)).view(torch.bfloat16).to(device)
+        cl = torch.full((dd.B,), Lc, dtype=torch.int32, device=device)
+        for _ in range(3):
+            dlayer.decode_step(xn, Kc, Vc, cl)
+        torch.cuda.synchronize()
+        nd = max(3, min(args.steps, 20))
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nd)]
+        tot = []
+        # attention-only timing: same call sequence, events around gqe_attn_decode
+        dims_c = gq.make_dims(dd, T=1)
+        ws = torch.empty((gq.gqe_workspace_size(dims_c, gq.GQE_OP_ATTN_DECODE, Lc),), dtype=torch.uint8, device=device)
+        qd = torch.randn((dd.B, dd.G, 1, dd.k, dd.d), device=device).to(torch.bfloat16)
+        qsd = torch.randn((dd.B, 1, dd.d), device=device).to(torch.bfloat16)
+        od = torch.empty_like(qd)
+        osd = torch.empty_like(qsd)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for i in range(nd):
+            ev[i][0].record(stream)
+            gq.gqe_attn_decode(dims_c, qd, qsd, Kc, Vc, Lc, cl, od, osd, ws)
+            ev[i][1].record(stream)
+        s0.record(stream)
+        for i in range(nd):
+            dlayer.decode_step(xn, Kc, Vc, cl)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        attn_dec_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        step_dec_ms = s0.elapsed_time(s1) / nd
+        bytes_ = decode_attn_bytes(dd, Lc)
+        gbs = bytes_ / (attn_dec_ms / 1e3) / 1e9
+        decode = {"workload": dw.desc, "tokens_per_s": world * dd.B / (max_over_ranks(step_dec_ms, dist, device) / 1e3),
+                  "ms_per_step": step_dec_ms,
+                  "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<64> + merge", "achieved": gbs,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                               "peak_source": f"{peaks['source']} HBM copy", "traffic": None,
+                               "algorithmic_bytes_per_launch": bytes_, "avg_launch_ms": attn_dec_ms},
+                  "data": "synthetic: cache ~N(0,1) from a seeded torch generator on the device"}
+        del Kc, Vc
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD}: {w.desc}", "B": dims.B, "T": dims.T, "d_model": dims.D,
+                       "G": dims.G, "E": dims.E, "k": dims.k, "d_head": dims.d, "n_shared": dims.n_shared,
+                       "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MB write)"},
+            "segments_ms": {n: float(seg_ms[:, i].mean()) for i, n in enumerate(seg_names)},
+            "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "decode": decode,
+            "clocks": clocks.summary(), "gpu_launches": launches_per_step * args.steps,
+            "device_error": err_code,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

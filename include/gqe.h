@@ -1,0 +1,162 @@
+/*
+ * gqe.h -- C ABI of the Grouped Query Experts (GQE) attention forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * GQE (as described in the "GQE" study note at dimensionstp.github.io, §3-2,
+ * and the chatpaper abstract "Experts de requêtes groupées") keeps the dense
+ * K/V heads of grouped-query attention and turns the E query heads of every
+ * KV group into experts: a per-group router picks k experts per token, only
+ * those query heads are projected and attend, and the layer output
+ * concatenates the hard-selected expert outputs, one router-weighted sum of
+ * them and one always-on shared query head.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is DEVICE memory owned by the caller, contiguous,
+ *     row-major, 16-byte aligned.  bf16 tensors are passed as pointers to
+ *     uint16_t bit patterns (gqe_bf16).
+ *   - Weights use the [out, in] layout of a linear layer, except Wr, which is
+ *     [d_model, G*E].
+ *   - No entry point allocates or frees device memory or synchronises the
+ *     device; work is enqueued on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  Scratch memory, where a call needs it, is the
+ *     caller's `ws` buffer of at least gqe_workspace_size() bytes.
+ *   - Argument errors return GQE_ERR_INVALID_ARG / GQE_ERR_UNSUPPORTED /
+ *     GQE_ERR_WORKSPACE before anything is launched; a failed launch returns
+ *     GQE_ERR_CUDA.  Errors inside a kernel surface at the caller's next
+ *     synchronisation; a kernel whose internal wait runs out of time records a
+ *     code that gqe_device_error() returns.
+ *   - Supported shapes: d_head in {64, 128}; 1 <= k <= E <= 8; G*E <= 64;
+ *     d_model a multiple of 64; n_shared in {0, 1}; 0 <= shared_kv_group < G.
+ */
+#ifndef GQE_H_
+#define GQE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t gqe_bf16;     /* bfloat16 bit pattern */
+typedef void* gqe_stream;      /* cudaStream_t */
+
+typedef enum {
+  GQE_OK = 0,
+  GQE_ERR_INVALID_ARG = 1,
+  GQE_ERR_UNSUPPORTED = 2,
+  GQE_ERR_WORKSPACE = 3,
+  GQE_ERR_CUDA = 4,
+  GQE_ERR_DEVICE_CHECK = 5
+} gqe_status;
+
+/* Shape of one layer call.  B sequences of T tokens (T = 1 for decode),
+ * model width d_model, G KV groups with E query experts each, k experts
+ * routed per (token, group), head width d_head.  renorm_scope 0 normalises
+ * the selected router probabilities over all k*G selections of a token, 1
+ * within each group.  scale 0 means 1/sqrt(d_head). */
+typedef struct {
+  int B, T, d_model, G, E, k, d_head;
+  int n_shared;          /* 0 or 1 always-on shared query heads */
+  int shared_kv_group;   /* KV group the shared head reads */
+  int renorm_scope;      /* 0 token, 1 group */
+  float scale;
+} gqe_dims;
+
+enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2 };
+
+/* Bytes of scratch the call `op` needs for these dims (L_max: the decode
+ * cache length, used by GQE_OP_ATTN_DECODE only).  Returns
+ * GQE_ERR_INVALID_ARG for bad dims or op. */
+gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* bytes);
+
+/* Router: "GQE" study note §3-2 2) (score, in-group softmax, TopK) and 4)
+ * (renormalised weights p~).
+ *   x [B*T, d_model] bf16, Wr [d_model, G*E] bf16, bias [G*E] fp32 or NULL.
+ *   topk_idx [B*T, G, k] int32: the selected experts of each (token, group)
+ *     in ascending expert order (ties in the logits go to the lower index).
+ *   topk_w   [B*T, G, k] fp32: p~ aligned with topk_idx.
+ *   probs    [B*T, G, E] fp32 softmax probabilities, or NULL.
+ * Logits are accumulated in fp32 from the bf16 inputs. */
+gqe_status gqe_router_topk(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wr,
+                           const float* bias, int32_t* topk_idx, float* topk_w, float* probs,
+                           gqe_stream stream);
+
+/* Routed and shared query projection: "GQE" study note §3-2 2) (only the
+ * selected experts compute their query) and 5) (shared head); ai-feeds
+ * summary, 方法 (unselected query heads are skipped).
+ *   x [B*T, d_model], Wq [G, E, d_head, d_model], Wsh [n_shared*d_head, d_model],
+ *   topk_idx [B*T, G, k] as written by gqe_router_topk.
+ *   q_routed [B, G, T, k, d_head]: slot j of (b, g, t) holds x_t Wq[g, topk_idx[t,g,j]]^T.
+ *   q_sh [B, T, d_head] (ignored when n_shared == 0).
+ *   expert_counts [G*E] int32 tokens per expert, or NULL.
+ *   ws: scratch of gqe_workspace_size(GQE_OP_ROUTED_QPROJ) bytes (the
+ *   token-to-expert permutation lives there). */
+gqe_status gqe_routed_qproj(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wq,
+                            const gqe_bf16* Wsh, const int32_t* topk_idx, gqe_bf16* q_routed,
+                            gqe_bf16* q_sh, int32_t* expert_counts, void* ws, size_t ws_bytes,
+                            gqe_stream stream);
+
+/* Dense, unchanged K/V projection ("GQE" study note §1-2 3) and §3-2 1)):
+ *   K[b, g, t, :] = x[b*T+t] Wk[g*d:(g+1)*d]^T, likewise V.
+ *   x [B*T, d_model]; Wk, Wv [G*d_head, d_model]; K, V [B, G, T, d_head]. */
+gqe_status gqe_kv_proj(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk,
+                       const gqe_bf16* Wv, gqe_bf16* K, gqe_bf16* V, gqe_stream stream);
+
+/* Decode-step K/V append: projects the B new tokens (T must be 1) and writes
+ * their rows at index cache_len[b]-1 of the caches Kc, Vc [B, G, L_max, d_head].
+ * cache_len [B] int32 device array, each value in [1, L_max]. */
+gqe_status gqe_kv_append(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk,
+                         const gqe_bf16* Wv, gqe_bf16* Kc, gqe_bf16* Vc, int L_max,
+                         const int32_t* cache_len, gqe_stream stream);
+
+/* Routed causal attention, prefill ("GQE" study note §1-1 attention
+ * equation; §3-2 2) every selected expert attends to its group's dense K/V;
+ * §3-2 5) the shared head, which reads KV group shared_kv_group).
+ *   q_routed [B, G, T, k, d], q_sh [B, T, d], K, V [B, G, T, d] (bf16).
+ *   o_routed [B, G, T, k, d], o_sh [B, T, d] (bf16).
+ *   lse: NULL, or fp32 [B*G*T*k + B*T*n_shared]: natural-log sum of
+ *   exp(scaled scores) per query row, routed rows first.
+ * Row (t, j) of a group attends to keys 0..t.  fp32 softmax and accumulation. */
+gqe_status gqe_attn_prefill(const gqe_dims* dims, const gqe_bf16* q_routed,
+                            const gqe_bf16* q_sh, const gqe_bf16* K, const gqe_bf16* V,
+                            gqe_bf16* o_routed, gqe_bf16* o_sh, float* lse, gqe_stream stream);
+
+/* Decode attention: one new token per sequence (dims->T must be 1) against a
+ * dense cache (freeguideonline GQA tutorial, "自回归推理中的内存带宽优势": a
+ * decode step reads the whole KV cache).
+ *   q_routed [B, G, k, d], q_sh [B, d]; Kc, Vc [B, G, L_max, d];
+ *   cache_len [B] int32 device array: rows [0, cache_len[b]) are attended.
+ *   o_routed [B, G, k, d], o_sh [B, d].
+ *   ws: scratch of gqe_workspace_size(GQE_OP_ATTN_DECODE) bytes (split-L
+ *   partial softmax states). */
+gqe_status gqe_attn_decode(const gqe_dims* dims, const gqe_bf16* q_routed,
+                           const gqe_bf16* q_sh, const gqe_bf16* Kc, const gqe_bf16* Vc,
+                           int L_max, const int32_t* cache_len, gqe_bf16* o_routed,
+                           gqe_bf16* o_sh, void* ws, size_t ws_bytes, gqe_stream stream);
+
+/* Output construction ("GQE" study note §3-2 3) hard slots, 4) weighted-sum
+ * slot, 5) final concat):
+ *   h[n] = [o(g=0, slot 0..k-1), ..., o(g=G-1, ...), sum_g sum_j w[n,g,j] o(g,j), o_sh]
+ *   o_routed [B, G, T, k, d], o_sh [B, T, d], topk_w [B*T, G, k] fp32
+ *   -> h [B*T, (k*G + 1 + n_shared) * d] bf16 (the weighted sum in fp32). */
+gqe_status gqe_combine(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe_bf16* o_sh,
+                       const float* topk_w, gqe_bf16* h, gqe_stream stream);
+
+/* Output projection and general linear map ("GQE" study note §3-2 7)):
+ *   C [M, N] = A [M, K] W^T with W [N, K]; bf16 in and out, fp32 accumulation.
+ *   K must be a multiple of 64 and N a multiple of 64. */
+gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W, gqe_bf16* C,
+                      gqe_stream stream);
+
+/* Reads and clears the device error word that kernels set when one of their
+ * internal waits runs out of time (0 = none).  Synchronises `stream`. */
+gqe_status gqe_device_error(int* code, gqe_stream stream);
+
+const char* gqe_status_string(gqe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* GQE_H_ */

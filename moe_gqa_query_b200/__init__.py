@@ -1,0 +1,15 @@
+"""Grouped Query Experts (GQE) attention forward on NVIDIA B200 (sm_100a).
+
+The computation lives in the CUDA library libgqe.so (C ABI in include/gqe.h);
+this package is its thin Python binding plus GQELayer, which chains the calls.
+Importing it without the built library raises ImportError: there is no CPU
+fallback.
+"""
+from ._lib import (  # noqa: F401
+    GQEError, gqe_dims, make_dims, header_functions, LIB_PATH,
+    GQE_OP_ROUTED_QPROJ, GQE_OP_ATTN_DECODE,
+    gqe_workspace_size, gqe_router_topk, gqe_routed_qproj, gqe_kv_proj, gqe_kv_append,
+    gqe_attn_prefill, gqe_attn_decode, gqe_combine, gqe_linear, gqe_device_error,
+    gqe_status_string,
+)
+from .layer import GQEConfig, GQELayer  # noqa: F401

@@ -1,0 +1,220 @@
+"""ctypes binding of libgqe.so (include/gqe.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors that already live on the GPU (or raw integer pointers), passes their
+device pointers, the shape struct and the current CUDA stream to the library,
+and raises GQEError on a non-zero status.  No step of the computation happens
+in Python.  The library must be built (python -m moe_gqa_query_b200.build);
+importing this module without it raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgqe.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "gqe.h")
+
+GQE_OK = 0
+GQE_OP_ROUTED_QPROJ = 1
+GQE_OP_ATTN_DECODE = 2
+STATUS_NAMES = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED",
+                3: "GQE_ERR_WORKSPACE", 4: "GQE_ERR_CUDA", 5: "GQE_ERR_DEVICE_CHECK"}
+
+
+class GQEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+
+
+class gqe_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("d_model", ctypes.c_int),
+                ("G", ctypes.c_int), ("E", ctypes.c_int), ("k", ctypes.c_int),
+                ("d_head", ctypes.c_int), ("n_shared", ctypes.c_int),
+                ("shared_kv_group", ctypes.c_int), ("renorm_scope", ctypes.c_int),
+                ("scale", ctypes.c_float)]
+
+
+def make_dims(cfg, **override) -> gqe_dims:
+    """Shape struct from any object with B, T, D, G, E, k, d (+ n_shared, sg,
+    renorm_scope, scale) attributes."""
+    v = dict(B=cfg.B, T=cfg.T, d_model=cfg.D, G=cfg.G, E=cfg.E, k=cfg.k, d_head=cfg.d,
+             n_shared=getattr(cfg, "n_shared", 1), shared_kv_group=getattr(cfg, "sg", 0),
+             renorm_scope=getattr(cfg, "renorm_scope", 0), scale=float(getattr(cfg, "scale", 0.0)))
+    v.update(override)
+    return gqe_dims(**v)
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+_D = ctypes.POINTER(gqe_dims)
+
+SIGNATURES = {
+    "gqe_workspace_size": [_D, _I, _I, ctypes.POINTER(_SZ)],
+    "gqe_router_topk": [_D, _P, _P, _P, _P, _P, _P, _P],
+    "gqe_routed_qproj": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
+    "gqe_kv_proj": [_D, _P, _P, _P, _P, _P, _P],
+    "gqe_kv_append": [_D, _P, _P, _P, _P, _P, _I, _P, _P],
+    "gqe_attn_prefill": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
+    "gqe_attn_decode": [_D, _P, _P, _P, _P, _I, _P, _P, _P, _P, _SZ, _P],
+    "gqe_combine": [_D, _P, _P, _P, _P, _P],
+    "gqe_linear": [_I, _I, _I, _P, _P, _P, _P],
+    "gqe_device_error": [ctypes.POINTER(_I), _P],
+    "gqe_status_string": [_I],
+}
+
+
+def header_functions(path: str = HEADER_PATH):
+    """Names of the functions include/gqe.h declares."""
+    with open(path) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(gqe_\w+)\s*\(", text, flags=re.M)))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m moe_gqa_query_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, args in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_char_p if name == "gqe_status_string" else ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+# ----------------------------------------------------------------------------
+# marshalling helpers
+
+def _ptr(t, name="tensor", dtype=None, optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, st):
+    if st != GQE_OK:
+        raise GQEError(fn, st)
+
+
+def _bf16():
+    import torch
+    return torch.bfloat16
+
+
+# ----------------------------------------------------------------------------
+# the entry points
+
+def gqe_workspace_size(dims: gqe_dims, op: int, L_max: int = 0) -> int:
+    n = _SZ(0)
+    _check("gqe_workspace_size", lib.gqe_workspace_size(ctypes.byref(dims), op, L_max, ctypes.byref(n)))
+    return int(n.value)
+
+
+def gqe_router_topk(dims, x, Wr, bias, topk_idx, topk_w, probs=None, stream=None):
+    import torch
+    _check("gqe_router_topk", lib.gqe_router_topk(
+        ctypes.byref(dims), _ptr(x, "x", _bf16()), _ptr(Wr, "Wr", _bf16()),
+        _ptr(bias, "bias", torch.float32, optional=True), _ptr(topk_idx, "topk_idx", torch.int32),
+        _ptr(topk_w, "topk_w", torch.float32), _ptr(probs, "probs", torch.float32, optional=True),
+        _stream(stream)))
+
+
+def gqe_routed_qproj(dims, x, Wq, Wsh, topk_idx, q_routed, q_sh, ws, expert_counts=None, stream=None):
+    import torch
+    ws_bytes = ws.numel() * ws.element_size()
+    _check("gqe_routed_qproj", lib.gqe_routed_qproj(
+        ctypes.byref(dims), _ptr(x, "x", _bf16()), _ptr(Wq, "Wq", _bf16()),
+        _ptr(Wsh, "Wsh", _bf16(), optional=True), _ptr(topk_idx, "topk_idx", torch.int32),
+        _ptr(q_routed, "q_routed", _bf16()), _ptr(q_sh, "q_sh", _bf16(), optional=True),
+        _ptr(expert_counts, "expert_counts", torch.int32, optional=True),
+        _ptr(ws, "ws"), ws_bytes, _stream(stream)))
+
+
+def gqe_kv_proj(dims, x, Wk, Wv, K, V, stream=None):
+    b = _bf16()
+    _check("gqe_kv_proj", lib.gqe_kv_proj(
+        ctypes.byref(dims), _ptr(x, "x", b), _ptr(Wk, "Wk", b), _ptr(Wv, "Wv", b),
+        _ptr(K, "K", b), _ptr(V, "V", b), _stream(stream)))
+
+
+def gqe_kv_append(dims, x, Wk, Wv, Kc, Vc, L_max, cache_len, stream=None):
+    import torch
+    b = _bf16()
+    _check("gqe_kv_append", lib.gqe_kv_append(
+        ctypes.byref(dims), _ptr(x, "x", b), _ptr(Wk, "Wk", b), _ptr(Wv, "Wv", b),
+        _ptr(Kc, "Kc", b), _ptr(Vc, "Vc", b), int(L_max), _ptr(cache_len, "cache_len", torch.int32),
+        _stream(stream)))
+
+
+def gqe_attn_prefill(dims, q_routed, q_sh, K, V, o_routed, o_sh, lse=None, stream=None):
+    import torch
+    b = _bf16()
+    _check("gqe_attn_prefill", lib.gqe_attn_prefill(
+        ctypes.byref(dims), _ptr(q_routed, "q_routed", b), _ptr(q_sh, "q_sh", b, optional=True),
+        _ptr(K, "K", b), _ptr(V, "V", b), _ptr(o_routed, "o_routed", b),
+        _ptr(o_sh, "o_sh", b, optional=True), _ptr(lse, "lse", torch.float32, optional=True),
+        _stream(stream)))
+
+
+def gqe_attn_decode(dims, q_routed, q_sh, Kc, Vc, L_max, cache_len, o_routed, o_sh, ws, stream=None):
+    import torch
+    b = _bf16()
+    ws_bytes = ws.numel() * ws.element_size()
+    _check("gqe_attn_decode", lib.gqe_attn_decode(
+        ctypes.byref(dims), _ptr(q_routed, "q_routed", b), _ptr(q_sh, "q_sh", b, optional=True),
+        _ptr(Kc, "Kc", b), _ptr(Vc, "Vc", b), int(L_max), _ptr(cache_len, "cache_len", torch.int32),
+        _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True), _ptr(ws, "ws"), ws_bytes,
+        _stream(stream)))
+
+
+def gqe_combine(dims, o_routed, o_sh, topk_w, h, stream=None):
+    import torch
+    b = _bf16()
+    _check("gqe_combine", lib.gqe_combine(
+        ctypes.byref(dims), _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True),
+        _ptr(topk_w, "topk_w", torch.float32), _ptr(h, "h", b), _stream(stream)))
+
+
+def gqe_linear(A, W, C, stream=None):
+    b = _bf16()
+    M, K = A.shape[-2] if A.dim() > 1 else 1, A.shape[-1]
+    M = A.numel() // K
+    N = W.shape[0]
+    _check("gqe_linear", lib.gqe_linear(M, N, K, _ptr(A, "A", b), _ptr(W, "W", b), _ptr(C, "C", b),
+                                        _stream(stream)))
+
+
+def gqe_device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check("gqe_device_error", lib.gqe_device_error(ctypes.byref(code), _stream(stream)))
+    return int(code.value)
+
+
+def gqe_status_string(status: int) -> str:
+    return lib.gqe_status_string(int(status)).decode()

@@ -1,0 +1,50 @@
+// gemm.cuh -- parameters and launchers of the tcgen05 GEMMs (gemm.cu).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace gqe {
+
+typedef uint16_t gqe_bf16_t;
+
+enum EpiMode : int {
+  kEpiRowMajor = 0,   // out[row * ldo + n]
+  kEpiHeads = 1,      // out[b, g, t, dd] with row = b*T + t, n = g*d + dd
+  kEpiCacheRow = 2,   // out[b, g, cache_len[b]-1, dd] with row = b
+  kEpiRows = 3,       // out[dst_row * ldo + n], dst_row given per tile row
+};
+
+struct EpiParams {
+  gqe_bf16_t* out0;
+  gqe_bf16_t* out1;      // second weight's output (K / V pair)
+  const int* cache_len;
+  int mode;
+  int ldo;
+  int n_limit;           // columns >= n_limit are not written
+  int T, G, d, L_max;
+  unsigned* err;         // device error word
+};
+
+// Token-to-expert permutation produced by perm.cu, consumed by the routed GEMM.
+struct RoutedParams {
+  const int* src_row;     // [n_routed] token row of x
+  const int* dst_row;     // [n_routed] row of q_routed [B, G, T, k]
+  const int* seg_off;     // [n_seg] first entry of each (group, expert) segment
+  const int* seg_cnt;     // [n_seg]
+  const int* tile_start;  // [n_seg + 1] first 128-row tile of each segment
+  int n_seg;              // G * E
+  int max_routed_tiles;   // upper bound on tile_start[n_seg] (grid slots)
+  int n_tokens;           // B * T (shared-head tiles)
+  int K;                  // d_model
+  int d;                  // head width (= tile N)
+};
+
+cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
+                              const CUtensorMap& mapB1, const EpiParams& ep, int M, int K,
+                              int n_tiles_b0, int n_tiles_total, cudaStream_t stream);
+
+cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh,
+                               const gqe_bf16_t* x, const RoutedParams& rp, const EpiParams& epr,
+                               const EpiParams& eps, int grid, cudaStream_t stream);
+
+}  // namespace gqe

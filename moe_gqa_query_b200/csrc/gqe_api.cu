@@ -1,0 +1,387 @@
+// gqe_api.cu -- the C ABI declared in include/gqe.h: argument validation,
+// TMA descriptor construction and kernel launches.  Nothing here allocates or
+// synchronises (except gqe_device_error, which is a synchronous query).
+#include <math.h>
+#include <string.h>
+
+#include "../../include/gqe.h"
+#include "attn.cuh"
+#include "gemm.cuh"
+#include "route.cuh"
+
+using namespace gqe;
+
+namespace {
+
+// Device error word set by kernels whose internal waits run out of time.
+__device__ unsigned int g_device_error = 0;
+
+// Device address of g_device_error for the current device (looked up once per
+// device; host code cannot take the address of a __device__ variable).
+unsigned* error_word() {
+  static unsigned* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) cache[dev] = static_cast<unsigned*>(p);
+  }
+  return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
+// dims/box innermost first; strides in bytes for dims 1..rank-1.
+bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
+  memset(m, 0, sizeof(*m));
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool map2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t strides[1] = {cols * 2};
+  const uint32_t box[2] = {64, box_rows};
+  return make_map(m, ptr, 2, dims, strides, box);
+}
+
+// [outer, rows, cols] contiguous, box 64 cols x box_rows rows x 1
+bool map3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t outer, uint32_t box_rows) {
+  const uint64_t dims[3] = {cols, rows, outer};
+  const uint64_t strides[2] = {cols * 2, cols * rows * 2};
+  const uint32_t box[3] = {64, box_rows, 1};
+  return make_map(m, ptr, 3, dims, strides, box);
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gqe_status check_dims(const gqe_dims* d) {
+  if (!d) return GQE_ERR_INVALID_ARG;
+  if (d->B < 1 || d->T < 1 || d->d_model < 1 || d->G < 1 || d->E < 1 || d->k < 1 || d->k > d->E)
+    return GQE_ERR_INVALID_ARG;
+  if (d->n_shared < 0 || d->n_shared > 1 || d->renorm_scope < 0 || d->renorm_scope > 1)
+    return GQE_ERR_INVALID_ARG;
+  if (d->shared_kv_group < 0 || d->shared_kv_group >= d->G) return GQE_ERR_INVALID_ARG;
+  if (!(d->scale >= 0.f) || isinf(d->scale)) return GQE_ERR_INVALID_ARG;
+  if (d->d_head != 64 && d->d_head != 128) return GQE_ERR_UNSUPPORTED;
+  if (d->E > 8 || d->G * d->E > 64) return GQE_ERR_UNSUPPORTED;
+  if (d->d_model % 64 != 0) return GQE_ERR_UNSUPPORTED;
+  const long long N = (long long)d->B * d->T;
+  if (N * d->G * d->k * d->d_head >= (1ll << 31) || N * d->d_model >= (1ll << 31)) return GQE_ERR_UNSUPPORTED;
+  return GQE_OK;
+}
+
+inline float scale_log2(const gqe_dims* d) {
+  const float s = d->scale > 0.f ? d->scale : 1.0f / sqrtf((float)d->d_head);
+  return s * 1.4426950408889634f;
+}
+
+inline cudaStream_t S(gqe_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+inline gqe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
+
+#define GQE_CHECK(x)               \
+  do {                             \
+    gqe_status _s = (x);           \
+    if (_s != GQE_OK) return _s;   \
+  } while (0)
+#define GQE_REQUIRE(c, code) \
+  do {                       \
+    if (!(c)) return code;   \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* gqe_status_string(gqe_status s) {
+  switch (s) {
+    case GQE_OK: return "ok";
+    case GQE_ERR_INVALID_ARG: return "invalid argument";
+    case GQE_ERR_UNSUPPORTED: return "unsupported shape";
+    case GQE_ERR_WORKSPACE: return "workspace too small";
+    case GQE_ERR_CUDA: return "CUDA error";
+    case GQE_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* bytes) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(bytes, GQE_ERR_INVALID_ARG);
+  const int N = dims->B * dims->T;
+  if (op == GQE_OP_ROUTED_QPROJ) {
+    *bytes = perm_layout(N, dims->G, dims->E, dims->k).bytes;
+    return GQE_OK;
+  }
+  if (op == GQE_OP_ATTN_DECODE) {
+    GQE_REQUIRE(L_max >= 1, GQE_ERR_INVALID_ARG);
+    *bytes = decode_workspace_bytes(dims->B, dims->G, dims->k, dims->d_head, dims->n_shared, L_max);
+    return GQE_OK;
+  }
+  return GQE_ERR_INVALID_ARG;
+}
+
+gqe_status gqe_router_topk(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wr, const float* bias,
+                           int32_t* topk_idx, float* topk_w, float* probs, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(x && Wr && topk_idx && topk_w, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(x), GQE_ERR_INVALID_ARG);
+  RouterParams p{};
+  p.x = x;
+  p.Wr = Wr;
+  p.bias = bias;
+  p.topk_idx = topk_idx;
+  p.topk_w = topk_w;
+  p.probs = probs;
+  p.N = dims->B * dims->T;
+  p.D = dims->d_model;
+  p.G = dims->G;
+  p.E = dims->E;
+  p.k = dims->k;
+  p.scope = dims->renorm_scope;
+  return cuda_status(launch_router(p, S(stream)));
+}
+
+gqe_status gqe_routed_qproj(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wq, const gqe_bf16* Wsh,
+                            const int32_t* topk_idx, gqe_bf16* q_routed, gqe_bf16* q_sh, int32_t* expert_counts,
+                            void* ws, size_t ws_bytes, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(x && Wq && topk_idx && q_routed, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || (Wsh && q_sh), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(x) && aligned16(Wq) && aligned16(q_routed), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || (aligned16(Wsh) && aligned16(q_sh)), GQE_ERR_INVALID_ARG);
+  const int N = dims->B * dims->T, G = dims->G, E = dims->E, k = dims->k, d = dims->d_head, D = dims->d_model;
+  const PermLayout L = perm_layout(N, G, E, k);
+  GQE_REQUIRE(ws && aligned16(ws), GQE_ERR_WORKSPACE);
+  GQE_REQUIRE(ws_bytes >= L.bytes, GQE_ERR_WORKSPACE);
+
+  cudaError_t e = launch_permutation(topk_idx, N, dims->T, G, E, k, ws, L, expert_counts, S(stream));
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+
+  CUtensorMap mWq, mWsh;
+  GQE_REQUIRE(map2d(&mWq, Wq, D, (uint64_t)G * E * d, d), GQE_ERR_CUDA);
+  if (dims->n_shared) GQE_REQUIRE(map2d(&mWsh, Wsh, D, d, d), GQE_ERR_CUDA);
+  else mWsh = mWq;
+
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  RoutedParams rp{};
+  rp.src_row = reinterpret_cast<const int*>(w + L.off_src_row);
+  rp.dst_row = reinterpret_cast<const int*>(w + L.off_dst_row);
+  rp.seg_off = reinterpret_cast<const int*>(w + L.off_seg_off);
+  rp.seg_cnt = reinterpret_cast<const int*>(w + L.off_seg_cnt);
+  rp.tile_start = reinterpret_cast<const int*>(w + L.off_tile_start);
+  rp.n_seg = G * E;
+  rp.max_routed_tiles = L.n_entries / 128 + G * E;
+  rp.n_tokens = N;
+  rp.K = D;
+  rp.d = d;
+  EpiParams epr{};
+  epr.out0 = q_routed;
+  epr.mode = kEpiRows;
+  epr.ldo = d;
+  epr.n_limit = d;
+  epr.err = error_word();
+  EpiParams eps = epr;
+  eps.out0 = q_sh;
+  const int shared_tiles = dims->n_shared ? (N + 127) / 128 : 0;
+  return cuda_status(launch_gemm_routed(mWq, mWsh, x, rp, epr, eps, rp.max_routed_tiles + shared_tiles, S(stream)));
+}
+
+static gqe_status kv_common(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk, const gqe_bf16* Wv,
+                            EpiParams& ep, int M, gqe_stream stream) {
+  const int G = dims->G, d = dims->d_head, D = dims->d_model;
+  CUtensorMap mA, mK, mV;
+  GQE_REQUIRE(map2d(&mA, x, D, M, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mK, Wk, D, (uint64_t)G * d, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mV, Wv, D, (uint64_t)G * d, 128), GQE_ERR_CUDA);
+  ep.n_limit = G * d;
+  ep.G = G;
+  ep.d = d;
+  ep.err = error_word();
+  const int nt = (G * d + 127) / 128;
+  return cuda_status(launch_gemm_dense(mA, mK, mV, ep, M, D, nt, 2 * nt, S(stream)));
+}
+
+gqe_status gqe_kv_proj(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk, const gqe_bf16* Wv,
+                       gqe_bf16* K, gqe_bf16* V, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(x && Wk && Wv && K && V, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(x) && aligned16(Wk) && aligned16(Wv) && aligned16(K) && aligned16(V), GQE_ERR_INVALID_ARG);
+  EpiParams ep{};
+  ep.out0 = K;
+  ep.out1 = V;
+  ep.mode = kEpiHeads;
+  ep.T = dims->T;
+  return kv_common(dims, x, Wk, Wv, ep, dims->B * dims->T, stream);
+}
+
+gqe_status gqe_kv_append(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk, const gqe_bf16* Wv,
+                         gqe_bf16* Kc, gqe_bf16* Vc, int L_max, const int32_t* cache_len, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(dims->T == 1 && L_max >= 1, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(x && Wk && Wv && Kc && Vc && cache_len, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(x) && aligned16(Wk) && aligned16(Wv) && aligned16(Kc) && aligned16(Vc), GQE_ERR_INVALID_ARG);
+  EpiParams ep{};
+  ep.out0 = Kc;
+  ep.out1 = Vc;
+  ep.mode = kEpiCacheRow;
+  ep.cache_len = cache_len;
+  ep.L_max = L_max;
+  ep.T = 1;
+  return kv_common(dims, x, Wk, Wv, ep, dims->B, stream);
+}
+
+gqe_status gqe_attn_prefill(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh,
+                            const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* o_routed, gqe_bf16* o_sh, float* lse,
+                            gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(q_routed && K && V && o_routed, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || (q_sh && o_sh), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(q_routed) && aligned16(K) && aligned16(V) && aligned16(o_routed), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || (aligned16(q_sh) && aligned16(o_sh)), GQE_ERR_INVALID_ARG);
+  const int B = dims->B, T = dims->T, G = dims->G, k = dims->k, d = dims->d_head;
+  CUtensorMap mQ, mQs, mK, mV;
+  GQE_REQUIRE(map3d(&mQ, q_routed, d, (uint64_t)T * k, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  if (dims->n_shared) GQE_REQUIRE(map3d(&mQs, q_sh, d, T, B, 128), GQE_ERR_CUDA);
+  else mQs = mQ;
+  GQE_REQUIRE(map3d(&mK, K, d, T, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map3d(&mV, V, d, T, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  AttnParams p{};
+  p.o_routed = o_routed;
+  p.o_sh = o_sh;
+  p.lse = lse;
+  p.B = B;
+  p.T = T;
+  p.G = G;
+  p.k = k;
+  p.n_shared = dims->n_shared;
+  p.sg = dims->shared_kv_group;
+  p.scale_log2 = scale_log2(dims);
+  p.err = error_word();
+  return cuda_status(launch_attn_prefill(mQ, mQs, mK, mV, p, d, S(stream)));
+}
+
+gqe_status gqe_attn_decode(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh, const gqe_bf16* Kc,
+                           const gqe_bf16* Vc, int L_max, const int32_t* cache_len, gqe_bf16* o_routed,
+                           gqe_bf16* o_sh, void* ws, size_t ws_bytes, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(dims->T == 1 && L_max >= 1, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(q_routed && Kc && Vc && cache_len && o_routed, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || (q_sh && o_sh), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(q_routed) && aligned16(Kc) && aligned16(Vc), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || aligned16(q_sh), GQE_ERR_INVALID_ARG);
+  const int B = dims->B, G = dims->G, d = dims->d_head;
+  const size_t need = decode_workspace_bytes(B, G, dims->k, d, dims->n_shared, L_max);
+  GQE_REQUIRE(ws && aligned16(ws) && ws_bytes >= need, GQE_ERR_WORKSPACE);
+  CUtensorMap mK, mV;
+  GQE_REQUIRE(map3d(&mK, Kc, d, L_max, (uint64_t)B * G, 64), GQE_ERR_CUDA);
+  GQE_REQUIRE(map3d(&mV, Vc, d, L_max, (uint64_t)B * G, 64), GQE_ERR_CUDA);
+  DecodeParams p{};
+  p.q_routed = q_routed;
+  p.q_sh = q_sh;
+  p.Kc = Kc;
+  p.Vc = Vc;
+  p.cache_len = cache_len;
+  p.o_routed = o_routed;
+  p.o_sh = o_sh;
+  p.part = static_cast<float*>(ws);
+  p.B = B;
+  p.G = G;
+  p.k = dims->k;
+  p.d = d;
+  p.n_shared = dims->n_shared;
+  p.sg = dims->shared_kv_group;
+  p.L_max = L_max;
+  decode_split_plan(L_max, &p.chunk, &p.n_chunks);
+  p.nq_max = dims->k + dims->n_shared;
+  p.scale_log2 = scale_log2(dims);
+  p.err = error_word();
+  return cuda_status(launch_attn_decode_maps(mK, mV, p, S(stream)));
+}
+
+gqe_status gqe_combine(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe_bf16* o_sh, const float* topk_w,
+                       gqe_bf16* h, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(o_routed && topk_w && h, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || o_sh, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(o_routed) && aligned16(h) && (!dims->n_shared || aligned16(o_sh)), GQE_ERR_INVALID_ARG);
+  CombineParams p{};
+  p.o_routed = o_routed;
+  p.o_sh = o_sh;
+  p.w = topk_w;
+  p.h = h;
+  p.B = dims->B;
+  p.T = dims->T;
+  p.G = dims->G;
+  p.k = dims->k;
+  p.d = dims->d_head;
+  p.n_shared = dims->n_shared;
+  return cuda_status(launch_combine(p, S(stream)));
+}
+
+gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W, gqe_bf16* C, gqe_stream stream) {
+  GQE_REQUIRE(M >= 1 && N >= 1 && K >= 1, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(A && W && C, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(K % 64 == 0 && N % 64 == 0, GQE_ERR_UNSUPPORTED);
+  GQE_REQUIRE((long long)M * N < (1ll << 31) && (long long)M * K < (1ll << 31), GQE_ERR_UNSUPPORTED);
+  GQE_REQUIRE(aligned16(A) && aligned16(W) && aligned16(C), GQE_ERR_INVALID_ARG);
+  CUtensorMap mA, mW;
+  GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mW, W, K, N, 128), GQE_ERR_CUDA);
+  EpiParams ep{};
+  ep.out0 = C;
+  ep.out1 = C;
+  ep.mode = kEpiRowMajor;
+  ep.ldo = N;
+  ep.n_limit = N;
+  ep.err = error_word();
+  const int nt = (N + 127) / 128;
+  return cuda_status(launch_gemm_dense(mA, mW, mW, ep, M, K, nt, nt, S(stream)));
+}
+
+gqe_status gqe_device_error(int* code, gqe_stream stream) {
+  GQE_REQUIRE(code, GQE_ERR_INVALID_ARG);
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(v), 0, cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess)
+    return GQE_ERR_CUDA;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return GQE_ERR_CUDA;
+  *code = (int)v;
+  if (v) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, S(stream)) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(S(stream)) != cudaSuccess)
+      return GQE_ERR_CUDA;
+  }
+  return GQE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,42 @@
+// route.cuh -- parameters and launchers of the router, the token-to-expert
+// permutation and the output-construction kernels.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace gqe {
+
+struct RouterParams {
+  const uint16_t* x;      // [N, D] bf16
+  const uint16_t* Wr;     // [D, G*E] bf16
+  const float* bias;      // [G*E] or null
+  int* topk_idx;          // [N, G, k]
+  float* topk_w;          // [N, G, k]
+  float* probs;           // [N, G, E] or null
+  int N, D, G, E, k, scope;
+};
+cudaError_t launch_router(const RouterParams& p, cudaStream_t stream);
+
+// Token-to-expert permutation workspace (int32 arrays, see perm.cu).
+struct PermLayout {
+  int n_entries;     // N*G*k
+  int n_seg;         // G*E
+  int n_blocks;      // permutation blocks (chunks of entries)
+  size_t off_block_counts, off_block_base, off_seg_cnt, off_seg_off, off_tile_start;
+  size_t off_src_row, off_dst_row;
+  size_t bytes;
+};
+PermLayout perm_layout(int N, int G, int E, int k);
+cudaError_t launch_permutation(const int* topk_idx, int N, int T, int G, int E, int k, void* ws,
+                               const PermLayout& L, int* expert_counts, cudaStream_t stream);
+
+struct CombineParams {
+  const uint16_t* o_routed;   // [B, G, T, k, d]
+  const uint16_t* o_sh;       // [B, T, d]
+  const float* w;             // [N, G, k]
+  uint16_t* h;                // [N, slots*d]
+  int B, T, G, k, d, n_shared;
+};
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+}  // namespace gqe

@@ -1,0 +1,155 @@
+"""GQELayer: one GQE attention layer driven through the C ABI.
+
+PyTorch supplies device memory (weights, activations, scratch) and the CUDA
+stream; every step of the forward runs in libgqe.so's kernels:
+
+  prefill  gqe_router_topk -> gqe_routed_qproj -> gqe_kv_proj ->
+           gqe_attn_prefill -> gqe_combine -> gqe_linear (output projection)
+  decode   gqe_router_topk -> gqe_routed_qproj -> gqe_kv_append ->
+           gqe_attn_decode -> gqe_combine -> gqe_linear
+
+Weight layouts (bf16): Wr [D, G*E]; Wq [G, E, d, D]; Wk, Wv [G*d, D];
+Wsh [n_shared*d, D]; Wo [D, (k*G + 1 + n_shared)*d].
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import _lib as L
+
+
+@dataclasses.dataclass(frozen=True)
+class GQEConfig:
+    B: int
+    T: int
+    D: int
+    G: int
+    E: int
+    k: int
+    d: int
+    n_shared: int = 1
+    sg: int = 0
+    renorm_scope: int = 0
+    scale: float = 0.0
+
+    @property
+    def slots(self) -> int:
+        return self.k * self.G + 1 + self.n_shared
+
+
+def config_from(obj) -> GQEConfig:
+    return GQEConfig(**{f.name: getattr(obj, f.name) for f in dataclasses.fields(GQEConfig)
+                        if hasattr(obj, f.name)})
+
+
+class GQELayer:
+    """Holds a layer's weights on one GPU and runs its forward passes."""
+
+    def __init__(self, cfg, weights: dict, bias=None, device="cuda"):
+        if not torch.cuda.is_available():
+            raise RuntimeError("GQELayer needs a CUDA device; there is no CPU path")
+        self.cfg = config_from(cfg)
+        self.device = torch.device(device)
+        c = self.cfg
+
+        def dev(t, shape, dtype=torch.bfloat16):
+            t = torch.as_tensor(t)
+            if t.dtype == torch.int16 or t.dtype == torch.uint16:
+                t = t.view(torch.bfloat16) if t.dtype == torch.int16 else t.view(torch.int16).view(torch.bfloat16)
+            t = t.to(self.device, dtype).contiguous()
+            if tuple(t.shape) != tuple(shape):
+                raise ValueError(f"weight shape {tuple(t.shape)} != {tuple(shape)}")
+            return t
+
+        self.Wr = dev(weights["Wr"], (c.D, c.G * c.E))
+        self.Wq = dev(weights["Wq"], (c.G, c.E, c.d, c.D))
+        self.Wk = dev(weights["Wk"], (c.G * c.d, c.D))
+        self.Wv = dev(weights["Wv"], (c.G * c.d, c.D))
+        self.Wsh = dev(weights["Wsh"], (c.n_shared * c.d, c.D)) if c.n_shared else None
+        self.Wo = dev(weights["Wo"], (c.D, c.slots * c.d))
+        self.bias = None if bias is None else torch.as_tensor(bias, dtype=torch.float32).to(self.device).contiguous()
+        self._bufs = {}
+
+    # ------------------------------------------------------------------ buffers
+    def _buf(self, name, shape, dtype=torch.bfloat16):
+        t = self._bufs.get(name)
+        if t is None or tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+            t = torch.empty(shape, dtype=dtype, device=self.device)
+            self._bufs[name] = t
+        return t
+
+    def _ws(self, name, nbytes):
+        return self._buf(name, ((max(nbytes, 16) + 255) // 256 * 256,), torch.uint8)
+
+    # ------------------------------------------------------------------ prefill
+    def forward(self, x: torch.Tensor, stream=None, keep=False) -> torch.Tensor:
+        """x [B, T, D] bf16 on the device -> y [B, T, D] bf16.
+
+        keep=True also returns the intermediates (router outputs, q, K, V, o, h).
+        """
+        c = self.cfg
+        B, T = x.shape[0], x.shape[1]
+        dims = L.make_dims(c, B=B, T=T)
+        N = B * T
+        idx = self._buf("idx", (N, c.G, c.k), torch.int32)
+        w = self._buf("w", (N, c.G, c.k), torch.float32)
+        q = self._buf("q", (B, c.G, T, c.k, c.d))
+        qs = self._buf("qs", (B, T, c.d)) if c.n_shared else None
+        K = self._buf("K", (B, c.G, T, c.d))
+        V = self._buf("V", (B, c.G, T, c.d))
+        o = self._buf("o", (B, c.G, T, c.k, c.d))
+        os_ = self._buf("os", (B, T, c.d)) if c.n_shared else None
+        h = self._buf("h", (N, c.slots * c.d))
+        y = self._buf("y", (B, T, c.D))
+        ws = self._ws("ws_q", L.gqe_workspace_size(dims, L.GQE_OP_ROUTED_QPROJ))
+        L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, None, stream)
+        L.gqe_routed_qproj(dims, x, self.Wq, self.Wsh, idx, q, qs, ws, None, stream)
+        L.gqe_kv_proj(dims, x, self.Wk, self.Wv, K, V, stream)
+        L.gqe_attn_prefill(dims, q, qs, K, V, o, os_, None, stream)
+        L.gqe_combine(dims, o, os_, w, h, stream)
+        L.gqe_linear(h, self.Wo, y, stream)
+        if keep:
+            return y, dict(idx=idx, w=w, q=q, q_sh=qs, K=K, V=V, o=o, o_sh=os_, h=h)
+        return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None):
+        """End-to-end call on host buffers (pinned for async copies): copy x in,
+        run forward, copy y out, all enqueued on the stream."""
+        c = self.cfg
+        xd = self._buf("x_in", tuple(x_host.shape))
+        xd.copy_(x_host, non_blocking=True)
+        y = self.forward(xd, stream)
+        y_host.copy_(y, non_blocking=True)
+        return y_host
+
+    # ------------------------------------------------------------------ decode
+    def decode_step(self, x_new: torch.Tensor, Kc: torch.Tensor, Vc: torch.Tensor,
+                    cache_len: torch.Tensor, stream=None, keep=False) -> torch.Tensor:
+        """One new token per sequence.  x_new [B, D]; Kc, Vc [B, G, L_max, d]
+        (the new token's K/V are written at row cache_len[b]-1); cache_len [B]
+        int32 on the device.  Returns y [B, D]."""
+        c = self.cfg
+        B = x_new.shape[0]
+        L_max = Kc.shape[2]
+        dims = L.make_dims(c, B=B, T=1)
+        idx = self._buf("d_idx", (B, c.G, c.k), torch.int32)
+        w = self._buf("d_w", (B, c.G, c.k), torch.float32)
+        q = self._buf("d_q", (B, c.G, 1, c.k, c.d))
+        qs = self._buf("d_qs", (B, 1, c.d)) if c.n_shared else None
+        o = self._buf("d_o", (B, c.G, 1, c.k, c.d))
+        os_ = self._buf("d_os", (B, 1, c.d)) if c.n_shared else None
+        h = self._buf("d_h", (B, c.slots * c.d))
+        y = self._buf("d_y", (B, c.D))
+        wsq = self._ws("d_ws_q", L.gqe_workspace_size(dims, L.GQE_OP_ROUTED_QPROJ))
+        wsd = self._ws("d_ws_a", L.gqe_workspace_size(dims, L.GQE_OP_ATTN_DECODE, L_max))
+        L.gqe_router_topk(dims, x_new, self.Wr, self.bias, idx, w, None, stream)
+        L.gqe_routed_qproj(dims, x_new, self.Wq, self.Wsh, idx, q, qs, wsq, None, stream)
+        L.gqe_kv_append(dims, x_new, self.Wk, self.Wv, Kc, Vc, L_max, cache_len, stream)
+        L.gqe_attn_decode(dims, q, qs, Kc, Vc, L_max, cache_len, o, os_, wsd, stream)
+        L.gqe_combine(dims, o, os_, w, h, stream)
+        L.gqe_linear(h, self.Wo, y, stream)
+        if keep:
+            return y, dict(idx=idx, w=w, q=q, q_sh=qs, o=o, o_sh=os_, h=h)
+        return y

@@ -1,0 +1,386 @@
+"""Parity of every C-ABI call with the fp64 oracle on the same seeded inputs.
+
+Small shapes span several tiles with ragged tails and are compared element by
+element; the full workload sizes are compared on sampled rows the oracle
+computes one by one.  Tolerances: TopK indices exact except near-ties (logit
+margin < 1e-4, counted, the GPU's choice checked valid); router weights 1e-5;
+projections 2^-8 |ref| + 1e-3; attention outputs, h and y max-abs 2e-2 and
+mean-abs 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gqe_inputs as gi
+import oracle as orc
+from helpers import (ATTN_MAX_ABS, NEAR_TIE, W_TOL, assert_close_attn, assert_close_proj, bf16_dev,
+                     to_f64)
+
+pytestmark = pytest.mark.gpu
+
+gq = pytest.importorskip("moe_gqa_query_b200")
+
+
+@pytest.fixture(autouse=True)
+def _cuda_and_error_word():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    yield
+    torch.cuda.synchronize()
+    assert gq.gqe_device_error() == 0
+
+
+def D(**kw):
+    base = dict(B=1, T=128, D=256, G=2, E=2, k=1, d=64)
+    base.update(kw)
+    return gi.GQEDims(**base)
+
+
+def dims_c(dims, **over):
+    return gq.make_dims(dims, **over)
+
+
+# ----------------------------------------------------------------------------
+# router
+
+ROUTER_CASES = {
+    "tiny": (gi.WORKLOADS["tiny_prefill"], None),
+    "ragged_odd_GE": (gi.Workload("r", D(B=2, T=77, D=128, G=3, E=3, k=2)), None),
+    "group_scope": (gi.Workload("g", D(B=1, T=200, D=192, G=4, E=4, k=2, renorm_scope=1)), None),
+    "main": (gi.WORKLOADS["main_prefill"], None),
+    "long": (gi.WORKLOADS["long_prefill"], None),
+    "wide_skewed": (gi.WORKLOADS["wide_skewed_prefill"], None),
+}
+
+
+def check_router(w: gi.Workload, seed=0):
+    dims = w.dims
+    x = gi.layer_input(dims, seed)
+    Wt = gi.layer_weights(dims, seed)
+    bias = gi.router_bias(w, seed)
+    N, G, E, k = dims.N, dims.G, dims.E, dims.k
+    idx = torch.empty((N, G, k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((N, G, k), dtype=torch.float32, device="cuda")
+    probs = torch.empty((N, G, E), dtype=torch.float32, device="cuda")
+    gq.gqe_router_topk(dims_c(dims), bf16_dev(x), bf16_dev(Wt["Wr"]),
+                       None if bias is None else torch.from_numpy(bias).cuda(), idx, wt, probs)
+    torch.cuda.synchronize()
+    r = orc.router_topk(orc.f64(x).reshape(N, -1), Wt["Wr"], G, E, k, bias, dims.renorm_scope)
+    gi_idx = idx.cpu().numpy()
+    tie = r["margin"] < NEAR_TIE
+    same = np.all(gi_idx == r["idx"], axis=-1)
+    assert np.all(same | tie), f"{int((~same & ~tie).sum())} routing decisions differ outside near-ties"
+    # near-ties: the GPU's set must contain every sure expert and only undecided others
+    for (t, g), (sure, undecided) in orc.near_tie_alternatives(r, k).items():
+        chosen = set(gi_idx[t, g].tolist())
+        assert set(sure.tolist()) <= chosen and chosen <= set(sure.tolist()) | set(undecided.tolist())
+    assert np.all(np.diff(gi_idx, axis=-1) > 0) if k > 1 else True
+    np.testing.assert_allclose(probs.cpu().numpy(), r["probs"], atol=W_TOL)
+    tok_ok = ~tie.any(axis=1)
+    np.testing.assert_allclose(wt.cpu().numpy()[tok_ok], r["w"][tok_ok], atol=W_TOL)
+    return int(tie.sum())
+
+
+@pytest.mark.parametrize("case", list(ROUTER_CASES))
+def test_router_topk(case):
+    w, _ = ROUTER_CASES[case]
+    n_ties = check_router(w)
+    print(f"[router {case}] near-ties: {n_ties}")
+
+
+# ----------------------------------------------------------------------------
+# routed + shared query projection
+
+QPROJ_CASES = {
+    "tiny": (gi.WORKLOADS["tiny_prefill"].dims, 0.0, None),
+    "ragged_k2": (D(B=2, T=77, D=128, G=3, E=4, k=2), 0.0, None),
+    "wide_k4_skew_d128": (D(B=1, T=300, D=256, G=2, E=8, k=4, d=128), 0.8, None),
+    "no_shared": (D(B=1, T=129, D=64, G=2, E=3, k=1, n_shared=0), 0.0, None),
+    "main": (gi.WORKLOADS["main_prefill"].dims, 0.0, None),
+    "wide_skewed_sampled": (gi.WORKLOADS["wide_skewed_prefill"].dims, 0.8, 96),
+}
+
+
+@pytest.mark.parametrize("case", list(QPROJ_CASES))
+def test_routed_qproj(case):
+    dims, skew, n_sample = QPROJ_CASES[case]
+    x = gi.layer_input(dims, 1)
+    Wt = gi.layer_weights(dims, 1)
+    idx = gi.random_routing(dims, 1, skew0=skew)
+    N, G, k, d = dims.N, dims.G, dims.k, dims.d
+    q = torch.empty((dims.B, G, dims.T, k, d), dtype=torch.bfloat16, device="cuda")
+    qs = torch.empty((dims.B, dims.T, d), dtype=torch.bfloat16, device="cuda") if dims.n_shared else None
+    cnt = torch.empty((G * dims.E,), dtype=torch.int32, device="cuda")
+    dc = dims_c(dims)
+    ws = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_ROUTED_QPROJ),), dtype=torch.uint8, device="cuda")
+    gq.gqe_routed_qproj(dc, bf16_dev(x), bf16_dev(Wt["Wq"]), bf16_dev(Wt["Wsh"]) if dims.n_shared else None,
+                        torch.from_numpy(idx).cuda(), q, qs, ws, cnt)
+    torch.cuda.synchronize()
+    hist = np.bincount((np.arange(G)[None, :, None] * dims.E + idx).reshape(-1), minlength=G * dims.E)
+    assert np.array_equal(cnt.cpu().numpy(), hist)
+    xf = orc.f64(x).reshape(N, -1)
+    rows = np.arange(N) if n_sample is None else np.sort(np.random.default_rng(5).choice(N, n_sample, replace=False))
+    sub = gi.GQEDims(B=1, T=len(rows), D=dims.D, G=G, E=dims.E, k=k, d=d, n_shared=dims.n_shared)
+    q_ref, qs_ref = orc.routed_qproj(xf[rows], Wt["Wq"], Wt["Wsh"], idx[rows], sub)
+    q_gpu = to_f64(q).transpose(0, 2, 1, 3, 4).reshape(N, G, k, d)[rows]
+    assert_close_proj(q_gpu, q_ref[0].transpose(1, 0, 2, 3), "q_routed")
+    if dims.n_shared:
+        assert_close_proj(to_f64(qs).reshape(N, d)[rows], qs_ref[0], "q_sh")
+
+
+# ----------------------------------------------------------------------------
+# dense K/V projection, output projection
+
+@pytest.mark.parametrize("dims", [gi.WORKLOADS["tiny_prefill"].dims, D(B=2, T=77, D=128, G=3, E=2, k=1),
+                                  D(B=1, T=130, D=192, G=1, E=2, k=1, d=128), gi.WORKLOADS["main_prefill"].dims],
+                         ids=["tiny", "ragged_G3", "G1_d128", "main"])
+def test_kv_proj(dims):
+    x = gi.layer_input(dims, 2)
+    Wt = gi.layer_weights(dims, 2)
+    K = torch.empty((dims.B, dims.G, dims.T, dims.d), dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    gq.gqe_kv_proj(dims_c(dims), bf16_dev(x), bf16_dev(Wt["Wk"]), bf16_dev(Wt["Wv"]), K, V)
+    torch.cuda.synchronize()
+    K_ref, V_ref = orc.kv_proj(orc.f64(x).reshape(dims.N, -1), Wt["Wk"], Wt["Wv"], dims)
+    assert_close_proj(to_f64(K), K_ref, "K")
+    assert_close_proj(to_f64(V), V_ref, "V")
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 192, 320), (16, 64, 64), (1000, 256, 640), (16384, 1024, 640)])
+def test_linear(M, N, K):
+    rng_dims = gi.GQEDims(B=1, T=M, D=K, G=1, E=1, k=1, d=64)
+    A = gi.normal_bf16(3, "x", (M, K), 1.0)
+    W = gi.normal_bf16(3, "Wo", (N, K), 0.02)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    gq.gqe_linear(bf16_dev(A), bf16_dev(W), C)
+    torch.cuda.synchronize()
+    assert_close_proj(to_f64(C), orc.linear(A, W), "linear")
+    del rng_dims
+
+
+# ----------------------------------------------------------------------------
+# routed causal attention (prefill)
+
+def _attn_inputs(dims, seed):
+    B, G, T, k, d = dims.B, dims.G, dims.T, dims.k, dims.d
+    q = gi.normal_bf16(seed, "q", (B, G, T, k, d))
+    qs = gi.normal_bf16(seed, "qsh", (B, T, d))
+    K = gi.normal_bf16(seed, "K", (B, G, T, d))
+    V = gi.normal_bf16(seed, "V", (B, G, T, d))
+    return q, qs, K, V
+
+
+def _run_prefill(dims, q, qs, K, V, want_lse=True):
+    B, G, T, k, d = dims.B, dims.G, dims.T, dims.k, dims.d
+    o = torch.full((B, G, T, k, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    os_ = torch.full((B, T, d), float("nan"), dtype=torch.bfloat16, device="cuda") if dims.n_shared else None
+    lse = torch.empty((B * G * T * k + B * T * dims.n_shared,), dtype=torch.float32, device="cuda") if want_lse else None
+    gq.gqe_attn_prefill(dims_c(dims), bf16_dev(q), bf16_dev(qs) if dims.n_shared else None, bf16_dev(K),
+                        bf16_dev(V), o, os_, lse)
+    torch.cuda.synchronize()
+    return o, os_, lse
+
+
+PREFILL_SMALL = {
+    "tiny": D(),
+    "ragged_k2_sg1": D(B=2, T=300, G=3, E=2, k=2, sg=1),
+    "k4_d128_ragged": D(B=1, T=257, G=2, E=4, k=4, d=128),
+    "single_token": D(B=2, T=1, G=2, E=2, k=2),
+    "k3_no_shared": D(B=2, T=50, G=1, E=3, k=3, n_shared=0),
+    "k1_d128_multi_tile": D(B=1, T=520, G=2, E=2, k=1, d=128, sg=1),
+    "k8_E8": D(B=1, T=70, G=1, E=8, k=8),
+}
+
+
+@pytest.mark.parametrize("case", list(PREFILL_SMALL))
+def test_attn_prefill_small(case):
+    dims = PREFILL_SMALL[case]
+    q, qs, K, V = _attn_inputs(dims, 7)
+    o, os_, lse = _run_prefill(dims, q, qs, K, V)
+    o_ref, os_ref, lse_ref, lsesh_ref = orc.attn_prefill(q, qs, K, V, dims)
+    assert_close_attn(to_f64(o), o_ref, "o_routed")
+    n_r = dims.B * dims.G * dims.T * dims.k
+    np.testing.assert_allclose(lse.cpu().numpy()[:n_r], lse_ref.reshape(-1), atol=2e-3, rtol=1e-3)
+    if dims.n_shared:
+        assert_close_attn(to_f64(os_), os_ref, "o_sh")
+        np.testing.assert_allclose(lse.cpu().numpy()[n_r:], lsesh_ref.reshape(-1), atol=2e-3, rtol=1e-3)
+
+
+def test_attn_prefill_constant_keys_prefix_mean():
+    """At any size: equal keys give the causal prefix mean of V."""
+    dims = D(B=1, T=1000, G=2, E=2, k=2, d=64)
+    q, qs, _, V = _attn_inputs(dims, 8)
+    K = np.broadcast_to(gi.normal_bf16(8, "K", (1, 2, 1, 64)), (1, 2, 1000, 64)).copy()
+    o, os_, _ = _run_prefill(dims, q, qs, K, V, want_lse=False)
+    Vf = orc.f64(V)
+    pm = np.cumsum(Vf, axis=2) / np.arange(1, 1001)[None, None, :, None]
+    assert_close_attn(to_f64(o), np.repeat(pm[:, :, :, None, :], 2, axis=3), "prefix mean")
+    assert_close_attn(to_f64(os_), pm[:, 0], "prefix mean shared")
+
+
+@pytest.mark.parametrize("wname", ["main_prefill", "long_prefill", "wide_skewed_prefill"])
+def test_attn_prefill_full_size_sampled(wname):
+    """Full workload size, bench launch configuration; sampled rows vs the oracle."""
+    dims = gi.WORKLOADS[wname].dims
+    B, G, T, k, d = dims.B, dims.G, dims.T, dims.k, dims.d
+    q, qs, K, V = _attn_inputs(dims, 9)
+    o, os_, lse = _run_prefill(dims, q, qs, K, V)
+    rng = np.random.default_rng(11)
+    picks = [(int(rng.integers(B)), int(rng.integers(G)), int(t)) for t in
+             list(rng.integers(0, T, 24)) + [0, T - 1, 127, 128]]
+    got = to_f64(o)
+    for b, g, t in picks:
+        ref = orc.causal_attention(q[b, g, t], np.full(k, t), K[b, g], V[b, g], dims.sm_scale)
+        err = np.abs(got[b, g, t] - ref).max()
+        assert err <= ATTN_MAX_ABS, (b, g, t, err)
+    gsh = to_f64(os_)
+    for b, _, t in picks:
+        ref = orc.causal_attention(qs[b, t][None], np.array([t]), K[b, dims.sg], V[b, dims.sg], dims.sm_scale)[0]
+        assert np.abs(gsh[b, t] - ref).max() <= ATTN_MAX_ABS
+    assert torch.isfinite(o.float()).all() and torch.isfinite(os_.float()).all()
+
+
+# ----------------------------------------------------------------------------
+# decode attention
+
+def _run_decode(dims, L_max, lens, seed, rows=None):
+    B, G, k, d = dims.B, dims.G, dims.k, dims.d
+    q = gi.normal_bf16(seed, "q", (B, G, k, d))
+    qs = gi.normal_bf16(seed, "qsh", (B, d))
+    dev_K = torch.empty((B, G, L_max, d), dtype=torch.bfloat16, device="cuda")
+    dev_V = torch.empty_like(dev_K)
+    host = {}
+    gen_rows = range(B) if rows is None else rows
+    if rows is not None:
+        g_ = torch.Generator(device="cuda").manual_seed(seed)
+        dev_K.normal_(generator=g_)
+        dev_V.normal_(generator=g_)
+    for b in gen_rows:
+        Kb = gi.normal_bf16(seed, "Kc", (B, G, L_max, d), rows=[b])[0]
+        Vb = gi.normal_bf16(seed, "Vc", (B, G, L_max, d), rows=[b])[0]
+        dev_K[b] = bf16_dev(Kb)
+        dev_V[b] = bf16_dev(Vb)
+        host[b] = (Kb, Vb)
+    dc = dims_c(dims)
+    ws = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_ATTN_DECODE, L_max),), dtype=torch.uint8, device="cuda")
+    o = torch.full((B, G, k, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    os_ = torch.full((B, d), float("nan"), dtype=torch.bfloat16, device="cuda") if dims.n_shared else None
+    cl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    gq.gqe_attn_decode(dc, bf16_dev(q), bf16_dev(qs) if dims.n_shared else None, dev_K, dev_V, L_max, cl, o, os_, ws)
+    torch.cuda.synchronize()
+    return q, qs, host, to_f64(o), (to_f64(os_) if dims.n_shared else None)
+
+
+@pytest.mark.parametrize("case", [
+    dict(dims=D(B=3, T=1, G=2, E=2, k=2, d=64), L=300, lens=[300, 1, 150]),
+    dict(dims=D(B=2, T=1, G=3, E=4, k=3, d=128, sg=2), L=257, lens=[257, 64]),
+    dict(dims=D(B=2, T=1, G=2, E=2, k=1, d=64, n_shared=0), L=4096, lens=[4096, 4000]),
+    dict(dims=D(B=1, T=1, G=1, E=8, k=8, d=64), L=1000, lens=[999]),
+], ids=["ragged", "d128_sg2", "no_shared_long", "k8"])
+def test_attn_decode_small(case):
+    dims, L_max, lens = case["dims"], case["L"], case["lens"]
+    q, qs, host, o, os_ = _run_decode(dims, L_max, lens, 21)
+    for b in range(dims.B):
+        n = lens[b]
+        Kb, Vb = host[b]
+        for g in range(dims.G):
+            ref = orc.causal_attention(q[b, g], np.full(dims.k, n - 1), Kb[g, :n], Vb[g, :n], dims.sm_scale)
+            assert_close_attn(o[b, g], ref, f"decode b{b} g{g}")
+        if dims.n_shared:
+            ref = orc.causal_attention(qs[b][None], np.array([n - 1]), Kb[dims.sg, :n], Vb[dims.sg, :n],
+                                       dims.sm_scale)[0]
+            assert_close_attn(os_[b], ref, f"decode shared b{b}")
+
+
+def test_attn_decode_full_size_sampled():
+    """The decode workload (64 x 8 x 32768 x 64 cache): sampled sequences vs the oracle."""
+    w = gi.WORKLOADS["decode"]
+    dims, L_max = w.dims, w.L
+    rows = [0, 37, 63]
+    q, qs, host, o, os_ = _run_decode(dims, L_max, [L_max] * dims.B, 31, rows=rows)
+    for b in rows:
+        Kb, Vb = host[b]
+        for g in range(dims.G):
+            ref = orc.causal_attention(q[b, g], np.full(dims.k, L_max - 1), Kb[g], Vb[g], dims.sm_scale)
+            assert_close_attn(o[b, g], ref, f"decode b{b} g{g}")
+        ref = orc.causal_attention(qs[b][None], np.array([L_max - 1]), Kb[dims.sg], Vb[dims.sg], dims.sm_scale)[0]
+        assert_close_attn(os_[b], ref, f"decode shared b{b}")
+    assert np.isfinite(o).all()
+
+
+# ----------------------------------------------------------------------------
+# output construction
+
+@pytest.mark.parametrize("dims", [D(), D(B=2, T=33, G=3, E=4, k=2, d=128), D(B=1, T=10, G=2, E=2, k=1, n_shared=0),
+                                  gi.WORKLOADS["main_prefill"].dims], ids=["tiny", "k2_d128", "no_shared", "main"])
+def test_combine(dims):
+    B, G, T, k, d = dims.B, dims.G, dims.T, dims.k, dims.d
+    o = gi.normal_bf16(4, "o", (B, G, T, k, d))
+    osh = gi.normal_bf16(4, "osh", (B, T, d))
+    w = gi.random_weights_simplex(dims, 4)
+    h = torch.full((dims.N, dims.slots * d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gq.gqe_combine(dims_c(dims), bf16_dev(o), bf16_dev(osh) if dims.n_shared else None,
+                   torch.from_numpy(w).cuda(), h)
+    torch.cuda.synchronize()
+    ref = orc.combine(o, osh, w.astype(np.float64), dims)
+    got = to_f64(h)
+    hard = G * k * d
+    assert np.array_equal(got[:, :hard], ref[:, :hard])                       # copies: exact
+    if dims.n_shared:
+        assert np.array_equal(got[:, hard + d:], ref[:, hard + d:])
+    np.testing.assert_allclose(got[:, hard:hard + d], ref[:, hard:hard + d], rtol=2 ** -8, atol=1e-6)
+
+
+# ----------------------------------------------------------------------------
+# whole layer
+
+def _layer(w: gi.Workload, seed=0):
+    dims = w.dims
+    x = gi.layer_input(dims, seed)
+    Wt = gi.layer_weights(dims, seed)
+    bias = gi.router_bias(w, seed)
+    layer = gq.GQELayer(dims, {k_: torch.from_numpy(v.view(np.int16)) for k_, v in Wt.items()}, bias)
+    return dims, x, Wt, bias, layer
+
+
+@pytest.mark.parametrize("wname", ["tiny_prefill", "main_prefill"])
+def test_layer_forward_end_to_end(wname):
+    w = gi.WORKLOADS[wname]
+    dims, x, Wt, bias, layer = _layer(w)
+    y, inter = layer.forward(bf16_dev(x), keep=True)
+    torch.cuda.synchronize()
+    ref = orc.gqe_forward(x, Wt, dims, bias)
+    r = ref["router"]
+    tie_tok = (r["margin"] < NEAR_TIE).any(axis=1)
+    gi_idx = inter["idx"].cpu().numpy()
+    agree = np.all(gi_idx == r["idx"], axis=(1, 2))
+    assert np.all(agree | tie_tok)
+    keep = agree          # rows routed identically; near-tie rows that differ are valid alternatives
+    yg = to_f64(y).reshape(dims.N, -1)
+    mx, mean = assert_close_attn(yg[keep], ref["y"][keep], "y")
+    assert_close_attn(to_f64(inter["h"])[keep], ref["h"][keep], "h")
+    print(f"[layer {wname}] y max-abs {mx:.3e} mean-abs {mean:.3e}; near-tie tokens {int(tie_tok.sum())}, "
+          f"differently routed {int((~agree).sum())}")
+
+
+def test_layer_decode_step_end_to_end():
+    w = gi.Workload("dec_small", D(B=4, T=1, D=256, G=2, E=4, k=2, d=64), decode=True, L=700)
+    dims = w.dims
+    x = gi.normal_bf16(0, "xdec", (dims.B, dims.D))
+    Wt = gi.layer_weights(dims, 0)
+    layer = gq.GQELayer(dims, {k_: torch.from_numpy(v.view(np.int16)) for k_, v in Wt.items()})
+    L_max = 700
+    lens = np.array([700, 1, 333, 512])
+    Kc = gi.normal_bf16(0, "Kc", (dims.B, dims.G, L_max, dims.d))
+    Vc = gi.normal_bf16(0, "Vc", (dims.B, dims.G, L_max, dims.d))
+    dK, dV = bf16_dev(Kc), bf16_dev(Vc)
+    y, inter = layer.decode_step(bf16_dev(x), dK, dV, torch.from_numpy(lens.astype(np.int32)).cuda(), keep=True)
+    torch.cuda.synchronize()
+    ref = orc.decode_step(x, Wt, Kc, Vc, lens, dims)
+    # the cache rows written by the step
+    for b in range(dims.B):
+        assert_close_attn(to_f64(dK[b, :, lens[b] - 1]), ref["Knew"][b, :, 0], "K append")
+    gi_idx = inter["idx"].cpu().numpy()
+    agree = np.all(gi_idx == ref["router"]["idx"], axis=(1, 2))
+    assert np.all(agree | (ref["router"]["margin"] < NEAR_TIE).any(axis=1))
+    assert_close_attn(to_f64(y)[agree], ref["y"][agree], "decode y")
