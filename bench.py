@@ -225,6 +225,85 @@ def run_reference(args):
     return 0
 
 
+def run_kernel(args):
+    """One call of the path in isolation on its workload's inputs (for profiling)."""
+    import torch
+    import moe_gqa_query_b200 as gq
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    if args.kernel == "decode":
+        w = gi.WORKLOADS[DECODE_WORKLOAD]
+        dd, Lc = w.dims, w.L
+        gen = torch.Generator(device=device).manual_seed(7)
+        Kc = torch.empty((dd.B, dd.G, Lc, dd.d), dtype=torch.bfloat16, device=device).normal_(generator=gen)
+        Vc = torch.empty_like(Kc).normal_(generator=gen)
+        dc = gq.make_dims(dd, T=1)
+        ws = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_ATTN_DECODE, Lc),), dtype=torch.uint8, device=device)
+        q = torch.randn((dd.B, dd.G, 1, dd.k, dd.d), device=device, generator=gen).to(torch.bfloat16)
+        qs = torch.randn((dd.B, 1, dd.d), device=device, generator=gen).to(torch.bfloat16)
+        o, os_ = torch.empty_like(q), torch.empty_like(qs)
+        cl = torch.full((dd.B,), Lc, dtype=torch.int32, device=device)
+        fn = lambda: gq.gqe_attn_decode(dc, q, qs, Kc, Vc, Lc, cl, o, os_, ws)  # noqa: E731
+        work = dict(bytes=decode_attn_bytes(dd, Lc))
+    else:
+        w = gi.WORKLOADS[args.workload]
+        dims = w.dims
+        dc = gq.make_dims(dims)
+        gen = torch.Generator(device=device).manual_seed(7)
+
+        def rn(*shape, std=1.0):
+            return (torch.randn(shape, device=device, generator=gen) * std).to(torch.bfloat16)
+        B, T, G, E, k, d, D = dims.B, dims.T, dims.G, dims.E, dims.k, dims.d, dims.D
+        if args.kernel == "attn":
+            q, qs, K, V = rn(B, G, T, k, d), rn(B, T, d), rn(B, G, T, d), rn(B, G, T, d)
+            o, os_ = torch.empty_like(q), torch.empty_like(qs)
+            fn = lambda: gq.gqe_attn_prefill(dc, q, qs, K, V, o, os_, None)  # noqa: E731
+            work = dict(flops=attn_useful_flops(dims))
+        elif args.kernel in ("router", "qproj", "kv", "linear", "combine"):
+            x = rn(B, T, D)
+            Wt = gi.layer_weights(dims)
+            lay = gq.GQELayer(dims, {kk: torch.from_numpy(v.view(np.int16)) for kk, v in Wt.items()},
+                              gi.router_bias(w), device=device)
+            y, inter = lay.forward(x, keep=True)
+            if args.kernel == "router":
+                fn = lambda: gq.gqe_router_topk(dc, x, lay.Wr, lay.bias, inter["idx"], inter["w"], None)  # noqa
+                work = dict(bytes=dims.N * D * 2.0)
+            elif args.kernel == "qproj":
+                ws = lay._bufs["ws_q"]
+                fn = lambda: gq.gqe_routed_qproj(dc, x, lay.Wq, lay.Wsh, inter["idx"], inter["q"], inter["q_sh"], ws)  # noqa
+                work = dict(flops=2.0 * dims.N * dims.h_active * d * D)
+            elif args.kernel == "kv":
+                fn = lambda: gq.gqe_kv_proj(dc, x, lay.Wk, lay.Wv, inter["K"], inter["V"])  # noqa
+                work = dict(flops=2.0 * 2 * dims.N * G * d * D)
+            elif args.kernel == "combine":
+                fn = lambda: gq.gqe_combine(dc, inter["o"], inter["o_sh"], inter["w"], inter["h"])  # noqa
+                work = dict(bytes=2.0 * dims.N * (G * k + 1) * d + 2.0 * dims.N * dims.slots * d)
+            else:
+                fn = lambda: gq.gqe_linear(inter["h"], lay.Wo, y)  # noqa
+                work = dict(flops=2.0 * dims.N * dims.slots * d * D)
+        else:
+            raise SystemExit(f"unknown kernel {args.kernel}")
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    out = {"kernel": args.kernel, "workload": DECODE_WORKLOAD if args.kernel == "decode" else args.workload,
+           "ms": ms, "device_error": gq.gqe_device_error()}
+    if "flops" in work:
+        out["TFLOP/s"] = work["flops"] / ms / 1e9
+    if "bytes" in work:
+        out["GB/s"] = work["bytes"] / ms / 1e6
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -233,9 +312,14 @@ def main():
     ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--kernel", default=None,
+                    help="time one call alone: attn | decode | router | qproj | kv | combine | linear")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[k for k, v in gi.WORKLOADS.items() if not v.decode])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.kernel:
+        return run_kernel(args)
     args.warmup = max(args.warmup, 3)
 
     world, rank, local = dist_env()

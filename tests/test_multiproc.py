@@ -1,0 +1,58 @@
+"""Host logic of the N-GPU benchmark (independent replicas) on CPU ranks.
+
+The GQE path does not shard across GPUs here: each rank runs its own replica.
+The only cross-rank steps are the barrier around the timed region and the max
+over ranks of the measured time; these run as world_size-2 gloo ranks.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import bench
+    w, r, local = bench.dist_env()
+    assert (w, r, local) == (world, rank, rank)
+    dist = bench.init_dist(world, "gloo")
+    bench.barrier(dist)
+    local_ms = 10.0 + 5.0 * rank            # rank 1 is the slow one
+    total = bench.max_over_ranks(local_ms, dist)
+    out[rank] = total
+    bench.barrier(dist)
+    dist.destroy_process_group()
+
+
+def test_two_rank_max_over_ranks():
+    world = 2
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+    assert out[0] == out[1] == 15.0
+
+
+def test_single_rank_has_no_process_group():
+    import bench
+    assert bench.init_dist(1, "gloo") is None
+    assert bench.max_over_ranks(3.5, None) == 3.5
+
+
+def test_work_counts():
+    import bench
+    import gqe_inputs as gi
+    main = gi.WORKLOADS["main_prefill"].dims
+    assert bench.attn_useful_flops(main) == pytest.approx(3.867e10, rel=1e-3)
+    dec = gi.WORKLOADS["decode"]
+    assert bench.decode_attn_bytes(dec.dims, dec.L) == pytest.approx(4.295e9, rel=1e-3)
