@@ -248,7 +248,8 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeParams p) {
     float L = 0.f, A = 0.f;
     for (int c = 0; c < p.n_chunks; ++c) {
       const float* s = base + (c * p.nq_max + qi) * (D + 2);
-      const float f = (s[0] == -INFINITY) ? 0.f : ex2(s[0] - M);
+      if (s[0] == -INFINITY) continue;   // chunk past cache_len: its acc was never written
+      const float f = ex2(s[0] - M);
       L += s[1] * f;
       A += s[2 + dim] * f;
     }

@@ -243,7 +243,7 @@ def test_attn_prefill_full_size_sampled(wname):
 # ----------------------------------------------------------------------------
 # decode attention
 
-def _run_decode(dims, L_max, lens, seed, rows=None):
+def _run_decode(dims, L_max, lens, seed, rows=None, ws_fill=None):
     B, G, k, d = dims.B, dims.G, dims.k, dims.d
     q = gi.normal_bf16(seed, "q", (B, G, k, d))
     qs = gi.normal_bf16(seed, "qsh", (B, d))
@@ -263,6 +263,8 @@ def _run_decode(dims, L_max, lens, seed, rows=None):
         host[b] = (Kb, Vb)
     dc = dims_c(dims)
     ws = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_ATTN_DECODE, L_max),), dtype=torch.uint8, device="cuda")
+    if ws_fill is not None:
+        ws.view(torch.float32).fill_(ws_fill)
     o = torch.full((B, G, k, d), float("nan"), dtype=torch.bfloat16, device="cuda")
     os_ = torch.full((B, d), float("nan"), dtype=torch.bfloat16, device="cuda") if dims.n_shared else None
     cl = torch.tensor(lens, dtype=torch.int32, device="cuda")
@@ -273,13 +275,14 @@ def _run_decode(dims, L_max, lens, seed, rows=None):
 
 @pytest.mark.parametrize("case", [
     dict(dims=D(B=3, T=1, G=2, E=2, k=2, d=64), L=300, lens=[300, 1, 150]),
+    dict(dims=D(B=2, T=1, G=2, E=2, k=1, d=64), L=40000, lens=[40000, 3000], nan_ws=True),
     dict(dims=D(B=2, T=1, G=3, E=4, k=3, d=128, sg=2), L=257, lens=[257, 64]),
     dict(dims=D(B=2, T=1, G=2, E=2, k=1, d=64, n_shared=0), L=4096, lens=[4096, 4000]),
     dict(dims=D(B=1, T=1, G=1, E=8, k=8, d=64), L=1000, lens=[999]),
-], ids=["ragged", "d128_sg2", "no_shared_long", "k8"])
+], ids=["ragged", "short_len_nan_scratch", "d128_sg2", "no_shared_long", "k8"])
 def test_attn_decode_small(case):
     dims, L_max, lens = case["dims"], case["L"], case["lens"]
-    q, qs, host, o, os_ = _run_decode(dims, L_max, lens, 21)
+    q, qs, host, o, os_ = _run_decode(dims, L_max, lens, 21, ws_fill=float("nan") if case.get("nan_ws") else None)
     for b in range(dims.B):
         n = lens[b]
         Kb, Vb = host[b]
