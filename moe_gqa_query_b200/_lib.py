@@ -4,7 +4,7 @@ Every function here has the name of the C entry point it calls, takes torch
 tensors that already live on the GPU (or raw integer pointers), passes their
 device pointers, the shape struct and the current CUDA stream to the library,
 and raises GQEError on a non-zero status.  No step of the computation happens
-in Python.  The library must be built (python -m moe_gqa_query_b200.build);
+in Python.  The library must be built (python moe_gqa_query_b200/build.py);
 importing this module without it raises ImportError.
 """
 from __future__ import annotations
@@ -77,7 +77,7 @@ def header_functions(path: str = HEADER_PATH):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m moe_gqa_query_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python moe_gqa_query_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     for name, args in SIGNATURES.items():
         fn = getattr(lib, name)

@@ -1,6 +1,6 @@
 """Builds the in-tree CUDA library libgqe.so for sm_100a (B200).
 
-Usage:  python -m moe_gqa_query_b200.build   (or build_library() from Python)
+Usage:  python moe_gqa_query_b200/build.py   (or build_library() from Python)
 """
 from __future__ import annotations
 
