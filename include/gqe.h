@@ -135,6 +135,33 @@ gqe_status gqe_attn_decode(const gqe_dims* dims, const gqe_bf16* q_routed,
                            int L_max, const int32_t* cache_len, gqe_bf16* o_routed,
                            gqe_bf16* o_sh, void* ws, size_t ws_bytes, gqe_stream stream);
 
+/* Decode attention that allocates nothing and takes no scratch buffer.  The
+ * GQE pages have no counterpart to this call: it exists for callers that
+ * cannot allocate device memory when they decode, such as a serving engine
+ * that reserved all device memory for its own pool at start-up (a
+ * library-side allocation would fail or bypass its accounting), or a
+ * latency-bound decode loop that cannot afford cudaMalloc's implicit device
+ * synchronisation.
+ *   Arguments and results are those of gqe_attn_decode without ws/ws_bytes.
+ *   The split-L partial states live in one array inside the library,
+ *   GQE_DECODE_NOALLOC_MAX_BYTES (8 MiB) of device memory that every GPU that
+ *   loads the library holds until the process exits.  Dims and L_max whose
+ *   partial states need more (gqe_workspace_size(GQE_OP_ATTN_DECODE) larger
+ *   than the maximum) are rejected with GQE_ERR_WORKSPACE before anything is
+ *   launched.  The 64-sequence, 8-group, 32768-key main-layer decode needs 4.3 MB.
+ *   The first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture.
+ *   Every call shares the array and it keeps the last call's contents (each
+ *   slot a call reads is written earlier in the same call, so nothing needs
+ *   clearing).  Calls that can overlap on the GPU, e.g. on two streams with no
+ *   ordering between them, race on the array and corrupt each other's
+ *   results: serialise them. */
+#define GQE_DECODE_NOALLOC_MAX_BYTES (8u << 20)
+gqe_status gqe_attn_decode_noalloc(const gqe_dims* dims, const gqe_bf16* q_routed,
+                                   const gqe_bf16* q_sh, const gqe_bf16* Kc, const gqe_bf16* Vc,
+                                   int L_max, const int32_t* cache_len, gqe_bf16* o_routed,
+                                   gqe_bf16* o_sh, gqe_stream stream);
+
 /* Output construction ("GQE" study note §3-2 3) hard slots, 4) weighted-sum
  * slot, 5) final concat):
  *   h[n] = [o(g=0, slot 0..k-1), ..., o(g=G-1, ...), sum_g sum_j w[n,g,j] o(g,j), o_sh]

@@ -61,6 +61,7 @@ SIGNATURES = {
     "gqe_kv_append": [_D, _P, _P, _P, _P, _P, _I, _P, _P],
     "gqe_attn_prefill": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
     "gqe_attn_decode": [_D, _P, _P, _P, _P, _I, _P, _P, _P, _P, _SZ, _P],
+    "gqe_attn_decode_noalloc": [_D, _P, _P, _P, _P, _I, _P, _P, _P, _P],
     "gqe_combine": [_D, _P, _P, _P, _P, _P],
     "gqe_linear": [_I, _I, _I, _P, _P, _P, _P],
     "gqe_device_error": [ctypes.POINTER(_I), _P],
@@ -191,6 +192,21 @@ def gqe_attn_decode(dims, q_routed, q_sh, Kc, Vc, L_max, cache_len, o_routed, o_
         _ptr(Kc, "Kc", b), _ptr(Vc, "Vc", b), int(L_max), _ptr(cache_len, "cache_len", torch.int32),
         _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True), _ptr(ws, "ws"), ws_bytes,
         _stream(stream)))
+
+
+def gqe_attn_decode_noalloc(dims, q_routed, q_sh, Kc, Vc, L_max, cache_len, o_routed, o_sh, stream=None):
+    """gqe_attn_decode with the partial states in the library's fixed device
+    array instead of a caller workspace: for callers that cannot allocate
+    device memory at decode time.  Calls must not overlap on the GPU."""
+    import torch
+    b = _bf16()
+    _check("gqe_attn_decode_noalloc", lib.gqe_attn_decode_noalloc(
+        ctypes.byref(dims), _ptr(q_routed, "q_routed", b), _ptr(q_sh, "q_sh", b, optional=True),
+        _ptr(Kc, "Kc", b), _ptr(Vc, "Vc", b), int(L_max), _ptr(cache_len, "cache_len", torch.int32),
+        _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True), _stream(stream)))
+
+
+DECODE_NOALLOC_MAX_BYTES = 8 << 20
 
 
 def gqe_combine(dims, o_routed, o_sh, topk_w, h, stream=None):

@@ -12,6 +12,9 @@
 //           keep an online-softmax state per query row in fp32; the CTA merges
 //           its 64 row-states with warp shuffles and writes (m, l, acc[d]).
 //   merge:  one CTA per (b, g) combines the chunk states and writes bf16.
+#include <mutex>
+
+#include "../../include/gqe.h"
 #include "attn.cuh"
 
 namespace gqe {
@@ -301,3 +304,64 @@ cudaError_t launch_attn_decode_maps(const CUtensorMap& mK, const CUtensorMap& mV
 }
 
 }  // namespace gqe
+
+// ---------------------------------------------------------------------------
+// Decode without a caller workspace, for callers that cannot allocate device
+// memory when they decode (an engine that reserved all device memory for its
+// own pool, a decode loop that cannot pay cudaMalloc's implicit
+// synchronisation).  The split-L partial states go to one fixed array in this
+// file instead of a caller buffer; the kernels are the ones above.
+
+namespace gqe {
+
+gqe_status decode_setup(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh, const gqe_bf16* Kc,
+                        const gqe_bf16* Vc, int L_max, const int32_t* cache_len, gqe_bf16* o_routed,
+                        gqe_bf16* o_sh, CUtensorMap* mK, CUtensorMap* mV, DecodeParams* p);
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = GQE_DECODE_NOALLOC_MAX_BYTES;
+
+// Held by every GPU that loads the library, from load until process exit.
+static __device__ __align__(256) float g_decode_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of the array on the current device.  Host code only sees a
+// host-side stand-in under the array's name, so the address is looked up once
+// per device, with that device current, and cached.
+float* noalloc_scratch() {
+  static std::mutex mu;
+  static float* cache[64] = {nullptr};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<float*>(ptr);
+  }
+  return cache[dev];
+}
+
+}  // namespace
+}  // namespace gqe
+
+extern "C" gqe_status gqe_attn_decode_noalloc(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh,
+                                              const gqe_bf16* Kc, const gqe_bf16* Vc, int L_max,
+                                              const int32_t* cache_len, gqe_bf16* o_routed, gqe_bf16* o_sh,
+                                              gqe_stream stream) {
+  using namespace gqe;
+  CUtensorMap mK, mV;
+  DecodeParams p;
+  const gqe_status st = decode_setup(dims, q_routed, q_sh, Kc, Vc, L_max, cache_len, o_routed, o_sh, &mK, &mV, &p);
+  if (st != GQE_OK) return st;
+  // The partial states for these dims must fit the fixed array.  Every slot
+  // the merge reads is written earlier in the same call (a chunk past
+  // cache_len writes its empty state), so nothing is cleared beforehand.
+  if (decode_workspace_bytes(p.B, p.G, p.k, p.d, p.n_shared, L_max) > kNoAllocScratchBytes)
+    return GQE_ERR_WORKSPACE;
+  float* scratch = noalloc_scratch();
+  if (!scratch) return GQE_ERR_CUDA;
+  p.part = scratch;
+  return launch_attn_decode_maps(mK, mV, p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? GQE_OK
+                                                                                                    : GQE_ERR_CUDA;
+}
