@@ -30,17 +30,33 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   typedef typename std::conditional<VPL == 2, uint32_t, uint2>::type vec_t;
-  for (int g = 0; g < p.G; ++g) {
-    for (int j = 0; j < p.k; ++j) {
-      const float w = p.w[((size_t)n * p.G + g) * p.k + j];
-      const uint16_t* orow = p.o_routed + ((((size_t)b * p.G + g) * p.T + t) * p.k + j) * d + lane * VPL;
-      const vec_t v = *reinterpret_cast<const vec_t*>(orow);
-      *reinterpret_cast<vec_t*>(hrow + (g * p.k + j) * d) = v;
-      const uint32_t* u = reinterpret_cast<const uint32_t*>(&v);
+  const int GK = p.G * p.k;
+  const uint16_t* obase = p.o_routed + (((size_t)b * p.G) * p.T + t) * p.k * d + lane * VPL;
+  const size_t gstride = (size_t)p.T * p.k * d;   // next group, same token
+  const float* wrow = p.w + (size_t)n * GK;
+  for (int s0 = 0; s0 < GK; s0 += 8) {
+    vec_t v[8];
+    float wv[8];
 #pragma unroll
-      for (int i = 0; i < VPL / 2; ++i) {
-        acc[2 * i] = fmaf(w, bf16_lo(u[i]), acc[2 * i]);
-        acc[2 * i + 1] = fmaf(w, bf16_hi(u[i]), acc[2 * i + 1]);
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      if (s < GK) {
+        const int g = s / p.k, j = s % p.k;
+        v[u] = __ldg(reinterpret_cast<const vec_t*>(obase + g * gstride + (size_t)j * d));
+        wv[u] = __ldg(wrow + s);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      if (s < GK) {
+        *reinterpret_cast<vec_t*>(hrow + s * d) = v[u];
+        const uint32_t* uu = reinterpret_cast<const uint32_t*>(&v[u]);
+#pragma unroll
+        for (int i = 0; i < VPL / 2; ++i) {
+          acc[2 * i] = fmaf(wv[u], bf16_lo(uu[i]), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(wv[u], bf16_hi(uu[i]), acc[2 * i + 1]);
+        }
       }
     }
   }

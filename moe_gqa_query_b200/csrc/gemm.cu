@@ -7,15 +7,18 @@
 //     slots ("GQE" study note §3-2 7));
 //   * routed path: the A rows are gathered per (group, expert) segment of the
 //     token-to-expert permutation with 16-byte cp.async (one 128-row tile of
-//     one expert per CTA), so only selected experts' query projections are
+//     one expert at a time), so only selected experts' query projections are
 //     computed ("GQE" study note §3-2 2)); the shared head's projection rides
 //     in the same launch as extra tiles.
 //
-// CTA layout (192 threads, one 128 x BN tile):
-//   warp 0      TMA producer (lane 0)
-//   warp 1      tensor-memory owner and MMA issuer (lane 0)
-//   warps 2..5  routed path: A-row gather producers; then the epilogue
-//               (tensor memory -> registers -> bf16 -> global), one row per thread.
+// Both are persistent (one CTA per SM walks a static tile list) with two
+// accumulators in tensor memory, so the epilogue of one tile overlaps the
+// main loop of the next.
+//
+// Dense CTA (192 threads):  warp 0 TMA producer, warp 1 MMA issuer (and
+//   tensor-memory owner), warps 2..5 epilogue (one output row per thread).
+// Routed CTA (320 threads): warp 0 TMA producer of W, warp 1 MMA issuer,
+//   warps 2..5 A-row gather producers, warps 6..9 epilogue.
 #include "gemm.cuh"
 
 namespace gqe {
@@ -25,133 +28,169 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;                 // 64 bf16 = one 128-byte swizzle row
 constexpr int kATileBytes = kBM * kBK * 2;
-constexpr int kThreads = 192;
 
-struct __align__(8) GemmSmemTail {
+struct __align__(8) GemmBarriers {
   uint64_t full[8];
   uint64_t empty[8];
-  uint64_t accum;
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
   uint32_t tmem_base;
   int abort;
-  int rowsrc[kBM];
-  int rowdst[kBM];
 };
 
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+// One 32-column chunk of an output row: fp32 from tensor memory -> bf16 -> global.
+__device__ __forceinline__ void store_chunk(const EpiParams& ep, int map_sel, int row_dst, int n,
+                                            const uint32_t* v) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+  gqe_bf16_t* base = map_sel ? ep.out1 : ep.out0;
+  gqe_bf16_t* dst;
+  switch (ep.mode) {
+    case kEpiHeads: {
+      const int g = n / ep.d, dd = n % ep.d;
+      const int b = row_dst / ep.T, t = row_dst % ep.T;
+      dst = base + (((size_t)b * ep.G + g) * ep.T + t) * ep.d + dd;
+      break;
+    }
+    case kEpiCacheRow: {
+      const int g = n / ep.d, dd = n % ep.d;
+      const int pos = ep.cache_len[row_dst] - 1;
+      dst = base + (((size_t)row_dst * ep.G + g) * ep.L_max + pos) * ep.d + dd;
+      break;
+    }
+    default:  // kEpiRowMajor, kEpiRows
+      dst = base + (size_t)row_dst * ep.ldo + n;
+      break;
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+}
+
 template <int BN>
-__device__ __forceinline__ void epilogue_store(const EpiParams& ep, int map_sel, int row,
-                                               int grow_dst, int n0, uint32_t tmem_row,
-                                               bool valid) {
-  // grow_dst: row index in the destination (dense: the A row)
+__device__ __forceinline__ void epilogue_tile(const EpiParams& ep, int map_sel, int row_dst, int n0,
+                                              uint32_t tmem_row, bool valid) {
+#pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 32) {
     uint32_t v[32];
     tmem_ld32(tmem_row + c0, v);
-    const int n = n0 + c0;
-    if (!valid || n >= ep.n_limit) continue;
-    uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-    gqe_bf16_t* dst = nullptr;
-    gqe_bf16_t* base = map_sel ? ep.out1 : ep.out0;
-    switch (ep.mode) {
-      case kEpiRowMajor:
-        dst = base + (size_t)grow_dst * ep.ldo + n;
-        break;
-      case kEpiHeads: {
-        const int g = n / ep.d, dd = n % ep.d;
-        const int b = grow_dst / ep.T, t = grow_dst % ep.T;
-        dst = base + (((size_t)b * ep.G + g) * ep.T + t) * ep.d + dd;
-        break;
-      }
-      case kEpiCacheRow: {
-        const int g = n / ep.d, dd = n % ep.d;
-        const int pos = ep.cache_len[grow_dst] - 1;
-        dst = base + (((size_t)grow_dst * ep.G + g) * ep.L_max + pos) * ep.d + dd;
-        break;
-      }
-      default:  // kEpiRows: destination row given per tile row
-        dst = base + (size_t)grow_dst * ep.ldo + n;
-        break;
-    }
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    if (valid && n0 + c0 < ep.n_limit) store_chunk(ep, map_sel, row_dst, n0 + c0, v);
   }
 }
 
 // ---------------------------------------------------------------------------
-// dense: A [M, K] and W [N, K] by TMA
+// dense: A [M, K] and W [N, K] by TMA; persistent over (m-tile, n-tile)
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
-gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA,
-                  const __grid_constant__ CUtensorMap mapB0,
-                  const __grid_constant__ CUtensorMap mapB1, EpiParams ep, int M, int K,
-                  int n_tiles_b0) {
+__global__ void __launch_bounds__(192, 1)
+gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
+                  const __grid_constant__ CUtensorMap mapB1, EpiParams ep, int M, int K, int n_tiles_b0,
+                  int n_tiles_total) {
+  constexpr int kBTileBytes = BN * kBK * 2;
+  constexpr uint32_t kTmemCols = 2 * BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kATileBytes;
-  constexpr int kBTileBytes = BN * kBK * 2;
-  GemmSmemTail* tail = reinterpret_cast<GemmSmemTail*>(sB + STAGES * kBTileBytes);
-  volatile int* abort = &tail->abort;
+  GemmBarriers* bar = reinterpret_cast<GemmBarriers*>(sB + STAGES * kBTileBytes);
+  volatile int* abort = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBM;
-  const int map_sel = (int)blockIdx.y >= n_tiles_b0 ? 1 : 0;
-  const int n0 = (map_sel ? (int)blockIdx.y - n_tiles_b0 : (int)blockIdx.y) * BN;
-  const CUtensorMap* mapB = map_sel ? &mapB1 : &mapB0;
   const int nk = K / kBK;
-  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  const int m_tiles = (M + kBM - 1) / kBM;
+  const int total = m_tiles * n_tiles_total;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&tail->full[s], 1);
-      mbar_init(&tail->empty[s], 1);
+      mbar_init(&bar->full[s], 1);
+      mbar_init(&bar->empty[s], 1);
     }
-    mbar_init(&tail->accum, 1);
-    tail->abort = 0;
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bar->acc_full[a], 1);
+      mbar_init(&bar->acc_empty[a], 4);
+    }
+    bar->abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&mapA);
-    tma_prefetch_desc(mapB);
+    tma_prefetch_desc(&mapB0);
+    tma_prefetch_desc(&mapB1);
   }
-  if (warp == 1) tmem_alloc(&tail->tmem_base, kTmemCols);
+  if (warp == 1) tmem_alloc(&bar->tmem_base, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tail->tmem_base;
+  const uint32_t tmem = bar->tmem_base;
 
-  if (warp == 0 && lane == 0) {
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (kb >= STAGES && !mbar_wait(&tail->empty[s], ph ^ 1, abort, ep.err, kErrTimeoutGemm)) break;
-      mbar_arrive_expect_tx(&tail->full[s], kATileBytes + kBTileBytes);
-      tma_load_2d(sA + s * kATileBytes, &mapA, &tail->full[s], kb * kBK, m0);
-      tma_load_2d(sB + s * kBTileBytes, mapB, &tail->full[s], kb * kBK, n0);
-    }
-  } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!mbar_wait(&tail->full[s], ph, abort, ep.err, kErrTimeoutGemm)) break;
-      tc_fence_after();
-      const uint32_t a0 = smem_u32(sA + s * kATileBytes);
-      const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
-#pragma unroll
-      for (int kk = 0; kk < kBK / 16; ++kk) {
-        umma_ss(tmem, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
-                idesc, (kb | kk) != 0);
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+        const int mt = t / n_tiles_total, nt = t % n_tiles_total;
+        const int sel = nt >= n_tiles_b0;
+        const CUtensorMap* mB = sel ? &mapB1 : &mapB0;
+        const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, ep.err, kErrTimeoutGemm))
+            break;
+          mbar_arrive_expect_tx(&bar->full[s], kATileBytes + kBTileBytes);
+          tma_load_2d(sA + s * kATileBytes, &mapA, &bar->full[s], kb * kBK, mt * kBM);
+          tma_load_2d(sB + s * kBTileBytes, mB, &bar->full[s], kb * kBK, n0);
+        }
       }
-      umma_commit(&tail->empty[s]);
     }
-    umma_commit(&tail->accum);
-  } else if (warp >= 2) {
-    const bool ok = mbar_wait(&tail->accum, 0, abort, ep.err, kErrTimeoutGemm);
-    tc_fence_after();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
+      int it = 0, tc = 0;
+      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tc) {
+        const int ab = tc & 1, use = tc >> 1;
+        if (tc >= 2 && !mbar_wait(&bar->acc_empty[ab], (use & 1) ^ 1, abort, ep.err, kErrTimeoutGemm)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(ab * BN);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&bar->full[s], (it / STAGES) & 1, abort, ep.err, kErrTimeoutGemm)) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kATileBytes);
+          const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_ss(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
+                    (kb | kk) != 0);
+          umma_commit(&bar->empty[s]);
+        }
+        umma_commit(&bar->acc_full[ab]);
+      }
+    }
+  } else {
     const int lg = warp & 3;
-    const int row = m0 + lg * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(lg * 32) << 16);
-    epilogue_store<BN>(ep, map_sel, row, row, n0, trow, ok && row < M);
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    int tc = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
+      const int ab = tc & 1, use = tc >> 1;
+      const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, ep.err, kErrTimeoutGemm);
+      tc_fence_after();
+      const int mt = t / n_tiles_total, nt = t % n_tiles_total;
+      const int sel = nt >= n_tiles_b0;
+      const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
+      const int row = mt * kBM + lg * 32 + lane;
+      epilogue_tile<BN>(ep, sel, row, n0, tmem + lane_off + (uint32_t)(ab * BN), ok && row < M);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->acc_empty[ab]);
+      if (!ok) break;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -163,142 +202,169 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA,
 }
 
 // ---------------------------------------------------------------------------
-// routed: A rows gathered per (group, expert) segment, W by TMA
+// routed: A rows gathered per (group, expert) segment, W by TMA; persistent
+struct RoutedTile {
+  int shared;   // 0 routed, 1 shared head
+  int seg;
+  int row0;     // first permutation entry (routed) or token row (shared)
+  int nrows;
+};
+
+__device__ __forceinline__ RoutedTile routed_tile(const RoutedParams& rp, int t, int n_routed) {
+  RoutedTile r{};
+  if (t < n_routed) {
+    int s = 0;
+    while (s + 1 < rp.n_seg && rp.tile_start[s + 1] <= t) ++s;
+    const int local = t - rp.tile_start[s];
+    r.shared = 0;
+    r.seg = s;
+    r.row0 = rp.seg_off[s] + local * kBM;
+    r.nrows = min(kBM, rp.seg_cnt[s] - local * kBM);
+  } else {
+    r.shared = 1;
+    r.seg = 0;
+    r.row0 = (t - n_routed) * kBM;
+    r.nrows = min(kBM, rp.n_tokens - r.row0);
+  }
+  return r;
+}
+
 template <int BN, int STAGES, int LAG>
-__global__ void __launch_bounds__(kThreads, 1)
-gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq,
-                   const __grid_constant__ CUtensorMap mapWsh, const gqe_bf16_t* __restrict__ x,
-                   RoutedParams rp, EpiParams ep_routed, EpiParams ep_shared) {
+__global__ void __launch_bounds__(320, 1)
+gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_constant__ CUtensorMap mapWsh,
+                   const gqe_bf16_t* __restrict__ x, RoutedParams rp, EpiParams ep_routed, EpiParams ep_shared) {
+  constexpr int kBTileBytes = BN * kBK * 2;
+  constexpr uint32_t kTmemCols = 2 * BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kATileBytes;
-  constexpr int kBTileBytes = BN * kBK * 2;
-  GemmSmemTail* tail = reinterpret_cast<GemmSmemTail*>(sB + STAGES * kBTileBytes);
-  volatile int* abort = &tail->abort;
+  GemmBarriers* bar = reinterpret_cast<GemmBarriers*>(sB + STAGES * kBTileBytes);
+  volatile int* abort = &bar->abort;
+  unsigned* err = ep_routed.err;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x;
   const int K = rp.K;
   const int nk = K / kBK;
+  const int n_routed = rp.tile_start[rp.n_seg];
+  const int total = n_routed + rp.shared_tiles;
 
-  // ---- which tile is this
-  bool shared_tile = false;
-  int seg = 0, row0 = 0, nrows = 0;
-  if (tile < rp.max_routed_tiles) {
-    const int total = rp.tile_start[rp.n_seg];
-    if (tile >= total) return;            // unused upper-bound slot
-    seg = 0;
-    while (seg + 1 < rp.n_seg && rp.tile_start[seg + 1] <= tile) ++seg;
-    const int local = tile - rp.tile_start[seg];
-    row0 = rp.seg_off[seg] + local * kBM;
-    nrows = min(kBM, rp.seg_cnt[seg] - local * kBM);
-  } else {
-    shared_tile = true;
-    row0 = (tile - rp.max_routed_tiles) * kBM;
-    nrows = min(kBM, rp.n_tokens - row0);
-    if (nrows <= 0) return;
-  }
-  const CUtensorMap* mapB = shared_tile ? &mapWsh : &mapWq;
-  const int nb0 = shared_tile ? 0 : seg * rp.d;
-
-  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&tail->full[s], 1 + 128);
-      mbar_init(&tail->empty[s], 1);
+      mbar_init(&bar->full[s], 1 + 128);
+      mbar_init(&bar->empty[s], 1);
     }
-    mbar_init(&tail->accum, 1);
-    tail->abort = 0;
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bar->acc_full[a], 1);
+      mbar_init(&bar->acc_empty[a], 4);
+    }
+    bar->abort = 0;
     fence_mbar_init();
-    tma_prefetch_desc(mapB);
+    tma_prefetch_desc(&mapWq);
+    tma_prefetch_desc(&mapWsh);
   }
-  if (threadIdx.x < kBM) {
-    const int r = threadIdx.x;
-    int src = -1, dst = -1;
-    if (r < nrows) {
-      if (shared_tile) {
-        src = row0 + r;
-        dst = row0 + r;
-      } else {
-        src = rp.src_row[row0 + r];
-        dst = rp.dst_row[row0 + r];
-      }
-    }
-    tail->rowsrc[r] = src;
-    tail->rowdst[r] = dst;
-  }
-  if (warp == 1) tmem_alloc(&tail->tmem_base, kTmemCols);
+  if (warp == 1) tmem_alloc(&bar->tmem_base, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tail->tmem_base;
+  const uint32_t tmem = bar->tmem_base;
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (kb >= STAGES && !mbar_wait(&tail->empty[s], ph ^ 1, abort, ep_routed.err, kErrTimeoutGemm)) break;
-        mbar_arrive_expect_tx(&tail->full[s], kBTileBytes);
-        tma_load_2d(sB + s * kBTileBytes, mapB, &tail->full[s], kb * kBK, nb0);
+      int it = 0;
+      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+        const RoutedTile tl = routed_tile(rp, t, n_routed);
+        const CUtensorMap* mB = tl.shared ? &mapWsh : &mapWq;
+        const int nb0 = tl.shared ? 0 : tl.seg * rp.d;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, err, kErrTimeoutGemm))
+            break;
+          mbar_arrive_expect_tx(&bar->full[s], kBTileBytes);
+          tma_load_2d(sB + s * kBTileBytes, mB, &bar->full[s], kb * kBK, nb0);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait(&tail->full[s], ph, abort, ep_routed.err, kErrTimeoutGemm)) break;
+      int it = 0, tc = 0;
+      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tc) {
+        const int ab = tc & 1, use = tc >> 1;
+        if (tc >= 2 && !mbar_wait(&bar->acc_empty[ab], (use & 1) ^ 1, abort, err, kErrTimeoutGemm)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * kATileBytes);
-        const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
+        const uint32_t acc = tmem + (uint32_t)(ab * BN);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&bar->full[s], (it / STAGES) & 1, abort, err, kErrTimeoutGemm)) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kATileBytes);
+          const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          umma_ss(tmem, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
-                  idesc, (kb | kk) != 0);
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_ss(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
+                    (kb | kk) != 0);
+          umma_commit(&bar->empty[s]);
         }
-        umma_commit(&tail->empty[s]);
+        umma_commit(&bar->acc_full[ab]);
       }
-      umma_commit(&tail->accum);
     }
-  } else {
+  } else if (warp < 6) {
     // ---- gather producers: 128 threads, 8 threads per 128-byte row segment
-    const int t = threadIdx.x - 64;
-    const int c = t & 7;
-    const int rsub = t >> 3;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (kb >= STAGES && !mbar_wait(&tail->empty[s], ph ^ 1, abort, ep_routed.err, kErrTimeoutGemm)) break;
-      uint8_t* st = sA + s * kATileBytes;
+    const int tg = threadIdx.x - 64;
+    const int c = tg & 7;
+    const int rsub = tg >> 3;
+    int it = 0;
+    for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+      const RoutedTile tl = routed_tile(rp, t, n_routed);
+      int src[kBM / 16];
 #pragma unroll
       for (int i = 0; i < kBM / 16; ++i) {
         const int r = rsub + 16 * i;
-        const int src = tail->rowsrc[r];
-        const gqe_bf16_t* g = x + (size_t)(src < 0 ? 0 : src) * K + kb * kBK + c * 8;
-        cp_async_16(st + r * 128 + ((c ^ (r & 7)) << 4), g, src >= 0);
+        src[i] = r < tl.nrows ? (tl.shared ? tl.row0 + r : rp.src_row[tl.row0 + r]) : -1;
       }
-      cp_async_commit();
-      if (kb >= LAG) {
-        cp_async_wait<LAG>();
-        fence_proxy_async_smem();
-        mbar_arrive(&tail->full[(kb - LAG) % STAGES]);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (it >= STAGES && !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, err, kErrTimeoutGemm))
+          break;
+        uint8_t* st = sA + s * kATileBytes;
+#pragma unroll
+        for (int i = 0; i < kBM / 16; ++i) {
+          const int r = rsub + 16 * i;
+          const gqe_bf16_t* g = x + (size_t)(src[i] < 0 ? 0 : src[i]) * K + kb * kBK + c * 8;
+          cp_async_16(st + r * 128 + ((c ^ (r & 7)) << 4), g, src[i] >= 0);
+        }
+        cp_async_commit();
+        if (it >= LAG) {
+          cp_async_wait<LAG>();
+          fence_proxy_async_smem();
+          mbar_arrive(&bar->full[(it - LAG) % STAGES]);
+        }
       }
     }
     cp_async_wait<0>();
     fence_proxy_async_smem();
-    for (int kb = (nk > LAG ? nk - LAG : 0); kb < nk; ++kb) mbar_arrive(&tail->full[kb % STAGES]);
-
-    // ---- epilogue
-    const bool ok = mbar_wait(&tail->accum, 0, abort, ep_routed.err, kErrTimeoutGemm);
-    tc_fence_after();
+    for (int j = (it > LAG ? it - LAG : 0); j < it; ++j) mbar_arrive(&bar->full[j % STAGES]);
+  } else {
+    // ---- epilogue: warps 6..9, tensor-memory lane quarters 2, 3, 0, 1
     const int lg = warp & 3;
-    const int r = lg * 32 + lane;
-    const int dst = tail->rowdst[r];
-    const uint32_t trow = tmem + ((uint32_t)(lg * 32) << 16);
-    epilogue_store<BN>(shared_tile ? ep_shared : ep_routed, 0, r, dst, 0, trow, ok && dst >= 0);
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    int tc = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
+      const RoutedTile tl = routed_tile(rp, t, n_routed);
+      const int ab = tc & 1, use = tc >> 1;
+      const int r = lg * 32 + lane;
+      int dst = -1;
+      if (r < tl.nrows) dst = tl.shared ? tl.row0 + r : rp.dst_row[tl.row0 + r];
+      const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, err, kErrTimeoutGemm);
+      tc_fence_after();
+      epilogue_tile<BN>(tl.shared ? ep_shared : ep_routed, 0, dst, 0, tmem + lane_off + (uint32_t)(ab * BN),
+                        ok && dst >= 0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->acc_empty[ab]);
+      if (!ok) break;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -315,42 +381,48 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq,
 // host launchers
 
 template <int BN, int STAGES>
-static size_t dense_smem_bytes() {
-  return 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmSmemTail);
-}
-
-cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
-                              const CUtensorMap& mapB1, const EpiParams& ep, int M, int K,
-                              int n_tiles_b0, int n_tiles_total, cudaStream_t stream) {
-  constexpr int BN = 128, STAGES = 4;
-  const size_t smem = dense_smem_bytes<BN, STAGES>();
+static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
+                                   const EpiParams& ep, int M, int K, int n_tiles_b0, int n_tiles_total,
+                                   cudaStream_t stream) {
+  const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmBarriers);
   auto kern = gemm_dense_kernel<BN, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((M + kBM - 1) / kBM, n_tiles_total);
-  kern<<<grid, kThreads, smem, stream>>>(mapA, mapB0, mapB1, ep, M, K, n_tiles_b0);
+  const int tiles = ((M + kBM - 1) / kBM) * n_tiles_total;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  kern<<<grid, 192, smem, stream>>>(mapA, mapB0, mapB1, ep, M, K, n_tiles_b0, n_tiles_total);
   return cudaGetLastError();
+}
+
+int dense_tile_n(int n_per_weight) { return (n_per_weight % 256 == 0) ? 256 : 128; }
+
+cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
+                              const EpiParams& ep, int M, int K, int n_tiles_b0, int n_tiles_total, int bn,
+                              cudaStream_t stream) {
+  if (bn == 256) return launch_dense_bn<256, 4>(mapA, mapB0, mapB1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
+  return launch_dense_bn<128, 6>(mapA, mapB0, mapB1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
 }
 
 template <int BN>
-static cudaError_t launch_routed_bn(const CUtensorMap& mapWq, const CUtensorMap& mapWsh,
-                                    const gqe_bf16_t* x, const RoutedParams& rp,
-                                    const EpiParams& epr, const EpiParams& eps, int grid,
+static cudaError_t launch_routed_bn(const CUtensorMap& mapWq, const CUtensorMap& mapWsh, const gqe_bf16_t* x,
+                                    const RoutedParams& rp, const EpiParams& epr, const EpiParams& eps,
                                     cudaStream_t stream) {
-  constexpr int STAGES = 4, LAG = 2;
-  const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmSmemTail);
+  constexpr int STAGES = 6, LAG = 2;
+  const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmBarriers);
   auto kern = gemm_routed_kernel<BN, STAGES, LAG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(mapWq, mapWsh, x, rp, epr, eps);
+  const int max_tiles = rp.max_routed_tiles + rp.shared_tiles;
+  const int grid = max_tiles < num_sms() ? max_tiles : num_sms();
+  kern<<<grid, 320, smem, stream>>>(mapWq, mapWsh, x, rp, epr, eps);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh,
-                               const gqe_bf16_t* x, const RoutedParams& rp, const EpiParams& epr,
-                               const EpiParams& eps, int grid, cudaStream_t stream) {
-  if (rp.d == 64) return launch_routed_bn<64>(mapWq, mapWsh, x, rp, epr, eps, grid, stream);
-  return launch_routed_bn<128>(mapWq, mapWsh, x, rp, epr, eps, grid, stream);
+cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh, const gqe_bf16_t* x,
+                               const RoutedParams& rp, const EpiParams& epr, const EpiParams& eps,
+                               cudaStream_t stream) {
+  if (rp.d == 64) return launch_routed_bn<64>(mapWq, mapWsh, x, rp, epr, eps, stream);
+  return launch_routed_bn<128>(mapWq, mapWsh, x, rp, epr, eps, stream);
 }
 
 }  // namespace gqe

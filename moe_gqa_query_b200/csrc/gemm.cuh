@@ -33,18 +33,22 @@ struct RoutedParams {
   const int* seg_cnt;     // [n_seg]
   const int* tile_start;  // [n_seg + 1] first 128-row tile of each segment
   int n_seg;              // G * E
-  int max_routed_tiles;   // upper bound on tile_start[n_seg] (grid slots)
+  int max_routed_tiles;   // upper bound on tile_start[n_seg]
+  int shared_tiles;       // 128-row tiles of the shared head (0 without one)
   int n_tokens;           // B * T (shared-head tiles)
   int K;                  // d_model
   int d;                  // head width (= tile N)
 };
 
+// Output tile width for a weight with n_per_weight rows: 256 when it divides, else 128.
+int dense_tile_n(int n_per_weight);
+
 cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
                               const CUtensorMap& mapB1, const EpiParams& ep, int M, int K,
-                              int n_tiles_b0, int n_tiles_total, cudaStream_t stream);
+                              int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream);
 
 cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh,
                                const gqe_bf16_t* x, const RoutedParams& rp, const EpiParams& epr,
-                               const EpiParams& eps, int grid, cudaStream_t stream);
+                               const EpiParams& eps, cudaStream_t stream);
 
 }  // namespace gqe

@@ -251,23 +251,24 @@ gqe_status gqe_routed_qproj(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
   epr.err = error_word();
   EpiParams eps = epr;
   eps.out0 = q_sh;
-  const int shared_tiles = dims->n_shared ? (N + 127) / 128 : 0;
-  return cuda_status(launch_gemm_routed(mWq, mWsh, x, rp, epr, eps, rp.max_routed_tiles + shared_tiles, S(stream)));
+  rp.shared_tiles = dims->n_shared ? (N + 127) / 128 : 0;
+  return cuda_status(launch_gemm_routed(mWq, mWsh, x, rp, epr, eps, S(stream)));
 }
 
 static gqe_status kv_common(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk, const gqe_bf16* Wv,
                             EpiParams& ep, int M, gqe_stream stream) {
   const int G = dims->G, d = dims->d_head, D = dims->d_model;
+  const int bn = dense_tile_n(G * d);
   CUtensorMap mA, mK, mV;
   GQE_REQUIRE(map2d(&mA, x, D, M, 128), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mK, Wk, D, (uint64_t)G * d, 128), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mV, Wv, D, (uint64_t)G * d, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mK, Wk, D, (uint64_t)G * d, bn), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mV, Wv, D, (uint64_t)G * d, bn), GQE_ERR_CUDA);
   ep.n_limit = G * d;
   ep.G = G;
   ep.d = d;
   ep.err = error_word();
-  const int nt = (G * d + 127) / 128;
-  return cuda_status(launch_gemm_dense(mA, mK, mV, ep, M, D, nt, 2 * nt, S(stream)));
+  const int nt = (G * d + bn - 1) / bn;
+  return cuda_status(launch_gemm_dense(mA, mK, mV, ep, M, D, nt, 2 * nt, bn, S(stream)));
 }
 
 gqe_status gqe_kv_proj(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk, const gqe_bf16* Wv,
@@ -393,9 +394,10 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   GQE_REQUIRE(K % 64 == 0 && N % 64 == 0, GQE_ERR_UNSUPPORTED);
   GQE_REQUIRE((long long)M * N < (1ll << 31) && (long long)M * K < (1ll << 31), GQE_ERR_UNSUPPORTED);
   GQE_REQUIRE(aligned16(A) && aligned16(W) && aligned16(C), GQE_ERR_INVALID_ARG);
+  const int bn = dense_tile_n(N);
   CUtensorMap mA, mW;
   GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mW, W, K, N, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mW, W, K, N, bn), GQE_ERR_CUDA);
   EpiParams ep{};
   ep.out0 = C;
   ep.out1 = C;
@@ -403,8 +405,8 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   ep.ldo = N;
   ep.n_limit = N;
   ep.err = error_word();
-  const int nt = (N + 127) / 128;
-  return cuda_status(launch_gemm_dense(mA, mW, mW, ep, M, K, nt, nt, S(stream)));
+  const int nt = (N + bn - 1) / bn;
+  return cuda_status(launch_gemm_dense(mA, mW, mW, ep, M, K, nt, nt, bn, S(stream)));
 }
 
 gqe_status gqe_device_error(int* code, gqe_stream stream) {

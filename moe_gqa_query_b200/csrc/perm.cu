@@ -7,23 +7,27 @@
 // segment), so the routed GEMM can run one expert's weight against a gathered
 // 128-row tile.
 //
-//   count:   each block counts its chunk of entries per segment with a
-//            warp-level histogram (__match_any_sync + one shared atomic per
-//            distinct key);
-//   scan:    per segment, an exclusive scan over blocks; segment offsets and
-//            128-row tile offsets;
-//   scatter: each block ranks its entries with the same warp histogram plus
-//            a scan over warps and writes (source token row, destination row
-//            of q_routed [B, G, T, k]).
+// A token contributes at most one entry to any segment (its k experts in a
+// group are distinct, and groups own disjoint segments).  So with one thread
+// per token, the rank of a token inside a segment is a prefix count of one
+// bit per token: a warp ballot per segment gives the in-warp rank, a scan over
+// the block's warps and over the preceding blocks gives the rest.
+//
+//   count:   per block of 256 tokens, tokens per segment (ballot + popc);
+//   scatter: each block sums the counts of the blocks before it (and of all
+//            blocks, for the segment offsets), ranks its tokens with ballots
+//            and writes (source token row, destination row of
+//            q_routed [B, G, T, k]).  Block 0 also writes the segment counts,
+//            offsets and 128-row tile offsets the GEMM reads.
 #include "route.cuh"
 
 namespace gqe {
 
 namespace {
 
-constexpr int kChunk = 4096;      // entries per block
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;     // tokens per block
 constexpr int kWarps = kThreads / 32;
+constexpr int kMaxSeg = 64;
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -31,97 +35,122 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
-__global__ void __launch_bounds__(kThreads) perm_count_kernel(const int* __restrict__ idx, int n_entries,
-                                                              int G, int E, int k, int* block_counts) {
-  __shared__ int hist[64];
-  const int nseg = G * E;
-  for (int s = threadIdx.x; s < nseg; s += kThreads) hist[s] = 0;
-  __syncthreads();
-  const int base = blockIdx.x * kChunk;
-  const int end = min(base + kChunk, n_entries);
-  for (int e0 = base; e0 < end; e0 += kThreads) {
-    const int e = e0 + threadIdx.x;
-    int key = -1;
-    if (e < end) {
-      const int ev = idx[e];   // out-of-range experts are skipped
-      if (ev >= 0 && ev < E) key = ((e / k) % G) * E + ev;
-    }
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    if (key >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[key], __popc(peers));
+// Bit s set when this token routes to segment s (out-of-range experts skipped).
+__device__ __forceinline__ unsigned long long token_segments(const int* __restrict__ idx, int n, int N, int G,
+                                                             int E, int k) {
+  unsigned long long bits = 0;
+  if (n < N) {
+    const int* row = idx + (size_t)n * G * k;
+    for (int g = 0; g < G; ++g)
+      for (int j = 0; j < k; ++j) {
+        const int e = row[g * k + j];
+        if (e >= 0 && e < E) bits |= 1ull << (g * E + e);
+      }
   }
-  __syncthreads();
-  for (int s = threadIdx.x; s < nseg; s += kThreads) block_counts[blockIdx.x * nseg + s] = hist[s];
+  return bits;
 }
 
-__global__ void __launch_bounds__(64) perm_scan_kernel(const int* block_counts, int n_blocks, int nseg,
-                                                       int* block_base, int* seg_cnt, int* seg_off,
-                                                       int* tile_start, int* expert_counts) {
-  __shared__ int cnt[64];
-  const int s = threadIdx.x;
-  if (s < nseg) {
-    int run = 0;
-    for (int b = 0; b < n_blocks; ++b) {
-      block_base[b * nseg + s] = run;
-      run += block_counts[b * nseg + s];
-    }
-    cnt[s] = run;
-    seg_cnt[s] = run;
-    if (expert_counts) expert_counts[s] = run;
-  }
-  __syncthreads();
-  if (s == 0) {
-    int off = 0, tiles = 0;
-    for (int i = 0; i < nseg; ++i) {
-      seg_off[i] = off;
-      tile_start[i] = tiles;
-      off += cnt[i];
-      tiles += (cnt[i] + 127) / 128;
-    }
-    tile_start[nseg] = tiles;
-  }
-}
-
-__global__ void __launch_bounds__(kThreads) perm_scatter_kernel(const int* __restrict__ idx, int n_entries,
-                                                                int T, int G, int E, int k,
-                                                                const int* block_base, const int* seg_off,
-                                                                int* src_row, int* dst_row) {
-  __shared__ int wcnt[kWarps][64];
-  __shared__ int run[64];
+__global__ void __launch_bounds__(kThreads) perm_count_kernel(const int* __restrict__ idx, int N, int G, int E,
+                                                              int k, int* block_counts) {
+  __shared__ int wcnt[kWarps][kMaxSeg];
   const int nseg = G * E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int s = threadIdx.x; s < nseg; s += kThreads) run[s] = 0;
-  const int base = blockIdx.x * kChunk;
-  const int end = min(base + kChunk, n_entries);
-  for (int e0 = base; e0 < end; e0 += kThreads) {
-    for (int i = threadIdx.x; i < kWarps * 64; i += kThreads) (&wcnt[0][0])[i] = 0;
-    __syncthreads();
-    const int e = e0 + threadIdx.x;
-    int key = -1;
-    if (e < end) {
-      const int ev = idx[e];   // out-of-range experts are skipped
-      if (ev >= 0 && ev < E) key = ((e / k) % G) * E + ev;
+  const int n = blockIdx.x * kThreads + threadIdx.x;
+  const unsigned long long bits = token_segments(idx, n, N, G, E, k);
+  for (int s = 0; s < nseg; ++s) {
+    const unsigned m = __ballot_sync(0xffffffffu, (bits >> s) & 1ull);
+    if (lane == 0) wcnt[warp][s] = __popc(m);
+  }
+  __syncthreads();
+  for (int s = threadIdx.x; s < nseg; s += kThreads) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) c += wcnt[w][s];
+    block_counts[blockIdx.x * nseg + s] = c;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) perm_scatter_kernel(const int* __restrict__ idx, int N, int T, int G,
+                                                                int E, int k, int n_blocks,
+                                                                const int* __restrict__ block_counts, int* seg_cnt,
+                                                                int* seg_off, int* tile_start, int* expert_counts,
+                                                                int* src_row, int* dst_row) {
+  __shared__ int wcnt[kWarps][kMaxSeg];
+  __shared__ int base[kMaxSeg];    // this block's first position inside each segment
+  __shared__ int off[kMaxSeg];     // segment offsets
+  const int nseg = G * E;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * kThreads + threadIdx.x;
+  const unsigned long long bits = token_segments(idx, n, N, G, E, k);
+
+  // ---- preceding blocks and totals: 4 threads per segment share the block loop
+  {
+    const int s = threadIdx.x >> 2, part = threadIdx.x & 3;
+    int before = 0, total = 0;
+    if (s < nseg) {
+      for (int b = part; b < n_blocks; b += 4) {
+        const int c = block_counts[b * nseg + s];
+        total += c;
+        before += (b < (int)blockIdx.x) ? c : 0;
+      }
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    const int rank = __popc(peers & lanemask_lt());
-    if (key >= 0 && rank == 0) wcnt[warp][key] = __popc(peers);
-    __syncthreads();
-    if (key >= 0) {
-      int pos = seg_off[key] + block_base[blockIdx.x * nseg + key] + run[key] + rank;
-      for (int w = 0; w < warp; ++w) pos += wcnt[w][key];
-      const int n = e / (G * k);
-      const int g = (e / k) % G;
-      const int j = e % k;
-      const int b = n / T, t = n % T;
-      src_row[pos] = n;
-      dst_row[pos] = ((b * G + g) * T + t) * k + j;
+    before += __shfl_xor_sync(0xffffffffu, before, 1);
+    before += __shfl_xor_sync(0xffffffffu, before, 2);
+    total += __shfl_xor_sync(0xffffffffu, total, 1);
+    total += __shfl_xor_sync(0xffffffffu, total, 2);
+    if (s < nseg && part == 0) {
+      base[s] = before;
+      off[s] = total;     // totals for now; turned into offsets below
     }
-    __syncthreads();
-    for (int s = threadIdx.x; s < nseg; s += kThreads) {
-      int add = 0;
-      for (int w = 0; w < kWarps; ++w) add += wcnt[w][s];
-      run[s] += add;
+  }
+  // ---- in-warp ranks: one ballot per segment
+  for (int s = 0; s < nseg; ++s) {
+    const unsigned m = __ballot_sync(0xffffffffu, (bits >> s) & 1ull);
+    if (lane == 0) wcnt[warp][s] = __popc(m);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int o = 0, tiles = 0;
+    for (int s = 0; s < nseg; ++s) {
+      const int c = off[s];
+      if (blockIdx.x == 0) {
+        seg_cnt[s] = c;
+        tile_start[s] = tiles;
+        if (expert_counts) expert_counts[s] = c;
+      }
+      off[s] = o;
+      o += c;
+      tiles += (c + 127) / 128;
     }
-    __syncthreads();
+    if (blockIdx.x == 0) {
+      for (int s = 0; s < nseg; ++s) seg_off[s] = off[s];
+      tile_start[nseg] = tiles;
+    }
+  }
+  // ---- ranks of this warp's first token in each segment: scan over the block's warps
+  for (int s2 = threadIdx.x; s2 < nseg; s2 += kThreads) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = wcnt[w][s2];
+      wcnt[w][s2] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const int b = n / T, t = n % T;
+  const int* row = idx + (size_t)(n < N ? n : 0) * G * k;
+  const unsigned lt = lanemask_lt();
+  for (int s = 0; s < nseg; ++s) {
+    const bool mine = (bits >> s) & 1ull;
+    const unsigned m = __ballot_sync(0xffffffffu, mine);
+    if (!mine) continue;
+    const int g = s / E, e = s % E;
+    int j = 0;
+    while (j < k - 1 && row[g * k + j] != e) ++j;
+    const int pos = off[s] + base[s] + wcnt[warp][s] + __popc(m & lt);
+    src_row[pos] = n;
+    dst_row[pos] = ((b * G + g) * T + t) * k + j;
   }
 }
 
@@ -133,10 +162,10 @@ PermLayout perm_layout(int N, int G, int E, int k) {
   PermLayout L{};
   L.n_entries = N * G * k;
   L.n_seg = G * E;
-  L.n_blocks = (L.n_entries + kChunk - 1) / kChunk;
+  L.n_blocks = (N + kThreads - 1) / kThreads;
   size_t o = 0;
   L.off_block_counts = o; o = align256(o + sizeof(int) * (size_t)L.n_blocks * L.n_seg);
-  L.off_block_base = o;   o = align256(o + sizeof(int) * (size_t)L.n_blocks * L.n_seg);
+  L.off_block_base = o;   // unused: the scatter kernel derives block bases from the counts
   L.off_seg_cnt = o;      o = align256(o + sizeof(int) * L.n_seg);
   L.off_seg_off = o;      o = align256(o + sizeof(int) * L.n_seg);
   L.off_tile_start = o;   o = align256(o + sizeof(int) * (L.n_seg + 1));
@@ -150,18 +179,15 @@ cudaError_t launch_permutation(const int* topk_idx, int N, int T, int G, int E, 
                                const PermLayout& L, int* expert_counts, cudaStream_t stream) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   int* block_counts = reinterpret_cast<int*>(w + L.off_block_counts);
-  int* block_base = reinterpret_cast<int*>(w + L.off_block_base);
   int* seg_cnt = reinterpret_cast<int*>(w + L.off_seg_cnt);
   int* seg_off = reinterpret_cast<int*>(w + L.off_seg_off);
   int* tile_start = reinterpret_cast<int*>(w + L.off_tile_start);
   int* src_row = reinterpret_cast<int*>(w + L.off_src_row);
   int* dst_row = reinterpret_cast<int*>(w + L.off_dst_row);
-  if (L.n_entries == 0) return cudaSuccess;
-  perm_count_kernel<<<L.n_blocks, kThreads, 0, stream>>>(topk_idx, L.n_entries, G, E, k, block_counts);
-  perm_scan_kernel<<<1, 64, 0, stream>>>(block_counts, L.n_blocks, L.n_seg, block_base, seg_cnt, seg_off,
-                                         tile_start, expert_counts);
-  perm_scatter_kernel<<<L.n_blocks, kThreads, 0, stream>>>(topk_idx, L.n_entries, T, G, E, k, block_base,
-                                                           seg_off, src_row, dst_row);
+  perm_count_kernel<<<L.n_blocks, kThreads, 0, stream>>>(topk_idx, N, G, E, k, block_counts);
+  perm_scatter_kernel<<<L.n_blocks, kThreads, 0, stream>>>(topk_idx, N, T, G, E, k, L.n_blocks, block_counts,
+                                                           seg_cnt, seg_off, tile_start, expert_counts, src_row,
+                                                           dst_row);
   return cudaGetLastError();
 }
 

@@ -5,11 +5,13 @@
 // p~ = p normalised over the selected experts (all k*G of the token by
 // default, or within the group).
 //
-// The router reads x once and is HBM bound.  A CTA of 4 warps owns 64 tokens:
-// x streams through a 3-deep cp.async ring (128-byte rows, XOR-swizzled), the
-// logits x Wr are accumulated in fp32 on the tensor cores (mma.sync m16n8k16:
-// the products of bf16 inputs are exact, so this is the fp32 dot product), and
-// one thread per token then runs the softmax and TopK of every group in fp32
+// The router reads x once and is HBM bound.  A CTA of 4 warps owns 32 tokens
+// (many CTAs per SM keep enough bytes in flight): x streams through a 4-deep
+// cp.async ring (128-byte rows, XOR-swizzled); the logits x Wr are accumulated
+// in fp32 on the tensor cores (mma.sync m16n8k16: the products of bf16 inputs
+// are exact, so this is the fp32 dot product), two warps per 16 tokens each
+// taking half of every 64-column chunk, the halves added in shared memory; one
+// thread per token then runs the softmax and TopK of every group in fp32
 // registers.  Selection uses the fp32 logits (softmax is monotone within a
 // group); ties go to the lower expert index; selected experts are emitted in
 // ascending index order.
@@ -19,9 +21,9 @@ namespace gqe {
 
 namespace {
 
-constexpr int kTok = 64;       // tokens per CTA
+constexpr int kTok = 32;       // tokens per CTA
 constexpr int kKC = 64;        // reduction chunk (d_model columns)
-constexpr int kXStages = 3;
+constexpr int kXStages = 4;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -49,20 +51,21 @@ __global__ void __launch_bounds__(128) router_kernel(RouterParams p) {
   constexpr int WPT = kKC * GEP / 128;   // Wr elements per thread per chunk
   __shared__ __align__(128) uint16_t xs[kXStages][kTok * kKC];
   __shared__ __align__(16) uint16_t ws[2][kKC * WS];
-  // the logits reuse the x ring once the reduction is done
-  float (*lg)[GEP + 1] = reinterpret_cast<float (*)[GEP + 1]>(&xs[0][0]);
-  static_assert(sizeof(float) * kTok * (GEP + 1) <= sizeof(uint16_t) * kXStages * kTok * kKC, "logits fit");
+  __shared__ float lg[kTok][GEP + 1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tok0 = blockIdx.x * kTok;
   const int GE = p.G * p.E;
   const int nkc = p.D / kKC;
+  // warp w: token rows (w & 1) * 16 .. +15, reduction half (w >> 1) of every chunk
+  const int mrow = (warp & 1) * 16;
+  const int khalf = warp >> 1;
 
   auto load_x = [&](int kc) {
     uint16_t* dst = xs[kc % kXStages];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = tid + 128 * i;     // 512 16-byte chunks
+    for (int i = 0; i < kTok * 8 / 128; ++i) {
+      const int e = tid + 128 * i;     // kTok * 8 16-byte chunks
       const int r = e >> 3, c = e & 7;
       const int n = tok0 + r;
       const uint16_t* src = p.x + (size_t)(n < p.N ? n : 0) * p.D + kc * kKC + c * 8;
@@ -106,9 +109,10 @@ __global__ void __launch_bounds__(128) router_kernel(RouterParams p) {
     const uint32_t xb = smem_u32(xs[kc % kXStages]);
     const uint32_t wb = smem_u32(ws[kc & 1]);
 #pragma unroll
-    for (int ks = 0; ks < kKC / 16; ++ks) {
+    for (int kh = 0; kh < kKC / 32; ++kh) {
+      const int ks = khalf * (kKC / 32) + kh;
       const int mi = lane >> 3;
-      const int ar = warp * 16 + (mi & 1) * 8 + (lane & 7);
+      const int ar = mrow + (mi & 1) * 8 + (lane & 7);
       const int ac = ks * 2 + (mi >> 1);
       uint32_t a0, a1, a2, a3;
       ldsm_x4(xb + ar * 128 + ((ac ^ (ar & 7)) << 4), a0, a1, a2, a3);
@@ -126,16 +130,30 @@ __global__ void __launch_bounds__(128) router_kernel(RouterParams p) {
     if (kc + 1 < nkc) store_w((kc + 1) & 1);
   }
   cp_async_wait<0>();
-  __syncthreads();
 
+  // the two reduction halves meet in shared memory
+  if (khalf == 1) {
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const int r = warp * 16 + (lane >> 2);
-    const int c = t * 8 + (lane & 3) * 2;
-    lg[r][c] = acc[t][0];
-    lg[r][c + 1] = acc[t][1];
-    lg[r + 8][c] = acc[t][2];
-    lg[r + 8][c + 1] = acc[t][3];
+    for (int t = 0; t < NT; ++t) {
+      const int r = mrow + (lane >> 2);
+      const int c = t * 8 + (lane & 3) * 2;
+      lg[r][c] = acc[t][0];
+      lg[r][c + 1] = acc[t][1];
+      lg[r + 8][c] = acc[t][2];
+      lg[r + 8][c + 1] = acc[t][3];
+    }
+  }
+  __syncthreads();
+  if (khalf == 0) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int r = mrow + (lane >> 2);
+      const int c = t * 8 + (lane & 3) * 2;
+      lg[r][c] += acc[t][0];
+      lg[r][c + 1] += acc[t][1];
+      lg[r + 8][c] += acc[t][2];
+      lg[r + 8][c + 1] += acc[t][3];
+    }
   }
   __syncthreads();
 
