@@ -180,6 +180,13 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
  * internal waits runs out of time (0 = none).  Synchronises `stream`. */
 gqe_status gqe_device_error(int* code, gqe_stream stream);
 
+/* Diagnostics.  Evaluates the attention kernel's exponential helpers on n
+ * fp32 inputs (device arrays): y_poly the polynomial exp2 used on the FMA
+ * pipe, y_pair its packed two-lane form, y_hw the hardware exp2 (MUFU).  For
+ * tests; not part of the layer. */
+gqe_status gqe_debug_exp2(const float* x, float* y_poly, float* y_pair, float* y_hw, int n,
+                          gqe_stream stream);
+
 const char* gqe_status_string(gqe_status status);
 
 #ifdef __cplusplus

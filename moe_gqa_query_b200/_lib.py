@@ -65,6 +65,7 @@ SIGNATURES = {
     "gqe_combine": [_D, _P, _P, _P, _P, _P],
     "gqe_linear": [_I, _I, _I, _P, _P, _P, _P],
     "gqe_device_error": [ctypes.POINTER(_I), _P],
+    "gqe_debug_exp2": [_P, _P, _P, _P, _I, _P],
     "gqe_status_string": [_I],
 }
 
@@ -230,6 +231,13 @@ def gqe_device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     _check("gqe_device_error", lib.gqe_device_error(ctypes.byref(code), _stream(stream)))
     return int(code.value)
+
+
+def gqe_debug_exp2(x, y_poly, y_pair, y_hw, stream=None):
+    import torch
+    f = torch.float32
+    _check("gqe_debug_exp2", lib.gqe_debug_exp2(_ptr(x, "x", f), _ptr(y_poly, "y_poly", f), _ptr(y_pair, "y_pair", f),
+                                                _ptr(y_hw, "y_hw", f), x.numel(), _stream(stream)))
 
 
 def gqe_status_string(status: int) -> str:

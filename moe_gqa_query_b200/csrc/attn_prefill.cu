@@ -4,40 +4,56 @@
 // that group's dense K/V ("GQE" study note §3-2 2) and §1-1 attention
 // equation); the shared head does the same against KV group sg (§3-2 5)).
 //
-// Work item = one 128-row tile of packed query rows of one sequence:
-//   routed: rows (t, j) of group (b, g), row = t*k + j, so one tile spans
-//           128/k tokens and every K/V tile loaded for it serves all of the
-//           group's selected experts at once;
-//   shared: 128 tokens of the shared head of sequence b.
-// Items are launched heaviest first (descending 128-token level), so the
-// causal triangle's long tiles start early.
+// Packing: the rows (t, j) of group (b, g) are contiguous (row = t*k + j), so
+// one 128-row query tile holds 128/k tokens x k selected experts and every
+// K/V tile loaded for it serves all of them at once.
 //
-// Per item: TMA brings Q once and K/V tiles (128 keys) through a ring of
-// shared-memory stages; tcgen05 computes S = Q K^T into one of three tensor-
-// memory S buffers; 4 softmax warps (one row per thread) apply the causal
-// mask, keep the running max in the base-2 domain, write P (bf16) over the S
-// columns, and rescale the O accumulator in tensor memory only when the max
-// grows by more than 2^8 (exact: l and O share the stale max); tcgen05 then
-// adds P V (A operand from tensor memory) into O.
+// Work item = two consecutive 128-row query tiles A and B of one sequence
+// (routed: one (b, g); shared: one b).  They share every K/V tile load and run
+// in ping-pong: while the softmax warpgroup of A works on S_A, the tensor core
+// computes P_B V and Q_B K^T, and the other way round.  Items are launched
+// heaviest first (descending 256-token level); the hardware block scheduler
+// hands each SM the next item when it frees up, which balances the causal
+// triangle's unequal items better than a static per-SM list.
 //
-// CTA: 192 threads.  warp 0 TMA producer, warp 1 MMA issuer (and tensor-memory
-// owner), warps 2..5 softmax + epilogue.  Tensor memory: S0|S1|S2|O at columns
-// 0|128|256|384.
+// Per item: TMA brings Q_A, Q_B once and K/V tiles (128 keys) through rings of
+// shared-memory stages.  tcgen05 computes S = Q K^T into tensor memory; the
+// softmax warps (one query row per thread) load their S row once (row max,
+// then exponentials from registers), apply the causal mask on diagonal tiles, keep
+// the running max in the base-2 domain, write P (bf16) to tensor memory, and
+// rescale the O accumulator only when the max grows by more than 2^8 (exact:
+// l and O share the stale max); tcgen05 then adds P V (A operand from tensor
+// memory) into O.
+//
+// CTA: 320 threads.  warps 0-3 softmax + epilogue of tile A, warps 4-7 of tile
+// B, warp 8 TMA producer, warp 9 MMA issuer and tensor-memory owner.  Tensor
+// memory (512 columns):
+//   d=64 : S_A 0 | S_B 128 | O_A 256 | O_B 320 | P_A 384 | P_B 448
+//   d=128: S_A 0 | S_B 128 | O_A 256 | O_B 384, P_X written over S_X's first
+//          64 columns (the next S_X waits for P_X V to finish).
 #include "attn.cuh"
 
 namespace gqe {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kTile = 128;          // query rows and keys per tile
 constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16, 16 KB
 constexpr float kRescaleLog2 = 8.0f;
+#ifndef GQE_ATTN_POLY_PAIRS
+#define GQE_ATTN_POLY_PAIRS 0
+#endif
+// Column pairs (of every 16) whose exponentials run as the FMA-pipe polynomial
+// instead of MUFU ex2.  On B200 the softmax here is bound by instruction issue,
+// not by MUFU throughput (measured: 0, 3, 5 and 8 of 16 within 3 % of each
+// other at d = 64), so the default keeps every exponential on MUFU.
+constexpr int kPolyPairs = GQE_ATTN_POLY_PAIRS;
 
 struct __align__(8) AttnBarriers {
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[3], p_full[3], pv_done[3];
+  uint64_t s_full[2], p_full[2], pv_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -46,10 +62,37 @@ template <int D>
 struct AttnCfg {
   static constexpr int NB = D / 64;                  // 64-column boxes per tile
   static constexpr int ST = (D == 64) ? 3 : 2;       // K/V ring depth
-  static constexpr int QBytes = NB * kBox;
+  static constexpr int QBytes = NB * kBox;           // one Q tile
   static constexpr int KVBytes = NB * kBox;
-  static constexpr size_t Smem = 1024 + QBytes + 2 * ST * KVBytes + sizeof(AttnBarriers);
+  static constexpr bool kPAliasS = (D != 64);
+  // tensor-memory columns of tile x's S, O and P
+  __host__ __device__ static constexpr uint32_t scol(int x) { return x ? 128u : 0u; }
+  __host__ __device__ static constexpr uint32_t ocol(int x) { return x ? (uint32_t)(256 + D) : 256u; }
+  __host__ __device__ static constexpr uint32_t pcol(int x) {
+    return kPAliasS ? scol(x) : (x ? 448u : 384u);
+  }
+  static constexpr size_t Smem = 1024 + 2 * QBytes + 2 * ST * KVBytes + sizeof(AttnBarriers);
 };
+
+struct TileInfo {
+  int row0;      // first packed row
+  int n_kv;      // key tiles 0..n_kv-1 (0: tile absent)
+  int t_first;   // first token of the tile
+};
+
+__device__ __forceinline__ TileInfo tile_info(int qt, int rows_total, int kk, int T) {
+  TileInfo ti;
+  ti.row0 = qt * kTile;
+  if (ti.row0 >= rows_total) {
+    ti.n_kv = 0;
+    ti.t_first = 0;
+    return ti;
+  }
+  ti.t_first = ti.row0 / kk;
+  const int t_last = min(T - 1, (ti.row0 + kTile - 1) / kk);
+  ti.n_kv = t_last / kTile + 1;
+  return ti;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -59,44 +102,41 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::QBytes;
+  uint8_t* sQ = smem;                                 // [2][QBytes]
+  uint8_t* sK = sQ + 2 * C::QBytes;
   uint8_t* sV = sK + C::ST * C::KVBytes;
   AttnBarriers* bar = reinterpret_cast<AttnBarriers*>(sV + C::ST * C::KVBytes);
   volatile int* abort = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work item
+  // ---- work item: level-major (heaviest first), then routed pairs, then shared
   const int BG = p.B * p.G;
   const int per_level = BG * p.k + p.B * p.n_shared;
-  const int ntq_sh = (p.T + kTile - 1) / kTile;
-  const int level = blockIdx.x / per_level;
+  const int n_levels = (p.T + 2 * kTile - 1) / (2 * kTile);
+  const int level = n_levels - 1 - (int)blockIdx.x / per_level;
   const int i = blockIdx.x % per_level;
-  const int qt_sh = ntq_sh - 1 - level;
   bool routed;
-  int seq, qt, kvseq, kk, rows_total;
+  int seq, pair, kvseq, kk, rows_total;
   if (i < BG * p.k) {
     routed = true;
-    const int r = i / BG;
     seq = i % BG;
-    qt = qt_sh * p.k + r;
+    pair = level * p.k + i / BG;
     kvseq = seq;
     kk = p.k;
     rows_total = p.T * p.k;
   } else {
     routed = false;
     seq = i - BG * p.k;
-    qt = qt_sh;
+    pair = level;
     kvseq = seq * p.G + p.sg;
     kk = 1;
     rows_total = p.T;
   }
-  const int row0 = qt * kTile;
-  if (row0 >= rows_total) return;
-  const int t_first = row0 / kk;
-  const int t_last = min(p.T - 1, (row0 + kTile - 1) / kk);
-  const int n_kv = t_last / kTile + 1;
+  const TileInfo tA = tile_info(2 * pair, rows_total, kk, p.T);
+  const TileInfo tB = tile_info(2 * pair + 1, rows_total, kk, p.T);
+  if (tA.n_kv == 0) return;
+  const int n_kv = max(tA.n_kv, tB.n_kv);
   const CUtensorMap* mq = routed ? &mapQ : &mapQs;
 
   if (threadIdx.x == 0) {
@@ -107,10 +147,10 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       mbar_init(&bar->v_full[s], 1);
       mbar_init(&bar->v_empty[s], 1);
     }
-    for (int s = 0; s < 3; ++s) {
-      mbar_init(&bar->s_full[s], 1);
-      mbar_init(&bar->p_full[s], 128);
-      mbar_init(&bar->pv_done[s], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bar->s_full[x], 1);
+      mbar_init(&bar->p_full[x], 128);
+      mbar_init(&bar->pv_done[x], 1);
     }
     bar->abort = 0;
     fence_mbar_init();
@@ -118,197 +158,217 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     tma_prefetch_desc(&mapK);
     tma_prefetch_desc(&mapV);
   }
-  if (warp == 1) tmem_alloc(&bar->tmem_base, 512);
+  if (warp == 9) tmem_alloc(&bar->tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
-  constexpr uint32_t kOcol = 384;
 
-  if (warp == 0) {
+  if (warp == 8) {
     if (lane == 0) {
-      // ---------------- producer: Q once, then K_0, K_1, V_0, K_2, V_1, ...
-      mbar_arrive_expect_tx(&bar->q_full, C::QBytes);
-      for (int bx = 0; bx < C::NB; ++bx)
-        tma_load_3d(sQ + bx * kBox, mq, &bar->q_full, bx * 64, row0, seq);
-      auto load_k = [&](int j) -> bool {
+      // ---------------- producer: Q_A, Q_B once; then K_0, V_0, K_1, V_1, ...
+      const int nq = tB.n_kv > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(&bar->q_full, nq * C::QBytes);
+      for (int x = 0; x < nq; ++x)
+        for (int bx = 0; bx < C::NB; ++bx)
+          tma_load_3d(sQ + x * C::QBytes + bx * kBox, mq, &bar->q_full, bx * 64, (x ? tB : tA).row0, seq);
+      for (int j = 0; j < n_kv; ++j) {
         const int s = j % C::ST;
-        if (j >= C::ST && !mbar_wait(&bar->k_empty[s], ((j / C::ST) & 1) ^ 1, abort, p.err, kErrTimeoutAttn))
-          return false;
+        const uint32_t ph = ((j / C::ST) & 1) ^ 1;
+        if (j >= C::ST && !mbar_wait(&bar->k_empty[s], ph, abort, p.err, kErrTimeoutAttn)) break;
         mbar_arrive_expect_tx(&bar->k_full[s], C::KVBytes);
         for (int bx = 0; bx < C::NB; ++bx)
           tma_load_3d(sK + s * C::KVBytes + bx * kBox, &mapK, &bar->k_full[s], bx * 64, j * kTile, kvseq);
-        return true;
-      };
-      auto load_v = [&](int j) -> bool {
-        const int s = j % C::ST;
-        if (j >= C::ST && !mbar_wait(&bar->v_empty[s], ((j / C::ST) & 1) ^ 1, abort, p.err, kErrTimeoutAttn))
-          return false;
+        if (j >= C::ST && !mbar_wait(&bar->v_empty[s], ph, abort, p.err, kErrTimeoutAttn)) break;
         mbar_arrive_expect_tx(&bar->v_full[s], C::KVBytes);
         for (int bx = 0; bx < C::NB; ++bx)
           tma_load_3d(sV + s * C::KVBytes + bx * kBox, &mapV, &bar->v_full[s], bx * 64, j * kTile, kvseq);
-        return true;
-      };
-      for (int j = 0; j < n_kv; ++j) {
-        if (!load_k(j)) break;
-        if (j >= 1 && !load_v(j - 1)) break;
       }
-      if (!*abort) load_v(n_kv - 1);
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     if (lane == 0) {
-      // ---------------- MMA issuer: S_0, S_1, PV_0, S_2, PV_1, ...
+      // ---------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kTile, D, false, true);
-      const uint32_t q0 = smem_u32(sQ);
-      auto issue_s = [&](int j) -> bool {
+      const int nA = tA.n_kv, nB = tB.n_kv;
+      bool ok = true;
+      auto issue_s = [&](int x, int j) {
         const int s = j % C::ST;
         if (!mbar_wait(&bar->k_full[s], (j / C::ST) & 1, abort, p.err, kErrTimeoutAttn)) return false;
         tc_fence_after();
+        const uint32_t q0 = smem_u32(sQ + x * C::QBytes);
         const uint32_t k0 = smem_u32(sK + s * C::KVBytes);
-        const uint32_t dst = tmem + (uint32_t)((j % 3) * kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * kBox + (ks & 3) * 32;
-          umma_ss(dst, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(k0 + off, 16, 1024), idesc_s,
-                  ks > 0);
+          umma_ss(tmem + C::scol(x), sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(k0 + off, 16, 1024),
+                  idesc_s, ks > 0);
         }
-        umma_commit(&bar->s_full[j % 3]);
-        umma_commit(&bar->k_empty[s]);
+        umma_commit(&bar->s_full[x]);
+        // K_j's last reader is tile B when it reaches j, else tile A
+        if (x == 1 || nB <= j) umma_commit(&bar->k_empty[s]);
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
+      auto issue_pv = [&](int x, int j) {
         const int s = j % C::ST;
         if (!mbar_wait(&bar->v_full[s], (j / C::ST) & 1, abort, p.err, kErrTimeoutAttn)) return false;
         tc_fence_after();
         const uint32_t v0 = smem_u32(sV + s * C::KVBytes);
-        const uint32_t pcol = tmem + (uint32_t)((j % 3) * kTile);
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks) {
-          // V rows 16*ks .. 16*ks+15 (K dim), all D columns (MN-major, 64-col boxes 16 KB apart)
-          umma_ts(tmem + kOcol, pcol + ks * 8, sdesc_sw128(v0 + ks * 2048, kBox, 1024), idesc_o,
-                  (j > 0 || ks > 0));
-        }
-        umma_commit(&bar->pv_done[j % 3]);
-        umma_commit(&bar->v_empty[s]);
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          umma_ts(tmem + C::ocol(x), tmem + C::pcol(x) + ks * 8, sdesc_sw128(v0 + ks * 2048, kBox, 1024),
+                  idesc_o, (j > 0 || ks > 0));
+        umma_commit(&bar->pv_done[x]);
+        if (x == 1 || nB <= j) umma_commit(&bar->v_empty[s]);
         return true;
       };
       if (mbar_wait(&bar->q_full, 0, abort, p.err, kErrTimeoutAttn)) {
-        bool ok = issue_s(0);
-        if (ok && n_kv > 1) ok = issue_s(1);
+        ok = issue_s(0, 0);
+        if (ok && nB > 0) ok = issue_s(1, 0);
         for (int j = 0; ok && j < n_kv; ++j) {
-          if (!mbar_wait(&bar->p_full[j % 3], (j / 3) & 1, abort, p.err, kErrTimeoutAttn)) break;
-          tc_fence_after();
-          if (!issue_pv(j)) break;
-          if (j + 2 < n_kv) {
-            if (j >= 1 && !mbar_wait(&bar->pv_done[(j - 1) % 3], ((j - 1) / 3) & 1, abort, p.err, kErrTimeoutAttn))
-              break;
-            if (!issue_s(j + 2)) break;
+          for (int x = 0; x < 2 && ok; ++x) {
+            const int nx = x ? nB : nA;
+            if (j >= nx) continue;
+            ok = mbar_wait(&bar->p_full[x], j & 1, abort, p.err, kErrTimeoutAttn);
+            tc_fence_after();
+            ok = ok && issue_pv(x, j);
+            if (ok && j + 1 < nx) {
+              if (C::kPAliasS) ok = mbar_wait(&bar->pv_done[x], j & 1, abort, p.err, kErrTimeoutAttn);
+              ok = ok && issue_s(x, j + 1);
+            }
           }
         }
       }
     }
   } else {
-    // ---------------- softmax warps: one query row per thread
-    const int lg = warp & 3;
-    const int r = lg * 32 + lane;
-    const int prow = row0 + r;
-    const bool valid = prow < rows_total;
-    const int t_r = prow / kk;
-    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
-    const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      ok = mbar_wait(&bar->s_full[j % 3], (j / 3) & 1, abort, p.err, kErrTimeoutAttn);
-      tc_fence_after();
-      const uint32_t sbase = tmem + lane_off + (uint32_t)((j % 3) * kTile);
-      uint32_t s[128];
-      tmem_ld32(sbase + 0, s);
-      tmem_ld32(sbase + 32, s + 32);
-      tmem_ld32(sbase + 64, s + 64);
-      tmem_ld32(sbase + 96, s + 96);
-      float mx = -INFINITY;
-      if (j * kTile + kTile - 1 > t_first) {
-        const int lim = t_r - j * kTile;   // columns > lim are in the future
+    // ---------------- softmax warpgroups: one query row per thread
+    const int x = warp >> 2;                 // 0: tile A, 1: tile B
+    const TileInfo ti = x ? tB : tA;
+    if (ti.n_kv > 0) {
+      const int lg = warp & 3;
+      const int r = lg * 32 + lane;
+      const int prow = ti.row0 + r;
+      const bool valid = prow < rows_total;
+      const int t_r = prow / kk;
+      const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+      const uint32_t s_base = tmem + lane_off + C::scol(x);
+      const uint32_t p_base = tmem + lane_off + C::pcol(x);
+      const uint32_t o_base = tmem + lane_off + C::ocol(x);
+      const float sl2 = p.scale_log2;
+      float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      for (int j = 0; j < ti.n_kv && ok; ++j) {
+        ok = mbar_wait(&bar->s_full[x], j & 1, abort, p.err, kErrTimeoutAttn);
+        tc_fence_after();
+        const bool diag = j * kTile + kTile - 1 > ti.t_first;
+        const int lim = t_r - j * kTile;     // columns > lim are in the future
+        // the whole S row, once (two loads, one wait), then the row max with
+        // 8 independent partial maxima
+        uint32_t s[128];
+        tmem_ld128(s_base, s);
+        if (diag) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          if (c > lim) s[c] = __float_as_uint(-INFINITY);
-          mx = fmaxf(mx, __uint_as_float(s[c]));
+          for (int c = 0; c < 128; ++c)
+            if (c > lim) s[c] = __float_as_uint(-INFINITY);
         }
-      } else {
+        float m8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
-      }
-      const float m_new = fmaxf(m_run, mx * sl2);
-      if (j == 0) {
-        m_run = m_new;
-      } else {
-        const bool need = m_new > m_run + kRescaleLog2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2(m_run - m_new) : 1.f;
+        for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          m8[c & 7] = fmax3(m8[c & 7], __uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]));
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        const float m_new = fmaxf(m_run, mx * sl2);
+        // lazy rescale: only when some row's max grew by more than 2^8; O itself
+        // is rescaled after the exponentials (S registers are dead by then) and
+        // before P is released to the MMA
+        bool rescale = false;
+        float alpha = 1.f;
+        if (j == 0) {
+          m_run = m_new;
+        } else {
+          const bool need = m_new > m_run + kRescaleLog2;
+          rescale = __any_sync(0xffffffffu, need);
           if (need) {
+            alpha = ex2(m_run - m_new);
             l_run *= alpha;
             m_run = m_new;
           }
-          ok = mbar_wait(&bar->pv_done[(j - 1) % 3], ((j - 1) / 3) & 1, abort, p.err, kErrTimeoutAttn) && ok;
-          tc_fence_after();
+        }
+        // exponentials (MUFU, or the FMA-pipe polynomial for kPolyPairs of every
+        // 16 pairs), row sum, P (bf16) into tensor memory
+        const float neg_m = -m_run;
+        float sum_lo = 0.f, sum_hi = 0.f;
 #pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int q = c0 + c;          // column pair
+            const float x0 = fmaf(__uint_as_float(s[2 * q]), sl2, neg_m);
+            const float x1 = fmaf(__uint_as_float(s[2 * q + 1]), sl2, neg_m);
+            float p0, p1;
+            if ((q & 15) < kPolyPairs) {
+              p0 = exp2_poly(x0);
+              p1 = exp2_poly(x1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            sum_lo += p0;
+            sum_hi += p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(p_base + c0, pk);
+        }
+        l_run += sum_lo + sum_hi;
+        if (rescale) {
+          ok = mbar_wait(&bar->pv_done[x], (j - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
+          tc_fence_after();
+#pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(tmem + lane_off + kOcol + c0, o);
+            tmem_ld32(o_base + c0, o);
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tmem + lane_off + kOcol + c0, o);
+            tmem_st32(o_base + c0, o);
           }
-          tmem_wait_st();
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar->p_full[x]);
+      }
+      // ---------------- epilogue: O / l -> bf16
+      ok = mbar_wait(&bar->pv_done[x], (ti.n_kv - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
+      tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      gqe_bf16_t* orow = routed ? p.o_routed + ((size_t)seq * rows_total + prow) * D
+                                : p.o_sh + ((size_t)seq * p.T + prow) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(o_base + c0, o);
+        if (valid && ok) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+          uint4* d4 = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
       }
-      float sum = 0.f;
-      const float neg_m = -m_run;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), sl2, neg_m));
-        const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), sl2, neg_m));
-        sum += p0 + p1;
-        s[c] = pack_bf16x2(p0, p1);
+      if (p.lse && valid && ok) {
+        const size_t li = routed ? (size_t)seq * rows_total + prow
+                                 : (size_t)BG * p.T * p.k + (size_t)seq * p.T + prow;
+        p.lse[li] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       }
-      l_run += sum;
-      tmem_st32(sbase + 0, s);
-      tmem_st32(sbase + 32, s + 32);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar->p_full[j % 3]);
-    }
-    // ---------------- epilogue: O / l -> bf16
-    ok = mbar_wait(&bar->pv_done[(n_kv - 1) % 3], ((n_kv - 1) / 3) & 1, abort, p.err, kErrTimeoutAttn) && ok;
-    tc_fence_after();
-    const float inv_l = 1.f / l_run;
-    gqe_bf16_t* orow = routed ? p.o_routed + ((size_t)seq * rows_total + prow) * D
-                              : p.o_sh + ((size_t)seq * p.T + prow) * D;
-#pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      tmem_ld32(tmem + lane_off + kOcol + c0, o);
-      if (valid && ok) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-        uint4* d4 = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-    }
-    if (p.lse && valid && ok) {
-      const size_t li = routed ? (size_t)seq * rows_total + prow
-                               : (size_t)BG * p.T * p.k + (size_t)seq * p.T + prow;
-      p.lse[li] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -324,15 +384,14 @@ static cudaError_t launch_d(const CUtensorMap& mQ, const CUtensorMap& mQs, const
   auto kern = attn_prefill_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int ntq_sh = (p.T + kTile - 1) / kTile;
+  const int n_levels = (p.T + 2 * kTile - 1) / (2 * kTile);
   const int per_level = p.B * p.G * p.k + p.B * p.n_shared;
-  kern<<<ntq_sh * per_level, kThreads, smem, stream>>>(mQ, mQs, mK, mV, p);
+  kern<<<n_levels * per_level, kThreads, smem, stream>>>(mQ, mQs, mK, mV, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_prefill(const CUtensorMap& mQ, const CUtensorMap& mQs, const CUtensorMap& mK,
-                                const CUtensorMap& mV, const AttnParams& p, int d,
-                                cudaStream_t stream) {
+                                const CUtensorMap& mV, const AttnParams& p, int d, cudaStream_t stream) {
   if (d == 64) return launch_d<64>(mQ, mQs, mK, mV, p, stream);
   return launch_d<128>(mQ, mQs, mK, mV, p, stream);
 }

@@ -1,0 +1,30 @@
+// diag.cu -- diagnostic entry point: evaluates the kernels' device exp2
+// helpers on caller data so tests can check them against the hardware exp2.
+#include "../../include/gqe.h"
+#include "sm100.cuh"
+
+namespace gqe {
+namespace {
+
+__global__ void exp2_diag_kernel(const float* __restrict__ x, float* y_poly, float* y_pair, float* y_hw, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float v = x[i];
+  y_poly[i] = exp2_poly(v);
+  float a, b;
+  exp2_poly2(f2_pack(v, v), a, b);
+  y_pair[i] = (a == b) ? a : __int_as_float(0x7fc00000);   // both lanes must agree
+  y_hw[i] = ex2(v);
+}
+
+}  // namespace
+}  // namespace gqe
+
+extern "C" gqe_status gqe_debug_exp2(const float* x, float* y_poly, float* y_pair, float* y_hw, int n,
+                                     gqe_stream stream) {
+  if (n < 0 || (n > 0 && (!x || !y_poly || !y_pair || !y_hw))) return GQE_ERR_INVALID_ARG;
+  if (n == 0) return GQE_OK;
+  gqe::exp2_diag_kernel<<<(n + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y_poly, y_pair,
+                                                                                             y_hw, n);
+  return cudaGetLastError() == cudaSuccess ? GQE_OK : GQE_ERR_CUDA;
+}

@@ -11,8 +11,8 @@
 // in fp32 on the tensor cores (mma.sync m16n8k16: the products of bf16 inputs
 // are exact, so this is the fp32 dot product), two warps per 16 tokens each
 // taking half of every 64-column chunk, the halves added in shared memory; one
-// thread per token then runs the softmax and TopK of every group in fp32
-// registers.  Selection uses the fp32 logits (softmax is monotone within a
+// thread per (token, group) then runs that group's softmax and TopK in fp32
+// registers, the token-scope denominator summed through shared memory.  Selection uses the fp32 logits (softmax is monotone within a
 // group); ties go to the lower expert index; selected experts are emitted in
 // ascending index order.
 #include "route.cuh"
@@ -44,6 +44,86 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Softmax and TopK of one (token, group) from the token's fp32 logits.
+// Returns the selected experts as a bit mask and the sum of their
+// probabilities; pr receives the group's probabilities.
+__device__ __forceinline__ unsigned route_group(const RouterParams& p, const float* logits, int g, float* pr,
+                                                float* gsum) {
+  const int E = p.E;
+  float s[8];
+  float mx = -INFINITY;
+  for (int e = 0; e < E; ++e) {
+    s[e] = logits[g * E + e] + (p.bias ? p.bias[g * E + e] : 0.f);
+    mx = fmaxf(mx, s[e]);
+  }
+  float Z = 0.f;
+  for (int e = 0; e < E; ++e) {
+    pr[e] = expf(s[e] - mx);
+    Z += pr[e];
+  }
+  const float invZ = 1.f / Z;
+  for (int e = 0; e < E; ++e) pr[e] *= invZ;
+  unsigned chosen = 0;
+  for (int it = 0; it < p.k; ++it) {
+    int best = -1;
+    float bv = -INFINITY;
+    for (int e = 0; e < E; ++e) {
+      if ((chosen >> e) & 1u) continue;
+      if (best < 0 || s[e] > bv) {   // strict: ties keep the lower index
+        best = e;
+        bv = s[e];
+      }
+    }
+    chosen |= 1u << best;
+  }
+  float sum = 0.f;
+  for (int e = 0; e < E; ++e)
+    if ((chosen >> e) & 1u) sum += pr[e];
+  *gsum = sum;
+  return chosen;
+}
+
+// Routes the kTok tokens of a tile cooperatively, one (token, group) pair per
+// thread: softmax and TopK per group, the token-scope denominator through
+// shared memory, then the selected experts (ascending), their renormalised
+// weights and optionally the probabilities.  `lg` holds the tile's logits
+// with row stride `ls`; `gs` is kTok*G floats of shared scratch.
+__device__ __forceinline__ void route_tile(const RouterParams& p, const float* lg, int ls, int tok0, float* gs) {
+  const int G = p.G, E = p.E, k = p.k;
+  const int npairs = kTok * G;
+  for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
+    const int t = e / G, g = e % G;
+    float pr[8], sum;
+    route_group(p, lg + t * ls, g, pr, &sum);
+    gs[e] = sum;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
+    const int t = e / G, g = e % G;
+    const int n = tok0 + t;
+    if (n >= p.N) continue;
+    float pr[8], sum;
+    const unsigned chosen = route_group(p, lg + t * ls, g, pr, &sum);
+    float den = sum;
+    if (p.scope == 0) {
+      den = 0.f;
+      for (int gg = 0; gg < G; ++gg) den += gs[t * G + gg];
+    }
+    const float inv_den = 1.f / den;
+    const size_t o = ((size_t)n * G + g) * k;
+    int j = 0;
+    for (int ee = 0; ee < E; ++ee) {
+      if ((chosen >> ee) & 1u) {
+        p.topk_idx[o + j] = ee;
+        p.topk_w[o + j] = pr[ee] * inv_den;
+        ++j;
+      }
+    }
+    if (p.probs)
+      for (int ee = 0; ee < E; ++ee) p.probs[((size_t)n * G + g) * E + ee] = pr[ee];
+  }
+}
+
 template <int GEP>
 __global__ void __launch_bounds__(128) router_kernel(RouterParams p) {
   constexpr int WS = GEP + 8;            // padded Wr row (bf16), 16-byte multiple
@@ -52,6 +132,9 @@ __global__ void __launch_bounds__(128) router_kernel(RouterParams p) {
   __shared__ __align__(128) uint16_t xs[kXStages][kTok * kKC];
   __shared__ __align__(16) uint16_t ws[2][kKC * WS];
   __shared__ float lg[kTok][GEP + 1];
+  // the per-(token, group) sums reuse the x ring once the reduction is done
+  float* gsum_s = reinterpret_cast<float*>(&xs[0][0]);
+  static_assert(sizeof(float) * kTok * 64 <= sizeof(uint16_t) * kXStages * kTok * kKC, "group sums fit");
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tok0 = blockIdx.x * kTok;
@@ -157,73 +240,175 @@ __global__ void __launch_bounds__(128) router_kernel(RouterParams p) {
   }
   __syncthreads();
 
-  if (tid >= kTok) return;
-  const int n = tok0 + tid;
-  if (n >= p.N) return;
-  const int E = p.E, k = p.k;
+  route_tile(p, &lg[0][0], GEP + 1, tok0, gsum_s);
+}
 
-  // pass 1 (token scope): sum of the selected probabilities over all groups
-  float total = 0.f;
-  for (int pass = (p.scope == 0 ? 0 : 1); pass < 2; ++pass) {
-    for (int g = 0; g < p.G; ++g) {
-      float s[8], pr[8];
-      float mx = -INFINITY;
-      for (int e = 0; e < E; ++e) {
-        s[e] = lg[tid][g * E + e] + (p.bias ? p.bias[g * E + e] : 0.f);
-        mx = fmaxf(mx, s[e]);
-      }
-      float Z = 0.f;
-      for (int e = 0; e < E; ++e) {
-        pr[e] = expf(s[e] - mx);
-        Z += pr[e];
-      }
-      const float invZ = 1.f / Z;
-      unsigned chosen = 0;
-      for (int it = 0; it < k; ++it) {
-        int best = -1;
-        float bv = -INFINITY;
-        for (int e = 0; e < E; ++e) {
-          if ((chosen >> e) & 1u) continue;
-          if (best < 0 || s[e] > bv) {
-            best = e;
-            bv = s[e];
-          }
-        }
-        chosen |= 1u << best;
-      }
-      float gsum = 0.f;
-      for (int e = 0; e < E; ++e)
-        if ((chosen >> e) & 1u) gsum += pr[e] * invZ;
-      if (pass == 0) {
-        total += gsum;
-        continue;
-      }
-      const float den = (p.scope == 0) ? total : gsum;
-      const float inv_den = 1.f / den;
-      const size_t o = ((size_t)n * p.G + g) * k;
-      int j = 0;
-      for (int e = 0; e < E; ++e) {
-        if ((chosen >> e) & 1u) {
-          p.topk_idx[o + j] = e;
-          p.topk_w[o + j] = pr[e] * invZ * inv_den;
-          ++j;
-        }
-      }
-      if (p.probs)
-        for (int e = 0; e < E; ++e) p.probs[((size_t)n * p.G + g) * E + e] = pr[e] * invZ;
+
+// Wr resident in shared memory (when it fits), persistent over 32-token tiles;
+// x streams through one cp.async ring that runs across tile boundaries.
+template <int GEP, int STAGES>
+__global__ void __launch_bounds__(128, 4) router_resident_kernel(RouterParams p) {
+  constexpr int WS = GEP + 8;
+  constexpr int NT = GEP / 8;
+  extern __shared__ __align__(128) uint8_t rsm[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(rsm);                           // [STAGES][kTok*kKC]
+  uint16_t* wsm = xs + STAGES * kTok * kKC;                                  // [D][WS]
+  float* lgf = reinterpret_cast<float*>(wsm + (size_t)p.D * WS);             // [kTok][GEP+1]
+  float* gsf = lgf + kTok * (GEP + 1);                                        // [kTok][G]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int GE = p.G * p.E;
+  const int nkc = p.D / kKC;
+  const int n_tiles = (p.N + kTok - 1) / kTok;
+  const int my_tiles = (n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int total = my_tiles * nkc;
+  const int mrow = (warp & 1) * 16;
+  const int khalf = warp >> 1;
+
+  auto load_x = [&](int it) {
+    const int tile = blockIdx.x + (it / nkc) * gridDim.x;
+    const int kc = it % nkc;
+    uint16_t* dst = xs + (it % STAGES) * kTok * kKC;
+#pragma unroll
+    for (int i = 0; i < kTok * 8 / 128; ++i) {
+      const int e = tid + 128 * i;
+      const int r = e >> 3, c = e & 7;
+      const int n = tile * kTok + r;
+      const uint16_t* src = p.x + (size_t)(n < p.N ? n : 0) * p.D + kc * kKC + c * 8;
+      cp_async_16(reinterpret_cast<uint8_t*>(dst) + r * 128 + ((c ^ (r & 7)) << 4), src, n < p.N);
+    }
+  };
+
+  for (int s = 0; s < STAGES - 1; ++s) {
+    if (s < total) load_x(s);
+    cp_async_commit();
+  }
+  // Wr into shared memory once (padded columns zero); 16-byte loads when the
+  // rows allow it
+  if ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0) {
+    const int n16 = p.D * GE / 8;
+    for (int e = tid; e < n16; e += 128) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.Wr) + e);
+      const int r = (e * 8) / GE, c = (e * 8) % GE;
+      *reinterpret_cast<uint4*>(wsm + (size_t)r * WS + c) = v;
+    }
+    if (GE < GEP)
+      for (int e = tid; e < p.D * (GEP - GE); e += 128)
+        wsm[(size_t)(e / (GEP - GE)) * WS + GE + e % (GEP - GE)] = 0;
+  } else {
+    for (int e = tid; e < p.D * GEP; e += 128) {
+      const int r = e / GEP, c = e % GEP;
+      wsm[r * WS + c] = (c < GE) ? p.Wr[(size_t)r * GE + c] : (uint16_t)0;
     }
   }
+
+  float acc[NT][4];
+  for (int it = 0; it < total; ++it) {
+    const int kc = it % nkc;
+    if (kc == 0) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    }
+    if (it + STAGES - 1 < total) load_x(it + STAGES - 1);
+    cp_async_commit();
+    cp_async_wait<STAGES - 1>();
+    __syncthreads();
+    const uint32_t xb = smem_u32(xs + (it % STAGES) * kTok * kKC);
+    const uint32_t wb = smem_u32(wsm + (size_t)kc * kKC * WS);
+#pragma unroll
+    for (int kh = 0; kh < kKC / 32; ++kh) {
+      const int ks = khalf * (kKC / 32) + kh;
+      const int mi = lane >> 3;
+      const int ar = mrow + (mi & 1) * 8 + (lane & 7);
+      const int ac = ks * 2 + (mi >> 1);
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(xb + ar * 128 + ((ac ^ (ar & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        const int kr = ks * 16 + (mi & 1) * 8 + (lane & 7);
+        const int nc = np * 16 + (mi >> 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(wb + (kr * WS + nc) * 2, b0, b1, b2, b3);
+        mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+    if (kc == nkc - 1) {
+      // tile done: add the two reduction halves, then route its tokens
+      const int tile = blockIdx.x + (it / nkc) * gridDim.x;
+      if (khalf == 1) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const int r = mrow + (lane >> 2);
+          const int c = t * 8 + (lane & 3) * 2;
+          lgf[r * (GEP + 1) + c] = acc[t][0];
+          lgf[r * (GEP + 1) + c + 1] = acc[t][1];
+          lgf[(r + 8) * (GEP + 1) + c] = acc[t][2];
+          lgf[(r + 8) * (GEP + 1) + c + 1] = acc[t][3];
+        }
+      }
+      __syncthreads();
+      if (khalf == 0) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const int r = mrow + (lane >> 2);
+          const int c = t * 8 + (lane & 3) * 2;
+          lgf[r * (GEP + 1) + c] += acc[t][0];
+          lgf[r * (GEP + 1) + c + 1] += acc[t][1];
+          lgf[(r + 8) * (GEP + 1) + c] += acc[t][2];
+          lgf[(r + 8) * (GEP + 1) + c + 1] += acc[t][3];
+        }
+      }
+      __syncthreads();
+      route_tile(p, lgf, GEP + 1, tile * kTok, gsf);
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+}
+
+template <int GEP>
+size_t resident_smem(int D, int stages) {
+  return (size_t)stages * kTok * kKC * 2 + (size_t)D * (GEP + 8) * 2 + (size_t)kTok * (GEP + 1) * 4 +
+         (size_t)kTok * 64 * 4;
+}
+
+int router_num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int GEP>
+cudaError_t launch_router_gep(const RouterParams& p, cudaStream_t stream) {
+  constexpr int STAGES = 8;
+  const size_t smem = resident_smem<GEP>(p.D, STAGES);
+  const int n_tiles = (p.N + kTok - 1) / kTok;
+  if (smem <= 100 * 1024) {
+    auto kern = router_resident_kernel<GEP, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int per_sm = (int)((220 * 1024) / (smem + 1024));
+    int grid = router_num_sms() * (per_sm < 1 ? 1 : per_sm);
+    if (grid > n_tiles) grid = n_tiles;
+    kern<<<grid, 128, smem, stream>>>(p);
+  } else {
+    router_kernel<GEP><<<n_tiles, 128, 0, stream>>>(p);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_router(const RouterParams& p, cudaStream_t stream) {
   const int GE = p.G * p.E;
-  const int grid = (p.N + kTok - 1) / kTok;
-  if (GE <= 16) router_kernel<16><<<grid, 128, 0, stream>>>(p);
-  else if (GE <= 32) router_kernel<32><<<grid, 128, 0, stream>>>(p);
-  else router_kernel<64><<<grid, 128, 0, stream>>>(p);
-  return cudaGetLastError();
+  if (GE <= 16) return launch_router_gep<16>(p, stream);
+  if (GE <= 32) return launch_router_gep<32>(p, stream);
+  return launch_router_gep<64>(p, stream);
 }
 
 }  // namespace gqe

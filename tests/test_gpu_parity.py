@@ -387,3 +387,26 @@ def test_layer_decode_step_end_to_end():
     agree = np.all(gi_idx == ref["router"]["idx"], axis=(1, 2))
     assert np.all(agree | (ref["router"]["margin"] < NEAR_TIE).any(axis=1))
     assert_close_attn(to_f64(y)[agree], ref["y"][agree], "decode y")
+
+
+# ----------------------------------------------------------------------------
+# the exponential helpers of the attention kernel
+
+def test_device_exp2_helpers():
+    xs = np.concatenate([np.linspace(-120, 20, 20001), np.linspace(-1, 1, 4001)]).astype(np.float32)
+    x = torch.from_numpy(xs).cuda()
+    yp, y2, yh = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+    gq.gqe_debug_exp2(x, yp, y2, yh)
+    torch.cuda.synchronize()
+    ref = np.exp2(xs.astype(np.float64))
+    rel_poly = np.abs(yp.cpu().numpy() - ref) / ref
+    rel_hw = np.abs(yh.cpu().numpy() - ref) / ref
+    assert rel_poly.max() < 1e-4, rel_poly.max()
+    assert rel_hw.max() < 1e-5, rel_hw.max()
+    assert torch.equal(yp, y2)
+    ninf = torch.tensor([-float("inf"), -500.0], device="cuda")
+    a, b, c = torch.empty_like(ninf), torch.empty_like(ninf), torch.empty_like(ninf)
+    gq.gqe_debug_exp2(ninf, a, b, c)
+    torch.cuda.synchronize()
+    assert (a.cpu() < 2.0 ** -124).all() and (a.cpu() > 0).all()
+    assert c.cpu()[0] == 0
