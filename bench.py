@@ -42,6 +42,7 @@ DECODE_WORKLOAD = "decode"
 METRIC = "GQE prefill tokens/s per layer"
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 L2_FLUSH_BYTES = 256 << 20
+HOST_LEAD_CYCLES = 600_000      # ~0.3 ms at B200 clocks: longer than the host needs to enqueue a step
 
 
 def load_peaks():
@@ -289,6 +290,7 @@ def run_kernel(args):
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for a, b in evs:
+        torch.cuda._sleep(HOST_LEAD_CYCLES)      # host runs ahead: events time device work only
         a.record(stream)
         fn()
         b.record(stream)
@@ -391,6 +393,9 @@ def main():
     with ClockSampler(local) as clocks:
         for s in range(args.steps):
             flush.zero_()                       # L2 flushed between timed steps (outside the events)
+            # a GPU-side pause (outside the events) lets the host enqueue the whole
+            # step before the GPU reaches it, so the events time device work only
+            torch.cuda._sleep(HOST_LEAD_CYCLES)
             step(events[s])
         torch.cuda.synchronize()
     barrier(dist, device)

@@ -16,6 +16,7 @@
 
 #include "../../include/gqe.h"
 #include "attn.cuh"
+#include "launch.cuh"
 
 namespace gqe {
 
@@ -288,7 +289,7 @@ static cudaError_t launch_dec(const CUtensorMap& mK, const CUtensorMap& mV, cons
                               cudaStream_t stream) {
   const size_t smem = DecCfg<D>::Smem;
   auto kern = decode_split_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(p.n_chunks, p.G, p.B), kThreads, smem, stream>>>(mK, mV, p);
   e = cudaGetLastError();

@@ -32,6 +32,7 @@
 //   d=128: S_A 0 | S_B 128 | O_A 256 | O_B 384, P_X written over S_X's first
 //          64 columns (the next S_X waits for P_X V to finish).
 #include "attn.cuh"
+#include "launch.cuh"
 
 namespace gqe {
 
@@ -382,7 +383,7 @@ static cudaError_t launch_d(const CUtensorMap& mQ, const CUtensorMap& mQs, const
                             const CUtensorMap& mV, const AttnParams& p, cudaStream_t stream) {
   const size_t smem = AttnCfg<D>::Smem;
   auto kern = attn_prefill_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int n_levels = (p.T + 2 * kTile - 1) / (2 * kTile);
   const int per_level = p.B * p.G * p.k + p.B * p.n_shared;

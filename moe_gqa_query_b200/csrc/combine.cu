@@ -5,69 +5,65 @@
 //                 sum_g sum_{e in S} p~_{t,g,e} o_{t,g,e}   (weighted-sum slot),
 //                 o_shared_t )                               (shared head slot)
 //
-// One warp per token; each lane owns d/32 contiguous columns of every slot.
-// The weighted sum accumulates in fp32 and is rounded to bf16 once.
-#include <type_traits>
-
+// One warp per token, 16-byte vectors: d/8 lanes cover one slot row, so a
+// warp moves 32/(d/8) slot rows per pass.  The weighted sum accumulates in
+// fp32 per lane, is reduced across the lane groups with shuffles, and is
+// rounded to bf16 once.
 #include "route.cuh"
 
 namespace gqe {
 
 namespace {
 
-template <int VPL>   // bf16 values per lane: d / 32
+template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
-  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  constexpr int LPR = D / 8;       // lanes per slot row: 8 bf16 (16 bytes) each
+  constexpr int RPW = 32 / LPR;    // slot rows per warp pass
+  const int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.B * p.T;
-  if (warp_global >= N) return;
-  const int n = warp_global;
+  if (n >= N) return;
   const int b = n / p.T, t = n % p.T;
-  const int d = p.d;
-  const int slots = p.k * p.G + 1 + p.n_shared;
-  uint16_t* hrow = p.h + (size_t)n * slots * d + lane * VPL;
-  float acc[VPL];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
-  typedef typename std::conditional<VPL == 2, uint32_t, uint2>::type vec_t;
   const int GK = p.G * p.k;
-  const uint16_t* obase = p.o_routed + (((size_t)b * p.G) * p.T + t) * p.k * d + lane * VPL;
-  const size_t gstride = (size_t)p.T * p.k * d;   // next group, same token
+  const int slots = GK + 1 + p.n_shared;
+  const int sub = lane / LPR, c8 = (lane % LPR) * 8;
+  uint16_t* hrow = p.h + (size_t)n * slots * D + c8;
+  const size_t gstride = (size_t)p.T * p.k * D;     // next group, same token
+  const uint16_t* obase = p.o_routed + (((size_t)b * p.G) * p.T + t) * p.k * D + c8;
   const float* wrow = p.w + (size_t)n * GK;
-  for (int s0 = 0; s0 < GK; s0 += 8) {
-    vec_t v[8];
-    float wv[8];
+  float acc[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int s = s0 + u;
-      if (s < GK) {
-        const int g = s / p.k, j = s % p.k;
-        v[u] = __ldg(reinterpret_cast<const vec_t*>(obase + g * gstride + (size_t)j * d));
-        wv[u] = __ldg(wrow + s);
-      }
-    }
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int s0 = 0; s0 < GK; s0 += RPW) {
+    const int s = s0 + sub;
+    if (s < GK) {
+      const int g = s / p.k, j = s % p.k;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(obase + g * gstride + (size_t)j * D));
+      const float w = __ldg(wrow + s);
+      *reinterpret_cast<uint4*>(hrow + (size_t)s * D) = v;     // hard slot: a copy
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int s = s0 + u;
-      if (s < GK) {
-        *reinterpret_cast<vec_t*>(hrow + s * d) = v[u];
-        const uint32_t* uu = reinterpret_cast<const uint32_t*>(&v[u]);
-#pragma unroll
-        for (int i = 0; i < VPL / 2; ++i) {
-          acc[2 * i] = fmaf(wv[u], bf16_lo(uu[i]), acc[2 * i]);
-          acc[2 * i + 1] = fmaf(wv[u], bf16_hi(uu[i]), acc[2 * i + 1]);
-        }
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(w, bf16_lo(u[i]), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(w, bf16_hi(u[i]), acc[2 * i + 1]);
       }
     }
   }
-  vec_t r;
-  uint32_t* ru = reinterpret_cast<uint32_t*>(&r);
+  // weighted-sum slot: add the RPW lane groups' partial sums
 #pragma unroll
-  for (int i = 0; i < VPL / 2; ++i) ru[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
-  *reinterpret_cast<vec_t*>(hrow + (p.k * p.G) * d) = r;
-  if (p.n_shared) {
-    const vec_t v = *reinterpret_cast<const vec_t*>(p.o_sh + (size_t)n * d + lane * VPL);
-    *reinterpret_cast<vec_t*>(hrow + (p.k * p.G + 1) * d) = v;
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+  if (sub == 0) {
+    uint4 r;
+    r.x = pack_bf16x2(acc[0], acc[1]);
+    r.y = pack_bf16x2(acc[2], acc[3]);
+    r.z = pack_bf16x2(acc[4], acc[5]);
+    r.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(hrow + (size_t)GK * D) = r;
+  } else if (sub == 1 && p.n_shared) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.o_sh + (size_t)n * D + c8));
+    *reinterpret_cast<uint4*>(hrow + (size_t)(GK + 1) * D) = v;
   }
 }
 
@@ -76,8 +72,8 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   const int N = p.B * p.T;
   const int grid = (N * 32 + 255) / 256;
-  if (p.d == 64) combine_kernel<2><<<grid, 256, 0, stream>>>(p);
-  else combine_kernel<4><<<grid, 256, 0, stream>>>(p);
+  if (p.d == 64) combine_kernel<64><<<grid, 256, 0, stream>>>(p);
+  else combine_kernel<128><<<grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

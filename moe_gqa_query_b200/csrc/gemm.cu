@@ -9,7 +9,8 @@
 //     token-to-expert permutation with 16-byte cp.async (one 128-row tile of
 //     one expert at a time), so only selected experts' query projections are
 //     computed ("GQE" study note §3-2 2)); the shared head's projection rides
-//     in the same launch as extra tiles.
+//     in the same launch as extra tiles.  (TMA tile::gather4 was measured 3.7x
+//     slower here: 128-byte rows are too small a request for the TMA unit.)
 //
 // Both are persistent (one CTA per SM walks a static tile list) with two
 // accumulators in tensor memory, so the epilogue of one tile overlaps the
@@ -20,6 +21,7 @@
 // Routed CTA (320 threads): warp 0 TMA producer of W, warp 1 MMA issuer,
 //   warps 2..5 A-row gather producers, warps 6..9 epilogue.
 #include "gemm.cuh"
+#include "launch.cuh"
 
 namespace gqe {
 
@@ -210,16 +212,25 @@ struct RoutedTile {
   int nrows;
 };
 
-__device__ __forceinline__ RoutedTile routed_tile(const RoutedParams& rp, int t, int n_routed) {
+// Segment tables staged in shared memory once per CTA (a tile's segment is
+// found by a scan that would otherwise cost one global load per step).
+struct SegTables {
+  int tile_start[65];
+  int seg_off[64];
+  int seg_cnt[64];
+};
+
+__device__ __forceinline__ RoutedTile routed_tile(const RoutedParams& rp, const SegTables& st, int t,
+                                                  int n_routed) {
   RoutedTile r{};
   if (t < n_routed) {
     int s = 0;
-    while (s + 1 < rp.n_seg && rp.tile_start[s + 1] <= t) ++s;
-    const int local = t - rp.tile_start[s];
+    while (s + 1 < rp.n_seg && st.tile_start[s + 1] <= t) ++s;
+    const int local = t - st.tile_start[s];
     r.shared = 0;
     r.seg = s;
-    r.row0 = rp.seg_off[s] + local * kBM;
-    r.nrows = min(kBM, rp.seg_cnt[s] - local * kBM);
+    r.row0 = st.seg_off[s] + local * kBM;
+    r.nrows = min(kBM, st.seg_cnt[s] - local * kBM);
   } else {
     r.shared = 1;
     r.seg = 0;
@@ -229,7 +240,7 @@ __device__ __forceinline__ RoutedTile routed_tile(const RoutedParams& rp, int t,
   return r;
 }
 
-template <int BN, int STAGES, int LAG>
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(320, 1)
 gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_constant__ CUtensorMap mapWsh,
                    const gqe_bf16_t* __restrict__ x, RoutedParams rp, EpiParams ep_routed, EpiParams ep_shared) {
@@ -240,13 +251,22 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kATileBytes;
   GemmBarriers* bar = reinterpret_cast<GemmBarriers*>(sB + STAGES * kBTileBytes);
+  SegTables* seg = reinterpret_cast<SegTables*>(bar + 1);
   volatile int* abort = &bar->abort;
   unsigned* err = ep_routed.err;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = rp.K;
   const int nk = K / kBK;
-  const int n_routed = rp.tile_start[rp.n_seg];
+  for (int i = threadIdx.x; i <= rp.n_seg; i += blockDim.x) {
+    seg->tile_start[i] = rp.tile_start[i];
+    if (i < rp.n_seg) {
+      seg->seg_off[i] = rp.seg_off[i];
+      seg->seg_cnt[i] = rp.seg_cnt[i];
+    }
+  }
+  __syncthreads();
+  const int n_routed = seg->tile_start[rp.n_seg];
   const int total = n_routed + rp.shared_tiles;
 
   if (threadIdx.x == 0) {
@@ -273,7 +293,7 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
     if (lane == 0) {
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        const RoutedTile tl = routed_tile(rp, t, n_routed);
+        const RoutedTile tl = routed_tile(rp, *seg, t, n_routed);
         const CUtensorMap* mB = tl.shared ? &mapWsh : &mapWq;
         const int nb0 = tl.shared ? 0 : tl.seg * rp.d;
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -297,6 +317,7 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&bar->full[s], (it / STAGES) & 1, abort, err, kErrTimeoutGemm)) break;
+          fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kATileBytes);
           const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
@@ -316,7 +337,7 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
     const int rsub = tg >> 3;
     int it = 0;
     for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-      const RoutedTile tl = routed_tile(rp, t, n_routed);
+      const RoutedTile tl = routed_tile(rp, *seg, t, n_routed);
       int src[kBM / 16];
 #pragma unroll
       for (int i = 0; i < kBM / 16; ++i) {
@@ -334,24 +355,19 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
           const gqe_bf16_t* g = x + (size_t)(src[i] < 0 ? 0 : src[i]) * K + kb * kBK + c * 8;
           cp_async_16(st + r * 128 + ((c ^ (r & 7)) << 4), g, src[i] >= 0);
         }
-        cp_async_commit();
-        if (it >= LAG) {
-          cp_async_wait<LAG>();
-          fence_proxy_async_smem();
-          mbar_arrive(&bar->full[(it - LAG) % STAGES]);
-        }
+        // the stage's barrier hears from this thread once its copies land; the
+        // MMA thread makes them visible to the tensor core's (async) proxy
+        cp_async_arrive_noinc(&bar->full[s]);
       }
     }
     cp_async_wait<0>();
-    fence_proxy_async_smem();
-    for (int j = (it > LAG ? it - LAG : 0); j < it; ++j) mbar_arrive(&bar->full[j % STAGES]);
   } else {
     // ---- epilogue: warps 6..9, tensor-memory lane quarters 2, 3, 0, 1
     const int lg = warp & 3;
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     int tc = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
-      const RoutedTile tl = routed_tile(rp, t, n_routed);
+      const RoutedTile tl = routed_tile(rp, *seg, t, n_routed);
       const int ab = tc & 1, use = tc >> 1;
       const int r = lg * 32 + lane;
       int dst = -1;
@@ -386,7 +402,7 @@ static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& m
                                    cudaStream_t stream) {
   const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmBarriers);
   auto kern = gemm_dense_kernel<BN, STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int tiles = ((M + kBM - 1) / kBM) * n_tiles_total;
   const int grid = tiles < num_sms() ? tiles : num_sms();
@@ -403,14 +419,13 @@ cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
   return launch_dense_bn<128, 6>(mapA, mapB0, mapB1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
 }
 
-template <int BN>
+template <int BN, int STAGES>
 static cudaError_t launch_routed_bn(const CUtensorMap& mapWq, const CUtensorMap& mapWsh, const gqe_bf16_t* x,
                                     const RoutedParams& rp, const EpiParams& epr, const EpiParams& eps,
                                     cudaStream_t stream) {
-  constexpr int STAGES = 6, LAG = 2;
-  const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmBarriers);
-  auto kern = gemm_routed_kernel<BN, STAGES, LAG>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmBarriers) + sizeof(SegTables);
+  auto kern = gemm_routed_kernel<BN, STAGES>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int max_tiles = rp.max_routed_tiles + rp.shared_tiles;
   const int grid = max_tiles < num_sms() ? max_tiles : num_sms();
@@ -421,8 +436,10 @@ static cudaError_t launch_routed_bn(const CUtensorMap& mapWq, const CUtensorMap&
 cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh, const gqe_bf16_t* x,
                                const RoutedParams& rp, const EpiParams& epr, const EpiParams& eps,
                                cudaStream_t stream) {
-  if (rp.d == 64) return launch_routed_bn<64>(mapWq, mapWsh, x, rp, epr, eps, stream);
-  return launch_routed_bn<128>(mapWq, mapWsh, x, rp, epr, eps, stream);
+  // deep rings: the gathered rows come from L2/HBM at 128 bytes per row, so
+  // many k-blocks stay in flight per gather thread
+  if (rp.d == 64) return launch_routed_bn<64, 8>(mapWq, mapWsh, x, rp, epr, eps, stream);
+  return launch_routed_bn<128, 6>(mapWq, mapWsh, x, rp, epr, eps, stream);
 }
 
 }  // namespace gqe

@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/gqe.h"
 #include "attn.cuh"
 #include "gemm.cuh"
@@ -47,8 +49,8 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
 // dims/box innermost first; strides in bytes for dims 1..rank-1.
-bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
-              const uint32_t* box) {
+bool encode_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
+                const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -64,6 +66,50 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, c
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Encoded maps are cached (a layer call re-encodes the same few maps every
+// step); a small direct-mapped table keyed by everything the encoding reads.
+struct MapKey {
+  const void* ptr;
+  int rank;
+  uint64_t dims[3];
+  uint32_t box[3];
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && rank == o.rank && !memcmp(dims, o.dims, sizeof(dims)) && !memcmp(box, o.box, sizeof(box));
+  }
+};
+
+bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box) {
+  constexpr int kSlots = 256;
+  static MapKey keys[kSlots];
+  static CUtensorMap maps[kSlots];
+  static bool used[kSlots];
+  static std::mutex mu;
+  MapKey k{};
+  k.ptr = ptr;
+  k.rank = rank;
+  for (int i = 0; i < rank && i < 3; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+  }
+  uint64_t h = reinterpret_cast<uintptr_t>(ptr) * 0x9E3779B97F4A7C15ull;
+  for (int i = 0; i < 3; ++i) h = (h ^ (k.dims[i] + 0x632BE5ABull * k.box[i])) * 0x100000001B3ull;
+  const int slot = (int)(h >> 56);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (used[slot] && keys[slot] == k) {
+      *m = maps[slot];
+      return true;
+    }
+  }
+  if (!encode_map(m, ptr, rank, dims, strides, box)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  keys[slot] = k;
+  maps[slot] = *m;
+  used[slot] = true;
+  return true;
 }
 
 bool map2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {

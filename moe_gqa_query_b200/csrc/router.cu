@@ -16,6 +16,7 @@
 // group); ties go to the lower expert index; selected experts are emitted in
 // ascending index order.
 #include "route.cuh"
+#include "launch.cuh"
 
 namespace gqe {
 
@@ -244,133 +245,147 @@ __global__ void __launch_bounds__(128) router_kernel(RouterParams p) {
 }
 
 
-// Wr resident in shared memory (when it fits), persistent over 32-token tiles;
-// x streams through one cp.async ring that runs across tile boundaries.
+// Wr resident in shared memory (when it fits); every warp streams its own
+// 16-token tile through a private cp.async ring (no block barriers), so eight
+// independent pipelines per CTA keep bytes in flight, then routes its tokens:
+// two lanes per token, each taking every other group, the token-scope sum
+// combined with one shuffle.
+constexpr int kWarpTok = 16;
+constexpr int kRouterWarps = 8;
+
 template <int GEP, int STAGES>
-__global__ void __launch_bounds__(128, 4) router_resident_kernel(RouterParams p) {
+__global__ void __launch_bounds__(kRouterWarps * 32, 1) router_resident_kernel(RouterParams p) {
   constexpr int WS = GEP + 8;
   constexpr int NT = GEP / 8;
+  constexpr int kStageBytes = kWarpTok * kKC * 2;                           // 2 KB
   extern __shared__ __align__(128) uint8_t rsm[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(rsm);                           // [STAGES][kTok*kKC]
-  uint16_t* wsm = xs + STAGES * kTok * kKC;                                  // [D][WS]
-  float* lgf = reinterpret_cast<float*>(wsm + (size_t)p.D * WS);             // [kTok][GEP+1]
-  float* gsf = lgf + kTok * (GEP + 1);                                        // [kTok][G]
+  uint16_t* wsm = reinterpret_cast<uint16_t*>(rsm);                           // [D][WS]
+  uint8_t* xring = rsm + (((size_t)p.D * WS * 2 + 127) & ~size_t(127));       // [warps][STAGES][2 KB]
+  float* lgw = reinterpret_cast<float*>(xring + (size_t)kRouterWarps * STAGES * kStageBytes);  // [warps][16][GEP+1]
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int GE = p.G * p.E;
   const int nkc = p.D / kKC;
-  const int n_tiles = (p.N + kTok - 1) / kTok;
-  const int my_tiles = (n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-  const int total = my_tiles * nkc;
-  const int mrow = (warp & 1) * 16;
-  const int khalf = warp >> 1;
+  const int n_tiles = (p.N + kWarpTok - 1) / kWarpTok;
+  uint8_t* ring = xring + (size_t)warp * STAGES * kStageBytes;
+  float* lg = lgw + (size_t)warp * kWarpTok * (GEP + 1);
 
-  auto load_x = [&](int it) {
-    const int tile = blockIdx.x + (it / nkc) * gridDim.x;
-    const int kc = it % nkc;
-    uint16_t* dst = xs + (it % STAGES) * kTok * kKC;
-#pragma unroll
-    for (int i = 0; i < kTok * 8 / 128; ++i) {
-      const int e = tid + 128 * i;
-      const int r = e >> 3, c = e & 7;
-      const int n = tile * kTok + r;
-      const uint16_t* src = p.x + (size_t)(n < p.N ? n : 0) * p.D + kc * kKC + c * 8;
-      cp_async_16(reinterpret_cast<uint8_t*>(dst) + r * 128 + ((c ^ (r & 7)) << 4), src, n < p.N);
-    }
-  };
-
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (s < total) load_x(s);
-    cp_async_commit();
-  }
-  // Wr into shared memory once (padded columns zero); 16-byte loads when the
-  // rows allow it
+  // Wr into shared memory once (padded columns zero)
   if ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0) {
     const int n16 = p.D * GE / 8;
-    for (int e = tid; e < n16; e += 128) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.Wr) + e);
+    for (int e = threadIdx.x; e < n16; e += blockDim.x) {
       const int r = (e * 8) / GE, c = (e * 8) % GE;
-      *reinterpret_cast<uint4*>(wsm + (size_t)r * WS + c) = v;
+      cp_async_16(wsm + (size_t)r * WS + c, reinterpret_cast<const uint4*>(p.Wr) + e, true);
     }
     if (GE < GEP)
-      for (int e = tid; e < p.D * (GEP - GE); e += 128)
+      for (int e = threadIdx.x; e < p.D * (GEP - GE); e += blockDim.x)
         wsm[(size_t)(e / (GEP - GE)) * WS + GE + e % (GEP - GE)] = 0;
   } else {
-    for (int e = tid; e < p.D * GEP; e += 128) {
+    for (int e = threadIdx.x; e < p.D * GEP; e += blockDim.x) {
       const int r = e / GEP, c = e % GEP;
       wsm[r * WS + c] = (c < GE) ? p.Wr[(size_t)r * GE + c] : (uint16_t)0;
     }
   }
-
-  float acc[NT][4];
-  for (int it = 0; it < total; ++it) {
-    const int kc = it % nkc;
-    if (kc == 0) {
-#pragma unroll
-      for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-    }
-    if (it + STAGES - 1 < total) load_x(it + STAGES - 1);
-    cp_async_commit();
-    cp_async_wait<STAGES - 1>();
-    __syncthreads();
-    const uint32_t xb = smem_u32(xs + (it % STAGES) * kTok * kKC);
-    const uint32_t wb = smem_u32(wsm + (size_t)kc * kKC * WS);
-#pragma unroll
-    for (int kh = 0; kh < kKC / 32; ++kh) {
-      const int ks = khalf * (kKC / 32) + kh;
-      const int mi = lane >> 3;
-      const int ar = mrow + (mi & 1) * 8 + (lane & 7);
-      const int ac = ks * 2 + (mi >> 1);
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(xb + ar * 128 + ((ac ^ (ar & 7)) << 4), a0, a1, a2, a3);
-#pragma unroll
-      for (int np = 0; np < NT / 2; ++np) {
-        const int kr = ks * 16 + (mi & 1) * 8 + (lane & 7);
-        const int nc = np * 16 + (mi >> 1) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(wb + (kr * WS + nc) * 2, b0, b1, b2, b3);
-        mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-    if (kc == nkc - 1) {
-      // tile done: add the two reduction halves, then route its tokens
-      const int tile = blockIdx.x + (it / nkc) * gridDim.x;
-      if (khalf == 1) {
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const int r = mrow + (lane >> 2);
-          const int c = t * 8 + (lane & 3) * 2;
-          lgf[r * (GEP + 1) + c] = acc[t][0];
-          lgf[r * (GEP + 1) + c + 1] = acc[t][1];
-          lgf[(r + 8) * (GEP + 1) + c] = acc[t][2];
-          lgf[(r + 8) * (GEP + 1) + c + 1] = acc[t][3];
-        }
-      }
-      __syncthreads();
-      if (khalf == 0) {
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const int r = mrow + (lane >> 2);
-          const int c = t * 8 + (lane & 3) * 2;
-          lgf[r * (GEP + 1) + c] += acc[t][0];
-          lgf[r * (GEP + 1) + c + 1] += acc[t][1];
-          lgf[(r + 8) * (GEP + 1) + c] += acc[t][2];
-          lgf[(r + 8) * (GEP + 1) + c + 1] += acc[t][3];
-        }
-      }
-      __syncthreads();
-      route_tile(p, lgf, GEP + 1, tile * kTok, gsf);
-    }
-    __syncthreads();
-  }
+  cp_async_commit();
   cp_async_wait<0>();
+  __syncthreads();
+
+  for (int tile = blockIdx.x * kRouterWarps + warp; tile < n_tiles; tile += gridDim.x * kRouterWarps) {
+    const int tok0 = tile * kWarpTok;
+    auto load_x = [&](int kc) {
+      uint8_t* dst = ring + (kc % STAGES) * kStageBytes;
+#pragma unroll
+      for (int i = 0; i < kWarpTok * 8 / 32; ++i) {       // 128 16-byte chunks, 4 per lane
+        const int e = lane + 32 * i;
+        const int r = e >> 3, c = e & 7;
+        const int n = tok0 + r;
+        const uint16_t* src = p.x + (size_t)(n < p.N ? n : 0) * p.D + kc * kKC + c * 8;
+        cp_async_16(dst + r * 128 + ((c ^ (r & 7)) << 4), src, n < p.N);
+      }
+    };
+    for (int kc = 0; kc < STAGES - 1; ++kc) {
+      if (kc < nkc) load_x(kc);
+      cp_async_commit();
+    }
+    float acc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    for (int kc = 0; kc < nkc; ++kc) {
+      cp_async_wait<STAGES - 2>();
+      __syncwarp();
+      if (kc + STAGES - 1 < nkc) load_x(kc + STAGES - 1);
+      cp_async_commit();
+      const uint32_t xb = smem_u32(ring + (kc % STAGES) * kStageBytes);
+      const uint32_t wb = smem_u32(wsm + (size_t)kc * kKC * WS);
+#pragma unroll
+      for (int ks = 0; ks < kKC / 16; ++ks) {
+        const int mi = lane >> 3;
+        const int ar = (mi & 1) * 8 + (lane & 7);
+        const int ac = ks * 2 + (mi >> 1);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(xb + ar * 128 + ((ac ^ (ar & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          const int kr = ks * 16 + (mi & 1) * 8 + (lane & 7);
+          const int nc = np * 16 + (mi >> 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(wb + (kr * WS + nc) * 2, b0, b1, b2, b3);
+          mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+    cp_async_wait<0>();
+    // logits of the 16 tokens into the warp's scratch
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int r = lane >> 2;
+      const int c = t * 8 + (lane & 3) * 2;
+      lg[r * (GEP + 1) + c] = acc[t][0];
+      lg[r * (GEP + 1) + c + 1] = acc[t][1];
+      lg[(r + 8) * (GEP + 1) + c] = acc[t][2];
+      lg[(r + 8) * (GEP + 1) + c + 1] = acc[t][3];
+    }
+    __syncwarp();
+    // routing: lanes 2i and 2i+1 share token i, each taking every other group
+    {
+      const int t = lane >> 1, half = lane & 1;
+      const int n = tok0 + t;
+      const float* row = lg + t * (GEP + 1);
+      float part = 0.f;
+      for (int g = half; g < p.G; g += 2) {
+        float pr[8], sum;
+        route_group(p, row, g, pr, &sum);
+        part += sum;
+      }
+      const float total = part + __shfl_xor_sync(0xffffffffu, part, 1);
+      if (n < p.N) {
+        for (int g = half; g < p.G; g += 2) {
+          float pr[8], sum;
+          const unsigned chosen = route_group(p, row, g, pr, &sum);
+          const float inv_den = 1.f / (p.scope == 0 ? total : sum);
+          const size_t o = ((size_t)n * p.G + g) * p.k;
+          int j = 0;
+          for (int ee = 0; ee < p.E; ++ee) {
+            if ((chosen >> ee) & 1u) {
+              p.topk_idx[o + j] = ee;
+              p.topk_w[o + j] = pr[ee] * inv_den;
+              ++j;
+            }
+          }
+          if (p.probs)
+            for (int ee = 0; ee < p.E; ++ee) p.probs[((size_t)n * p.G + g) * p.E + ee] = pr[ee];
+        }
+      }
+    }
+    __syncwarp();
+  }
 }
 
 template <int GEP>
 size_t resident_smem(int D, int stages) {
-  return (size_t)stages * kTok * kKC * 2 + (size_t)D * (GEP + 8) * 2 + (size_t)kTok * (GEP + 1) * 4 +
-         (size_t)kTok * 64 * 4;
+  return (((size_t)D * (GEP + 8) * 2 + 127) & ~size_t(127)) + (size_t)kRouterWarps * stages * kWarpTok * kKC * 2 +
+         (size_t)kRouterWarps * kWarpTok * (GEP + 1) * 4;
 }
 
 int router_num_sms() {
@@ -387,17 +402,17 @@ template <int GEP>
 cudaError_t launch_router_gep(const RouterParams& p, cudaStream_t stream) {
   constexpr int STAGES = 8;
   const size_t smem = resident_smem<GEP>(p.D, STAGES);
-  const int n_tiles = (p.N + kTok - 1) / kTok;
-  if (smem <= 100 * 1024) {
+  if (smem <= 200 * 1024) {
     auto kern = router_resident_kernel<GEP, STAGES>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
-    const int per_sm = (int)((220 * 1024) / (smem + 1024));
-    int grid = router_num_sms() * (per_sm < 1 ? 1 : per_sm);
-    if (grid > n_tiles) grid = n_tiles;
-    kern<<<grid, 128, smem, stream>>>(p);
+    const int n_tiles = (p.N + kWarpTok - 1) / kWarpTok;
+    int grid = router_num_sms();
+    const int need = (n_tiles + kRouterWarps - 1) / kRouterWarps;
+    if (grid > need) grid = need;
+    kern<<<grid, kRouterWarps * 32, smem, stream>>>(p);
   } else {
-    router_kernel<GEP><<<n_tiles, 128, 0, stream>>>(p);
+    router_kernel<GEP><<<(p.N + kTok - 1) / kTok, 128, 0, stream>>>(p);
   }
   return cudaGetLastError();
 }

@@ -71,6 +71,7 @@ class GQELayer:
         self.Wo = dev(weights["Wo"], (c.D, c.slots * c.d))
         self.bias = None if bias is None else torch.as_tensor(bias, dtype=torch.float32).to(self.device).contiguous()
         self._bufs = {}
+        self._graphs = {}
 
     # ------------------------------------------------------------------ buffers
     def _buf(self, name, shape, dtype=torch.bfloat16):
@@ -114,13 +115,31 @@ class GQELayer:
             return y, dict(idx=idx, w=w, q=q, q_sh=qs, K=K, V=V, o=o, o_sh=os_, h=h)
         return y
 
-    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None):
+    def forward_graph(self, x: torch.Tensor) -> torch.Tensor:
+        """forward() replayed from a CUDA graph captured on first use for this
+        input buffer and shape (the six library calls become one graph launch).
+        The returned tensor is the layer's own output buffer, overwritten by the
+        next call."""
+        key = (x.data_ptr(), tuple(x.shape))
+        entry = self._graphs.get(key)
+        if entry is None:
+            self.forward(x)                       # eager first: buffers, kernel attributes
+            torch.cuda.synchronize(self.device)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                y = self.forward(x)
+            entry = self._graphs[key] = (g, y)
+        g, y = entry
+        g.replay()
+        return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, graph: bool = True):
         """End-to-end call on host buffers (pinned for async copies): copy x in,
-        run forward, copy y out, all enqueued on the stream."""
-        c = self.cfg
+        run the forward (from a CUDA graph by default), copy y out, all on the
+        current stream."""
         xd = self._buf("x_in", tuple(x_host.shape))
         xd.copy_(x_host, non_blocking=True)
-        y = self.forward(xd, stream)
+        y = self.forward_graph(xd) if graph else self.forward(xd)
         y_host.copy_(y, non_blocking=True)
         return y_host
 

@@ -410,3 +410,19 @@ def test_device_exp2_helpers():
     torch.cuda.synchronize()
     assert (a.cpu() < 2.0 ** -124).all() and (a.cpu() > 0).all()
     assert c.cpu()[0] == 0
+
+
+def test_layer_graph_replay_matches_eager():
+    w = gi.WORKLOADS["tiny_prefill"]
+    dims, x, Wt, bias, layer = _layer(w, seed=3)
+    xd = bf16_dev(x)
+    y_eager = layer.forward(xd).clone()
+    y_graph = layer.forward_graph(xd).clone()
+    y_graph2 = layer.forward_graph(xd).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y_eager, y_graph) and torch.equal(y_graph, y_graph2)
+    x_pin = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_pin = torch.empty((dims.B, dims.T, dims.D), dtype=torch.bfloat16).pin_memory()
+    layer.forward_host(x_pin, y_pin)
+    torch.cuda.synchronize()
+    assert torch.equal(y_pin, y_eager.cpu())
