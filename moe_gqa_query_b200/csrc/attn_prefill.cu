@@ -300,7 +300,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         // exponentials (MUFU, or the FMA-pipe polynomial for kPolyPairs of every
         // 16 pairs), row sum, P (bf16) into tensor memory
         const float neg_m = -m_run;
-        float sum_lo = 0.f, sum_hi = 0.f;
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 16) {
           uint32_t pk[16];
@@ -317,13 +317,13 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
               p0 = ex2(x0);
               p1 = ex2(x1);
             }
-            sum_lo += p0;
-            sum_hi += p1;
+            sum4[(c & 1) * 2] += p0;
+            sum4[(c & 1) * 2 + 1] += p1;
             pk[c] = pack_bf16x2(p0, p1);
           }
           tmem_st16(p_base + c0, pk);
         }
-        l_run += sum_lo + sum_hi;
+        l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
         if (rescale) {
           ok = mbar_wait(&bar->pv_done[x], (j - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
           tc_fence_after();
