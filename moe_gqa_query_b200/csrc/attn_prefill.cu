@@ -376,6 +376,261 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   drain_after_abort(abort);
 }
 
+// ---------------------------------------------------------------------------
+// d = 64: one 128-row query tile per CTA in 256 tensor-memory columns
+// (S 0-127 | P 128-191 | O 192-255), so two CTAs share an SM.  The hardware
+// block scheduler then overlaps one item's set-up and epilogue with another
+// item's work, which matters when causal rows are short.  The MMA warp issues
+// P(j) V and Q K_{j+1}^T back to back; the commit after the latter also
+// covers the former, so when the softmax sees S(j+1), P(j) has been consumed
+// and O is final up to j.
+struct __align__(8) Attn1Barriers {
+  uint64_t q_full;
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t s_full, p_full, pv_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr int kSingleST = 2;   // two CTAs per SM must fit in 228 KB of shared memory
+constexpr size_t kSingleSmem = 1024 + kBox + 2 * kSingleST * kBox + sizeof(Attn1Barriers);
+
+__global__ void __launch_bounds__(192, 2)
+attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapQs,
+                           const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                           AttnParams p) {
+  constexpr int D = 64;
+  constexpr int ST = kSingleST;
+  constexpr uint32_t kS = 0, kP = 128, kO = 192;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + kBox;
+  uint8_t* sV = sK + ST * kBox;
+  Attn1Barriers* bar = reinterpret_cast<Attn1Barriers*>(sV + ST * kBox);
+  volatile int* abort = &bar->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item: one q-tile, level-major (heaviest first)
+  const int BG = p.B * p.G;
+  const int per_level = BG * p.k + p.B * p.n_shared;
+  const int n_levels = (p.T + kTile - 1) / kTile;
+  const int level = n_levels - 1 - (int)blockIdx.x / per_level;
+  const int i = blockIdx.x % per_level;
+  bool routed;
+  int seq, qt, kvseq, kk, rows_total;
+  if (i < BG * p.k) {
+    routed = true;
+    seq = i % BG;
+    qt = level * p.k + i / BG;
+    kvseq = seq;
+    kk = p.k;
+    rows_total = p.T * p.k;
+  } else {
+    routed = false;
+    seq = i - BG * p.k;
+    qt = level;
+    kvseq = seq * p.G + p.sg;
+    kk = 1;
+    rows_total = p.T;
+  }
+  const TileInfo ti = tile_info(qt, rows_total, kk, p.T);
+  if (ti.n_kv == 0) return;
+  const int n_kv = ti.n_kv;
+  const CUtensorMap* mq = routed ? &mapQ : &mapQs;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar->q_full, 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_empty[s], 1);
+      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->v_empty[s], 1);
+    }
+    mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->p_full, 128);
+    mbar_init(&bar->pv_done, 1);
+    bar->abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(mq);
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  if (warp == 5) tmem_alloc(&bar->tmem_base, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------- producer: Q once, then K_0, V_0, K_1, V_1, ...
+      mbar_arrive_expect_tx(&bar->q_full, kBox);
+      tma_load_3d(sQ, mq, &bar->q_full, 0, ti.row0, seq);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % ST;
+        const uint32_t ph = ((j / ST) & 1) ^ 1;
+        if (j >= ST && !mbar_wait(&bar->k_empty[s], ph, abort, p.err, kErrTimeoutAttn)) break;
+        mbar_arrive_expect_tx(&bar->k_full[s], kBox);
+        tma_load_3d(sK + s * kBox, &mapK, &bar->k_full[s], 0, j * kTile, kvseq);
+        if (j >= ST && !mbar_wait(&bar->v_empty[s], ph, abort, p.err, kErrTimeoutAttn)) break;
+        mbar_arrive_expect_tx(&bar->v_full[s], kBox);
+        tma_load_3d(sV + s * kBox, &mapV, &bar->v_full[s], 0, j * kTile, kvseq);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: S_0 | PV_0 S_1 | PV_1 S_2 | ...
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kTile, D, false, true);
+      const uint32_t q0 = smem_u32(sQ);
+      auto issue_s = [&](int j) {
+        const int s = j % ST;
+        if (!mbar_wait(&bar->k_full[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn)) return false;
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(sK + s * kBox);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          umma_ss(tmem + kS, sdesc_sw128(q0 + ks * 32, 16, 1024), sdesc_sw128(k0 + ks * 32, 16, 1024), idesc_s,
+                  ks > 0);
+        umma_commit(&bar->s_full);
+        umma_commit(&bar->k_empty[s]);
+        return true;
+      };
+      bool ok = mbar_wait(&bar->q_full, 0, abort, p.err, kErrTimeoutAttn) && issue_s(0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        ok = mbar_wait(&bar->p_full, j & 1, abort, p.err, kErrTimeoutAttn);
+        tc_fence_after();
+        const int s = j % ST;
+        ok = ok && mbar_wait(&bar->v_full[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(sV + s * kBox);
+#pragma unroll
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          umma_ts(tmem + kO, tmem + kP + ks * 8, sdesc_sw128(v0 + ks * 2048, kBox, 1024), idesc_o,
+                  (j > 0 || ks > 0));
+        umma_commit(&bar->pv_done);
+        umma_commit(&bar->v_empty[s]);
+        if (j + 1 < n_kv) ok = issue_s(j + 1);
+      }
+    }
+  } else {
+    // ---------------- softmax: warps 0-3, one query row per thread
+    const int lg = warp;
+    const int r = lg * 32 + lane;
+    const int prow = ti.row0 + r;
+    const bool valid = prow < rows_total;
+    const int t_r = prow / kk;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    const uint32_t s_base = tmem + lane_off + kS;
+    const uint32_t p_base = tmem + lane_off + kP;
+    const uint32_t o_base = tmem + lane_off + kO;
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      // S(j) ready; its commit also covers P(j-1) V, so P and O are free
+      ok = mbar_wait(&bar->s_full, j & 1, abort, p.err, kErrTimeoutAttn);
+      tc_fence_after();
+      const bool diag = j * kTile + kTile - 1 > ti.t_first;
+      const int lim = t_r - j * kTile;
+      uint32_t s[128];
+      tmem_ld128(s_base, s);
+      if (diag) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c > lim) s[c] = __float_as_uint(-INFINITY);
+      }
+      float m8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        m8[c & 7] = fmax3(m8[c & 7], __uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]));
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float m_new = fmaxf(m_run, mx * sl2);
+      bool rescale = false;
+      float alpha = 1.f;
+      if (j == 0) {
+        m_run = m_new;
+      } else {
+        const bool need = m_new > m_run + kRescaleLog2;
+        rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          alpha = ex2(m_run - m_new);
+          l_run *= alpha;
+          m_run = m_new;
+        }
+      }
+      const float neg_m = -m_run;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c0 = 0; c0 < 64; c0 += 16) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int q = c0 + c;
+          const float x0 = fmaf(__uint_as_float(s[2 * q]), sl2, neg_m);
+          const float x1 = fmaf(__uint_as_float(s[2 * q + 1]), sl2, neg_m);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          sum4[(c & 1) * 2] += p0;
+          sum4[(c & 1) * 2 + 1] += p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(p_base + c0, pk);
+      }
+      l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      if (rescale) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(o_base + c0, o);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(o_base + c0, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar->p_full);
+    }
+    // ---------------- epilogue: O / l -> bf16
+    ok = mbar_wait(&bar->pv_done, (n_kv - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
+    tc_fence_after();
+    const float inv_l = 1.f / l_run;
+    gqe_bf16_t* orow = routed ? p.o_routed + ((size_t)seq * rows_total + prow) * D
+                              : p.o_sh + ((size_t)seq * p.T + prow) * D;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t o[32];
+      tmem_ld32(o_base + c0, o);
+      if (valid && ok) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+        uint4* d4 = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+    }
+    if (p.lse && valid && ok) {
+      const size_t li = routed ? (size_t)seq * rows_total + prow
+                               : (size_t)BG * p.T * p.k + (size_t)seq * p.T + prow;
+      p.lse[li] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+  drain_after_abort(abort);
+}
+
 }  // namespace
 
 template <int D>
@@ -391,8 +646,22 @@ static cudaError_t launch_d(const CUtensorMap& mQ, const CUtensorMap& mQs, const
   return cudaGetLastError();
 }
 
+static cudaError_t launch_single(const CUtensorMap& mQ, const CUtensorMap& mQs, const CUtensorMap& mK,
+                                 const CUtensorMap& mV, const AttnParams& p, cudaStream_t stream) {
+  auto kern = attn_prefill_single_kernel;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), kSingleSmem);
+  if (e != cudaSuccess) return e;
+  const int n_levels = (p.T + kTile - 1) / kTile;
+  const int per_level = p.B * p.G * p.k + p.B * p.n_shared;
+  kern<<<n_levels * per_level, 192, kSingleSmem, stream>>>(mQ, mQs, mK, mV, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_prefill(const CUtensorMap& mQ, const CUtensorMap& mQs, const CUtensorMap& mK,
                                 const CUtensorMap& mV, const AttnParams& p, int d, cudaStream_t stream) {
+#ifndef GQE_ATTN_PAIRED_D64
+  if (d == 64) return launch_single(mQ, mQs, mK, mV, p, stream);
+#endif
   if (d == 64) return launch_d<64>(mQ, mQs, mK, mV, p, stream);
   return launch_d<128>(mQ, mQs, mK, mV, p, stream);
 }
