@@ -411,7 +411,8 @@ def main():
     attn_ms = float(seg_ms[:, 3].mean())
     flops = attn_useful_flops(dims)
     achieved_tf = flops / (attn_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "attn_prefill_kernel<64>", "achieved": achieved_tf,
+    attn_kernel = "attn_prefill_single_kernel (d=64)" if dims.d == 64 else f"attn_prefill_kernel<{dims.d}>"
+    roofline = {"bound": "tensor", "kernel": attn_kernel, "achieved": achieved_tf,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
                 "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": None,
                 "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_ms}

@@ -380,14 +380,17 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
 // d = 64: one 128-row query tile per CTA in 256 tensor-memory columns
 // (S 0-127 | P 128-191 | O 192-255), so two CTAs share an SM.  The hardware
 // block scheduler then overlaps one item's set-up and epilogue with another
-// item's work, which matters when causal rows are short.  The MMA warp issues
-// P(j) V and Q K_{j+1}^T back to back; the commit after the latter also
-// covers the former, so when the softmax sees S(j+1), P(j) has been consumed
-// and O is final up to j.
+// item's work, which matters when causal rows are short.
+//
+// The softmax warps copy S(j) into registers and release its columns at once
+// (s_free), so the MMA warp computes S(j+1) = Q K_{j+1}^T while the
+// exponentials of tile j run; P(j) V follows when P(j) is in tensor memory.
+// Before writing P(j+1) (and rescaling O) the softmax waits for P(j) V to
+// finish (pv_done).
 struct __align__(8) Attn1Barriers {
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full, p_full, pv_done;
+  uint64_t s_full, s_free, p_full, pv_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -448,6 +451,7 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       mbar_init(&bar->v_empty[s], 1);
     }
     mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->s_free, 128);
     mbar_init(&bar->p_full, 128);
     mbar_init(&bar->pv_done, 1);
     bar->abort = 0;
@@ -480,7 +484,7 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      // ---------------- MMA issuer: S_0 | PV_0 S_1 | PV_1 S_2 | ...
+      // ---------------- MMA issuer: S_0 | S_1 PV_0 | S_2 PV_1 | ...
       constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kTile, D, false, true);
       const uint32_t q0 = smem_u32(sQ);
@@ -499,6 +503,12 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       };
       bool ok = mbar_wait(&bar->q_full, 0, abort, p.err, kErrTimeoutAttn) && issue_s(0);
       for (int j = 0; ok && j < n_kv; ++j) {
+        if (j + 1 < n_kv) {
+          // S(j) is in the softmax registers: overwrite its columns with S(j+1)
+          ok = mbar_wait(&bar->s_free, j & 1, abort, p.err, kErrTimeoutAttn);
+          tc_fence_after();
+          if (!ok || !issue_s(j + 1)) break;
+        }
         ok = mbar_wait(&bar->p_full, j & 1, abort, p.err, kErrTimeoutAttn);
         tc_fence_after();
         const int s = j % ST;
@@ -512,7 +522,6 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
                   (j > 0 || ks > 0));
         umma_commit(&bar->pv_done);
         umma_commit(&bar->v_empty[s]);
-        if (j + 1 < n_kv) ok = issue_s(j + 1);
       }
     }
   } else {
@@ -530,13 +539,14 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
-      // S(j) ready; its commit also covers P(j-1) V, so P and O are free
       ok = mbar_wait(&bar->s_full, j & 1, abort, p.err, kErrTimeoutAttn);
       tc_fence_after();
       const bool diag = j * kTile + kTile - 1 > ti.t_first;
       const int lim = t_r - j * kTile;
       uint32_t s[128];
       tmem_ld128(s_base, s);
+      tc_fence_before();
+      mbar_arrive(&bar->s_free);     // S(j) is in registers; the MMA warp may overwrite it
       if (diag) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
@@ -567,11 +577,11 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       const float neg_m = -m_run;
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c0 = 0; c0 < 64; c0 += 16) {
-        uint32_t pk[16];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int q = c0 + c;
+        for (int c = 0; c < 32; ++c) {
+          const int q = h * 32 + c;
           const float x0 = fmaf(__uint_as_float(s[2 * q]), sl2, neg_m);
           const float x1 = fmaf(__uint_as_float(s[2 * q + 1]), sl2, neg_m);
           const float p0 = ex2(x0), p1 = ex2(x1);
@@ -579,7 +589,12 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
           sum4[(c & 1) * 2 + 1] += p1;
           pk[c] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(p_base + c0, pk);
+        // P(j-1) V must be done before P is overwritten (and O rescaled)
+        if (h == 0 && j > 0) {
+          ok = mbar_wait(&bar->pv_done, (j - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
+          tc_fence_after();
+        }
+        tmem_st32(p_base + h * 32, pk);
       }
       l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       if (rescale) {
