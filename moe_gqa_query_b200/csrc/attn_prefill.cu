@@ -42,13 +42,24 @@ constexpr int kThreads = 320;
 constexpr int kTile = 128;          // query rows and keys per tile
 constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16, 16 KB
 constexpr float kRescaleLog2 = 8.0f;
+// Single-tile kernel (d = 64): GQE_ATTN1_F2 computes the scaled logits and the
+// row sums with packed f32x2 FMA/ADD (half the instructions), and
+// GQE_ATTN1_POLY column pairs of every 16 take the FMA-pipe polynomial 2^x
+// instead of MUFU ex2.  Measured on B200: 2 of 16 is 3-5 % faster than 0,
+// 4 of 16 no better (register pressure).
+#ifndef GQE_ATTN1_F2
+#define GQE_ATTN1_F2 1
+#endif
+#ifndef GQE_ATTN1_POLY
+#define GQE_ATTN1_POLY 2
+#endif
 #ifndef GQE_ATTN_POLY_PAIRS
 #define GQE_ATTN_POLY_PAIRS 0
 #endif
-// Column pairs (of every 16) whose exponentials run as the FMA-pipe polynomial
-// instead of MUFU ex2.  On B200 the softmax here is bound by instruction issue,
-// not by MUFU throughput (measured: 0, 3, 5 and 8 of 16 within 3 % of each
-// other at d = 64), so the default keeps every exponential on MUFU.
+// Paired kernel (d = 128): column pairs (of every 16) whose exponentials run as
+// the polynomial.  There the softmax is bound by instruction issue, not by MUFU
+// throughput (measured: 0, 3, 5 and 8 of 16 within 3 % of each other), so the
+// default keeps every exponential on MUFU.
 constexpr int kPolyPairs = GQE_ATTN_POLY_PAIRS;
 
 struct __align__(8) AttnBarriers {
@@ -575,18 +586,38 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
         }
       }
       const float neg_m = -m_run;
+#if GQE_ATTN1_F2
+      const unsigned long long sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+      unsigned long long sum2[2] = {0ull, 0ull};
+#else
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#endif
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int q = h * 32 + c;
+#if GQE_ATTN1_F2
+          const unsigned long long x =
+              f2_fma(f2_pack(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), sl2x2, negm2);
+          float p0, p1;
+          if ((c & 15) < GQE_ATTN1_POLY) {
+            exp2_poly2(x, p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          sum2[c & 1] = f2_add(sum2[c & 1], f2_pack(p0, p1));
+#else
           const float x0 = fmaf(__uint_as_float(s[2 * q]), sl2, neg_m);
           const float x1 = fmaf(__uint_as_float(s[2 * q + 1]), sl2, neg_m);
           const float p0 = ex2(x0), p1 = ex2(x1);
           sum4[(c & 1) * 2] += p0;
           sum4[(c & 1) * 2 + 1] += p1;
+#endif
           pk[c] = pack_bf16x2(p0, p1);
         }
         // P(j-1) V must be done before P is overwritten (and O rescaled)
@@ -596,7 +627,16 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
         }
         tmem_st32(p_base + h * 32, pk);
       }
+#if GQE_ATTN1_F2
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(sum2[0], a0, a1);
+        f2_unpack(sum2[1], b0, b1);
+        l_run += (a0 + a1) + (b0 + b1);
+      }
+#else
       l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+#endif
       if (rescale) {
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
