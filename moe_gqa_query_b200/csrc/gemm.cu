@@ -91,12 +91,56 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, int map_sel, 
   }
 }
 
+// Coalesced epilogue: each 64-column chunk of the warp's 32 rows goes through
+// a 4 KB 128-byte-swizzled staging buffer (two per warp, alternating) and out
+// with one TMA store; rows past the output are clipped by the tensor map.
+constexpr int kStageOutBytes = 32 * 64 * 2;
+constexpr int kEpiStagingBytes = 4 * 2 * kStageOutBytes;   // four epilogue warps
+
+template <int BN>
+__device__ __forceinline__ void epilogue_tile_tma(const EpiParams& ep, const CUtensorMap* mo, int row0, int n0,
+                                                  uint32_t tmem_row, uint8_t* stg, int& chunk, bool ok) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    if (n0 + c0 >= ep.n_limit) break;
+    uint32_t v[64];
+    tmem_ld64(tmem_row + c0, v);
+    if (!ok) continue;
+    uint8_t* buf = stg + (chunk & 1) * kStageOutBytes;
+    if (chunk >= 2) {
+      if (lane == 0) bulk_wait_read<1>();   // the store that used this buffer has read it
+      __syncwarp();
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      st_shared_v4(buf + lane * 128 + ((j ^ (lane & 7)) << 4), pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                   pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                   pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                   pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int n = n0 + c0;
+      if (ep.store_mode == kStoreTma2d) {
+        tma_store_2d(mo, buf, n, row0);
+      } else {
+        const int b = row0 / ep.T, t = row0 - b * ep.T;
+        tma_store_3d(mo, buf, n % ep.d, t, b * ep.G + n / ep.d);
+      }
+      bulk_commit();
+    }
+    ++chunk;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // dense: A [M, K] and W [N, K] by TMA; persistent over (m-tile, n-tile)
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
 gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
-                  const __grid_constant__ CUtensorMap mapB1, EpiParams ep, int M, int K, int n_tiles_b0,
+                  const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapO0,
+                  const __grid_constant__ CUtensorMap mapO1, EpiParams ep, int M, int K, int n_tiles_b0,
                   int n_tiles_total) {
   constexpr int kBTileBytes = BN * kBK * 2;
   constexpr uint32_t kTmemCols = 2 * BN;
@@ -104,7 +148,8 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kATileBytes;
-  GemmBarriers* bar = reinterpret_cast<GemmBarriers*>(sB + STAGES * kBTileBytes);
+  uint8_t* sOut = sB + STAGES * kBTileBytes;
+  GemmBarriers* bar = reinterpret_cast<GemmBarriers*>(sOut + kEpiStagingBytes);
   volatile int* abort = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -178,7 +223,8 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
   } else {
     const int lg = warp & 3;
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
-    int tc = 0;
+    uint8_t* stg = sOut + lg * 2 * kStageOutBytes;
+    int tc = 0, chunk = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
       const int ab = tc & 1, use = tc >> 1;
       const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, ep.err, kErrTimeoutGemm);
@@ -187,12 +233,17 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
       const int sel = nt >= n_tiles_b0;
       const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
       const int row = mt * kBM + lg * 32 + lane;
-      epilogue_tile<BN>(ep, sel, row, n0, tmem + lane_off + (uint32_t)(ab * BN), ok && row < M);
+      const uint32_t tacc = tmem + lane_off + (uint32_t)(ab * BN);
+      if (ep.store_mode != kStorePerThread)
+        epilogue_tile_tma<BN>(ep, sel ? &mapO1 : &mapO0, mt * kBM + lg * 32, n0, tacc, stg, chunk, ok);
+      else
+        epilogue_tile<BN>(ep, sel, row, n0, tacc, ok && row < M);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->acc_empty[ab]);
       if (!ok) break;
     }
+    if (lane == 0) bulk_wait<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -201,6 +252,145 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
     tmem_dealloc(tmem, kTmemCols);
   }
   drain_after_abort(abort);
+}
+
+// ---------------------------------------------------------------------------
+// dense, CTA pairs: one 256 x 256 output tile per pair and step, issued as
+// M = 256 tcgen05 MMAs over both SMs.  Each CTA loads 128 rows of A and 128
+// rows of W per k-block (32 KB) where the single-CTA 128 x 256 tile loads
+// 16 + 32 KB for the same MMA work: a third fewer bytes through L2 per FLOP.
+// Both CTAs' loads count on the even CTA's `full` barrier; the even CTA's MMA
+// thread releases stages and accumulators in both CTAs with one commit each.
+template <int STAGES>
+__global__ void __launch_bounds__(192, 1)
+gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
+                       const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapO0,
+                       const __grid_constant__ CUtensorMap mapO1, EpiParams ep, int M, int K, int n_tiles_b0,
+                       int n_tiles_total) {
+  constexpr int BN = 256;
+  constexpr int kPM = 2 * kBM;                       // pair tile rows
+  constexpr int kHalfB = (BN / 2) * kBK * 2;         // 16 KB
+  constexpr uint32_t kTmemCols = 2 * BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kATileBytes;
+  uint8_t* sOut = sB + STAGES * kHalfB;
+  GemmBarriers* bar = reinterpret_cast<GemmBarriers*>(sOut + kEpiStagingBytes);
+  volatile int* abort = &bar->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int nk = K / kBK;
+  const int m_tiles = (M + kPM - 1) / kPM;
+  const int total = m_tiles * n_tiles_total;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bar->full[s], 1);      // used in the even CTA only
+      mbar_init(&bar->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bar->acc_full[a], 1);
+      mbar_init(&bar->acc_empty[a], 8);  // even CTA: 4 epilogue warps of each CTA
+    }
+    bar->abort = 0;
+    fence_mbar_init_cluster();
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB0);
+    tma_prefetch_desc(&mapB1);
+  }
+  if (warp == 1) tmem_alloc_pair(&bar->tmem_base, kTmemCols);
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t full0 = cluster_addr(&bar->full[0], 0);
+      int it = 0;
+      for (int t = pair; t < total && !*abort; t += n_pairs) {
+        const int mt = t / n_tiles_total, nt = t % n_tiles_total;
+        const int sel = nt >= n_tiles_b0;
+        const CUtensorMap* mB = sel ? &mapB1 : &mapB0;
+        const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN + (int)rank * (BN / 2);
+        const int m0 = mt * kPM + (int)rank * kBM;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, ep.err, kErrTimeoutGemm))
+            break;
+          if (rank == 0) mbar_arrive_expect_tx(&bar->full[s], 2 * (kATileBytes + kHalfB));
+          const uint32_t fb = full0 + (uint32_t)(s * sizeof(uint64_t));
+          tma_load_2d_pair(sA + s * kATileBytes, &mapA, fb, kb * kBK, m0);
+          tma_load_2d_pair(sB + s * kHalfB, mB, fb, kb * kBK, n0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kPM, BN, false, false);
+      const uint32_t empty_peer0 = cluster_addr(&bar->empty[0], peer);
+      const uint32_t accf_peer0 = cluster_addr(&bar->acc_full[0], peer);
+      int it = 0, tc = 0;
+      for (int t = pair; t < total && !*abort; t += n_pairs, ++tc) {
+        const int ab = tc & 1, use = tc >> 1;
+        if (tc >= 2 && !mbar_wait(&bar->acc_empty[ab], (use & 1) ^ 1, abort, ep.err, kErrTimeoutGemm)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(ab * BN);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&bar->full[s], (it / STAGES) & 1, abort, ep.err, kErrTimeoutGemm)) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kATileBytes);
+          const uint32_t b0 = smem_u32(sB + s * kHalfB);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_ss_pair(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
+                         (kb | kk) != 0);
+          umma_commit_pair(smem_u32(&bar->empty[s]));
+          umma_commit_pair(empty_peer0 + (uint32_t)(s * sizeof(uint64_t)));
+        }
+        umma_commit_pair(smem_u32(&bar->acc_full[ab]));
+        umma_commit_pair(accf_peer0 + (uint32_t)(ab * sizeof(uint64_t)));
+      }
+    }
+  } else {
+    const int lg = warp & 3;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    const uint32_t acce0 = cluster_addr(&bar->acc_empty[0], 0);
+    uint8_t* stg = sOut + lg * 2 * kStageOutBytes;
+    int tc = 0, chunk = 0;
+    for (int t = pair; t < total; t += n_pairs, ++tc) {
+      const int ab = tc & 1, use = tc >> 1;
+      const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, ep.err, kErrTimeoutGemm);
+      tc_fence_after();
+      const int mt = t / n_tiles_total, nt = t % n_tiles_total;
+      const int sel = nt >= n_tiles_b0;
+      const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
+      const int row0 = mt * kPM + (int)rank * kBM + lg * 32;
+      const uint32_t tacc = tmem + lane_off + (uint32_t)(ab * BN);
+      if (ep.store_mode != kStorePerThread)
+        epilogue_tile_tma<BN>(ep, sel ? &mapO1 : &mapO0, row0, n0, tacc, stg, chunk, ok);
+      else
+        epilogue_tile<BN>(ep, sel, row0 + lane, n0, tacc, ok && row0 + lane < M);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce0 + (uint32_t)(ab * sizeof(uint64_t)));
+      if (!ok) break;
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+  // an aborted CTA lets copies in flight land before its pair partner may exit
+  drain_after_abort(abort);
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -398,25 +588,71 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
 
 template <int BN, int STAGES>
 static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
-                                   const EpiParams& ep, int M, int K, int n_tiles_b0, int n_tiles_total,
-                                   cudaStream_t stream) {
-  const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmBarriers);
+                                   const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M,
+                                   int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream) {
+  const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
   auto kern = gemm_dense_kernel<BN, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int tiles = ((M + kBM - 1) / kBM) * n_tiles_total;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  kern<<<grid, 192, smem, stream>>>(mapA, mapB0, mapB1, ep, M, K, n_tiles_b0, n_tiles_total);
+  kern<<<grid, 192, smem, stream>>>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total);
   return cudaGetLastError();
+}
+
+template <int STAGES>
+static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
+                                        const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M, int K, int n_tiles_b0, int n_tiles_total,
+                                        cudaStream_t stream) {
+  const size_t smem = 1024 + STAGES * (kATileBytes + 128 * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
+  auto kern = gemm_dense_pair_kernel<STAGES>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // co-resident pairs on this device (a cluster needs both SMs in one GPC)
+  static int max_pairs[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& mp = max_pairs[dev & 63];
+  if (mp <= 0) {
+    cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kern), &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    mp = n;
+  }
+  const int total = ((M + 255) / 256) * n_tiles_total;
+  const int pairs = total < mp ? total : mp;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  return cudaLaunchKernelEx(&cfg, kern, mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total);
+}
+
+cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
+                                   const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M,
+                                   int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream) {
+  return launch_dense_pair_st<6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
 }
 
 int dense_tile_n(int n_per_weight) { return (n_per_weight % 256 == 0) ? 256 : 128; }
 
 cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
-                              const EpiParams& ep, int M, int K, int n_tiles_b0, int n_tiles_total, int bn,
-                              cudaStream_t stream) {
-  if (bn == 256) return launch_dense_bn<256, 4>(mapA, mapB0, mapB1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
-  return launch_dense_bn<128, 6>(mapA, mapB0, mapB1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
+                              const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
+                              int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream) {
+  if (bn == 256)
+    return launch_dense_bn<256, 4>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
+  return launch_dense_bn<128, 6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
 }
 
 template <int BN, int STAGES>

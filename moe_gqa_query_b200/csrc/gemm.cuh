@@ -23,6 +23,14 @@ struct EpiParams {
   int n_limit;           // columns >= n_limit are not written
   int T, G, d, L_max;
   unsigned* err;         // device error word
+  int store_mode;        // dense kernels: kStorePerThread or a TMA store layout
+};
+
+// How the dense kernels write their output.
+enum StoreMode : int {
+  kStorePerThread = 0,   // each thread stores its row (any EpiMode)
+  kStoreTma2d = 1,       // kEpiRowMajor through maps over [M, N], box 64 cols x 32 rows
+  kStoreTmaHeads = 2,    // kEpiHeads through maps over [B*G, T, d], box 64 x 32 x 1 (T % 32 == 0)
 };
 
 // Token-to-expert permutation produced by perm.cu, consumed by the routed GEMM.
@@ -43,9 +51,18 @@ struct RoutedParams {
 // Output tile width for a weight with n_per_weight rows: 256 when it divides, else 128.
 int dense_tile_n(int n_per_weight);
 
+// mapO0 / mapO1: output maps for ep.store_mode != kStorePerThread.
 cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
-                              const CUtensorMap& mapB1, const EpiParams& ep, int M, int K,
+                              const CUtensorMap& mapB1, const CUtensorMap& mapO0,
+                              const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
                               int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream);
+
+// 256 x 256 tiles over CTA pairs; W maps with 128-row boxes, weights' rows a
+// multiple of 256.
+cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapB0,
+                                   const CUtensorMap& mapB1, const CUtensorMap& mapO0,
+                                   const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
+                                   int n_tiles_b0, int n_tiles_total, cudaStream_t stream);
 
 cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh,
                                const gqe_bf16_t* x, const RoutedParams& rp, const EpiParams& epr,

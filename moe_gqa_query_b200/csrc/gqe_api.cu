@@ -301,20 +301,37 @@ gqe_status gqe_routed_qproj(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
   return cuda_status(launch_gemm_routed(mWq, mWsh, x, rp, epr, eps, S(stream)));
 }
 
+// CTA-pair GEMM (256 x 256 tiles) when the weights tile by 256 and there are
+// enough rows to fill the pairs; single-CTA 128-row tiles otherwise.
+#ifndef GQE_GEMM_PAIR
+#define GQE_GEMM_PAIR 1
+#endif
+static bool use_pair_gemm(int M, int bn) { return GQE_GEMM_PAIR && bn == 256 && M >= 2048; }
+
 static gqe_status kv_common(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk, const gqe_bf16* Wv,
                             EpiParams& ep, int M, gqe_stream stream) {
   const int G = dims->G, d = dims->d_head, D = dims->d_model;
   const int bn = dense_tile_n(G * d);
+  const bool pair = use_pair_gemm(M, bn);
   CUtensorMap mA, mK, mV;
   GQE_REQUIRE(map2d(&mA, x, D, M, 128), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mK, Wk, D, (uint64_t)G * d, bn), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mV, Wv, D, (uint64_t)G * d, bn), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mK, Wk, D, (uint64_t)G * d, pair ? 128 : bn), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mV, Wv, D, (uint64_t)G * d, pair ? 128 : bn), GQE_ERR_CUDA);
   ep.n_limit = G * d;
   ep.G = G;
   ep.d = d;
   ep.err = error_word();
+  // head-layout output through TMA stores when 32-row groups stay inside one sequence
+  CUtensorMap mOK{}, mOV{};
+  ep.store_mode = kStorePerThread;
+  if (ep.mode == kEpiHeads && ep.T % 32 == 0) {
+    GQE_REQUIRE(map3d(&mOK, ep.out0, d, ep.T, (uint64_t)(M / ep.T) * G, 32), GQE_ERR_CUDA);
+    GQE_REQUIRE(map3d(&mOV, ep.out1, d, ep.T, (uint64_t)(M / ep.T) * G, 32), GQE_ERR_CUDA);
+    ep.store_mode = kStoreTmaHeads;
+  }
   const int nt = (G * d + bn - 1) / bn;
-  return cuda_status(launch_gemm_dense(mA, mK, mV, ep, M, D, nt, 2 * nt, bn, S(stream)));
+  if (pair) return cuda_status(launch_gemm_dense_pair(mA, mK, mV, mOK, mOV, ep, M, D, nt, 2 * nt, S(stream)));
+  return cuda_status(launch_gemm_dense(mA, mK, mV, mOK, mOV, ep, M, D, nt, 2 * nt, bn, S(stream)));
 }
 
 gqe_status gqe_kv_proj(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk, const gqe_bf16* Wv,
@@ -441,9 +458,10 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   GQE_REQUIRE((long long)M * N < (1ll << 31) && (long long)M * K < (1ll << 31), GQE_ERR_UNSUPPORTED);
   GQE_REQUIRE(aligned16(A) && aligned16(W) && aligned16(C), GQE_ERR_INVALID_ARG);
   const int bn = dense_tile_n(N);
+  const bool pair = use_pair_gemm(M, bn);
   CUtensorMap mA, mW;
   GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mW, W, K, N, bn), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mW, W, K, N, pair ? 128 : bn), GQE_ERR_CUDA);
   EpiParams ep{};
   ep.out0 = C;
   ep.out1 = C;
@@ -451,8 +469,12 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   ep.ldo = N;
   ep.n_limit = N;
   ep.err = error_word();
+  CUtensorMap mO;
+  GQE_REQUIRE(map2d(&mO, C, N, M, 32), GQE_ERR_CUDA);
+  ep.store_mode = kStoreTma2d;
   const int nt = (N + bn - 1) / bn;
-  return cuda_status(launch_gemm_dense(mA, mW, mW, ep, M, K, nt, nt, bn, S(stream)));
+  if (pair) return cuda_status(launch_gemm_dense_pair(mA, mW, mW, mO, mO, ep, M, K, nt, nt, S(stream)));
+  return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, K, nt, nt, bn, S(stream)));
 }
 
 gqe_status gqe_device_error(int* code, gqe_stream stream) {

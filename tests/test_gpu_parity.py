@@ -132,8 +132,10 @@ def test_routed_qproj(case):
 # dense K/V projection, output projection
 
 @pytest.mark.parametrize("dims", [gi.WORKLOADS["tiny_prefill"].dims, D(B=2, T=77, D=128, G=3, E=2, k=1),
-                                  D(B=1, T=130, D=192, G=1, E=2, k=1, d=128), gi.WORKLOADS["main_prefill"].dims],
-                         ids=["tiny", "ragged_G3", "G1_d128", "main"])
+                                  D(B=1, T=130, D=192, G=1, E=2, k=1, d=128),
+                                  D(B=3, T=700, D=256, G=4, E=2, k=1),
+                                  gi.WORKLOADS["main_prefill"].dims],
+                         ids=["tiny", "ragged_G3", "G1_d128", "pair_ragged_M", "main"])
 def test_kv_proj(dims):
     x = gi.layer_input(dims, 2)
     Wt = gi.layer_weights(dims, 2)
@@ -146,7 +148,8 @@ def test_kv_proj(dims):
     assert_close_proj(to_f64(V), V_ref, "V")
 
 
-@pytest.mark.parametrize("M,N,K", [(200, 192, 320), (16, 64, 64), (1000, 256, 640), (16384, 1024, 640)])
+@pytest.mark.parametrize("M,N,K", [(200, 192, 320), (16, 64, 64), (1000, 256, 640), (2125, 512, 192),
+                                   (4133, 768, 1024), (16384, 1024, 640)])
 def test_linear(M, N, K):
     rng_dims = gi.GQEDims(B=1, T=M, D=K, G=1, E=1, k=1, d=64)
     A = gi.normal_bf16(3, "x", (M, K), 1.0)
