@@ -363,7 +363,12 @@ def main():
         h = layer._buf("h", (N, c.slots * c.d))
         y = layer._buf("y", (B, T, c.D))
         ws = layer._ws("ws_q", L.gqe_workspace_size(d_, L.GQE_OP_ROUTED_QPROJ))
-        rec = (lambda i: evs[i].record(stream)) if evs is not None else (lambda i: None)
+        if evs is None:
+            rec = lambda i: None
+        elif len(evs) == 2:                     # whole step: start and end only
+            rec = lambda i: evs[min(i, 1)].record(stream) if i in (0, 6) else None
+        else:                                   # per call
+            rec = lambda i: evs[i].record(stream)
         rec(0)
         L.gqe_router_topk(d_, x, layer.Wr, layer.bias, idx, wt, None)
         rec(1)
@@ -379,7 +384,7 @@ def main():
         rec(6)
         return y
 
-    launches_per_step = 9   # router, 3 permutation kernels, routed GEMM, K/V GEMM, attention, combine, Wo GEMM
+    launches_per_step = 8   # router, 2 permutation kernels, routed GEMM, K/V GEMM, attention, combine, Wo GEMM
 
     for _ in range(args.warmup):
         step()
@@ -387,7 +392,9 @@ def main():
     torch.cuda.synchronize()
     assert gq.gqe_device_error() == 0
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    # timed steps: one event pair around each whole step (events between the
+    # calls would stop each kernel from launching while its predecessor drains)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier(dist, device)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
@@ -399,9 +406,17 @@ def main():
             step(events[s])
         torch.cuda.synchronize()
     barrier(dist, device)
-    seg_ms = np.array([[events[s][i].elapsed_time(events[s][i + 1]) for i in range(6)] for s in range(args.steps)])
-    step_ms = seg_ms.sum(axis=1)
+    step_ms = np.array([events[s][0].elapsed_time(events[s][1]) for s in range(args.steps)])
     local_total_ms = float(step_ms.sum())
+    # per-call split, from separate steps with an event between every call
+    n_seg = min(args.steps, 10)
+    seg_events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(n_seg)]
+    for s in range(n_seg):
+        flush.zero_()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
+        step(seg_events[s])
+    torch.cuda.synchronize()
+    seg_ms = np.array([[seg_events[s][i].elapsed_time(seg_events[s][i + 1]) for i in range(6)] for s in range(n_seg)])
     total_ms = max_over_ranks(local_total_ms, dist, device)
     tokens = world * dims.N * args.steps
     value = tokens / (total_ms / 1e3)
@@ -499,6 +514,8 @@ def main():
                        "G": dims.G, "E": dims.E, "k": dims.k, "d_head": dims.d, "n_shared": dims.n_shared,
                        "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MB write)"},
             "segments_ms": {n: float(seg_ms[:, i].mean()) for i, n in enumerate(seg_names)},
+            "segments_note": "per-call CUDA events in separate L2-flushed steps; their sum exceeds "
+                             "ms_per_step by the overlap of each kernel's launch with its predecessor",
             "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "decode": decode,
             "clocks": clocks.summary(), "gpu_launches": launches_per_step * args.steps,
             "device_error": err_code,

@@ -57,6 +57,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_const
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rr = tid >> 1, half = tid & 1;
+  pdl_launch_dependents();
+  pdl_wait();
   const int len = p.cache_len[b];
   const int start = c * p.chunk;
   const int end = min(start + p.chunk, len);
@@ -241,6 +243,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_const
 
 template <int D>
 __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int bg = blockIdx.x;
   const int b = bg / p.G, g = bg % p.G;
   const int nq = p.k + ((p.n_shared && g == p.sg) ? 1 : 0);
@@ -291,11 +295,9 @@ static cudaError_t launch_dec(const CUtensorMap& mK, const CUtensorMap& mV, cons
   auto kern = decode_split_kernel<D>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(p.n_chunks, p.G, p.B), kThreads, smem, stream>>>(mK, mV, p);
-  e = cudaGetLastError();
+  e = launch_kernel(kern, dim3(p.n_chunks, p.G, p.B), dim3(kThreads), smem, stream, 1, mK, mV, p);
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<D><<<p.B * p.G, 128, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(decode_merge_kernel<D>, dim3(p.B * p.G), dim3(128), 0, stream, 1, p);
 }
 
 cudaError_t launch_attn_decode_maps(const CUtensorMap& mK, const CUtensorMap& mV, const DecodeParams& p,

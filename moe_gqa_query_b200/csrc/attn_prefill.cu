@@ -175,6 +175,8 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == 8) {
     if (lane == 0) {
@@ -476,6 +478,8 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == 4) {
     if (lane == 0) {
@@ -697,8 +701,7 @@ static cudaError_t launch_d(const CUtensorMap& mQ, const CUtensorMap& mQs, const
   if (e != cudaSuccess) return e;
   const int n_levels = (p.T + 2 * kTile - 1) / (2 * kTile);
   const int per_level = p.B * p.G * p.k + p.B * p.n_shared;
-  kern<<<n_levels * per_level, kThreads, smem, stream>>>(mQ, mQs, mK, mV, p);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(n_levels * per_level), dim3(kThreads), smem, stream, 1, mQ, mQs, mK, mV, p);
 }
 
 static cudaError_t launch_single(const CUtensorMap& mQ, const CUtensorMap& mQs, const CUtensorMap& mK,
@@ -708,8 +711,7 @@ static cudaError_t launch_single(const CUtensorMap& mQ, const CUtensorMap& mQs, 
   if (e != cudaSuccess) return e;
   const int n_levels = (p.T + kTile - 1) / kTile;
   const int per_level = p.B * p.G * p.k + p.B * p.n_shared;
-  kern<<<n_levels * per_level, 192, kSingleSmem, stream>>>(mQ, mQs, mK, mV, p);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(n_levels * per_level), dim3(192), kSingleSmem, stream, 1, mQ, mQs, mK, mV, p);
 }
 
 cudaError_t launch_attn_prefill(const CUtensorMap& mQ, const CUtensorMap& mQs, const CUtensorMap& mK,

@@ -9,6 +9,7 @@
 // warp moves 32/(d/8) slot rows per pass.  The weighted sum accumulates in
 // fp32 per lane, is reduced across the lane groups with shuffles, and is
 // rounded to bf16 once.
+#include "launch.cuh"
 #include "route.cuh"
 
 namespace gqe {
@@ -22,7 +23,9 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
   const int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.B * p.T;
+  pdl_launch_dependents();
   if (n >= N) return;
+  pdl_wait();
   const int b = n / p.T, t = n % p.T;
   const int GK = p.G * p.k;
   const int slots = GK + 1 + p.n_shared;
@@ -72,9 +75,8 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   const int N = p.B * p.T;
   const int grid = (N * 32 + 255) / 256;
-  if (p.d == 64) combine_kernel<64><<<grid, 256, 0, stream>>>(p);
-  else combine_kernel<128><<<grid, 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  if (p.d == 64) return launch_kernel(combine_kernel<64>, dim3(grid), dim3(256), 0, stream, 1, p);
+  return launch_kernel(combine_kernel<128>, dim3(grid), dim3(256), 0, stream, 1, p);
 }
 
 }  // namespace gqe

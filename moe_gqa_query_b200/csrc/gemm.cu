@@ -177,6 +177,8 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -261,15 +263,14 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
 // 16 + 32 KB for the same MMA work: a third fewer bytes through L2 per FLOP.
 // Both CTAs' loads count on the even CTA's `full` barrier; the even CTA's MMA
 // thread releases stages and accumulators in both CTAs with one commit each.
-template <int STAGES>
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
 gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                        const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapO0,
                        const __grid_constant__ CUtensorMap mapO1, EpiParams ep, int M, int K, int n_tiles_b0,
                        int n_tiles_total) {
-  constexpr int BN = 256;
   constexpr int kPM = 2 * kBM;                       // pair tile rows
-  constexpr int kHalfB = (BN / 2) * kBK * 2;         // 16 KB
+  constexpr int kHalfB = (BN / 2) * kBK * 2;         // this CTA's half of the W k-block
   constexpr uint32_t kTmemCols = 2 * BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -307,6 +308,8 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -448,6 +451,8 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = rp.K;
   const int nk = K / kBK;
+  pdl_launch_dependents();
+  pdl_wait();
   for (int i = threadIdx.x; i <= rp.n_seg; i += blockDim.x) {
     seg->tile_start[i] = rp.tile_start[i];
     if (i < rp.n_seg) {
@@ -596,16 +601,16 @@ static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& m
   if (e != cudaSuccess) return e;
   const int tiles = ((M + kBM - 1) / kBM) * n_tiles_total;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  kern<<<grid, 192, smem, stream>>>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(grid), dim3(192), smem, stream, 1, mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K,
+                       n_tiles_b0, n_tiles_total);
 }
 
-template <int STAGES>
+template <int BN, int STAGES>
 static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                                         const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M, int K, int n_tiles_b0, int n_tiles_total,
                                         cudaStream_t stream) {
-  const size_t smem = 1024 + STAGES * (kATileBytes + 128 * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
-  auto kern = gemm_dense_pair_kernel<STAGES>;
+  const size_t smem = 1024 + STAGES * (kATileBytes + (BN / 2) * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
+  auto kern = gemm_dense_pair_kernel<BN, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
@@ -620,7 +625,7 @@ static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorM
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // co-resident pairs on this device (a cluster needs both SMs in one GPC)
-  static int max_pairs[64] = {0};
+  static int max_pairs[64] = {0};   // per instantiation (static in the template)
   int dev = 0;
   cudaGetDevice(&dev);
   int& mp = max_pairs[dev & 63];
@@ -635,14 +640,16 @@ static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorM
   }
   const int total = ((M + 255) / 256) * n_tiles_total;
   const int pairs = total < mp ? total : mp;
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  return cudaLaunchKernelEx(&cfg, kern, mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total);
+  return launch_kernel(kern, dim3(2 * pairs), dim3(192), smem, stream, 2, mapA, mapB0, mapB1, mapO0, mapO1, ep, M,
+                       K, n_tiles_b0, n_tiles_total);
 }
 
 cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                                    const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M,
-                                   int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream) {
-  return launch_dense_pair_st<6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
+                                   int K, int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream) {
+  if (bn != 256) return cudaErrorInvalidValue;
+  return launch_dense_pair_st<256, 6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total,
+                                      stream);
 }
 
 int dense_tile_n(int n_per_weight) { return (n_per_weight % 256 == 0) ? 256 : 128; }
@@ -665,8 +672,7 @@ static cudaError_t launch_routed_bn(const CUtensorMap& mapWq, const CUtensorMap&
   if (e != cudaSuccess) return e;
   const int max_tiles = rp.max_routed_tiles + rp.shared_tiles;
   const int grid = max_tiles < num_sms() ? max_tiles : num_sms();
-  kern<<<grid, 320, smem, stream>>>(mapWq, mapWsh, x, rp, epr, eps);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(grid), dim3(320), smem, stream, 1, mapWq, mapWsh, x, rp, epr, eps);
 }
 
 cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh, const gqe_bf16_t* x,

@@ -57,12 +57,12 @@ cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
                               const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
                               int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream);
 
-// 256 x 256 tiles over CTA pairs; W maps with 128-row boxes, weights' rows a
-// multiple of 256.
+// 256 x 256 tiles over CTA pairs (bn must be 256); W maps with 128-row boxes,
+// weights' rows a multiple of 256.
 cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapB0,
                                    const CUtensorMap& mapB1, const CUtensorMap& mapO0,
                                    const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
-                                   int n_tiles_b0, int n_tiles_total, cudaStream_t stream);
+                                   int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream);
 
 cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh,
                                const gqe_bf16_t* x, const RoutedParams& rp, const EpiParams& epr,

@@ -302,21 +302,26 @@ gqe_status gqe_routed_qproj(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
 }
 
 // CTA-pair GEMM (256 x 256 tiles) when the weights tile by 256 and there are
-// enough rows to fill the pairs; single-CTA 128-row tiles otherwise.
+// enough rows to fill the pairs; single-CTA 128-row tiles otherwise.  (256 x
+// 128 pair tiles fill the last wave better on 64 x 16 x 1024 shapes but ran
+// 1.4x slower on B200: the k-block pipeline, not the tile count, bounds them.)
+// Returns the pair tile width, 0 for the single-CTA kernel.
 #ifndef GQE_GEMM_PAIR
 #define GQE_GEMM_PAIR 1
 #endif
-static bool use_pair_gemm(int M, int bn) { return GQE_GEMM_PAIR && bn == 256 && M >= 2048; }
+static int pair_tile_n(int M, int n_per_weight) {
+  return (GQE_GEMM_PAIR && M >= 2048 && n_per_weight % 256 == 0) ? 256 : 0;
+}
 
 static gqe_status kv_common(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wk, const gqe_bf16* Wv,
                             EpiParams& ep, int M, gqe_stream stream) {
   const int G = dims->G, d = dims->d_head, D = dims->d_model;
-  const int bn = dense_tile_n(G * d);
-  const bool pair = use_pair_gemm(M, bn);
+  const int pbn = pair_tile_n(M, G * d);
+  const int bn = pbn ? pbn : dense_tile_n(G * d);
   CUtensorMap mA, mK, mV;
   GQE_REQUIRE(map2d(&mA, x, D, M, 128), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mK, Wk, D, (uint64_t)G * d, pair ? 128 : bn), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mV, Wv, D, (uint64_t)G * d, pair ? 128 : bn), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mK, Wk, D, (uint64_t)G * d, pbn ? pbn / 2 : bn), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mV, Wv, D, (uint64_t)G * d, pbn ? pbn / 2 : bn), GQE_ERR_CUDA);
   ep.n_limit = G * d;
   ep.G = G;
   ep.d = d;
@@ -330,7 +335,7 @@ static gqe_status kv_common(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
     ep.store_mode = kStoreTmaHeads;
   }
   const int nt = (G * d + bn - 1) / bn;
-  if (pair) return cuda_status(launch_gemm_dense_pair(mA, mK, mV, mOK, mOV, ep, M, D, nt, 2 * nt, S(stream)));
+  if (pbn) return cuda_status(launch_gemm_dense_pair(mA, mK, mV, mOK, mOV, ep, M, D, nt, 2 * nt, pbn, S(stream)));
   return cuda_status(launch_gemm_dense(mA, mK, mV, mOK, mOV, ep, M, D, nt, 2 * nt, bn, S(stream)));
 }
 
@@ -457,11 +462,11 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   GQE_REQUIRE(K % 64 == 0 && N % 64 == 0, GQE_ERR_UNSUPPORTED);
   GQE_REQUIRE((long long)M * N < (1ll << 31) && (long long)M * K < (1ll << 31), GQE_ERR_UNSUPPORTED);
   GQE_REQUIRE(aligned16(A) && aligned16(W) && aligned16(C), GQE_ERR_INVALID_ARG);
-  const int bn = dense_tile_n(N);
-  const bool pair = use_pair_gemm(M, bn);
+  const int pbn = pair_tile_n(M, N);
+  const int bn = pbn ? pbn : dense_tile_n(N);
   CUtensorMap mA, mW;
   GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
-  GQE_REQUIRE(map2d(&mW, W, K, N, pair ? 128 : bn), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mW, W, K, N, pbn ? pbn / 2 : bn), GQE_ERR_CUDA);
   EpiParams ep{};
   ep.out0 = C;
   ep.out1 = C;
@@ -473,7 +478,7 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   GQE_REQUIRE(map2d(&mO, C, N, M, 32), GQE_ERR_CUDA);
   ep.store_mode = kStoreTma2d;
   const int nt = (N + bn - 1) / bn;
-  if (pair) return cuda_status(launch_gemm_dense_pair(mA, mW, mW, mO, mO, ep, M, K, nt, nt, S(stream)));
+  if (pbn) return cuda_status(launch_gemm_dense_pair(mA, mW, mW, mO, mO, ep, M, K, nt, nt, pbn, S(stream)));
   return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, K, nt, nt, bn, S(stream)));
 }
 

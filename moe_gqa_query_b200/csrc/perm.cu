@@ -19,6 +19,7 @@
 //            and writes (source token row, destination row of
 //            q_routed [B, G, T, k]).  Block 0 also writes the segment counts,
 //            offsets and 128-row tile offsets the GEMM reads.
+#include "launch.cuh"
 #include "route.cuh"
 
 namespace gqe {
@@ -56,6 +57,8 @@ __global__ void __launch_bounds__(kThreads) perm_count_kernel(const int* __restr
   const int nseg = G * E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = blockIdx.x * kThreads + threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   const unsigned long long bits = token_segments(idx, n, N, G, E, k);
   for (int s = 0; s < nseg; ++s) {
     const unsigned m = __ballot_sync(0xffffffffu, (bits >> s) & 1ull);
@@ -81,6 +84,8 @@ __global__ void __launch_bounds__(kThreads) perm_scatter_kernel(const int* __res
   const int nseg = G * E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = blockIdx.x * kThreads + threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   const unsigned long long bits = token_segments(idx, n, N, G, E, k);
 
   // ---- preceding blocks and totals: 4 threads per segment share the block loop
@@ -184,11 +189,12 @@ cudaError_t launch_permutation(const int* topk_idx, int N, int T, int G, int E, 
   int* tile_start = reinterpret_cast<int*>(w + L.off_tile_start);
   int* src_row = reinterpret_cast<int*>(w + L.off_src_row);
   int* dst_row = reinterpret_cast<int*>(w + L.off_dst_row);
-  perm_count_kernel<<<L.n_blocks, kThreads, 0, stream>>>(topk_idx, N, G, E, k, block_counts);
-  perm_scatter_kernel<<<L.n_blocks, kThreads, 0, stream>>>(topk_idx, N, T, G, E, k, L.n_blocks, block_counts,
-                                                           seg_cnt, seg_off, tile_start, expert_counts, src_row,
-                                                           dst_row);
-  return cudaGetLastError();
+  cudaError_t e = launch_kernel(perm_count_kernel, dim3(L.n_blocks), dim3(kThreads), 0, stream, 1, topk_idx, N, G,
+                                E, k, block_counts);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(perm_scatter_kernel, dim3(L.n_blocks), dim3(kThreads), 0, stream, 1, topk_idx, N, T, G, E, k,
+                       L.n_blocks, static_cast<const int*>(block_counts), seg_cnt, seg_off, tile_start,
+                       expert_counts, src_row, dst_row);
 }
 
 }  // namespace gqe

@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(128) router_kernel(RouterParams p) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tok0 = blockIdx.x * kTok;
+  pdl_launch_dependents();
+  pdl_wait();
   const int GE = p.G * p.E;
   const int nkc = p.D / kKC;
   // warp w: token rows (w & 1) * 16 .. +15, reduction half (w >> 1) of every chunk
@@ -269,6 +271,8 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) router_resident_kernel(R
   const int n_tiles = (p.N + kWarpTok - 1) / kWarpTok;
   uint8_t* ring = xring + (size_t)warp * STAGES * kStageBytes;
   float* lg = lgw + (size_t)warp * kWarpTok * (GEP + 1);
+  pdl_launch_dependents();
+  pdl_wait();
 
   // Wr into shared memory once (padded columns zero)
   if ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0) {
@@ -410,11 +414,9 @@ cudaError_t launch_router_gep(const RouterParams& p, cudaStream_t stream) {
     int grid = router_num_sms();
     const int need = (n_tiles + kRouterWarps - 1) / kRouterWarps;
     if (grid > need) grid = need;
-    kern<<<grid, kRouterWarps * 32, smem, stream>>>(p);
-  } else {
-    router_kernel<GEP><<<(p.N + kTok - 1) / kTok, 128, 0, stream>>>(p);
+    return launch_kernel(kern, dim3(grid), dim3(kRouterWarps * 32), smem, stream, 1, p);
   }
-  return cudaGetLastError();
+  return launch_kernel(router_kernel<GEP>, dim3((p.N + kTok - 1) / kTok), dim3(128), 0, stream, 1, p);
 }
 
 }  // namespace

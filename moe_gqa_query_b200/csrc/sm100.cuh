@@ -35,6 +35,15 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
+// ---------------------------------------------------------------- dependent launch
+// Wait until the kernels this one depends on (the previous kernel on the
+// stream) have completed and their memory is visible; no-op without a
+// programmatic dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream begin launching (its CTAs then wait in
+// pdl_wait before touching this kernel's data).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
