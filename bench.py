@@ -433,24 +433,27 @@ def main():
                 "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_ms}
 
     # ---------------- end to end through host buffers (pinned), on the same step
+    # each step copies its input batch in and its output batch out; the copies
+    # of neighbouring steps overlap each other and the compute (three streams)
     e2e = None
     x_pin = x_host.pin_memory()
-    y_pin = torch.empty((dims.B, dims.T, dims.D), dtype=torch.bfloat16).pin_memory()
-    for _ in range(2):
-        layer.forward_host(x_pin, y_pin)
+    y_pins = [torch.empty((dims.B, dims.T, dims.D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    n_e2e = max(3, min(args.steps, 20))
+    xs_h = [x_pin] * n_e2e
+    ys_h = [y_pins[i & 1] for i in range(n_e2e)]
+    layer.forward_host_pipelined(xs_h[:4], ys_h[:4])     # warm-up: graphs captured, streams created
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = max(3, min(args.steps, 20))
     barrier(dist, device)
+    torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(n_e2e):
-        layer.forward_host(x_pin, y_pin)
+    layer.forward_host_pipelined(xs_h, ys_h)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     e2e = {"value": world * dims.N * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s",
-           "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(y_pin.numel() * 2),
-           "steps": n_e2e}
+           "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(y_pins[0].numel() * 2),
+           "steps": n_e2e, "api": "GQELayer.forward_host_pipelined (pinned host batches, graph replay)"}
 
     # ---------------- decode sub-measurement (64 sequences x 32768-entry cache)
     decode = None

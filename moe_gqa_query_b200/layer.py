@@ -85,8 +85,8 @@ class GQELayer:
         return self._buf(name, ((max(nbytes, 16) + 255) // 256 * 256,), torch.uint8)
 
     # ------------------------------------------------------------------ prefill
-    def forward(self, x: torch.Tensor, stream=None, keep=False) -> torch.Tensor:
-        """x [B, T, D] bf16 on the device -> y [B, T, D] bf16.
+    def forward(self, x: torch.Tensor, stream=None, keep=False, out=None) -> torch.Tensor:
+        """x [B, T, D] bf16 on the device -> y [B, T, D] bf16 (into `out` when given).
 
         keep=True also returns the intermediates (router outputs, q, K, V, o, h).
         """
@@ -103,7 +103,7 @@ class GQELayer:
         o = self._buf("o", (B, c.G, T, c.k, c.d))
         os_ = self._buf("os", (B, T, c.d)) if c.n_shared else None
         h = self._buf("h", (N, c.slots * c.d))
-        y = self._buf("y", (B, T, c.D))
+        y = self._buf("y", (B, T, c.D)) if out is None else out
         ws = self._ws("ws_q", L.gqe_workspace_size(dims, L.GQE_OP_ROUTED_QPROJ))
         L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, None, stream)
         L.gqe_routed_qproj(dims, x, self.Wq, self.Wsh, idx, q, qs, ws, None, stream)
@@ -115,19 +115,19 @@ class GQELayer:
             return y, dict(idx=idx, w=w, q=q, q_sh=qs, K=K, V=V, o=o, o_sh=os_, h=h)
         return y
 
-    def forward_graph(self, x: torch.Tensor) -> torch.Tensor:
+    def forward_graph(self, x: torch.Tensor, out=None) -> torch.Tensor:
         """forward() replayed from a CUDA graph captured on first use for this
-        input buffer and shape (the six library calls become one graph launch).
-        The returned tensor is the layer's own output buffer, overwritten by the
-        next call."""
-        key = (x.data_ptr(), tuple(x.shape))
+        input buffer, output buffer and shape (the six library calls become one
+        graph launch), on the current stream.  Without `out` the returned tensor
+        is the layer's own output buffer, overwritten by the next call."""
+        key = (x.data_ptr(), tuple(x.shape), None if out is None else out.data_ptr())
         entry = self._graphs.get(key)
         if entry is None:
-            self.forward(x)                       # eager first: buffers, kernel attributes
+            self.forward(x, out=out)              # eager first: buffers, kernel attributes
             torch.cuda.synchronize(self.device)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                y = self.forward(x)
+                y = self.forward(x, out=out)
             entry = self._graphs[key] = (g, y)
         g, y = entry
         g.replay()
@@ -142,6 +142,55 @@ class GQELayer:
         y = self.forward_graph(xd) if graph else self.forward(xd)
         y_host.copy_(y, non_blocking=True)
         return y_host
+
+    def forward_host_pipelined(self, x_hosts, y_hosts):
+        """End to end over a sequence of batches in (pinned) host memory:
+        y_hosts[i] <- forward(x_hosts[i]).  The host->device copy of batch i,
+        the forward of batch i-1 and the read-back of batch i-2 run at once on
+        three streams over two device buffer sets, so the copies in the two
+        directions overlap each other and the compute.  Everything is enqueued;
+        the current stream waits for the last read-back, so synchronising it
+        (or an event recorded on it) means every y_hosts[i] is written."""
+        if len(x_hosts) != len(y_hosts):
+            raise ValueError("x_hosts and y_hosts differ in length")
+        if not x_hosts:
+            return y_hosts
+        cur = torch.cuda.current_stream(self.device)
+        if getattr(self, "_pipe_streams", None) is None:
+            self._pipe_streams = tuple(torch.cuda.Stream(self.device) for _ in range(3))
+        s_in, s_cmp, s_out = self._pipe_streams
+        B, T = x_hosts[0].shape[0], x_hosts[0].shape[1]
+        xs = [self._buf(f"pipe_x{j}", (B, T, self.cfg.D)) for j in range(2)]
+        ys = [self._buf(f"pipe_y{j}", (B, T, self.cfg.D)) for j in range(2)]
+        start = torch.cuda.Event()
+        start.record(cur)
+        for s_ in (s_in, s_cmp, s_out):
+            s_.wait_event(start)
+        done_cmp = [None, None]   # forward of the slot's last batch finished (x slot free)
+        done_out = [None, None]   # read-back of the slot's last batch finished (y slot free)
+        for i, (xh, yh) in enumerate(zip(x_hosts, y_hosts)):
+            j = i & 1
+            with torch.cuda.stream(s_in):
+                if done_cmp[j] is not None:
+                    s_in.wait_event(done_cmp[j])
+                xs[j].copy_(xh, non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ready)
+                if done_out[j] is not None:
+                    s_cmp.wait_event(done_out[j])
+                self.forward_graph(xs[j], out=ys[j])
+                done_cmp[j] = torch.cuda.Event()
+                done_cmp[j].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done_cmp[j])
+                yh.copy_(ys[j], non_blocking=True)
+                done_out[j] = torch.cuda.Event()
+                done_out[j].record(s_out)
+        for s_ in (s_in, s_cmp, s_out):
+            cur.wait_stream(s_)
+        return y_hosts
 
     # ------------------------------------------------------------------ decode
     def decode_step(self, x_new: torch.Tensor, Kc: torch.Tensor, Vc: torch.Tensor,

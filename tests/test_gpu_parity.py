@@ -429,3 +429,19 @@ def test_layer_graph_replay_matches_eager():
     layer.forward_host(x_pin, y_pin)
     torch.cuda.synchronize()
     assert torch.equal(y_pin, y_eager.cpu())
+
+
+def test_layer_host_pipeline_matches_eager():
+    """Five batches through the three-stream host pipeline: each output equals
+    the eager forward of its own input (no slot reuse races)."""
+    w = gi.WORKLOADS["tiny_prefill"]
+    dims, x, Wt, bias, layer = _layer(w, seed=4)
+    xs = [gi.layer_input(dims, seed=10 + i) for i in range(5)]
+    x_pins = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in xs]
+    y_pins = [torch.full((dims.B, dims.T, dims.D), float("nan"), dtype=torch.bfloat16).pin_memory() for _ in xs]
+    layer.forward_host_pipelined(x_pins, y_pins)
+    torch.cuda.synchronize()
+    for a, yp in zip(xs, y_pins):
+        y_ref = layer.forward(bf16_dev(a)).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(yp, y_ref.cpu())
