@@ -433,8 +433,8 @@ __device__ __forceinline__ RoutedTile routed_tile(const RoutedParams& rp, const 
   return r;
 }
 
-template <int BN, int STAGES>
-__global__ void __launch_bounds__(320, 1)
+template <int BN, int STAGES, int CPS>
+__global__ void __launch_bounds__(320, CPS)
 gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_constant__ CUtensorMap mapWsh,
                    const gqe_bf16_t* __restrict__ x, RoutedParams rp, EpiParams ep_routed, EpiParams ep_shared) {
   constexpr int kBTileBytes = BN * kBK * 2;
@@ -662,26 +662,42 @@ cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
   return launch_dense_bn<128, 6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int CPS>
 static cudaError_t launch_routed_bn(const CUtensorMap& mapWq, const CUtensorMap& mapWsh, const gqe_bf16_t* x,
                                     const RoutedParams& rp, const EpiParams& epr, const EpiParams& eps,
                                     cudaStream_t stream) {
   const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + sizeof(GemmBarriers) + sizeof(SegTables);
-  auto kern = gemm_routed_kernel<BN, STAGES>;
+  auto kern = gemm_routed_kernel<BN, STAGES, CPS>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int max_tiles = rp.max_routed_tiles + rp.shared_tiles;
-  const int grid = max_tiles < num_sms() ? max_tiles : num_sms();
+  const int slots = CPS * num_sms();
+  const int grid = max_tiles < slots ? max_tiles : slots;
   return launch_kernel(kern, dim3(grid), dim3(320), smem, stream, 1, mapWq, mapWsh, x, rp, epr, eps);
 }
+
+// Ring depth and CTAs per SM of the routed GEMM.  A tcgen05.mma of N = 64 or
+// 128 keeps the tensor pipe busy for less time than one issuing thread needs
+// per instruction (about 100 cycles), so two CTAs per SM, each with its own
+// MMA thread, feed the pipe where one cannot.
+#ifndef GQE_ROUTED64_ST
+#define GQE_ROUTED64_ST 4
+#endif
+#ifndef GQE_ROUTED64_CPS
+#define GQE_ROUTED64_CPS 2
+#endif
+#ifndef GQE_ROUTED128_ST
+#define GQE_ROUTED128_ST 3
+#endif
+#ifndef GQE_ROUTED128_CPS
+#define GQE_ROUTED128_CPS 2
+#endif
 
 cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh, const gqe_bf16_t* x,
                                const RoutedParams& rp, const EpiParams& epr, const EpiParams& eps,
                                cudaStream_t stream) {
-  // deep rings: the gathered rows come from L2/HBM at 128 bytes per row, so
-  // many k-blocks stay in flight per gather thread
-  if (rp.d == 64) return launch_routed_bn<64, 8>(mapWq, mapWsh, x, rp, epr, eps, stream);
-  return launch_routed_bn<128, 6>(mapWq, mapWsh, x, rp, epr, eps, stream);
+  if (rp.d == 64) return launch_routed_bn<64, GQE_ROUTED64_ST, GQE_ROUTED64_CPS>(mapWq, mapWsh, x, rp, epr, eps, stream);
+  return launch_routed_bn<128, GQE_ROUTED128_ST, GQE_ROUTED128_CPS>(mapWq, mapWsh, x, rp, epr, eps, stream);
 }
 
 }  // namespace gqe
