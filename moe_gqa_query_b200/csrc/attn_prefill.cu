@@ -483,29 +483,23 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
 
   if (warp == 4) {
     if (lane == 0) {
-      // ---------------- producer: Q once, then K_0, V_0, K_1, V_1, ...
+      // ---------------- K side: Q and K tiles by TMA, S(j) = Q K_j^T.  S(j+1)
+      // is issued as soon as the softmax holds S(j) in registers (s_free), so
+      // it runs while the exponentials of tile j do.
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       mbar_arrive_expect_tx(&bar->q_full, kBox);
       tma_load_3d(sQ, mq, &bar->q_full, 0, ti.row0, seq);
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % ST;
-        const uint32_t ph = ((j / ST) & 1) ^ 1;
-        if (j >= ST && !mbar_wait(&bar->k_empty[s], ph, abort, p.err, kErrTimeoutAttn)) break;
-        mbar_arrive_expect_tx(&bar->k_full[s], kBox);
-        tma_load_3d(sK + s * kBox, &mapK, &bar->k_full[s], 0, j * kTile, kvseq);
-        if (j >= ST && !mbar_wait(&bar->v_empty[s], ph, abort, p.err, kErrTimeoutAttn)) break;
-        mbar_arrive_expect_tx(&bar->v_full[s], kBox);
-        tma_load_3d(sV + s * kBox, &mapV, &bar->v_full[s], 0, j * kTile, kvseq);
+      for (int j = 0; j < ST && j < n_kv; ++j) {
+        mbar_arrive_expect_tx(&bar->k_full[j], kBox);
+        tma_load_3d(sK + j * kBox, &mapK, &bar->k_full[j], 0, j * kTile, kvseq);
       }
-    }
-  } else if (warp == 5) {
-    if (lane == 0) {
-      // ---------------- MMA issuer: S_0 | S_1 PV_0 | S_2 PV_1 | ...
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kTile, D, false, true);
       const uint32_t q0 = smem_u32(sQ);
-      auto issue_s = [&](int j) {
+      bool ok = mbar_wait(&bar->q_full, 0, abort, p.err, kErrTimeoutAttn);
+      for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % ST;
-        if (!mbar_wait(&bar->k_full[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn)) return false;
+        if (j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, abort, p.err, kErrTimeoutAttn);
+        ok = ok && mbar_wait(&bar->k_full[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn);
+        if (!ok) break;
         tc_fence_after();
         const uint32_t k0 = smem_u32(sK + s * kBox);
 #pragma unroll
@@ -514,19 +508,29 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
                   ks > 0);
         umma_commit(&bar->s_full);
         umma_commit(&bar->k_empty[s]);
-        return true;
-      };
-      bool ok = mbar_wait(&bar->q_full, 0, abort, p.err, kErrTimeoutAttn) && issue_s(0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv) {
-          // S(j) is in the softmax registers: overwrite its columns with S(j+1)
-          ok = mbar_wait(&bar->s_free, j & 1, abort, p.err, kErrTimeoutAttn);
-          tc_fence_after();
-          if (!ok || !issue_s(j + 1)) break;
+        if (j + ST < n_kv) {
+          // refill this stage with K_{j+ST} once S(j) has read it
+          ok = mbar_wait(&bar->k_empty[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar->k_full[s], kBox);
+          tma_load_3d(sK + s * kBox, &mapK, &bar->k_full[s], 0, (j + ST) * kTile, kvseq);
         }
-        ok = mbar_wait(&bar->p_full, j & 1, abort, p.err, kErrTimeoutAttn);
-        tc_fence_after();
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------- V side: V tiles by TMA, O += P(j) V_j once P(j) is in
+      // tensor memory (a second issuing thread: an MMA of N = 64 takes the
+      // tensor pipe for less time than one thread needs to issue it)
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kTile, D, false, true);
+      for (int j = 0; j < ST && j < n_kv; ++j) {
+        mbar_arrive_expect_tx(&bar->v_full[j], kBox);
+        tma_load_3d(sV + j * kBox, &mapV, &bar->v_full[j], 0, j * kTile, kvseq);
+      }
+      bool ok = true;
+      for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % ST;
+        ok = mbar_wait(&bar->p_full, j & 1, abort, p.err, kErrTimeoutAttn);
         ok = ok && mbar_wait(&bar->v_full[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn);
         if (!ok) break;
         tc_fence_after();
@@ -537,6 +541,12 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
                   (j > 0 || ks > 0));
         umma_commit(&bar->pv_done);
         umma_commit(&bar->v_empty[s]);
+        if (j + ST < n_kv) {
+          ok = mbar_wait(&bar->v_empty[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar->v_full[s], kBox);
+          tma_load_3d(sV + s * kBox, &mapV, &bar->v_full[s], 0, (j + ST) * kTile, kvseq);
+        }
       }
     }
   } else {
