@@ -21,6 +21,7 @@ path has no exchange step), and reports the aggregate.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -43,6 +44,23 @@ METRIC = "GQE prefill tokens/s per layer"
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 L2_FLUSH_BYTES = 256 << 20
 HOST_LEAD_CYCLES = 600_000      # ~0.3 ms at B200 clocks: longer than the host needs to enqueue a step
+
+
+def profiled_traffic(kernel_label):
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
+    or None when there is none or the kernel's source changed since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f).get(kernel_label)
+        if not entry:
+            return None
+        with open(os.path.join(ROOT, entry["source"]), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+        if digest != entry["source_sha256_16"]:
+            return None
+        return int(entry["dram_read_bytes"]) + int(entry["dram_write_bytes"])
+    except (OSError, ValueError, KeyError):
+        return None
 
 
 def load_peaks():
@@ -429,7 +447,7 @@ def main():
     attn_kernel = "attn_prefill_single_kernel (d=64)" if dims.d == 64 else f"attn_prefill_kernel<{dims.d}>"
     roofline = {"bound": "tensor", "kernel": attn_kernel, "achieved": achieved_tf,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
-                "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": profiled_traffic(attn_kernel),
                 "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_ms}
 
     # ---------------- end to end through host buffers (pinned), on the same step
