@@ -253,6 +253,14 @@ gqe_status gqe_router_topk(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf
   p.E = dims->E;
   p.k = dims->k;
   p.scope = dims->renorm_scope;
+  p.err = error_word();
+  // tcgen05 router with TMA-streamed x for prefill-sized batches
+  if (p.N >= 1024 && p.D % 64 == 0) {
+    CUtensorMap mX;
+    GQE_REQUIRE(map2d(&mX, x, p.D, p.N, 128), GQE_ERR_CUDA);
+    const cudaError_t e = launch_router_tc(mX, p, S(stream));
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+  }
   return cuda_status(launch_router(p, S(stream)));
 }
 

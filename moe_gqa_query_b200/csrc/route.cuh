@@ -14,8 +14,12 @@ struct RouterParams {
   float* topk_w;          // [N, G, k]
   float* probs;           // [N, G, E] or null
   int N, D, G, E, k, scope;
+  unsigned* err;          // device error word (bounded waits of the tcgen05 router)
 };
 cudaError_t launch_router(const RouterParams& p, cudaStream_t stream);
+// tcgen05 router streaming x by TMA (map over x [N, D], box 64 x 128); returns
+// cudaErrorNotSupported for shapes it does not take (the caller falls back).
+cudaError_t launch_router_tc(const CUtensorMap& mapX, const RouterParams& p, cudaStream_t stream);
 
 // Token-to-expert permutation workspace (int32 arrays, see perm.cu).
 struct PermLayout {

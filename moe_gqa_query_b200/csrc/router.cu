@@ -421,6 +421,355 @@ cudaError_t launch_router_gep(const RouterParams& p, cudaStream_t stream) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// tcgen05 router: 128-token x tiles stream in by TMA (128-byte swizzle); Wr^T
+// sits in shared memory for the whole kernel as the MMA's B operand (GEP
+// expert rows, zero-padded, one 128-byte row per 64-column k-block); the
+// logits of a tile accumulate in fp32 in tensor memory (two accumulators, so
+// one tile's routing overlaps the next tile's MMAs), and the epilogue routes
+// one token per thread: per-group softmax and TopK on logit + bias, the
+// renormalised weights of the selected experts.
+//
+// CTA (192 threads): warp 0 TMA producer, warp 1 MMA issuer (and tensor-memory
+// owner), warps 2..5 routing epilogue.
+namespace {
+
+constexpr int kRtBM = 128;
+constexpr int kRtBK = 64;
+constexpr int kRtTile = kRtBM * kRtBK * 2;   // 16 KB x tile
+
+struct __align__(8) RouterTcBarriers {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int GEP>
+__device__ __forceinline__ void route_token(const RouterParams& p, const float* lg, int n) {
+  const int G = p.G, E = p.E, k = p.k;
+  float den_tok = 0.f;
+  if (p.scope == 0) {
+    for (int g = 0; g < G; ++g) {
+      float pr[8], sum;
+      route_group(p, lg, g, pr, &sum);
+      den_tok += sum;
+    }
+  }
+  for (int g = 0; g < G; ++g) {
+    float pr[8], sum;
+    const unsigned chosen = route_group(p, lg, g, pr, &sum);
+    const float inv_den = 1.f / (p.scope == 0 ? den_tok : sum);
+    const size_t o = ((size_t)n * G + g) * k;
+    int j = 0;
+    for (int e = 0; e < E; ++e) {
+      if ((chosen >> e) & 1u) {
+        p.topk_idx[o + j] = e;
+        p.topk_w[o + j] = pr[e] * inv_den;
+        ++j;
+      }
+    }
+    if (p.probs)
+      for (int e = 0; e < E; ++e) p.probs[((size_t)n * G + g) * E + e] = pr[e];
+  }
+}
+
+// One token's routing with the group width E fixed at compile time: every
+// array index is static, the exponentials are ex2.approx on pre-scaled
+// arguments, and each group is evaluated once.
+template <int GEP, int E>
+__device__ __forceinline__ void route_token_e(const RouterParams& p, const float* lg, const float* bias, int n) {
+  constexpr int GM = GEP / E;          // groups that fit the padded width
+  const int G = p.G, k = p.k;
+  float pr[GEP];
+  unsigned chosen[GM];
+  float gsum[GM];
+  float den_tok = 0.f;
+#pragma unroll
+  for (int g = 0; g < GM; ++g) {
+    chosen[g] = 0;
+    gsum[g] = 1.f;
+    if (g < G) {
+      float sv[E];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        sv[e] = lg[g * E + e] + bias[g * E + e];
+        mx = fmaxf(mx, sv[e]);
+      }
+      float Z = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        pr[g * E + e] = ex2((sv[e] - mx) * 1.4426950408889634f);
+        Z += pr[g * E + e];
+      }
+      const float invZ = 1.f / Z;
+#pragma unroll
+      for (int e = 0; e < E; ++e) pr[g * E + e] *= invZ;
+      unsigned ch = 0;
+      for (int it = 0; it < k; ++it) {
+        int best = 0;
+        float bv = -INFINITY;
+        bool found = false;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const bool free_e = !((ch >> e) & 1u);
+          if (free_e && (!found || sv[e] > bv)) {   // strict: ties keep the lower index
+            best = e;
+            bv = sv[e];
+            found = true;
+          }
+        }
+        ch |= 1u << best;
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if ((ch >> e) & 1u) sum += pr[g * E + e];
+      chosen[g] = ch;
+      gsum[g] = sum;
+      den_tok += sum;
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < GM; ++g) {
+    if (g < G) {
+      const float inv_den = 1.f / (p.scope == 0 ? den_tok : gsum[g]);
+      const size_t o = ((size_t)n * G + g) * k;
+      int j = 0;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        if ((chosen[g] >> e) & 1u) {
+          p.topk_idx[o + j] = e;
+          p.topk_w[o + j] = pr[g * E + e] * inv_den;
+          ++j;
+        }
+      }
+      if (p.probs) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) p.probs[((size_t)n * G + g) * E + e] = pr[g * E + e];
+      }
+    }
+  }
+}
+
+// CTA (224 threads): warp 0 TMA producer; warps 1 and 6 issue the MMAs of the
+// even and odd k-blocks into two partial accumulators (an N <= 64 MMA keeps
+// the tensor pipe busy for less time than one thread needs to issue it);
+// warps 2..5 sum the partials and route, one token per thread.
+template <int GEP, int STAGES>
+__global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant__ CUtensorMap mapX, RouterParams p) {
+  constexpr int kWBlk = GEP * 128;                 // one k-block of Wr^T
+  constexpr uint32_t kTmemCols = 4 * GEP;          // 2 buffers x 2 partial accumulators
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nk = p.D / kRtBK;
+  uint8_t* sW = smem;                                        // nk x [GEP rows x 128 B]
+  uint8_t* sX = sW + ((nk * kWBlk + 1023) & ~1023);          // STAGES x 16 KB
+  RouterTcBarriers* bar = reinterpret_cast<RouterTcBarriers*>(sX + STAGES * kRtTile);
+  float* sBias = reinterpret_cast<float*>(bar + 1);          // GEP
+  volatile int* abort = &bar->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int GE = p.G * p.E;
+  const int n_tiles = (p.N + kRtBM - 1) / kRtBM;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bar->full[s], 1);
+      mbar_init(&bar->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bar->acc_full[a], 2);     // one commit from each MMA thread
+      mbar_init(&bar->acc_empty[a], 4);
+    }
+    bar->abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&mapX);
+  }
+  if (warp == 1) tmem_alloc(&bar->tmem_base, kTmemCols);
+  pdl_launch_dependents();
+  pdl_wait();
+  __syncthreads();   // barriers initialised
+  // the first x tiles are requested before Wr^T is built (they do not need it)
+  const int first_tiles = min(STAGES, (blockIdx.x < n_tiles ? ((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0) * nk);
+  if (threadIdx.x == 0) {
+    for (int it = 0; it < first_tiles; ++it) {
+      const int t = blockIdx.x + (it / nk) * gridDim.x, kb = it % nk;
+      mbar_arrive_expect_tx(&bar->full[it], kRtTile);
+      tma_load_2d(sX + it * kRtTile, &mapX, &bar->full[it], kb * kRtBK, t * kRtBM);
+    }
+  }
+  // Wr [D, GE] -> Wr^T in the swizzled K-major layout (rows GE..GEP-1 zero);
+  // 16-byte loads of 8 consecutive experts of one model dimension
+  if ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0) {
+    const int per_row = GE / 8;
+    const int total = p.D * per_row;
+    for (int e0 = threadIdx.x; e0 < total; e0 += 4 * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * blockDim.x;
+        if (e < total)
+          v[u] = __ldg(reinterpret_cast<const uint4*>(p.Wr + (size_t)(e / per_row) * GE + (e % per_row) * 8));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * blockDim.x;
+        if (e >= total) break;
+        const int dd = e / per_row, n0 = (e % per_row) * 8;
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(&v[u]);
+        const int kb = dd >> 6, c = dd & 63;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int n = n0 + i;
+          *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) =
+              h[i];
+        }
+      }
+    }
+    for (int e = threadIdx.x; e < p.D * (GEP - GE); e += blockDim.x) {
+      const int dd = e / (GEP - GE), n = GE + e % (GEP - GE);
+      const int kb = dd >> 6, c = dd & 63;
+      *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) = 0;
+    }
+  } else {
+    for (int e = threadIdx.x; e < p.D * GEP; e += blockDim.x) {
+      const int dd = e / GEP, n = e % GEP;
+      const int kb = dd >> 6, c = dd & 63;
+      const uint16_t v = n < GE ? p.Wr[(size_t)dd * GE + n] : (uint16_t)0;
+      *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) = v;
+    }
+  }
+  for (int e = threadIdx.x; e < GEP; e += blockDim.x) sBias[e] = (p.bias && e < GE) ? p.bias[e] : 0.f;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          if (it < first_tiles) continue;   // requested before Wr^T was built
+          const int s = it % STAGES;
+          if (it >= STAGES &&
+              !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, p.err, kErrTimeoutRouter))
+            break;
+          mbar_arrive_expect_tx(&bar->full[s], kRtTile);
+          tma_load_2d(sX + s * kRtTile, &mapX, &bar->full[s], kb * kRtBK, t * kRtBM);
+        }
+      }
+    }
+  } else if (warp == 1 || warp == 6) {
+    if (lane == 0) {
+      // warp 1: k-blocks 0, 2, 4, ... into partial 0; warp 6: 1, 3, 5, ... into partial 1
+      const int half = warp == 6 ? 1 : 0;
+      constexpr uint32_t idesc = idesc_bf16_f32(kRtBM, GEP, false, false);
+      const uint32_t w0 = smem_u32(sW);
+      int tc = 0;
+      for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tc) {
+        const int ab = tc & 1, use = tc >> 1;
+        if (tc >= 2 && !mbar_wait(&bar->acc_empty[ab], (use & 1) ^ 1, abort, p.err, kErrTimeoutRouter)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)((2 * ab + half) * GEP);
+        bool ok = true;
+        for (int kb = half; kb < nk; kb += 2) {
+          const int it = tc * nk + kb;
+          const int s = it % STAGES;
+          if (!mbar_wait(&bar->full[s], (it / STAGES) & 1, abort, p.err, kErrTimeoutRouter)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sX + s * kRtTile);
+          const uint32_t b0 = w0 + (uint32_t)(kb * kWBlk);
+#pragma unroll
+          for (int kk = 0; kk < kRtBK / 16; ++kk)
+            umma_ss(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
+                    (kb != half) || kk != 0);
+          umma_commit(&bar->empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&bar->acc_full[ab]);
+      }
+    }
+  } else {
+    const int lg = warp & 3;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    int tc = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
+      const int ab = tc & 1, use = tc >> 1;
+      const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, p.err, kErrTimeoutRouter);
+      tc_fence_after();
+      float logit[GEP];
+#pragma unroll
+      for (int c0 = 0; c0 < GEP; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_off + (uint32_t)(2 * ab * GEP + c0), v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) logit[c0 + i] = __uint_as_float(v[i]);
+        if (nk > 1) {   // the odd k-blocks' partial
+          tmem_ld16(tmem + lane_off + (uint32_t)((2 * ab + 1) * GEP + c0), v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) logit[c0 + i] += __uint_as_float(v[i]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->acc_empty[ab]);
+      const int n = t * kRtBM + lg * 32 + lane;
+      if (ok && n < p.N) {
+        if (p.E == 2) route_token_e<GEP, 2>(p, logit, sBias, n);
+        else if (p.E == 4) route_token_e<GEP, 4>(p, logit, sBias, n);
+        else if (p.E == 8) route_token_e<GEP, 8>(p, logit, sBias, n);
+        else route_token<GEP>(p, logit, n);
+      }
+      if (!ok) break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  drain_after_abort(abort);
+}
+
+template <int GEP>
+size_t router_tc_smem(int D, int stages) {
+  return 1024 + (((size_t)(D / kRtBK) * GEP * 128 + 1023) & ~size_t(1023)) + (size_t)stages * kRtTile +
+         sizeof(RouterTcBarriers) + GEP * sizeof(float);
+}
+
+template <int GEP>
+cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const RouterParams& p, cudaStream_t stream) {
+  constexpr int STAGES = 6;
+  const size_t smem = router_tc_smem<GEP>(p.D, STAGES);
+  if (smem > 220 * 1024) return cudaErrorNotSupported;
+  auto kern = router_tc_kernel<GEP, STAGES>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  const int n_tiles = (p.N + kRtBM - 1) / kRtBM;
+  const int sms = router_num_sms();
+  const int grid = n_tiles < sms ? n_tiles : sms;
+  return launch_kernel(kern, dim3(grid), dim3(224), smem, stream, 1, mapX, p);
+}
+
+}  // namespace
+
+cudaError_t launch_router_tc(const CUtensorMap& mapX, const RouterParams& p, cudaStream_t stream) {
+  const int GE = p.G * p.E;
+  if (p.D % kRtBK != 0 || p.E > 8) return cudaErrorNotSupported;
+  if (GE <= 16) return launch_router_tc_gep<16>(mapX, p, stream);
+  if (GE <= 32) return launch_router_tc_gep<32>(mapX, p, stream);
+  return launch_router_tc_gep<64>(mapX, p, stream);
+}
+
 cudaError_t launch_router(const RouterParams& p, cudaStream_t stream) {
   const int GE = p.G * p.E;
   if (GE <= 16) return launch_router_gep<16>(p, stream);

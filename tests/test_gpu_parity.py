@@ -50,6 +50,10 @@ ROUTER_CASES = {
     "main": (gi.WORKLOADS["main_prefill"], None),
     "long": (gi.WORKLOADS["long_prefill"], None),
     "wide_skewed": (gi.WORKLOADS["wide_skewed_prefill"], None),
+    # 1024 tokens and more take the tcgen05 router: generic E, group scope, ragged last tile
+    "tc_E3_group_scope": (gi.Workload("t3", D(B=2, T=640, D=256, G=5, E=3, k=2, renorm_scope=1)), None),
+    "tc_E8_k4_ragged": (gi.Workload("t8", D(B=1, T=1100, D=192, G=4, E=8, k=4)), None),
+    "tc_E4_GE64": (gi.Workload("t4", D(B=1, T=1536, D=128, G=16, E=4, k=1)), None),
 }
 
 
