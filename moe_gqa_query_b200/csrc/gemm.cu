@@ -453,12 +453,20 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
   const int nk = K / kBK;
   pdl_launch_dependents();
   pdl_wait();
-  for (int i = threadIdx.x; i <= rp.n_seg; i += blockDim.x) {
-    seg->tile_start[i] = rp.tile_start[i];
-    if (i < rp.n_seg) {
-      seg->seg_off[i] = rp.seg_off[i];
-      seg->seg_cnt[i] = rp.seg_cnt[i];
+  for (int i = threadIdx.x; i < rp.n_seg; i += blockDim.x) {
+    const int c = rp.seg_cnt[i];
+    seg->seg_cnt[i] = c;
+    seg->seg_off[i] = i * rp.seg_cap;
+    if (blockIdx.x == 0 && rp.expert_counts) rp.expert_counts[i] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tiles = 0;
+    for (int i = 0; i < rp.n_seg; ++i) {
+      seg->tile_start[i] = tiles;
+      tiles += (seg->seg_cnt[i] + kBM - 1) / kBM;
     }
+    seg->tile_start[rp.n_seg] = tiles;
   }
   __syncthreads();
   const int n_routed = seg->tile_start[rp.n_seg];

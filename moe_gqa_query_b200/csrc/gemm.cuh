@@ -34,14 +34,15 @@ enum StoreMode : int {
 };
 
 // Token-to-expert permutation produced by perm.cu, consumed by the routed GEMM.
+// Segment s = g*E + e holds its entries at [s*seg_cap, s*seg_cap + seg_cnt[s]).
 struct RoutedParams {
-  const int* src_row;     // [n_routed] token row of x
-  const int* dst_row;     // [n_routed] row of q_routed [B, G, T, k]
-  const int* seg_off;     // [n_seg] first entry of each (group, expert) segment
+  const int* src_row;     // [n_seg * seg_cap] token row of x
+  const int* dst_row;     // [n_seg * seg_cap] row of q_routed [B, G, T, k]
   const int* seg_cnt;     // [n_seg]
-  const int* tile_start;  // [n_seg + 1] first 128-row tile of each segment
+  int* expert_counts;     // [n_seg] copy of seg_cnt for the caller, or null
+  int seg_cap;            // entries reserved per segment (= tokens)
   int n_seg;              // G * E
-  int max_routed_tiles;   // upper bound on tile_start[n_seg]
+  int max_routed_tiles;   // upper bound on the routed 128-row tiles
   int shared_tiles;       // 128-row tiles of the shared head (0 without one)
   int n_tokens;           // B * T (shared-head tiles)
   int K;                  // d_model

@@ -277,7 +277,7 @@ gqe_status gqe_routed_qproj(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
   GQE_REQUIRE(ws && aligned16(ws), GQE_ERR_WORKSPACE);
   GQE_REQUIRE(ws_bytes >= L.bytes, GQE_ERR_WORKSPACE);
 
-  cudaError_t e = launch_permutation(topk_idx, N, dims->T, G, E, k, ws, L, expert_counts, S(stream));
+  cudaError_t e = launch_permutation(topk_idx, N, dims->T, G, E, k, ws, L, S(stream));
   if (e != cudaSuccess) return GQE_ERR_CUDA;
 
   CUtensorMap mWq, mWsh;
@@ -289,11 +289,11 @@ gqe_status gqe_routed_qproj(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
   RoutedParams rp{};
   rp.src_row = reinterpret_cast<const int*>(w + L.off_src_row);
   rp.dst_row = reinterpret_cast<const int*>(w + L.off_dst_row);
-  rp.seg_off = reinterpret_cast<const int*>(w + L.off_seg_off);
   rp.seg_cnt = reinterpret_cast<const int*>(w + L.off_seg_cnt);
-  rp.tile_start = reinterpret_cast<const int*>(w + L.off_tile_start);
+  rp.expert_counts = expert_counts;
+  rp.seg_cap = L.cap;
   rp.n_seg = G * E;
-  rp.max_routed_tiles = L.n_entries / 128 + G * E;
+  rp.max_routed_tiles = (int)(((long long)N * G * k) / 128) + G * E;
   rp.n_tokens = N;
   rp.K = D;
   rp.d = d;

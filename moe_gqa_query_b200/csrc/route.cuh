@@ -21,18 +21,18 @@ cudaError_t launch_router(const RouterParams& p, cudaStream_t stream);
 // cudaErrorNotSupported for shapes it does not take (the caller falls back).
 cudaError_t launch_router_tc(const CUtensorMap& mapX, const RouterParams& p, cudaStream_t stream);
 
-// Token-to-expert permutation workspace (int32 arrays, see perm.cu).
+// Token-to-expert permutation workspace (int32 arrays, see perm.cu): segment
+// counters, then per segment `cap` slots of source and destination rows.
 struct PermLayout {
-  int n_entries;     // N*G*k
   int n_seg;         // G*E
-  int n_blocks;      // permutation blocks (chunks of entries)
-  size_t off_block_counts, off_block_base, off_seg_cnt, off_seg_off, off_tile_start;
-  size_t off_src_row, off_dst_row;
+  int cap;           // slots per segment (= tokens: a token enters a segment at most once)
+  size_t off_seg_cnt, off_src_row, off_dst_row;
   size_t bytes;
 };
 PermLayout perm_layout(int N, int G, int E, int k);
+// Zeroes the counters and fills the segments in one kernel.
 cudaError_t launch_permutation(const int* topk_idx, int N, int T, int G, int E, int k, void* ws,
-                               const PermLayout& L, int* expert_counts, cudaStream_t stream);
+                               const PermLayout& L, cudaStream_t stream);
 
 struct CombineParams {
   const uint16_t* o_routed;   // [B, G, T, k, d]
