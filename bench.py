@@ -279,7 +279,7 @@ def run_kernel(args):
             o, os_ = torch.empty_like(q), torch.empty_like(qs)
             fn = lambda: gq.gqe_attn_prefill(dc, q, qs, K, V, o, os_, None)  # noqa: E731
             work = dict(flops=attn_useful_flops(dims))
-        elif args.kernel in ("router", "qproj", "kv", "linear", "combine"):
+        elif args.kernel in ("router", "qproj", "kv", "linear", "combine", "combine_out"):
             x = rn(B, T, D)
             Wt = gi.layer_weights(dims)
             lay = gq.GQELayer(dims, {kk: torch.from_numpy(v.view(np.int16)) for kk, v in Wt.items()},
@@ -298,6 +298,10 @@ def run_kernel(args):
             elif args.kernel == "combine":
                 fn = lambda: gq.gqe_combine(dc, inter["o"], inter["o_sh"], inter["w"], inter["h"])  # noqa
                 work = dict(bytes=2.0 * dims.N * (G * k + 1) * d + 2.0 * dims.N * dims.slots * d)
+            elif args.kernel == "combine_out":
+                ws_o = lay._bufs["ws_o"]
+                fn = lambda: gq.gqe_combine_out_proj(dc, inter["o"], inter["o_sh"], inter["w"], lay.Wo, y, ws_o)  # noqa
+                work = dict(flops=2.0 * dims.N * dims.slots * d * D)
             else:
                 fn = lambda: gq.gqe_linear(inter["h"], lay.Wo, y)  # noqa
                 work = dict(flops=2.0 * dims.N * dims.slots * d * D)
@@ -333,7 +337,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--kernel", default=None,
-                    help="time one call alone: attn | decode | router | qproj | kv | combine | linear")
+                    help="time one call alone: attn | decode | router | qproj | kv | combine | linear | combine_out")
     ap.add_argument("--workload", default=WORKLOAD, choices=[k for k, v in gi.WORKLOADS.items() if not v.decode])
     args = ap.parse_args()
     if args.impl == "reference":
@@ -363,7 +367,7 @@ def main():
     stream = torch.cuda.current_stream(device)
 
     # per-call events inside every timed step (router, q-proj, kv-proj, attention, combine, out-proj)
-    seg_names = ["router", "routed_qproj", "kv_proj", "attn_prefill", "combine", "out_proj"]
+    seg_names = ["router", "routed_qproj", "kv_proj", "attn_prefill", "combine_out_proj"]
 
     def step(evs=None):
         c = layer.cfg
@@ -378,13 +382,13 @@ def main():
         V = layer._buf("V", (B, c.G, T, c.d))
         o = layer._buf("o", (B, c.G, T, c.k, c.d))
         os_ = layer._buf("os", (B, T, c.d))
-        h = layer._buf("h", (N, c.slots * c.d))
         y = layer._buf("y", (B, T, c.D))
         ws = layer._ws("ws_q", L.gqe_workspace_size(d_, L.GQE_OP_ROUTED_QPROJ))
+        ws_o = layer._ws("ws_o", L.gqe_workspace_size(d_, L.GQE_OP_COMBINE_OUT_PROJ))
         if evs is None:
             rec = lambda i: None
         elif len(evs) == 2:                     # whole step: start and end only
-            rec = lambda i: evs[min(i, 1)].record(stream) if i in (0, 6) else None
+            rec = lambda i: evs[min(i, 1)].record(stream) if i in (0, 5) else None
         else:                                   # per call
             rec = lambda i: evs[i].record(stream)
         rec(0)
@@ -396,10 +400,8 @@ def main():
         rec(3)
         L.gqe_attn_prefill(d_, q, qs, K, V, o, os_, None)
         rec(4)
-        L.gqe_combine(d_, o, os_, wt, h)
+        L.gqe_combine_out_proj(d_, o, os_, wt, layer.Wo, y, ws_o)
         rec(5)
-        L.gqe_linear(h, layer.Wo, y)
-        rec(6)
         return y
 
     launches_per_step = 7   # router, permutation, routed GEMM, K/V GEMM, attention, combine, Wo GEMM (+ one memset)
@@ -428,13 +430,14 @@ def main():
     local_total_ms = float(step_ms.sum())
     # per-call split, from separate steps with an event between every call
     n_seg = min(args.steps, 10)
-    seg_events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(n_seg)]
+    seg_events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(seg_names) + 1)] for _ in range(n_seg)]
     for s in range(n_seg):
         flush.zero_()
         torch.cuda._sleep(HOST_LEAD_CYCLES)
         step(seg_events[s])
     torch.cuda.synchronize()
-    seg_ms = np.array([[seg_events[s][i].elapsed_time(seg_events[s][i + 1]) for i in range(6)] for s in range(n_seg)])
+    seg_ms = np.array([[seg_events[s][i].elapsed_time(seg_events[s][i + 1]) for i in range(len(seg_names))]
+                       for s in range(n_seg)])
     total_ms = max_over_ranks(local_total_ms, dist, device)
     tokens = world * dims.N * args.steps
     value = tokens / (total_ms / 1e3)

@@ -63,7 +63,7 @@ typedef struct {
   float scale;
 } gqe_dims;
 
-enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2 };
+enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3 };
 
 /* Bytes of scratch the call `op` needs for these dims (L_max: the decode
  * cache length, used by GQE_OP_ATTN_DECODE only).  Returns
@@ -175,6 +175,22 @@ gqe_status gqe_combine(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe
  *   K must be a multiple of 64 and N a multiple of 64. */
 gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W, gqe_bf16* C,
                       gqe_stream stream);
+
+/* Output construction and projection in one call ("GQE" study note §3-2
+ * 3)-5) and 7)): y [B*T, d_model] = h W_o^T with h as gqe_combine builds it,
+ * without writing h.  When T is a multiple of 128 and d_model a multiple of
+ * 256 (and B*T >= 2048) only the weighted-sum slot is materialised (in `ws`)
+ * and the projection reads the hard slots from o_routed and the shared slot
+ * from o_sh directly; otherwise h is built in `ws` and projected.
+ *   o_routed [B, G, T, k, d], o_sh [B, T, d] (NULL without a shared head),
+ *   topk_w [B*T, G, k] fp32, Wo [d_model, (k*G + 1 + n_shared) * d] bf16,
+ *   y [B*T, d_model] bf16; all device pointers, 16-byte aligned.
+ *   ws: scratch of gqe_workspace_size(GQE_OP_COMBINE_OUT_PROJ) bytes.
+ * Errors: GQE_ERR_INVALID_ARG (null/misaligned pointers, bad dims),
+ * GQE_ERR_WORKSPACE (ws too small), GQE_ERR_CUDA (launch failure). */
+gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe_bf16* o_sh,
+                                const float* topk_w, const gqe_bf16* Wo, gqe_bf16* y, void* ws,
+                                size_t ws_bytes, gqe_stream stream);
 
 /* Reads and clears the device error word that kernels set when one of their
  * internal waits runs out of time (0 = none).  Synchronises `stream`. */

@@ -20,6 +20,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "gqe.h")
 GQE_OK = 0
 GQE_OP_ROUTED_QPROJ = 1
 GQE_OP_ATTN_DECODE = 2
+GQE_OP_COMBINE_OUT_PROJ = 3
 STATUS_NAMES = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED",
                 3: "GQE_ERR_WORKSPACE", 4: "GQE_ERR_CUDA", 5: "GQE_ERR_DEVICE_CHECK"}
 
@@ -63,6 +64,7 @@ SIGNATURES = {
     "gqe_attn_decode": [_D, _P, _P, _P, _P, _I, _P, _P, _P, _P, _SZ, _P],
     "gqe_attn_decode_noalloc": [_D, _P, _P, _P, _P, _I, _P, _P, _P, _P],
     "gqe_combine": [_D, _P, _P, _P, _P, _P],
+    "gqe_combine_out_proj": [_D, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "gqe_linear": [_I, _I, _I, _P, _P, _P, _P],
     "gqe_device_error": [ctypes.POINTER(_I), _P],
     "gqe_debug_exp2": [_P, _P, _P, _P, _I, _P],
@@ -216,6 +218,16 @@ def gqe_combine(dims, o_routed, o_sh, topk_w, h, stream=None):
     _check("gqe_combine", lib.gqe_combine(
         ctypes.byref(dims), _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True),
         _ptr(topk_w, "topk_w", torch.float32), _ptr(h, "h", b), _stream(stream)))
+
+
+def gqe_combine_out_proj(dims, o_routed, o_sh, topk_w, Wo, y, ws, stream=None):
+    import torch
+    b = _bf16()
+    ws_bytes = ws.numel() * ws.element_size()
+    _check("gqe_combine_out_proj", lib.gqe_combine_out_proj(
+        ctypes.byref(dims), _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True),
+        _ptr(topk_w, "topk_w", torch.float32), _ptr(Wo, "Wo", b), _ptr(y, "y", b),
+        _ptr(ws, "ws"), ws_bytes, _stream(stream)))
 
 
 def gqe_linear(A, W, C, stream=None):

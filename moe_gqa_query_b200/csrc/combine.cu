@@ -30,7 +30,10 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
   const int GK = p.G * p.k;
   const int slots = GK + 1 + p.n_shared;
   const int sub = lane / LPR, c8 = (lane % LPR) * 8;
-  uint16_t* hrow = p.h + (size_t)n * slots * D + c8;
+  // route_only: h is the [N, d] weighted-sum slot; the hard and shared slots
+  // are read from o_routed and o_sh by the projection itself
+  uint16_t* hrow = p.h + (size_t)n * (p.route_only ? D : slots * D) + c8;
+  uint16_t* route_dst = p.route_only ? hrow : hrow + (size_t)GK * D;
   const size_t gstride = (size_t)p.T * p.k * D;     // next group, same token
   const uint16_t* obase = p.o_routed + (((size_t)b * p.G) * p.T + t) * p.k * D + c8;
   const float* wrow = p.w + (size_t)n * GK;
@@ -43,7 +46,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
       const int g = s / p.k, j = s % p.k;
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(obase + g * gstride + (size_t)j * D));
       const float w = __ldg(wrow + s);
-      *reinterpret_cast<uint4*>(hrow + (size_t)s * D) = v;     // hard slot: a copy
+      if (!p.route_only) *reinterpret_cast<uint4*>(hrow + (size_t)s * D) = v;     // hard slot: a copy
       const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -63,8 +66,8 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
     r.y = pack_bf16x2(acc[2], acc[3]);
     r.z = pack_bf16x2(acc[4], acc[5]);
     r.w = pack_bf16x2(acc[6], acc[7]);
-    *reinterpret_cast<uint4*>(hrow + (size_t)GK * D) = r;
-  } else if (sub == 1 && p.n_shared) {
+    *reinterpret_cast<uint4*>(route_dst) = r;
+  } else if (sub == 1 && p.n_shared && !p.route_only) {
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.o_sh + (size_t)n * D + c8));
     *reinterpret_cast<uint4*>(hrow + (size_t)(GK + 1) * D) = v;
   }

@@ -265,7 +265,9 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
 // thread releases stages and accumulators in both CTAs with one commit each.
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
-gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
+gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapR,
+                       const __grid_constant__ CUtensorMap mapS, ASource as,
+                       const __grid_constant__ CUtensorMap mapB0,
                        const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapO0,
                        const __grid_constant__ CUtensorMap mapO1, EpiParams ep, int M, int K, int n_tiles_b0,
                        int n_tiles_total) {
@@ -300,6 +302,10 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
     bar->abort = 0;
     fence_mbar_init_cluster();
     tma_prefetch_desc(&mapA);
+    if (as.mode == kASlots) {
+      tma_prefetch_desc(&mapR);
+      tma_prefetch_desc(&mapS);
+    }
     tma_prefetch_desc(&mapB0);
     tma_prefetch_desc(&mapB1);
   }
@@ -327,7 +333,19 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             break;
           if (rank == 0) mbar_arrive_expect_tx(&bar->full[s], 2 * (kATileBytes + kHalfB));
           const uint32_t fb = full0 + (uint32_t)(s * sizeof(uint64_t));
-          tma_load_2d_pair(sA + s * kATileBytes, &mapA, fb, kb * kBK, m0);
+          if (as.mode == kASingle) {
+            tma_load_2d_pair(sA + s * kATileBytes, &mapA, fb, kb * kBK, m0);
+          } else {
+            const int col = kb * kBK, slot = col / as.d, sub = col - slot * as.d;
+            const int kG = as.k * as.G;
+            if (slot < kG) {
+              const int g = slot / as.k, kk = slot - g * as.k;
+              const int b = m0 / as.T, t = m0 - b * as.T;
+              tma_load_3d_pair(sA + s * kATileBytes, &mapA, fb, kk * as.d + sub, t, b * as.G + g);
+            } else {
+              tma_load_2d_pair(sA + s * kATileBytes, slot == kG ? &mapR : &mapS, fb, sub, m0);
+            }
+          }
           tma_load_2d_pair(sB + s * kHalfB, mB, fb, kb * kBK, n0);
         }
       }
@@ -614,9 +632,10 @@ static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& m
 }
 
 template <int BN, int STAGES>
-static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
-                                        const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M, int K, int n_tiles_b0, int n_tiles_total,
-                                        cudaStream_t stream) {
+static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorMap& mapR, const CUtensorMap& mapS,
+                                        const ASource& as, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
+                                        const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep,
+                                        int M, int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream) {
   const size_t smem = 1024 + STAGES * (kATileBytes + (BN / 2) * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
   auto kern = gemm_dense_pair_kernel<BN, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
@@ -648,16 +667,17 @@ static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorM
   }
   const int total = ((M + 255) / 256) * n_tiles_total;
   const int pairs = total < mp ? total : mp;
-  return launch_kernel(kern, dim3(2 * pairs), dim3(192), smem, stream, 2, mapA, mapB0, mapB1, mapO0, mapO1, ep, M,
-                       K, n_tiles_b0, n_tiles_total);
+  return launch_kernel(kern, dim3(2 * pairs), dim3(192), smem, stream, 2, mapA, mapR, mapS, as, mapB0, mapB1,
+                       mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total);
 }
 
-cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
+cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapR, const CUtensorMap& mapS,
+                                   const ASource& as, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                                    const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M,
                                    int K, int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream) {
   if (bn != 256) return cudaErrorInvalidValue;
-  return launch_dense_pair_st<256, 6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total,
-                                      stream);
+  return launch_dense_pair_st<256, 6>(mapA, mapR, mapS, as, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0,
+                                      n_tiles_total, stream);
 }
 
 int dense_tile_n(int n_per_weight) { return (n_per_weight % 256 == 0) ? 256 : 128; }

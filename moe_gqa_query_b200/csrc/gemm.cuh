@@ -58,9 +58,22 @@ cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
                               const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
                               int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream);
 
+// Where the pair GEMM's A operand comes from.  kASingle: one map over A [M, K]
+// (box 64 x 128).  kASlots: the output projection's h = [hard slots, weighted
+// sum, shared] read without h: k-block kb (64 columns of slot kb*64/d) comes
+// from o_routed through a map over [B*G, T, k*d] (box 64 x 128 x 1; needs
+// T % 128 == 0), from the weighted-sum buffer [M, d] or from o_sh [M, d].
+enum ASourceMode : int { kASingle = 0, kASlots = 1 };
+struct ASource {
+  int mode;
+  int k, G, T, d;
+};
+
 // 256 x 256 tiles over CTA pairs (bn must be 256); W maps with 128-row boxes,
-// weights' rows a multiple of 256.
-cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapB0,
+// weights' rows a multiple of 256.  mapR / mapS: the weighted-sum and shared
+// slot maps of kASlots (ignored for kASingle).
+cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapR, const CUtensorMap& mapS,
+                                   const ASource& as, const CUtensorMap& mapB0,
                                    const CUtensorMap& mapB1, const CUtensorMap& mapO0,
                                    const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
                                    int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream);

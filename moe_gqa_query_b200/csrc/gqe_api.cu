@@ -227,6 +227,11 @@ gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* b
     *bytes = perm_layout(N, dims->G, dims->E, dims->k).bytes;
     return GQE_OK;
   }
+  if (op == GQE_OP_COMBINE_OUT_PROJ) {
+    const size_t slots = (size_t)dims->k * dims->G + 1 + dims->n_shared;
+    *bytes = (size_t)N * slots * dims->d_head * 2;
+    return GQE_OK;
+  }
   if (op == GQE_OP_ATTN_DECODE) {
     GQE_REQUIRE(L_max >= 1, GQE_ERR_INVALID_ARG);
     *bytes = decode_workspace_bytes(dims->B, dims->G, dims->k, dims->d_head, dims->n_shared, L_max);
@@ -343,7 +348,9 @@ static gqe_status kv_common(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
     ep.store_mode = kStoreTmaHeads;
   }
   const int nt = (G * d + bn - 1) / bn;
-  if (pbn) return cuda_status(launch_gemm_dense_pair(mA, mK, mV, mOK, mOV, ep, M, D, nt, 2 * nt, pbn, S(stream)));
+  if (pbn)
+    return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0}, mK, mV, mOK, mOV, ep, M, D, nt,
+                                              2 * nt, pbn, S(stream)));
   return cuda_status(launch_gemm_dense(mA, mK, mV, mOK, mOV, ep, M, D, nt, 2 * nt, bn, S(stream)));
 }
 
@@ -464,6 +471,61 @@ gqe_status gqe_combine(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe
   return cuda_status(launch_combine(p, S(stream)));
 }
 
+gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe_bf16* o_sh,
+                                const float* topk_w, const gqe_bf16* Wo, gqe_bf16* y, void* ws, size_t ws_bytes,
+                                gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(o_routed && topk_w && Wo && y, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || o_sh, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(o_routed) && aligned16(Wo) && aligned16(y) && (!dims->n_shared || aligned16(o_sh)),
+              GQE_ERR_INVALID_ARG);
+  const int B = dims->B, T = dims->T, G = dims->G, k = dims->k, d = dims->d_head, D = dims->d_model;
+  const int N = B * T;
+  const int slots = k * G + 1 + dims->n_shared;
+  const int Kdim = slots * d;
+  size_t need = 0;
+  GQE_CHECK(gqe_workspace_size(dims, GQE_OP_COMBINE_OUT_PROJ, 0, &need));
+  GQE_REQUIRE(ws && aligned16(ws), GQE_ERR_WORKSPACE);
+  GQE_REQUIRE(ws_bytes >= need, GQE_ERR_WORKSPACE);
+  gqe_bf16* h = static_cast<gqe_bf16*>(ws);
+  // without h: the hard slots come from o_routed in 128-token boxes (T % 128),
+  // only the weighted-sum slot is written (into ws)
+  const bool direct = (T % 128 == 0) && pair_tile_n(N, D) == 256;
+  CombineParams cp{};
+  cp.o_routed = o_routed;
+  cp.o_sh = o_sh;
+  cp.w = topk_w;
+  cp.h = h;
+  cp.B = B;
+  cp.T = T;
+  cp.G = G;
+  cp.k = k;
+  cp.d = d;
+  cp.n_shared = dims->n_shared;
+  cp.route_only = direct ? 1 : 0;
+  cudaError_t e = launch_combine(cp, S(stream));
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  if (!direct) return gqe_linear(N, D, Kdim, h, Wo, y, stream);
+  CUtensorMap mO, mR, mS, mW, mY;
+  GQE_REQUIRE(map3d(&mO, o_routed, (uint64_t)k * d, T, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mR, h, d, N, 128), GQE_ERR_CUDA);
+  if (dims->n_shared) GQE_REQUIRE(map2d(&mS, o_sh, d, N, 128), GQE_ERR_CUDA);
+  else mS = mR;
+  GQE_REQUIRE(map2d(&mW, Wo, Kdim, D, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mY, y, D, N, 32), GQE_ERR_CUDA);
+  EpiParams ep{};
+  ep.out0 = y;
+  ep.out1 = y;
+  ep.mode = kEpiRowMajor;
+  ep.ldo = D;
+  ep.n_limit = D;
+  ep.err = error_word();
+  ep.store_mode = kStoreTma2d;
+  const int nt = D / 256;
+  return cuda_status(launch_gemm_dense_pair(mO, mR, mS, ASource{kASlots, k, G, T, d}, mW, mW, mY, mY, ep, N, Kdim,
+                                            nt, nt, 256, S(stream)));
+}
+
 gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W, gqe_bf16* C, gqe_stream stream) {
   GQE_REQUIRE(M >= 1 && N >= 1 && K >= 1, GQE_ERR_INVALID_ARG);
   GQE_REQUIRE(A && W && C, GQE_ERR_INVALID_ARG);
@@ -486,7 +548,9 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   GQE_REQUIRE(map2d(&mO, C, N, M, 32), GQE_ERR_CUDA);
   ep.store_mode = kStoreTma2d;
   const int nt = (N + bn - 1) / bn;
-  if (pbn) return cuda_status(launch_gemm_dense_pair(mA, mW, mW, mO, mO, ep, M, K, nt, nt, pbn, S(stream)));
+  if (pbn)
+    return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0}, mW, mW, mO, mO, ep, M, K, nt,
+                                              nt, pbn, S(stream)));
   return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, K, nt, nt, bn, S(stream)));
 }
 

@@ -38,8 +38,9 @@ struct CombineParams {
   const uint16_t* o_routed;   // [B, G, T, k, d]
   const uint16_t* o_sh;       // [B, T, d]
   const float* w;             // [N, G, k]
-  uint16_t* h;                // [N, slots*d]
+  uint16_t* h;                // [N, slots*d], or the weighted-sum slot alone [N, d] when route_only
   int B, T, G, k, d, n_shared;
+  int route_only;
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 

@@ -4,7 +4,8 @@ PyTorch supplies device memory (weights, activations, scratch) and the CUDA
 stream; every step of the forward runs in libgqe.so's kernels:
 
   prefill  gqe_router_topk -> gqe_routed_qproj -> gqe_kv_proj ->
-           gqe_attn_prefill -> gqe_combine -> gqe_linear (output projection)
+           gqe_attn_prefill -> gqe_combine_out_proj (output construction and
+           projection, without materialising h where the shape allows)
   decode   gqe_router_topk -> gqe_routed_qproj -> gqe_kv_append ->
            gqe_attn_decode -> gqe_combine -> gqe_linear
 
@@ -102,16 +103,17 @@ class GQELayer:
         V = self._buf("V", (B, c.G, T, c.d))
         o = self._buf("o", (B, c.G, T, c.k, c.d))
         os_ = self._buf("os", (B, T, c.d)) if c.n_shared else None
-        h = self._buf("h", (N, c.slots * c.d))
         y = self._buf("y", (B, T, c.D)) if out is None else out
         ws = self._ws("ws_q", L.gqe_workspace_size(dims, L.GQE_OP_ROUTED_QPROJ))
+        ws_o = self._ws("ws_o", L.gqe_workspace_size(dims, L.GQE_OP_COMBINE_OUT_PROJ))
         L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, None, stream)
         L.gqe_routed_qproj(dims, x, self.Wq, self.Wsh, idx, q, qs, ws, None, stream)
         L.gqe_kv_proj(dims, x, self.Wk, self.Wv, K, V, stream)
         L.gqe_attn_prefill(dims, q, qs, K, V, o, os_, None, stream)
-        L.gqe_combine(dims, o, os_, w, h, stream)
-        L.gqe_linear(h, self.Wo, y, stream)
+        L.gqe_combine_out_proj(dims, o, os_, w, self.Wo, y, ws_o, stream)
         if keep:
+            h = self._buf("h", (N, c.slots * c.d))
+            L.gqe_combine(dims, o, os_, w, h, stream)     # h itself, for inspection only
             return y, dict(idx=idx, w=w, q=q, q_sh=qs, K=K, V=V, o=o, o_sh=os_, h=h)
         return y
 

@@ -341,6 +341,40 @@ def test_combine(dims):
     np.testing.assert_allclose(got[:, hard:hard + d], ref[:, hard:hard + d], rtol=2 ** -8, atol=1e-6)
 
 
+@pytest.mark.parametrize("dims", [gi.WORKLOADS["main_prefill"].dims,
+                                  D(B=2, T=1024, D=512, G=3, E=4, k=2, n_shared=0),
+                                  D(B=1, T=2048, D=256, G=2, E=2, k=1, d=128),
+                                  D(B=3, T=896, D=256, G=4, E=2, k=1, sg=2),
+                                  D(B=2, T=77, D=128, G=3, E=2, k=1)],
+                         ids=["main_direct", "k2_no_shared_direct", "d128_direct", "B3_ragged_pair_direct",
+                              "T77_through_h"])
+def test_combine_out_proj(dims):
+    """Output construction + projection in one call, against the oracle's
+    h = combine(o, o_sh, w) and y = h Wo^T (h is never written when T % 128 == 0)."""
+    B, G, T, k, d = dims.B, dims.G, dims.T, dims.k, dims.d
+    o = gi.normal_bf16(6, "o", (B, G, T, k, d))
+    osh = gi.normal_bf16(6, "osh", (B, T, d))
+    w = gi.random_weights_simplex(dims, 6)
+    Wo = gi.normal_bf16(6, "Wo", (dims.D, dims.slots * d), 0.02)
+    y = torch.full((dims.N, dims.D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dc = dims_c(dims)
+    ws = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_COMBINE_OUT_PROJ),), dtype=torch.uint8, device="cuda")
+    gq.gqe_combine_out_proj(dc, bf16_dev(o), bf16_dev(osh) if dims.n_shared else None,
+                            torch.from_numpy(w).cuda(), bf16_dev(Wo), y, ws)
+    torch.cuda.synchronize()
+    # y carries the bf16 rounding of the weighted-sum slot (as h does) and of y
+    # itself: the layer-output tolerance applies, not the single-GEMM one
+    h_ref = orc.combine(o, osh, w.astype(np.float64), dims)
+    assert_close_attn(to_f64(y), orc.out_proj(h_ref, Wo), "y")
+    # the same MMAs over the same bf16 operands as building h and projecting it
+    h = torch.empty((dims.N, dims.slots * d), dtype=torch.bfloat16, device="cuda")
+    gq.gqe_combine(dc, bf16_dev(o), bf16_dev(osh) if dims.n_shared else None, torch.from_numpy(w).cuda(), h)
+    y2 = torch.empty_like(y)
+    gq.gqe_linear(h, bf16_dev(Wo), y2)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+
+
 # ----------------------------------------------------------------------------
 # whole layer
 
