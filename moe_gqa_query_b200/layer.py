@@ -73,6 +73,8 @@ class GQELayer:
         self.bias = None if bias is None else torch.as_tensor(bias, dtype=torch.float32).to(self.device).contiguous()
         self._bufs = {}
         self._graphs = {}
+        self._side = None
+        self.concurrent_kv = True
 
     # ------------------------------------------------------------------ buffers
     def _buf(self, name, shape, dtype=torch.bfloat16):
@@ -106,9 +108,27 @@ class GQELayer:
         y = self._buf("y", (B, T, c.D)) if out is None else out
         ws = self._ws("ws_q", L.gqe_workspace_size(dims, L.GQE_OP_ROUTED_QPROJ))
         ws_o = self._ws("ws_o", L.gqe_workspace_size(dims, L.GQE_OP_COMBINE_OUT_PROJ))
-        L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, None, stream)
-        L.gqe_routed_qproj(dims, x, self.Wq, self.Wsh, idx, q, qs, ws, None, stream)
-        L.gqe_kv_proj(dims, x, self.Wk, self.Wv, K, V, stream)
+        if stream is None and self.concurrent_kv:
+            # K/V depend on x alone: project them on a side stream while the
+            # router, permutation and routed projection run (they leave SMs
+            # idle in their ramps and tails); attention waits for both
+            main = torch.cuda.current_stream(self.device)
+            if self._side is None:
+                self._side = torch.cuda.Stream(self.device)
+            fork = torch.cuda.Event()
+            fork.record(main)
+            self._side.wait_event(fork)
+            with torch.cuda.stream(self._side):
+                L.gqe_kv_proj(dims, x, self.Wk, self.Wv, K, V)
+                join = torch.cuda.Event()
+                join.record(self._side)
+            L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, None)
+            L.gqe_routed_qproj(dims, x, self.Wq, self.Wsh, idx, q, qs, ws, None)
+            main.wait_event(join)
+        else:
+            L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, None, stream)
+            L.gqe_routed_qproj(dims, x, self.Wq, self.Wsh, idx, q, qs, ws, None, stream)
+            L.gqe_kv_proj(dims, x, self.Wk, self.Wv, K, V, stream)
         L.gqe_attn_prefill(dims, q, qs, K, V, o, os_, None, stream)
         L.gqe_combine_out_proj(dims, o, os_, w, self.Wo, y, ws_o, stream)
         if keep:

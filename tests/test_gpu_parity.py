@@ -469,6 +469,20 @@ def test_layer_graph_replay_matches_eager():
     assert torch.equal(y_pin, y_eager.cpu())
 
 
+def test_layer_concurrent_kv_matches_sequential():
+    """The K/V projection on a side stream gives the same bits as the calls in
+    sequence on one stream."""
+    w = gi.WORKLOADS["main_prefill"]
+    dims, x, Wt, bias, layer = _layer(w, seed=5)
+    xd = bf16_dev(x)
+    layer.concurrent_kv = False
+    y_seq = layer.forward(xd).clone()
+    layer.concurrent_kv = True
+    y_con = layer.forward(xd).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y_seq, y_con)
+
+
 def test_layer_host_pipeline_matches_eager():
     """Five batches through the three-stream host pipeline: each output equals
     the eager forward of its own input (no slot reuse races)."""
