@@ -339,9 +339,10 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             const int col = kb * kBK, slot = col / as.d, sub = col - slot * as.d;
             const int kG = as.k * as.G;
             if (slot < kG) {
+              // o_routed as [B*G*T, k*d]: the 128 tokens of this box share (b, g)
               const int g = slot / as.k, kk = slot - g * as.k;
               const int b = m0 / as.T, t = m0 - b * as.T;
-              tma_load_3d_pair(sA + s * kATileBytes, &mapA, fb, kk * as.d + sub, t, b * as.G + g);
+              tma_load_2d_pair(sA + s * kATileBytes, &mapA, fb, kk * as.d + sub, (b * as.G + g) * as.T + t);
             } else {
               tma_load_2d_pair(sA + s * kATileBytes, slot == kG ? &mapR : &mapS, fb, sub, m0);
             }

@@ -61,8 +61,9 @@ cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
 // Where the pair GEMM's A operand comes from.  kASingle: one map over A [M, K]
 // (box 64 x 128).  kASlots: the output projection's h = [hard slots, weighted
 // sum, shared] read without h: k-block kb (64 columns of slot kb*64/d) comes
-// from o_routed through a map over [B*G, T, k*d] (box 64 x 128 x 1; needs
-// T % 128 == 0), from the weighted-sum buffer [M, d] or from o_sh [M, d].
+// from o_routed through a map over [B*G*T, k*d] (box 64 x 128; needs
+// T % 128 == 0 so a box stays inside one (b, g)), from the weighted-sum buffer
+// [M, d] or from o_sh [M, d].
 enum ASourceMode : int { kASingle = 0, kASlots = 1 };
 struct ASource {
   int mode;

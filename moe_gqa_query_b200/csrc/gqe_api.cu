@@ -507,7 +507,7 @@ gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, 
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   if (!direct) return gqe_linear(N, D, Kdim, h, Wo, y, stream);
   CUtensorMap mO, mR, mS, mW, mY;
-  GQE_REQUIRE(map3d(&mO, o_routed, (uint64_t)k * d, T, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d(&mO, o_routed, (uint64_t)k * d, (uint64_t)B * G * T, 128), GQE_ERR_CUDA);
   GQE_REQUIRE(map2d(&mR, h, d, N, 128), GQE_ERR_CUDA);
   if (dims->n_shared) GQE_REQUIRE(map2d(&mS, o_sh, d, N, 128), GQE_ERR_CUDA);
   else mS = mR;
