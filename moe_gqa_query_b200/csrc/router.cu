@@ -723,7 +723,7 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
       if (lane == 0) mbar_arrive(&bar->acc_empty[ab]);
       const int n = t * kRtBM + lg * 32 + lane;
       if (ok && n < p.N) {
-        if (p.E == 2) route_token_e<GEP, 2>(p, logit, sBias, n);
+        if (p.E == 2 && GEP <= 32) route_token_e<GEP, 2>(p, logit, sBias, n);
         else if (p.E == 4) route_token_e<GEP, 4>(p, logit, sBias, n);
         else if (p.E == 8) route_token_e<GEP, 8>(p, logit, sBias, n);
         else route_token<GEP>(p, logit, n);
