@@ -225,6 +225,26 @@ def test_attn_prefill_constant_keys_prefix_mean():
     assert_close_attn(to_f64(os_), pm[:, 0], "prefix mean shared")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_attn_prefill_growing_scores(d):
+    """Keys whose norm grows along the sequence: later key tiles raise the
+    running row maximum far past the lazy-rescale margin, so the rescale of
+    P, the row sum and O is exercised on most rows."""
+    dims = D(B=1, T=700, G=2, E=2, k=2, d=d)
+    q, qs, K, V = _attn_inputs(dims, 12)
+    growth = (1.0 + np.arange(dims.T) / 24.0)[None, None, :, None]
+    K = gi.f32_to_bf16_bits((gi.bf16_bits_to_f32(K) * growth).astype(np.float32))
+    # the softmax becomes nearly one-hot, so o is close to single V rows: V at a
+    # quarter scale keeps |o| where bf16 rounding of o stays inside the tolerance
+    V = gi.f32_to_bf16_bits((gi.bf16_bits_to_f32(V) * 0.25).astype(np.float32))
+    o, os_, lse = _run_prefill(dims, q, qs, K, V)
+    o_ref, os_ref, lse_ref, lsesh_ref = orc.attn_prefill(q, qs, K, V, dims)
+    assert_close_attn(to_f64(o), o_ref, "o_routed")
+    assert_close_attn(to_f64(os_), os_ref, "o_sh")
+    n_r = dims.B * dims.G * dims.T * dims.k
+    np.testing.assert_allclose(lse.cpu().numpy()[:n_r], lse_ref.reshape(-1), atol=2e-2, rtol=1e-3)
+
+
 @pytest.mark.parametrize("wname", ["main_prefill", "long_prefill", "wide_skewed_prefill"])
 def test_attn_prefill_full_size_sampled(wname):
     """Full workload size, bench launch configuration; sampled rows vs the oracle."""
