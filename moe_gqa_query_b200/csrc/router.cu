@@ -443,6 +443,7 @@ struct __align__(8) RouterTcBarriers {
   uint64_t empty[8];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t w_full;           // Wr copied into shared memory (bulk copy)
   uint32_t tmem_base;
   int abort;
 };
@@ -560,7 +561,8 @@ __device__ __forceinline__ void route_token_e(const RouterParams& p, const float
 // the tensor pipe busy for less time than one thread needs to issue it);
 // warps 2..5 sum the partials and route, one token per thread.
 template <int GEP, int STAGES>
-__global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant__ CUtensorMap mapX, RouterParams p) {
+__global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant__ CUtensorMap mapX, RouterParams p,
+                                                           int wr_staged) {
   constexpr int kWBlk = GEP * 128;                 // one k-block of Wr^T
   constexpr uint32_t kTmemCols = 4 * GEP;          // 2 buffers x 2 partial accumulators
   extern __shared__ uint8_t smem_raw[];
@@ -570,6 +572,8 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
   uint8_t* sX = sW + ((nk * kWBlk + 1023) & ~1023);          // STAGES x 16 KB
   RouterTcBarriers* bar = reinterpret_cast<RouterTcBarriers*>(sX + STAGES * kRtTile);
   float* sBias = reinterpret_cast<float*>(bar + 1);          // GEP
+  // Wr as it is in memory ([D, GE]), when it is brought in by one bulk copy
+  uint8_t* sWr = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sBias + GEP) + 127) & ~uintptr_t(127));
   volatile int* abort = &bar->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int GE = p.G * p.E;
@@ -584,6 +588,7 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
       mbar_init(&bar->acc_full[a], 2);     // one commit from each MMA thread
       mbar_init(&bar->acc_empty[a], 4);
     }
+    mbar_init(&bar->w_full, 1);
     bar->abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&mapX);
@@ -594,16 +599,41 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
   __syncthreads();   // barriers initialised
   // the first x tiles are requested before Wr^T is built (they do not need it)
   const int first_tiles = min(STAGES, (blockIdx.x < n_tiles ? ((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0) * nk);
+  const uint32_t wr_bytes = (uint32_t)p.D * GE * 2;
   if (threadIdx.x == 0) {
     for (int it = 0; it < first_tiles; ++it) {
       const int t = blockIdx.x + (it / nk) * gridDim.x, kb = it % nk;
       mbar_arrive_expect_tx(&bar->full[it], kRtTile);
       tma_load_2d(sX + it * kRtTile, &mapX, &bar->full[it], kb * kRtBK, t * kRtBM);
     }
+    if (wr_staged) {
+      mbar_arrive_expect_tx(&bar->w_full, wr_bytes);
+      bulk_load(sWr, p.Wr, wr_bytes, &bar->w_full);
+    }
   }
-  // Wr [D, GE] -> Wr^T in the swizzled K-major layout (rows GE..GEP-1 zero);
-  // 16-byte loads of 8 consecutive experts of one model dimension
-  if ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0) {
+  // Wr [D, GE] -> Wr^T in the swizzled K-major layout (rows GE..GEP-1 zero)
+  if (wr_staged) {
+    // from the bulk copy in shared memory: 16 bytes = 8 experts of one model dimension
+    mbar_wait(&bar->w_full, 0, abort, p.err, kErrTimeoutRouter);
+    const int per_row = GE / 8;
+    for (int e = threadIdx.x; e < p.D * per_row; e += blockDim.x) {
+      const int dd = e / per_row, n0 = (e % per_row) * 8;
+      const uint4 v = *reinterpret_cast<const uint4*>(sWr + ((size_t)dd * GE + n0) * 2);
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
+      const int kb = dd >> 6, c = dd & 63;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int n = n0 + i;
+        *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) = h[i];
+      }
+    }
+    for (int e = threadIdx.x; e < p.D * (GEP - GE); e += blockDim.x) {
+      const int dd = e / (GEP - GE), n = GE + e % (GEP - GE);
+      const int kb = dd >> 6, c = dd & 63;
+      *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) = 0;
+    }
+  } else if ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0) {
+    // 16-byte loads of 8 consecutive experts of one model dimension
     const int per_row = GE / 8;
     const int total = p.D * per_row;
     for (int e0 = threadIdx.x; e0 < total; e0 += 4 * blockDim.x) {
@@ -741,15 +771,20 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
 }
 
 template <int GEP>
-size_t router_tc_smem(int D, int stages) {
+size_t router_tc_smem(int D, int stages, size_t staging) {
   return 1024 + (((size_t)(D / kRtBK) * GEP * 128 + 1023) & ~size_t(1023)) + (size_t)stages * kRtTile +
-         sizeof(RouterTcBarriers) + GEP * sizeof(float);
+         sizeof(RouterTcBarriers) + GEP * sizeof(float) + 128 + staging;
 }
 
 template <int GEP>
 cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const RouterParams& p, cudaStream_t stream) {
   constexpr int STAGES = 6;
-  const size_t smem = router_tc_smem<GEP>(p.D, STAGES);
+  // Wr by one bulk copy when it and its staging fit (16-byte aligned, whole 16-byte rows of 8 experts)
+  const int GE = p.G * p.E;
+  const size_t wr_bytes = (size_t)p.D * GE * 2;
+  int staged = ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0 && wr_bytes % 16 == 0) ? 1 : 0;
+  if (staged && router_tc_smem<GEP>(p.D, STAGES, wr_bytes) > 220 * 1024) staged = 0;
+  const size_t smem = router_tc_smem<GEP>(p.D, STAGES, staged ? wr_bytes : 0);
   if (smem > 220 * 1024) return cudaErrorNotSupported;
   auto kern = router_tc_kernel<GEP, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
@@ -757,7 +792,7 @@ cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const RouterParams& p,
   const int n_tiles = (p.N + kRtBM - 1) / kRtBM;
   const int sms = router_num_sms();
   const int grid = n_tiles < sms ? n_tiles : sms;
-  return launch_kernel(kern, dim3(grid), dim3(224), smem, stream, 1, mapX, p);
+  return launch_kernel(kern, dim3(grid), dim3(224), smem, stream, 1, mapX, p, staged);
 }
 
 }  // namespace
