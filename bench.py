@@ -328,6 +328,74 @@ def run_kernel(args):
     return 0
 
 
+SWEEP_T = (2048, 4096, 8192, 16384, 32768, 65536, 131072)
+
+
+def run_sweep_gqa(args):
+    """GQE against dense GQA on the same layer shape (B=1, D=1024, 8 KV groups,
+    E=2 query heads per group, d=64), prefill T from 2K to 128K tokens.  GQE:
+    top-1 of 2 per group plus the shared head (9 active query heads).  Dense
+    GQA: the same kernels with k = E and no shared head (all 16 heads, the
+    weighted-sum slot kept).  Attention alone and the whole layer forward, each
+    timed with CUDA events on device-generated inputs (the pages' prefill
+    speedup claim, re-measured on this GPU)."""
+    import torch
+    import moe_gqa_query_b200 as gq
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    gen = torch.Generator(device=device).manual_seed(3)
+    ts = [int(t) for t in args.sweep_t.split(",")] if args.sweep_t else list(SWEEP_T)
+
+    def rn(*shape, std=1.0):
+        return (torch.randn(shape, device=device, generator=gen) * std).to(torch.bfloat16)
+
+    def time_ms(fn, reps):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in evs:
+            torch.cuda._sleep(HOST_LEAD_CYCLES)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+    for T in ts:
+        line = {"sweep": "gqe_vs_dense_gqa", "T": T, "B": 1}
+        for name, k, n_sh in (("gqe", 1, 1), ("gqa", 2, 0)):
+            dims = gi.GQEDims(B=1, T=T, D=1024, G=8, E=2, k=k, d=64, n_shared=n_sh)
+            dc = gq.make_dims(dims)
+            q = rn(1, 8, T, k, 64)
+            qs = rn(1, T, 64)
+            K, V = rn(1, 8, T, 64), rn(1, 8, T, 64)
+            o, os_ = torch.empty_like(q), torch.empty_like(qs)
+            reps = 3 if T >= 65536 else 5
+            a_ms = time_ms(lambda: gq.gqe_attn_prefill(dc, q, qs if n_sh else None, K, V, o,
+                                                      os_ if n_sh else None, None), reps)
+            del q, qs, K, V, o, os_
+            Wt = {"Wr": rn(1024, 16, std=0.02), "Wq": rn(8, 2, 64, 1024, std=0.02),
+                  "Wk": rn(512, 1024, std=0.02), "Wv": rn(512, 1024, std=0.02),
+                  "Wsh": rn(64, 1024, std=0.02), "Wo": rn(1024, dims.slots * 64, std=0.02)}
+            if not n_sh:
+                Wt["Wsh"] = rn(0, 1024)
+            lay = gq.GQELayer(dims, Wt, None, device=device)
+            x = rn(1, T, 1024)
+            y = torch.empty_like(x)
+            l_ms = time_ms(lambda: lay.forward(x, out=y), reps)
+            del lay, x, y
+            torch.cuda.empty_cache()
+            line[name] = {"attn_ms": a_ms, "attn_tflops": attn_useful_flops(dims) / a_ms / 1e9,
+                          "layer_ms": l_ms, "active_query_heads": dims.h_active}
+        line["attn_speedup"] = line["gqa"]["attn_ms"] / line["gqe"]["attn_ms"]
+        line["layer_speedup"] = line["gqa"]["layer_ms"] / line["gqe"]["layer_ms"]
+        line["device_error"] = gq.gqe_device_error()
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -339,11 +407,16 @@ def main():
     ap.add_argument("--kernel", default=None,
                     help="time one call alone: attn | decode | router | qproj | kv | combine | linear | combine_out")
     ap.add_argument("--workload", default=WORKLOAD, choices=[k for k, v in gi.WORKLOADS.items() if not v.decode])
+    ap.add_argument("--sweep", default=None, choices=["gqa"],
+                    help="gqa: GQE against dense GQA, prefill T from 2K to 128K (one JSON line per T)")
+    ap.add_argument("--sweep-t", default=None, help="comma-separated T values for --sweep")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.kernel:
         return run_kernel(args)
+    if args.sweep == "gqa":
+        return run_sweep_gqa(args)
     args.warmup = max(args.warmup, 3)
 
     world, rank, local = dist_env()

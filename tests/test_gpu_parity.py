@@ -427,6 +427,22 @@ def test_layer_forward_end_to_end(wname):
           f"differently routed {int((~agree).sum())}")
 
 
+def test_layer_dense_gqa_mode():
+    """k = E with no shared head is dense GQA through the same kernels: every
+    query head of every group is computed, and the hard slots of h are the GQA
+    heads in order g*E + e (the oracle reduces to dense GQA there, pinned on
+    the CPU); y against the oracle layer."""
+    dims = D(B=2, T=300, D=256, G=4, E=2, k=2, n_shared=0)
+    w = gi.Workload("dense_gqa", dims)
+    dims, x, Wt, bias, layer = _layer(w, seed=8)
+    y, inter = layer.forward(bf16_dev(x), keep=True)
+    torch.cuda.synchronize()
+    ref = orc.gqe_forward(x, Wt, dims, bias)
+    assert np.array_equal(inter["idx"].cpu().numpy(), np.broadcast_to(np.arange(2), (dims.N, 4, 2)))
+    assert_close_attn(to_f64(y).reshape(dims.N, -1), ref["y"], "y")
+    assert_close_attn(to_f64(inter["h"]), ref["h"], "h")
+
+
 def test_layer_decode_step_end_to_end():
     w = gi.Workload("dec_small", D(B=4, T=1, D=256, G=2, E=4, k=2, d=64), decode=True, L=700)
     dims = w.dims
