@@ -38,7 +38,9 @@ class GQEDims:
     k experts routed per (token, group), head width d, n_shared always-on
     shared query heads (0 or 1) reading KV group ``sg``.  ``renorm_scope`` 0
     normalises the selected router probabilities over all k*G selections of a
-    token, 1 within each group.  ``scale`` 0 means 1/sqrt(d).
+    token, 1 within each group, 2 not at all.  ``scale`` 0 means 1/sqrt(d).
+    ``output_mode`` 0 is GQE's output (hard slots, weighted-sum slot, shared
+    head); 1 hard slots only (+ shared); 2 router-weighted hard slots (+ shared).
     """
     B: int
     T: int
@@ -51,6 +53,7 @@ class GQEDims:
     sg: int = 0
     renorm_scope: int = 0
     scale: float = 0.0
+    output_mode: int = 0
 
     @property
     def N(self) -> int:
@@ -58,8 +61,8 @@ class GQEDims:
 
     @property
     def slots(self) -> int:
-        """Output-projection input slots: k*G hard + 1 weighted + n_shared."""
-        return self.k * self.G + 1 + self.n_shared
+        """Output-projection input slots: k*G hard (+ 1 weighted sum in mode 0) + n_shared."""
+        return self.k * self.G + (1 if self.output_mode == 0 else 0) + self.n_shared
 
     @property
     def h_active(self) -> int:

@@ -54,13 +54,20 @@ typedef enum {
  * model width d_model, G KV groups with E query experts each, k experts
  * routed per (token, group), head width d_head.  renorm_scope 0 normalises
  * the selected router probabilities over all k*G selections of a token, 1
- * within each group.  scale 0 means 1/sqrt(d_head). */
+ * within each group, 2 not at all (the weights are the in-group softmax
+ * probabilities).  scale 0 means 1/sqrt(d_head).  output_mode selects the
+ * output construction ("GQE" study note §3-2 3)-5) and the ablation rows of
+ * §5-1's accuracy table): 0 GQE, h = [hard slots, weighted-sum slot,
+ * shared]; 1 "hard concat only", h = [hard slots, shared]; 2 "weighted
+ * concat, no renormalised slot", h = [weight * hard slot each, shared].  The
+ * number of slots of h is k*G + (output_mode == 0) + n_shared. */
 typedef struct {
   int B, T, d_model, G, E, k, d_head;
   int n_shared;          /* 0 or 1 always-on shared query heads */
   int shared_kv_group;   /* KV group the shared head reads */
-  int renorm_scope;      /* 0 token, 1 group */
+  int renorm_scope;      /* 0 token, 1 group, 2 none */
   float scale;
+  int output_mode;       /* 0 GQE, 1 hard concat only, 2 weighted concat */
 } gqe_dims;
 
 enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3 };

@@ -36,15 +36,16 @@ class gqe_dims(ctypes.Structure):
                 ("G", ctypes.c_int), ("E", ctypes.c_int), ("k", ctypes.c_int),
                 ("d_head", ctypes.c_int), ("n_shared", ctypes.c_int),
                 ("shared_kv_group", ctypes.c_int), ("renorm_scope", ctypes.c_int),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("output_mode", ctypes.c_int)]
 
 
 def make_dims(cfg, **override) -> gqe_dims:
     """Shape struct from any object with B, T, D, G, E, k, d (+ n_shared, sg,
-    renorm_scope, scale) attributes."""
+    renorm_scope, scale, output_mode) attributes."""
     v = dict(B=cfg.B, T=cfg.T, d_model=cfg.D, G=cfg.G, E=cfg.E, k=cfg.k, d_head=cfg.d,
              n_shared=getattr(cfg, "n_shared", 1), shared_kv_group=getattr(cfg, "sg", 0),
-             renorm_scope=getattr(cfg, "renorm_scope", 0), scale=float(getattr(cfg, "scale", 0.0)))
+             renorm_scope=getattr(cfg, "renorm_scope", 0), scale=float(getattr(cfg, "scale", 0.0)),
+             output_mode=getattr(cfg, "output_mode", 0))
     v.update(override)
     return gqe_dims(**v)
 

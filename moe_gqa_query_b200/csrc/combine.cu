@@ -1,4 +1,7 @@
-// combine.cu -- GQE output construction ("GQE" study note §3-2 3)-5)).
+// combine.cu -- GQE output construction ("GQE" study note §3-2 3)-5)) and the
+// two ablation variants of §5-1's accuracy table (output_mode 1: hard slots
+// and shared head only; 2: hard slots each times its router weight, shared
+// head, no weighted-sum slot).
 //
 //   h_t = Concat( o_{t,g,e} for the selected e of every group g (group-major,
 //                 ascending expert index: one head slot each, never averaged),
@@ -28,7 +31,8 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
   pdl_wait();
   const int b = n / p.T, t = n % p.T;
   const int GK = p.G * p.k;
-  const int slots = GK + 1 + p.n_shared;
+  const int has_route = p.output_mode == 0 ? 1 : 0;
+  const int slots = GK + has_route + p.n_shared;
   const int sub = lane / LPR, c8 = (lane % LPR) * 8;
   // route_only: h is the [N, d] weighted-sum slot; the hard and shared slots
   // are read from o_routed and o_sh by the projection itself
@@ -46,8 +50,17 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
       const int g = s / p.k, j = s % p.k;
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(obase + g * gstride + (size_t)j * D));
       const float w = __ldg(wrow + s);
-      if (!p.route_only) *reinterpret_cast<uint4*>(hrow + (size_t)s * D) = v;     // hard slot: a copy
       const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+      if (p.output_mode == 2) {
+        // weighted concat: the hard slot times its router weight
+        const uint4 wv = make_uint4(pack_bf16x2(w * bf16_lo(u[0]), w * bf16_hi(u[0])),
+                                    pack_bf16x2(w * bf16_lo(u[1]), w * bf16_hi(u[1])),
+                                    pack_bf16x2(w * bf16_lo(u[2]), w * bf16_hi(u[2])),
+                                    pack_bf16x2(w * bf16_lo(u[3]), w * bf16_hi(u[3])));
+        *reinterpret_cast<uint4*>(hrow + (size_t)s * D) = wv;
+      } else if (!p.route_only) {
+        *reinterpret_cast<uint4*>(hrow + (size_t)s * D) = v;     // hard slot: a copy
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         acc[2 * i] = fmaf(w, bf16_lo(u[i]), acc[2 * i]);
@@ -60,7 +73,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
   for (int o = LPR; o < 32; o <<= 1)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-  if (sub == 0) {
+  if (sub == 0 && has_route) {
     uint4 r;
     r.x = pack_bf16x2(acc[0], acc[1]);
     r.y = pack_bf16x2(acc[2], acc[3]);
@@ -69,7 +82,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
     *reinterpret_cast<uint4*>(route_dst) = r;
   } else if (sub == 1 && p.n_shared && !p.route_only) {
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.o_sh + (size_t)n * D + c8));
-    *reinterpret_cast<uint4*>(hrow + (size_t)(GK + 1) * D) = v;
+    *reinterpret_cast<uint4*>(hrow + (size_t)(GK + has_route) * D) = v;
   }
 }
 

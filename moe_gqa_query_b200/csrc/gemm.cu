@@ -344,7 +344,7 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
               const int b = m0 / as.T, t = m0 - b * as.T;
               tma_load_2d_pair(sA + s * kATileBytes, &mapA, fb, kk * as.d + sub, (b * as.G + g) * as.T + t);
             } else {
-              tma_load_2d_pair(sA + s * kATileBytes, slot == kG ? &mapR : &mapS, fb, sub, m0);
+              tma_load_2d_pair(sA + s * kATileBytes, (slot == kG && as.route) ? &mapR : &mapS, fb, sub, m0);
             }
           }
           tma_load_2d_pair(sB + s * kHalfB, mB, fb, kb * kBK, n0);

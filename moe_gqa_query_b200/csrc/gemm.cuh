@@ -68,6 +68,7 @@ enum ASourceMode : int { kASingle = 0, kASlots = 1 };
 struct ASource {
   int mode;
   int k, G, T, d;
+  int route;    // kASlots: 1 when slot k*G is the weighted-sum slot, 0 when the shared slot follows the hard ones
 };
 
 // 256 x 256 tiles over CTA pairs (bn must be 256); W maps with 128-row boxes,

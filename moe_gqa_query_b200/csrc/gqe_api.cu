@@ -133,8 +133,9 @@ gqe_status check_dims(const gqe_dims* d) {
   if (!d) return GQE_ERR_INVALID_ARG;
   if (d->B < 1 || d->T < 1 || d->d_model < 1 || d->G < 1 || d->E < 1 || d->k < 1 || d->k > d->E)
     return GQE_ERR_INVALID_ARG;
-  if (d->n_shared < 0 || d->n_shared > 1 || d->renorm_scope < 0 || d->renorm_scope > 1)
+  if (d->n_shared < 0 || d->n_shared > 1 || d->renorm_scope < 0 || d->renorm_scope > 2)
     return GQE_ERR_INVALID_ARG;
+  if (d->output_mode < 0 || d->output_mode > 2) return GQE_ERR_INVALID_ARG;
   if (d->shared_kv_group < 0 || d->shared_kv_group >= d->G) return GQE_ERR_INVALID_ARG;
   if (!(d->scale >= 0.f) || isinf(d->scale)) return GQE_ERR_INVALID_ARG;
   if (d->d_head != 64 && d->d_head != 128) return GQE_ERR_UNSUPPORTED;
@@ -228,7 +229,7 @@ gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* b
     return GQE_OK;
   }
   if (op == GQE_OP_COMBINE_OUT_PROJ) {
-    const size_t slots = (size_t)dims->k * dims->G + 1 + dims->n_shared;
+    const size_t slots = (size_t)dims->k * dims->G + (dims->output_mode == 0 ? 1 : 0) + dims->n_shared;
     *bytes = (size_t)N * slots * dims->d_head * 2;
     return GQE_OK;
   }
@@ -349,7 +350,7 @@ static gqe_status kv_common(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
   }
   const int nt = (G * d + bn - 1) / bn;
   if (pbn)
-    return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0}, mK, mV, mOK, mOV, ep, M, D, nt,
+    return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0, 0}, mK, mV, mOK, mOV, ep, M, D, nt,
                                               2 * nt, pbn, S(stream)));
   return cuda_status(launch_gemm_dense(mA, mK, mV, mOK, mOV, ep, M, D, nt, 2 * nt, bn, S(stream)));
 }
@@ -468,6 +469,7 @@ gqe_status gqe_combine(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe
   p.k = dims->k;
   p.d = dims->d_head;
   p.n_shared = dims->n_shared;
+  p.output_mode = dims->output_mode;
   return cuda_status(launch_combine(p, S(stream)));
 }
 
@@ -481,7 +483,8 @@ gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, 
               GQE_ERR_INVALID_ARG);
   const int B = dims->B, T = dims->T, G = dims->G, k = dims->k, d = dims->d_head, D = dims->d_model;
   const int N = B * T;
-  const int slots = k * G + 1 + dims->n_shared;
+  const int has_route = dims->output_mode == 0 ? 1 : 0;
+  const int slots = k * G + has_route + dims->n_shared;
   const int Kdim = slots * d;
   size_t need = 0;
   GQE_CHECK(gqe_workspace_size(dims, GQE_OP_COMBINE_OUT_PROJ, 0, &need));
@@ -490,7 +493,8 @@ gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, 
   gqe_bf16* h = static_cast<gqe_bf16*>(ws);
   // without h: the hard slots come from o_routed in 128-token boxes (T % 128),
   // only the weighted-sum slot is written (into ws)
-  const bool direct = (T % 128 == 0) && pair_tile_n(N, D) == 256;
+  // (the weighted hard slots of output_mode 2 are built in h)
+  const bool direct = (T % 128 == 0) && pair_tile_n(N, D) == 256 && dims->output_mode != 2;
   CombineParams cp{};
   cp.o_routed = o_routed;
   cp.o_sh = o_sh;
@@ -503,8 +507,11 @@ gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, 
   cp.d = d;
   cp.n_shared = dims->n_shared;
   cp.route_only = direct ? 1 : 0;
-  cudaError_t e = launch_combine(cp, S(stream));
-  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  cp.output_mode = dims->output_mode;
+  if (!direct || has_route) {     // direct without a weighted-sum slot needs no combine pass
+    cudaError_t e = launch_combine(cp, S(stream));
+    if (e != cudaSuccess) return GQE_ERR_CUDA;
+  }
   if (!direct) return gqe_linear(N, D, Kdim, h, Wo, y, stream);
   CUtensorMap mO, mR, mS, mW, mY;
   GQE_REQUIRE(map2d(&mO, o_routed, (uint64_t)k * d, (uint64_t)B * G * T, 128), GQE_ERR_CUDA);
@@ -522,7 +529,7 @@ gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, 
   ep.err = error_word();
   ep.store_mode = kStoreTma2d;
   const int nt = D / 256;
-  return cuda_status(launch_gemm_dense_pair(mO, mR, mS, ASource{kASlots, k, G, T, d}, mW, mW, mY, mY, ep, N, Kdim,
+  return cuda_status(launch_gemm_dense_pair(mO, mR, mS, ASource{kASlots, k, G, T, d, has_route}, mW, mW, mY, mY, ep, N, Kdim,
                                             nt, nt, 256, S(stream)));
 }
 
@@ -549,7 +556,7 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   ep.store_mode = kStoreTma2d;
   const int nt = (N + bn - 1) / bn;
   if (pbn)
-    return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0}, mW, mW, mO, mO, ep, M, K, nt,
+    return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0, 0}, mW, mW, mO, mO, ep, M, K, nt,
                                               nt, pbn, S(stream)));
   return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, K, nt, nt, bn, S(stream)));
 }

@@ -13,7 +13,7 @@ struct RouterParams {
   int* topk_idx;          // [N, G, k]
   float* topk_w;          // [N, G, k]
   float* probs;           // [N, G, E] or null
-  int N, D, G, E, k, scope;
+  int N, D, G, E, k, scope;   // scope: 0 token, 1 group, 2 none (w = p)
   unsigned* err;          // device error word (bounded waits of the tcgen05 router)
 };
 cudaError_t launch_router(const RouterParams& p, cudaStream_t stream);
@@ -41,6 +41,7 @@ struct CombineParams {
   uint16_t* h;                // [N, slots*d], or the weighted-sum slot alone [N, d] when route_only
   int B, T, G, k, d, n_shared;
   int route_only;
+  int output_mode;            // 0 GQE, 1 hard slots only, 2 weighted hard slots (no weighted-sum slot)
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 

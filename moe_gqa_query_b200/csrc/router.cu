@@ -110,7 +110,7 @@ __device__ __forceinline__ void route_tile(const RouterParams& p, const float* l
       den = 0.f;
       for (int gg = 0; gg < G; ++gg) den += gs[t * G + gg];
     }
-    const float inv_den = 1.f / den;
+    const float inv_den = p.scope == 2 ? 1.f : 1.f / den;
     const size_t o = ((size_t)n * G + g) * k;
     int j = 0;
     for (int ee = 0; ee < E; ++ee) {
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) router_resident_kernel(R
         for (int g = half; g < p.G; g += 2) {
           float pr[8], sum;
           const unsigned chosen = route_group(p, row, g, pr, &sum);
-          const float inv_den = 1.f / (p.scope == 0 ? total : sum);
+          const float inv_den = p.scope == 2 ? 1.f : 1.f / (p.scope == 0 ? total : sum);
           const size_t o = ((size_t)n * p.G + g) * p.k;
           int j = 0;
           for (int ee = 0; ee < p.E; ++ee) {
@@ -462,7 +462,7 @@ __device__ __forceinline__ void route_token(const RouterParams& p, const float* 
   for (int g = 0; g < G; ++g) {
     float pr[8], sum;
     const unsigned chosen = route_group(p, lg, g, pr, &sum);
-    const float inv_den = 1.f / (p.scope == 0 ? den_tok : sum);
+    const float inv_den = p.scope == 2 ? 1.f : 1.f / (p.scope == 0 ? den_tok : sum);
     const size_t o = ((size_t)n * G + g) * k;
     int j = 0;
     for (int e = 0; e < E; ++e) {
@@ -537,7 +537,7 @@ __device__ __forceinline__ void route_token_e(const RouterParams& p, const float
 #pragma unroll
   for (int g = 0; g < GM; ++g) {
     if (g < G) {
-      const float inv_den = 1.f / (p.scope == 0 ? den_tok : gsum[g]);
+      const float inv_den = p.scope == 2 ? 1.f : 1.f / (p.scope == 0 ? den_tok : gsum[g]);
       const size_t o = ((size_t)n * G + g) * k;
       int j = 0;
 #pragma unroll

@@ -10,7 +10,8 @@ stream; every step of the forward runs in libgqe.so's kernels:
            gqe_attn_decode -> gqe_combine -> gqe_linear
 
 Weight layouts (bf16): Wr [D, G*E]; Wq [G, E, d, D]; Wk, Wv [G*d, D];
-Wsh [n_shared*d, D]; Wo [D, (k*G + 1 + n_shared)*d].
+Wsh [n_shared*d, D]; Wo [D, slots*d] with slots = k*G + 1 + n_shared (GQE's
+output; k*G + n_shared for the two ablation output modes).
 """
 from __future__ import annotations
 
@@ -34,10 +35,11 @@ class GQEConfig:
     sg: int = 0
     renorm_scope: int = 0
     scale: float = 0.0
+    output_mode: int = 0
 
     @property
     def slots(self) -> int:
-        return self.k * self.G + 1 + self.n_shared
+        return self.k * self.G + (1 if self.output_mode == 0 else 0) + self.n_shared
 
 
 def config_from(obj) -> GQEConfig:

@@ -19,7 +19,13 @@ it.  Pages cited:
 Readings where the pages leave a step open (each one is listed in the design
 notes of the repository):
   * p~ is normalised over all k*G selections of a token (scope 0); scope 1
-    normalises within a group.
+    normalises within a group; scope 2 leaves the in-group softmax
+    probability p as it is (for the ablation variants below).
+  * the two ablation variants of [SN] §5-1 (accuracy table), which the pages
+    name but do not define, read plainly: "hard concat only" (output_mode 1)
+    drops the weighted-sum slot, h = [hard slots, shared]; "weighted concat,
+    no renormalised slot" (output_mode 2) scales each hard slot by its router
+    weight and has no weighted-sum slot, h = [w * hard slots, shared].
   * hard slots are group-major, and inside a group in ascending expert index.
   * TopK ties go to the lower expert index.
   * the shared head has no K/V of its own and reads KV group ``sg``.
@@ -103,9 +109,12 @@ def renormalise(p, sel, scope=0):
 
     scope 0: p~_{t,g,e} = p_{t,g,e} / sum_{g'} sum_{e' in S_{t,g'}} p_{t,g',e'}
     scope 1: the same sum restricted to the token's own group g.
+    scope 2: no renormalisation, p~ = p (ablation variants).
     Returns float64 [N, G, k] aligned with ``sel``.
     """
     psel = np.take_along_axis(p, sel.astype(np.int64), axis=-1)
+    if scope == 2:
+        return psel.copy()
     if scope == 0:
         den = psel.sum(axis=(1, 2), keepdims=True)
     else:
@@ -256,20 +265,28 @@ def combine(o_routed, o_sh, w, dims):
     h_route = sum_g sum_{e in S} p~_{t,g,e} o_{t,g,e}  ([SN] §3-2 4));
     h_shared = the shared head's output ([SN] §3-2 5)).
     o_routed [B, G, T, k, d] (or decode [B, G, k, d] with T=1), w [N, G, k]
-    -> h [N, (k*G + 1 + n_shared) * d].
+    -> h [N, slots * d], slots = k*G + 1 + n_shared.
+
+    output_mode 1 ([SN] §5-1, "hard concat only"): h = [h_hard, h_shared];
+    output_mode 2 ([SN] §5-1, "weighted concat, no renormalised slot"):
+    h = [w_{t,g,e} o_{t,g,e} slot by slot, h_shared].
     """
     B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
+    mode = getattr(dims, "output_mode", 0)
     o = f64(o_routed).reshape(B, G, T, k, d).transpose(0, 2, 1, 3, 4).reshape(B * T, G, k, d)
-    hard = o.reshape(B * T, G * k * d)
-    route = np.einsum("ngk,ngkd->nd", f64(w), o)
-    parts = [hard, route]
+    if mode == 2:
+        parts = [(f64(w)[..., None] * o).reshape(B * T, G * k * d)]
+    else:
+        parts = [o.reshape(B * T, G * k * d)]
+    if mode == 0:
+        parts.append(np.einsum("ngk,ngkd->nd", f64(w), o))
     if dims.n_shared:
         parts.append(f64(o_sh).reshape(B * T, d))
     return np.concatenate(parts, axis=1)
 
 
 def out_proj(h, Wo):
-    """y = h Wo^T over the k*G + 2 slots ([SN] §3-2 7))."""
+    """y = h Wo^T over the slots of h ([SN] §3-2 7))."""
     return linear(h, Wo)
 
 

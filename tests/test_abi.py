@@ -53,9 +53,21 @@ def test_bad_shared_group_and_scope():
     with pytest.raises(gq.GQEError):
         gq.gqe_workspace_size(gq.make_dims(_cfg(), shared_kv_group=2), 1)
     with pytest.raises(gq.GQEError):
-        gq.gqe_workspace_size(gq.make_dims(_cfg(), renorm_scope=2), 1)
+        gq.gqe_workspace_size(gq.make_dims(_cfg(), renorm_scope=3), 1)
+    with pytest.raises(gq.GQEError):
+        gq.gqe_workspace_size(gq.make_dims(_cfg(), output_mode=3), 1)
+    with pytest.raises(gq.GQEError):
+        gq.gqe_workspace_size(gq.make_dims(_cfg(), output_mode=-1), 1)
     with pytest.raises(gq.GQEError):
         gq.gqe_workspace_size(gq.make_dims(_cfg(), scale=-1.0), 1)
+
+
+def test_output_mode_changes_the_fused_projection_scratch():
+    base = _cfg(B=2, T=256, D=256, G=4, E=2, k=1)
+    sizes = [gq.gqe_workspace_size(gq.make_dims(base, output_mode=m), gq.GQE_OP_COMBINE_OUT_PROJ) for m in range(3)]
+    # h has k*G + 1 + n_shared slots in mode 0 and one fewer in the ablation modes
+    assert sizes[0] == 512 * (4 + 1 + 1) * 64 * 2
+    assert sizes[1] == sizes[2] == 512 * (4 + 1) * 64 * 2
 
 
 def test_workspace_sizes():

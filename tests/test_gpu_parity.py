@@ -50,6 +50,8 @@ ROUTER_CASES = {
     "main": (gi.WORKLOADS["main_prefill"], None),
     "long": (gi.WORKLOADS["long_prefill"], None),
     "wide_skewed": (gi.WORKLOADS["wide_skewed_prefill"], None),
+    "no_renorm": (gi.Workload("n0", D(B=1, T=90, D=128, G=2, E=4, k=2, renorm_scope=2)), None),
+    "tc_no_renorm": (gi.Workload("n1", D(B=1, T=1500, D=128, G=8, E=2, k=1, renorm_scope=2)), None),
     # 1024 tokens and more take the tcgen05 router: generic E, group scope, ragged last tile
     "tc_E3_group_scope": (gi.Workload("t3", D(B=2, T=640, D=256, G=5, E=3, k=2, renorm_scope=1)), None),
     "tc_E8_k4_ragged": (gi.Workload("t8", D(B=1, T=1100, D=192, G=4, E=8, k=4)), None),
@@ -395,6 +397,38 @@ def test_combine_out_proj(dims):
     assert torch.equal(y, y2)
 
 
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("dims", [D(B=2, T=33, G=3, E=4, k=2, d=128), D(B=1, T=256, G=4, E=2, k=1, n_shared=0),
+                                  D(B=1, T=2048, D=512, G=4, E=2, k=1)],
+                         ids=["k2_d128", "no_shared_T256", "T2048_direct"])
+def test_output_modes(dims, mode):
+    """The ablation output constructions: h from gqe_combine and y from
+    gqe_combine_out_proj (which reads the hard slots in place for mode 1 when
+    T % 128 == 0) against the oracle."""
+    dims = dims.replace(output_mode=mode)
+    B, G, T, k, d = dims.B, dims.G, dims.T, dims.k, dims.d
+    o = gi.normal_bf16(13, "o", (B, G, T, k, d))
+    osh = gi.normal_bf16(13, "osh", (B, T, d))
+    w = gi.random_weights_simplex(dims, 13)
+    dc = dims_c(dims)
+    wt = torch.from_numpy(w).cuda()
+    osh_d = bf16_dev(osh) if dims.n_shared else None
+    h = torch.full((dims.N, dims.slots * d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gq.gqe_combine(dc, bf16_dev(o), osh_d, wt, h)
+    Wo = gi.normal_bf16(13, "Wo", (dims.D, dims.slots * d), 0.02)
+    y = torch.full((dims.N, dims.D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_COMBINE_OUT_PROJ),), dtype=torch.uint8, device="cuda")
+    gq.gqe_combine_out_proj(dc, bf16_dev(o), osh_d, wt, bf16_dev(Wo), y, ws)
+    torch.cuda.synchronize()
+    h_ref = orc.combine(o, osh, w.astype(np.float64), dims)
+    got = to_f64(h)
+    if mode == 1:
+        assert np.array_equal(got, h_ref)                  # copies: exact
+    else:
+        np.testing.assert_allclose(got, h_ref, rtol=2 ** -8, atol=1e-6)
+    assert_close_attn(to_f64(y), orc.out_proj(h_ref, Wo), "y")
+
+
 # ----------------------------------------------------------------------------
 # whole layer
 
@@ -441,6 +475,23 @@ def test_layer_dense_gqa_mode():
     assert np.array_equal(inter["idx"].cpu().numpy(), np.broadcast_to(np.arange(2), (dims.N, 4, 2)))
     assert_close_attn(to_f64(y).reshape(dims.N, -1), ref["y"], "y")
     assert_close_attn(to_f64(inter["h"]), ref["h"], "h")
+
+
+@pytest.mark.parametrize("mode,scope", [(1, 0), (2, 2)], ids=["hard_concat", "weighted_concat_no_renorm"])
+def test_layer_ablation_modes(mode, scope):
+    """The two ablation layers of the accuracy table end to end."""
+    dims = D(B=2, T=256, D=256, G=4, E=2, k=1, n_shared=0, renorm_scope=scope, output_mode=mode)
+    w = gi.Workload("ablation", dims)
+    dims, x, Wt, bias, layer = _layer(w, seed=9)
+    y, inter = layer.forward(bf16_dev(x), keep=True)
+    torch.cuda.synchronize()
+    ref = orc.gqe_forward(x, Wt, dims, bias)
+    r = ref["router"]
+    tie_tok = (r["margin"] < NEAR_TIE).any(axis=1)
+    agree = np.all(inter["idx"].cpu().numpy() == r["idx"], axis=(1, 2))
+    assert np.all(agree | tie_tok)
+    assert_close_attn(to_f64(y).reshape(dims.N, -1)[agree], ref["y"][agree], "y")
+    assert_close_attn(to_f64(inter["h"])[agree], ref["h"][agree], "h")
 
 
 def test_layer_decode_step_end_to_end():

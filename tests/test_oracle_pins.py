@@ -398,3 +398,75 @@ def test_skewed_router_bias_realises_expert0_share():
     in_topk = float((r["idx"] == 0).any(-1).mean())
     assert 0.7 < frac0 < 0.9
     assert in_topk > 0.95
+
+
+# ----------------------------------------------------------------------------
+# output-construction variants ("GQE" study note §5-1, ablation rows) and the
+# un-renormalised router weights
+
+
+def _brute_force_h(o, osh, w, dims):
+    """h token by token and slot by slot with plain Python loops."""
+    B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
+    rows = []
+    for b in range(B):
+        for t in range(T):
+            row = []
+            route = [0.0] * d
+            for g in range(G):
+                for j in range(k):
+                    v = [float(gi.bf16_bits_to_f32(o[b, g, t, j, c:c + 1])[0]) for c in range(d)]
+                    wt = float(w[b * T + t, g, j])
+                    row += [wt * x for x in v] if dims.output_mode == 2 else v
+                    route = [r + wt * x for r, x in zip(route, v)]
+            if dims.output_mode == 0:
+                row += route
+            if dims.n_shared:
+                row += [float(gi.bf16_bits_to_f32(osh[b, t, c:c + 1])[0]) for c in range(d)]
+            rows.append(row)
+    return np.array(rows)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("n_shared", [0, 1])
+def test_output_modes_match_brute_force(mode, n_shared):
+    dims = gi.GQEDims(B=2, T=3, D=64, G=3, E=3, k=2, d=4, n_shared=n_shared, output_mode=mode)
+    o = gi.normal_bf16(21, "o", (dims.B, dims.G, dims.T, dims.k, dims.d))
+    osh = gi.normal_bf16(21, "osh", (dims.B, dims.T, dims.d))
+    w = gi.random_weights_simplex(dims, 21).astype(np.float64)
+    h = orc.combine(o, osh, w, dims)
+    assert h.shape == (dims.N, dims.slots * dims.d)
+    np.testing.assert_allclose(h, _brute_force_h(o, osh, w, dims), rtol=0, atol=1e-12)
+
+
+def test_weighted_concat_slots_sum_to_the_weighted_sum_slot():
+    """Mode 2's weighted hard slots, added over the slots, give mode 0's
+    weighted-sum slot; mode 1's h is mode 0's without that slot."""
+    base = gi.GQEDims(B=1, T=5, D=64, G=4, E=2, k=1, d=8, n_shared=1)
+    o = gi.normal_bf16(22, "o", (1, 4, 5, 1, 8))
+    osh = gi.normal_bf16(22, "osh", (1, 5, 8))
+    w = gi.random_weights_simplex(base, 22).astype(np.float64)
+    h0 = orc.combine(o, osh, w, base)
+    h1 = orc.combine(o, osh, w, base.replace(output_mode=1))
+    h2 = orc.combine(o, osh, w, base.replace(output_mode=2))
+    G, k, d = 4, 1, 8
+    route = h0[:, G * k * d:(G * k + 1) * d]
+    np.testing.assert_allclose(h2[:, :G * k * d].reshape(5, G * k, d).sum(axis=1), route, atol=1e-12)
+    np.testing.assert_array_equal(h1, np.delete(h0, np.s_[G * k * d:(G * k + 1) * d], axis=1))
+    np.testing.assert_array_equal(h1[:, -d:], h2[:, -d:])
+
+
+def test_renorm_scope_none_keeps_group_softmax_probabilities():
+    rng = np.random.default_rng(23)
+    x = gi.f32_to_bf16_bits(rng.normal(size=(6, 32)).astype(np.float32))
+    Wr = gi.f32_to_bf16_bits(rng.normal(size=(32, 8), scale=0.3).astype(np.float32))
+    r = orc.router_topk(orc.f64(x), Wr, 2, 4, 2, None, 2)
+    xs, W = orc.f64(x), orc.f64(Wr)
+    for t in range(6):
+        for g in range(2):
+            s = xs[t] @ W[:, g * 4:(g + 1) * 4]
+            p = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
+            np.testing.assert_allclose(r["w"][t, g], p[r["idx"][t, g]], rtol=1e-12)
+    # a single expert per group: the weight is exactly 1
+    r1 = orc.router_topk(orc.f64(x), Wr[:, :2], 2, 1, 1, None, 2)
+    assert np.all(r1["w"] == 1.0)
