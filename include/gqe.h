@@ -89,6 +89,20 @@ gqe_status gqe_router_topk(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf
                            const float* bias, int32_t* topk_idx, float* topk_w, float* probs,
                            gqe_stream stream);
 
+/* Router statistics for collapse monitoring and a load-balancing loss
+ * ("GQE" study note §4-3 routing auxiliary loss, §4-4 "router collapse
+ * should be monitored"; ai-feeds summary, 局限: a loss on the tokens'
+ * allocation proportions).  The loss itself is not specified by the pages;
+ * this returns its inputs, per (group g, expert e), s = g*E + e:
+ *   counts[s]   tokens whose selection in group g includes e   (int32 [G*E])
+ *   prob_sum[s] sum over tokens of the in-group probability p (fp32 [G*E])
+ * from probs [B*T, G, E] fp32 and topk_idx [B*T, G, k] int32 as
+ * gqe_router_topk writes them.  Fractions and means are these over B*T.
+ * The outputs are zeroed and accumulated on `stream` (fp32 sums in an order
+ * that may differ between runs).  Errors: GQE_ERR_INVALID_ARG. */
+gqe_status gqe_router_stats(const gqe_dims* dims, const float* probs, const int32_t* topk_idx,
+                            int32_t* counts, float* prob_sum, gqe_stream stream);
+
 /* Routed and shared query projection: "GQE" study note §3-2 2) (only the
  * selected experts compute their query) and 5) (shared head); ai-feeds
  * summary, 方法 (unselected query heads are skipped).

@@ -58,6 +58,7 @@ _D = ctypes.POINTER(gqe_dims)
 SIGNATURES = {
     "gqe_workspace_size": [_D, _I, _I, ctypes.POINTER(_SZ)],
     "gqe_router_topk": [_D, _P, _P, _P, _P, _P, _P, _P],
+    "gqe_router_stats": [_D, _P, _P, _P, _P, _P],
     "gqe_routed_qproj": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "gqe_kv_proj": [_D, _P, _P, _P, _P, _P, _P],
     "gqe_kv_append": [_D, _P, _P, _P, _P, _P, _I, _P, _P],
@@ -148,6 +149,13 @@ def gqe_router_topk(dims, x, Wr, bias, topk_idx, topk_w, probs=None, stream=None
         _ptr(bias, "bias", torch.float32, optional=True), _ptr(topk_idx, "topk_idx", torch.int32),
         _ptr(topk_w, "topk_w", torch.float32), _ptr(probs, "probs", torch.float32, optional=True),
         _stream(stream)))
+
+
+def gqe_router_stats(dims, probs, topk_idx, counts, prob_sum, stream=None):
+    import torch
+    _check("gqe_router_stats", lib.gqe_router_stats(
+        ctypes.byref(dims), _ptr(probs, "probs", torch.float32), _ptr(topk_idx, "topk_idx", torch.int32),
+        _ptr(counts, "counts", torch.int32), _ptr(prob_sum, "prob_sum", torch.float32), _stream(stream)))
 
 
 def gqe_routed_qproj(dims, x, Wq, Wsh, topk_idx, q_routed, q_sh, ws, expert_counts=None, stream=None):

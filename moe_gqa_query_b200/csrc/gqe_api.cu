@@ -270,6 +270,14 @@ gqe_status gqe_router_topk(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf
   return cuda_status(launch_router(p, S(stream)));
 }
 
+gqe_status gqe_router_stats(const gqe_dims* dims, const float* probs, const int32_t* topk_idx, int32_t* counts,
+                            float* prob_sum, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(probs && topk_idx && counts && prob_sum, GQE_ERR_INVALID_ARG);
+  return cuda_status(launch_router_stats(probs, topk_idx, dims->B * dims->T, dims->G, dims->E, dims->k, counts,
+                                         prob_sum, S(stream)));
+}
+
 gqe_status gqe_routed_qproj(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16* Wq, const gqe_bf16* Wsh,
                             const int32_t* topk_idx, gqe_bf16* q_routed, gqe_bf16* q_sh, int32_t* expert_counts,
                             void* ws, size_t ws_bytes, gqe_stream stream) {

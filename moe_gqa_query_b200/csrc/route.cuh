@@ -34,6 +34,9 @@ PermLayout perm_layout(int N, int G, int E, int k);
 cudaError_t launch_permutation(const int* topk_idx, int N, int T, int G, int E, int k, void* ws,
                                const PermLayout& L, cudaStream_t stream);
 
+cudaError_t launch_router_stats(const float* probs, const int* topk_idx, int N, int G, int E, int k,
+                                int* counts, float* prob_sum, cudaStream_t stream);
+
 struct CombineParams {
   const uint16_t* o_routed;   // [B, G, T, k, d]
   const uint16_t* o_sh;       // [B, T, d]

@@ -805,6 +805,50 @@ cudaError_t launch_router_tc(const CUtensorMap& mapX, const RouterParams& p, cud
   return launch_router_tc_gep<64>(mapX, p, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Router statistics: one thread per token adds its selections and in-group
+// probabilities into shared-memory totals per (group, expert); each block then
+// adds its totals into the outputs.
+namespace {
+__global__ void __launch_bounds__(256) router_stats_kernel(const float* __restrict__ probs,
+                                                           const int* __restrict__ idx, int N, int G, int E,
+                                                           int k, int* counts, float* prob_sum) {
+  __shared__ int c_s[64];
+  __shared__ float p_s[64];
+  const int GE = G * E;
+  for (int i = threadIdx.x; i < GE; i += blockDim.x) {
+    c_s[i] = 0;
+    p_s[i] = 0.f;
+  }
+  pdl_launch_dependents();
+  pdl_wait();
+  __syncthreads();
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n < N) {
+    for (int s = 0; s < GE; ++s) atomicAdd(&p_s[s], probs[(size_t)n * GE + s]);
+    for (int g = 0; g < G; ++g)
+      for (int j = 0; j < k; ++j) {
+        const int e = idx[((size_t)n * G + g) * k + j];
+        if (e >= 0 && e < E) atomicAdd(&c_s[g * E + e], 1);
+      }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < GE; i += blockDim.x) {
+    if (c_s[i]) atomicAdd(&counts[i], c_s[i]);
+    atomicAdd(&prob_sum[i], p_s[i]);
+  }
+}
+}  // namespace
+
+cudaError_t launch_router_stats(const float* probs, const int* topk_idx, int N, int G, int E, int k,
+                                int* counts, float* prob_sum, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int) * G * E, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(prob_sum, 0, sizeof(float) * G * E, stream);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(router_stats_kernel, dim3((N + 255) / 256), dim3(256), 0, stream, 1, probs, topk_idx, N, G,
+                       E, k, counts, prob_sum);
+}
+
 cudaError_t launch_router(const RouterParams& p, cudaStream_t stream) {
   const int GE = p.G * p.E;
   if (GE <= 16) return launch_router_gep<16>(p, stream);

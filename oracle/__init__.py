@@ -5,6 +5,6 @@ import this package; the product path never does.
 """
 from .gqe_oracle import (  # noqa: F401
     f64, router_logits, group_softmax, topk_select, selection_margin, renormalise,
-    router_topk, linear, routed_qproj, kv_proj, causal_attention, attn_prefill,
+    router_topk, router_stats, linear, routed_qproj, kv_proj, causal_attention, attn_prefill,
     attn_decode, combine, out_proj, gqe_forward, decode_step, near_tie_alternatives,
 )

@@ -140,6 +140,20 @@ def linear(x, W):
     return f64(x) @ f64(W).T
 
 
+def router_stats(probs, idx, G, E):
+    """Per (group, expert): tokens that selected it and the sum of its in-group
+    probability over the tokens ([SN] §4-3, §4-4: load balance and collapse
+    monitoring; the loss built from them is not given).  probs [N, G, E],
+    idx [N, G, k] -> (counts int64 [G*E], prob_sum float64 [G*E])."""
+    N = probs.shape[0]
+    counts = np.zeros(G * E, dtype=np.int64)
+    for g in range(G):
+        for e in range(E):
+            counts[g * E + e] = int(np.sum(idx[:, g, :] == e))
+    prob_sum = np.asarray(probs, dtype=np.float64).reshape(N, G * E).sum(axis=0)
+    return counts, prob_sum
+
+
 def routed_qproj(x, Wq, Wsh, idx, dims):
     """q_{t,g,e} = x_t Wq[g,e]^T for e in S_{t,g} only; q_sh = x_t Wsh^T.
 

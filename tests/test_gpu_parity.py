@@ -87,6 +87,32 @@ def check_router(w: gi.Workload, seed=0):
     return int(tie.sum())
 
 
+@pytest.mark.parametrize("wname", ["main_prefill", "wide_skewed_prefill"])
+def test_router_stats(wname):
+    """Per-(group, expert) selection counts (exact) and probability sums
+    against the oracle; the skewed workload's expert-0 share shows in both."""
+    w = gi.WORKLOADS[wname]
+    dims = w.dims
+    x = gi.layer_input(dims, 0)
+    Wt = gi.layer_weights(dims, 0)
+    bias = gi.router_bias(w, 0)
+    N, G, E, k = dims.N, dims.G, dims.E, dims.k
+    idx = torch.empty((N, G, k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((N, G, k), dtype=torch.float32, device="cuda")
+    probs = torch.empty((N, G, E), dtype=torch.float32, device="cuda")
+    dc = dims_c(dims)
+    gq.gqe_router_topk(dc, bf16_dev(x), bf16_dev(Wt["Wr"]), None if bias is None else torch.from_numpy(bias).cuda(),
+                       idx, wt, probs)
+    counts = torch.full((G * E,), -1, dtype=torch.int32, device="cuda")
+    psum = torch.full((G * E,), float("nan"), dtype=torch.float32, device="cuda")
+    gq.gqe_router_stats(dc, probs, idx, counts, psum)
+    torch.cuda.synchronize()
+    c_ref, p_ref = orc.router_stats(probs.cpu().numpy(), idx.cpu().numpy(), G, E)
+    np.testing.assert_array_equal(counts.cpu().numpy(), c_ref)
+    np.testing.assert_allclose(psum.cpu().numpy(), p_ref, rtol=1e-4)
+    assert np.all(counts.cpu().numpy().reshape(G, E).sum(axis=1) == N * k)
+
+
 @pytest.mark.parametrize("case", list(ROUTER_CASES))
 def test_router_topk(case):
     w, _ = ROUTER_CASES[case]

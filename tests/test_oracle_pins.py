@@ -470,3 +470,23 @@ def test_renorm_scope_none_keeps_group_softmax_probabilities():
     # a single expert per group: the weight is exactly 1
     r1 = orc.router_topk(orc.f64(x), Wr[:, :2], 2, 1, 1, None, 2)
     assert np.all(r1["w"] == 1.0)
+
+
+def test_router_stats_closed_forms_and_brute_force():
+    """Per group the selection counts add to N*k and the probability sums to N
+    (each token's in-group probabilities add to 1); counts match a loop."""
+    rng = np.random.default_rng(24)
+    N, G, E, k, D = 40, 3, 4, 2, 32
+    x = gi.f32_to_bf16_bits(rng.normal(size=(N, D)).astype(np.float32))
+    Wr = gi.f32_to_bf16_bits(rng.normal(size=(D, G * E), scale=0.3).astype(np.float32))
+    r = orc.router_topk(orc.f64(x), Wr, G, E, k)
+    counts, psum = orc.router_stats(r["probs"], r["idx"], G, E)
+    for g in range(G):
+        assert counts[g * E:(g + 1) * E].sum() == N * k
+        assert abs(psum[g * E:(g + 1) * E].sum() - N) < 1e-9
+    loop = np.zeros(G * E, dtype=np.int64)
+    for t in range(N):
+        for g in range(G):
+            for e in r["idx"][t, g]:
+                loop[g * E + int(e)] += 1
+    np.testing.assert_array_equal(counts, loop)
