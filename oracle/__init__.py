@@ -1,4 +1,4 @@
-"""fp64 CPU oracle of the GQE attention forward (test infrastructure only).
+"""fp64 CPU oracle of the GQE attention forward and backward (test infrastructure only).
 
 Only the test suite, the smoke check and the benchmark's CPU-baseline leg may
 import this package; the product path never does.
@@ -8,3 +8,4 @@ from .gqe_oracle import (  # noqa: F401
     router_topk, router_stats, linear, routed_qproj, kv_proj, causal_attention, attn_prefill,
     attn_decode, combine, out_proj, gqe_forward, decode_step, near_tie_alternatives,
 )
+from . import gqe_backward  # noqa: F401,E402
