@@ -279,6 +279,17 @@ def run_kernel(args):
             o, os_ = torch.empty_like(q), torch.empty_like(qs)
             fn = lambda: gq.gqe_attn_prefill(dc, q, qs, K, V, o, os_, None)  # noqa: E731
             work = dict(flops=attn_useful_flops(dims))
+        elif args.kernel == "attn_bwd":
+            q, qs, K, V = rn(B, G, T, k, d), rn(B, T, d), rn(B, G, T, d), rn(B, G, T, d)
+            o, os_ = torch.empty_like(q), torch.empty_like(qs)
+            lse = torch.empty((B * G * T * k + B * T * dims.n_shared,), dtype=torch.float32, device=device)
+            gq.gqe_attn_prefill(dc, q, qs, K, V, o, os_, lse)
+            dO, dOs = rn(B, G, T, k, d), rn(B, T, d)
+            dq, dqs, dK, dV = torch.empty_like(q), torch.empty_like(qs), torch.empty_like(K), torch.empty_like(V)
+            ws = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_ATTN_BWD),), dtype=torch.uint8, device=device)
+            fn = lambda: gq.gqe_attn_prefill_bwd(dc, q, qs, K, V, o, os_, lse, dO, dOs, dq, dqs, dK, dV, ws)  # noqa
+            # five products per (query tile, key tile) against the forward's two
+            work = dict(flops=2.5 * attn_useful_flops(dims))
         elif args.kernel in ("router", "qproj", "kv", "linear", "combine", "combine_out"):
             x = rn(B, T, D)
             Wt = gi.layer_weights(dims)

@@ -25,7 +25,8 @@ import numpy as np
 
 # tensor ids for the seeded streams
 TID = dict(x=1, Wr=2, Wq=3, Wk=4, Wv=5, Wsh=6, Wo=7, bias=8, Kc=9, Vc=10,
-           route=11, q=12, K=13, V=14, qsh=15, o=16, osh=17, w=18, xdec=19)
+           route=11, q=12, K=13, V=14, qsh=15, o=16, osh=17, w=18, xdec=19,
+           do=20, dosh=21, dy=22, dh=23, dw=24)
 
 WEIGHT_STD = 0.02
 

@@ -70,7 +70,7 @@ typedef struct {
   int output_mode;       /* 0 GQE, 1 hard concat only, 2 weighted concat */
 } gqe_dims;
 
-enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3 };
+enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3, GQE_OP_ATTN_BWD = 4 };
 
 /* Bytes of scratch the call `op` needs for these dims (L_max: the decode
  * cache length, used by GQE_OP_ATTN_DECODE only).  Returns
@@ -142,6 +142,25 @@ gqe_status gqe_kv_append(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf16
 gqe_status gqe_attn_prefill(const gqe_dims* dims, const gqe_bf16* q_routed,
                             const gqe_bf16* q_sh, const gqe_bf16* K, const gqe_bf16* V,
                             gqe_bf16* o_routed, gqe_bf16* o_sh, float* lse, gqe_stream stream);
+
+/* Backward of gqe_attn_prefill ("GQE" study note §1-1 attention equation,
+ * differentiated; §3-2 2) and 5): the gradients of every selected expert's
+ * rows and of the shared head's rows flow into the K/V of the group they
+ * read).  With P the causal softmax and Delta_r = sum_c dO_rc O_rc:
+ *   dV = P^T dO,  dS = scale * P o (dO V^T - Delta),  dK = dS^T q,  dq = dS K.
+ *   q_routed, q_sh, K, V: the forward's inputs; o_routed, o_sh: its outputs;
+ *   lse: its fp32 LSE output (required here; the layout gqe_attn_prefill
+ *   writes).  do_routed [B, G, T, k, d], do_sh [B, T, d]: upstream gradients.
+ *   dq_routed, dq_sh (shapes of q), dK, dV [B, G, T, d]: bf16 outputs,
+ *   overwritten.  fp32 accumulation; dq is summed over key tiles in an fp32
+ *   workspace, in an order that may differ between runs.
+ *   ws: scratch of gqe_workspace_size(GQE_OP_ATTN_BWD) bytes, 256-byte
+ *   aligned.  d_head 64 only (GQE_ERR_UNSUPPORTED otherwise). */
+gqe_status gqe_attn_prefill_bwd(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh,
+                                const gqe_bf16* K, const gqe_bf16* V, const gqe_bf16* o_routed,
+                                const gqe_bf16* o_sh, const float* lse, const gqe_bf16* do_routed,
+                                const gqe_bf16* do_sh, gqe_bf16* dq_routed, gqe_bf16* dq_sh, gqe_bf16* dK,
+                                gqe_bf16* dV, void* ws, size_t ws_bytes, gqe_stream stream);
 
 /* Decode attention: one new token per sequence (dims->T must be 1) against a
  * dense cache (freeguideonline GQA tutorial, "自回归推理中的内存带宽优势": a

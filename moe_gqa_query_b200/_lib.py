@@ -21,6 +21,7 @@ GQE_OK = 0
 GQE_OP_ROUTED_QPROJ = 1
 GQE_OP_ATTN_DECODE = 2
 GQE_OP_COMBINE_OUT_PROJ = 3
+GQE_OP_ATTN_BWD = 4
 STATUS_NAMES = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED",
                 3: "GQE_ERR_WORKSPACE", 4: "GQE_ERR_CUDA", 5: "GQE_ERR_DEVICE_CHECK"}
 
@@ -63,6 +64,7 @@ SIGNATURES = {
     "gqe_kv_proj": [_D, _P, _P, _P, _P, _P, _P],
     "gqe_kv_append": [_D, _P, _P, _P, _P, _P, _I, _P, _P],
     "gqe_attn_prefill": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
+    "gqe_attn_prefill_bwd": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "gqe_attn_decode": [_D, _P, _P, _P, _P, _I, _P, _P, _P, _P, _SZ, _P],
     "gqe_attn_decode_noalloc": [_D, _P, _P, _P, _P, _I, _P, _P, _P, _P],
     "gqe_combine": [_D, _P, _P, _P, _P, _P],
@@ -193,6 +195,19 @@ def gqe_attn_prefill(dims, q_routed, q_sh, K, V, o_routed, o_sh, lse=None, strea
         _ptr(K, "K", b), _ptr(V, "V", b), _ptr(o_routed, "o_routed", b),
         _ptr(o_sh, "o_sh", b, optional=True), _ptr(lse, "lse", torch.float32, optional=True),
         _stream(stream)))
+
+
+def gqe_attn_prefill_bwd(dims, q_routed, q_sh, K, V, o_routed, o_sh, lse, do_routed, do_sh,
+                         dq_routed, dq_sh, dK, dV, ws, stream=None):
+    import torch
+    b = _bf16()
+    ws_bytes = ws.numel() * ws.element_size()
+    _check("gqe_attn_prefill_bwd", lib.gqe_attn_prefill_bwd(
+        ctypes.byref(dims), _ptr(q_routed, "q_routed", b), _ptr(q_sh, "q_sh", b, optional=True),
+        _ptr(K, "K", b), _ptr(V, "V", b), _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True),
+        _ptr(lse, "lse", torch.float32), _ptr(do_routed, "do_routed", b), _ptr(do_sh, "do_sh", b, optional=True),
+        _ptr(dq_routed, "dq_routed", b), _ptr(dq_sh, "dq_sh", b, optional=True), _ptr(dK, "dK", b),
+        _ptr(dV, "dV", b), _ptr(ws, "ws"), ws_bytes, _stream(stream)))
 
 
 def gqe_attn_decode(dims, q_routed, q_sh, Kc, Vc, L_max, cache_len, o_routed, o_sh, ws, stream=None):

@@ -47,10 +47,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
+// Tensor map (bf16 unless `f32`), 128-byte swizzle, zero fill out of bounds.
 // dims/box innermost first; strides in bytes for dims 1..rank-1.
 bool encode_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
-                const uint32_t* box) {
+                const uint32_t* box, bool f32 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -62,7 +62,7 @@ bool encode_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
   memset(m, 0, sizeof(*m));
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), gd, gs, bx, es,
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -73,15 +73,17 @@ bool encode_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
 struct MapKey {
   const void* ptr;
   int rank;
+  bool f32;
   uint64_t dims[3];
   uint32_t box[3];
   bool operator==(const MapKey& o) const {
-    return ptr == o.ptr && rank == o.rank && !memcmp(dims, o.dims, sizeof(dims)) && !memcmp(box, o.box, sizeof(box));
+    return ptr == o.ptr && rank == o.rank && f32 == o.f32 && !memcmp(dims, o.dims, sizeof(dims)) &&
+           !memcmp(box, o.box, sizeof(box));
   }
 };
 
 bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
-              const uint32_t* box) {
+              const uint32_t* box, bool f32 = false) {
   constexpr int kSlots = 256;
   static MapKey keys[kSlots];
   static CUtensorMap maps[kSlots];
@@ -90,11 +92,12 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, c
   MapKey k{};
   k.ptr = ptr;
   k.rank = rank;
+  k.f32 = f32;
   for (int i = 0; i < rank && i < 3; ++i) {
     k.dims[i] = dims[i];
     k.box[i] = box[i];
   }
-  uint64_t h = reinterpret_cast<uintptr_t>(ptr) * 0x9E3779B97F4A7C15ull;
+  uint64_t h = (reinterpret_cast<uintptr_t>(ptr) + (f32 ? 1 : 0)) * 0x9E3779B97F4A7C15ull;
   for (int i = 0; i < 3; ++i) h = (h ^ (k.dims[i] + 0x632BE5ABull * k.box[i])) * 0x100000001B3ull;
   const int slot = (int)(h >> 56);
   {
@@ -104,12 +107,20 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, c
       return true;
     }
   }
-  if (!encode_map(m, ptr, rank, dims, strides, box)) return false;
+  if (!encode_map(m, ptr, rank, dims, strides, box, f32)) return false;
   std::lock_guard<std::mutex> lock(mu);
   keys[slot] = k;
   maps[slot] = *m;
   used[slot] = true;
   return true;
+}
+
+// fp32 [rows, cols], box 32 cols (128 bytes) x box_rows rows
+bool map2d_f32(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t strides[1] = {cols * 4};
+  const uint32_t box[2] = {32, box_rows};
+  return make_map(m, ptr, 2, dims, strides, box, true);
 }
 
 bool map2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
@@ -231,6 +242,12 @@ gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* b
   if (op == GQE_OP_COMBINE_OUT_PROJ) {
     const size_t slots = (size_t)dims->k * dims->G + (dims->output_mode == 0 ? 1 : 0) + dims->n_shared;
     *bytes = (size_t)N * slots * dims->d_head * 2;
+    return GQE_OK;
+  }
+  if (op == GQE_OP_ATTN_BWD) {
+    AttnBwdLayout L;
+    attn_bwd_layout(dims->B, dims->T, dims->G, dims->k, dims->n_shared, dims->d_head, &L);
+    *bytes = L.bytes;
     return GQE_OK;
   }
   if (op == GQE_OP_ATTN_DECODE) {
@@ -420,6 +437,69 @@ gqe_status gqe_attn_prefill(const gqe_dims* dims, const gqe_bf16* q_routed, cons
   p.scale_log2 = scale_log2(dims);
   p.err = error_word();
   return cuda_status(launch_attn_prefill(mQ, mQs, mK, mV, p, d, S(stream)));
+}
+
+gqe_status gqe_attn_prefill_bwd(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh,
+                                const gqe_bf16* K, const gqe_bf16* V, const gqe_bf16* o_routed,
+                                const gqe_bf16* o_sh, const float* lse, const gqe_bf16* do_routed,
+                                const gqe_bf16* do_sh, gqe_bf16* dq_routed, gqe_bf16* dq_sh, gqe_bf16* dK,
+                                gqe_bf16* dV, void* ws, size_t ws_bytes, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  if (dims->d_head != 64) return GQE_ERR_UNSUPPORTED;
+  GQE_REQUIRE(q_routed && K && V && o_routed && lse && do_routed && dq_routed && dK && dV, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || (q_sh && o_sh && do_sh && dq_sh), GQE_ERR_INVALID_ARG);
+  const void* ptrs[] = {q_routed, K, V, o_routed, do_routed, dq_routed, dK, dV, lse};
+  for (const void* q : ptrs) GQE_REQUIRE(aligned16(q), GQE_ERR_INVALID_ARG);
+  if (dims->n_shared) {
+    const void* sp[] = {q_sh, o_sh, do_sh, dq_sh};
+    for (const void* q : sp) GQE_REQUIRE(aligned16(q), GQE_ERR_INVALID_ARG);
+  }
+  const int B = dims->B, T = dims->T, G = dims->G, k = dims->k, d = dims->d_head;
+  AttnBwdLayout L;
+  attn_bwd_layout(B, T, G, k, dims->n_shared, d, &L);
+  GQE_REQUIRE(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 && ws_bytes >= L.bytes, GQE_ERR_WORKSPACE);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  CUtensorMap mQ, mQs, mdO, mdOs, mK, mV, mdQ;
+  GQE_REQUIRE(map3d(&mQ, q_routed, d, (uint64_t)T * k, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map3d(&mdO, do_routed, d, (uint64_t)T * k, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  if (dims->n_shared) {
+    GQE_REQUIRE(map3d(&mQs, q_sh, d, T, B, 128), GQE_ERR_CUDA);
+    GQE_REQUIRE(map3d(&mdOs, do_sh, d, T, B, 128), GQE_ERR_CUDA);
+  } else {
+    mQs = mQ;
+    mdOs = mdO;
+  }
+  GQE_REQUIRE(map3d(&mK, K, d, T, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  GQE_REQUIRE(map3d(&mV, V, d, T, (uint64_t)B * G, 128), GQE_ERR_CUDA);
+  float* dq_acc = reinterpret_cast<float*>(w + L.off_dq);
+  GQE_REQUIRE(map2d_f32(&mdQ, dq_acc, d, (uint64_t)L.n_rows_pad, 32), GQE_ERR_CUDA);
+  AttnBwdParams p{};
+  p.lse = lse;
+  p.o_routed = o_routed;
+  p.o_sh = o_sh;
+  p.do_routed = do_routed;
+  p.do_sh = do_sh;
+  p.lse2 = reinterpret_cast<float*>(w + L.off_lse2);
+  p.delta = reinterpret_cast<float*>(w + L.off_delta);
+  p.dq_acc = dq_acc;
+  p.dq_routed = dq_routed;
+  p.dq_sh = dq_sh;
+  p.dK = dK;
+  p.dV = dV;
+  p.B = B;
+  p.T = T;
+  p.G = G;
+  p.k = k;
+  p.n_shared = dims->n_shared;
+  p.sg = dims->shared_kv_group;
+  p.d = d;
+  p.rows_pad = L.rows_pad;
+  p.rows_pad_sh = L.rows_pad_sh;
+  p.n_rows_pad = L.n_rows_pad;
+  p.scale_log2 = scale_log2(dims);
+  p.scale = p.scale_log2 / 1.4426950408889634f;
+  p.err = error_word();
+  return cuda_status(launch_attn_bwd(mQ, mQs, mdO, mdOs, mK, mV, mdQ, p, S(stream)));
 }
 
 gqe_status gqe_attn_decode(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh, const gqe_bf16* Kc,

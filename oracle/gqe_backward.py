@@ -15,11 +15,12 @@ where the pages leave the backward open:
     In output_mode 1 the router receives no gradient at all.
   * the shared head has no K/V of its own, so its dK/dV land in group sg.
 
-Pinned by tests/test_oracle_pins.py: central finite differences in fp64 of
-every forward step and of the whole layer (inputs chosen with TopK margins far
-above the step size, so the selection does not move), and closed forms
-(softmax and renormalisation gradients sum to zero; a constant upstream
-gradient gives dV = column sums of P).
+Pinned by tests/test_oracle_backward_pins.py: central finite differences in
+fp64 of every forward step and of the whole layer (inputs chosen with TopK
+margins far above the step size, so the selection does not move), torch
+autograd through a library attention, and closed forms (constant values give
+dq = dK = 0; in-group softmax gradients sum to zero; renormalisation is scale
+invariant; output_mode 1 gives the router nothing).
 """
 from __future__ import annotations
 
@@ -34,13 +35,17 @@ from .gqe_oracle import (
 # ----------------------------------------------------------------------------
 # attention: [SN] §1-1, o = softmax(q K^T * scale) V, causal
 
-def causal_attention_bwd(q, pos, K, V, dO, scale):
+def causal_attention_bwd(q, pos, K, V, dO, scale, O=None):
     """Gradients of o_r = sum_{j <= pos_r} P_rj V_j, P = softmax_j(q_r . K_j * scale).
 
     With S = q K^T * scale (masked to j <= pos_r) and P its row softmax:
       dV = P^T dO,   dP = dO V^T,
-      dS_rj = P_rj (dP_rj - sum_i P_ri dP_ri)          (softmax Jacobian),
+      dS_rj = P_rj (dP_rj - Delta_r)                    (softmax Jacobian),
+      Delta_r = sum_i P_ri dP_ri = dO_r . o_r,
       dq = scale * dS K,   dK = scale * dS^T q.
+    Delta is the first sum unless the forward output O is given, then the
+    second (identical for the exact O; a call that receives a rounded O
+    computes it from that O).
     q, dO [R, d]; pos [R]; K, V [L, d].  Returns dq [R, d], dK, dV [L, d].
     """
     q, K, V, dO = f64(q), f64(K), f64(V), f64(dO)
@@ -50,16 +55,67 @@ def causal_attention_bwd(q, pos, K, V, dO, scale):
     P = z / z.sum(axis=1, keepdims=True)
     dV = P.T @ dO
     dP = dO @ V.T
-    dS = P * (dP - np.sum(P * dP, axis=1, keepdims=True))
+    if O is None:
+        delta = np.sum(P * dP, axis=1, keepdims=True)
+    else:
+        delta = np.sum(dO * f64(O), axis=1, keepdims=True)
+    dS = P * (dP - delta)
     return scale * (dS @ K), scale * (dS.T @ q), dV
 
 
-def attn_prefill_bwd(q_routed, q_sh, K, V, do_routed, do_sh, dims):
+def causal_attention_bwd_magnitudes(q, pos, K, V, dO, scale, O=None):
+    """The absolute-value sums behind the rounding bound of causal_attention_bwd
+    computed with bf16 MMA operands: a sum of products whose factors are rounded
+    to bf16 (relative error <= 2^-8) errs by at most 2^-8 times the sum of the
+    products' magnitudes.  Returns |dS*scale| |K|, |dS*scale|^T |q|, |P|^T |dO|
+    (the magnitudes for dq, dK, dV)."""
+    q, K, V, dO = f64(q), f64(K), f64(V), f64(dO)
+    s = (q @ K.T) * scale
+    s[np.arange(K.shape[0])[None, :] > np.asarray(pos)[:, None]] = -np.inf
+    z = np.exp(s - s.max(axis=1, keepdims=True))
+    P = z / z.sum(axis=1, keepdims=True)
+    dP = dO @ V.T
+    delta = np.sum(P * dP, axis=1, keepdims=True) if O is None else np.sum(dO * f64(O), axis=1, keepdims=True)
+    aS = np.abs(scale * P * (dP - delta))
+    return aS @ np.abs(K), aS.T @ np.abs(q), P.T @ np.abs(dO)
+
+
+def attn_prefill_bwd_magnitudes(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_routed=None, o_sh=None):
+    """causal_attention_bwd_magnitudes laid out like attn_prefill_bwd's outputs."""
+    B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
+    sc = dims.sm_scale
+    pos = np.repeat(np.arange(T), k)
+    mq = np.empty((B, G, T, k, d))
+    mK = np.zeros((B, G, T, d))
+    mV = np.zeros((B, G, T, d))
+    for b in range(B):
+        for g in range(G):
+            o_rows = None if o_routed is None else np.asarray(o_routed[b, g]).reshape(T * k, d)
+            a, bk, bv = causal_attention_bwd_magnitudes(np.asarray(q_routed[b, g]).reshape(T * k, d), pos, K[b, g],
+                                                        V[b, g], np.asarray(do_routed[b, g]).reshape(T * k, d), sc,
+                                                        o_rows)
+            mq[b, g] = a.reshape(T, k, d)
+            mK[b, g] += bk
+            mV[b, g] += bv
+    mqs = None
+    if dims.n_shared:
+        mqs = np.empty((B, T, d))
+        for b in range(B):
+            a, bk, bv = causal_attention_bwd_magnitudes(q_sh[b], np.arange(T), K[b, dims.sg], V[b, dims.sg],
+                                                        do_sh[b], sc, None if o_sh is None else o_sh[b])
+            mqs[b] = a
+            mK[b, dims.sg] += bk
+            mV[b, dims.sg] += bv
+    return mq, mqs, mK, mV
+
+
+def attn_prefill_bwd(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_routed=None, o_sh=None):
     """Backward of attn_prefill: every selected expert's rows and the shared
     head's rows send their dK/dV into the KV group they read ([SN] §3-2 2), 5)).
 
     q_routed, do_routed [B, G, T, k, d]; q_sh, do_sh [B, T, d] or None;
-    K, V [B, G, T, d].  Returns dq_routed, dq_sh, dK, dV (float64).
+    K, V [B, G, T, d]; o_routed, o_sh: the forward output to take Delta from
+    (see causal_attention_bwd), or None.  Returns dq_routed, dq_sh, dK, dV.
     """
     B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
     sc = dims.sm_scale
@@ -69,8 +125,9 @@ def attn_prefill_bwd(q_routed, q_sh, K, V, do_routed, do_sh, dims):
     dV = np.zeros((B, G, T, d))
     for b in range(B):
         for g in range(G):
+            o_rows = None if o_routed is None else np.asarray(o_routed[b, g]).reshape(T * k, d)
             a, bk, bv = causal_attention_bwd(np.asarray(q_routed[b, g]).reshape(T * k, d), pos, K[b, g], V[b, g],
-                                             np.asarray(do_routed[b, g]).reshape(T * k, d), sc)
+                                             np.asarray(do_routed[b, g]).reshape(T * k, d), sc, o_rows)
             dq[b, g] = a.reshape(T, k, d)
             dK[b, g] += bk
             dV[b, g] += bv
@@ -78,7 +135,8 @@ def attn_prefill_bwd(q_routed, q_sh, K, V, do_routed, do_sh, dims):
     if dims.n_shared:
         dq_sh = np.empty((B, T, d))
         for b in range(B):
-            a, bk, bv = causal_attention_bwd(q_sh[b], np.arange(T), K[b, dims.sg], V[b, dims.sg], do_sh[b], sc)
+            a, bk, bv = causal_attention_bwd(q_sh[b], np.arange(T), K[b, dims.sg], V[b, dims.sg], do_sh[b], sc,
+                                             None if o_sh is None else o_sh[b])
             dq_sh[b] = a
             dK[b, dims.sg] += bk
             dV[b, dims.sg] += bv

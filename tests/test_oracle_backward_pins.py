@@ -54,6 +54,19 @@ def test_attention_gradients_match_finite_differences(k):
     _check(lambda a: L(q, K, a), V, dV, rng)
 
 
+def test_delta_from_the_forward_output_is_the_same_sum():
+    """Delta_r = sum_j P_rj dP_rj equals dO_r . o_r for the exact forward output."""
+    rng = np.random.default_rng(6)
+    T, d, k = 7, 4, 2
+    pos = np.repeat(np.arange(T), k)
+    q, dO = rng.standard_normal((T * k, d)), rng.standard_normal((T * k, d))
+    K, V = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    o = orc.causal_attention(q, pos, K, V, 0.6)
+    for a, b in zip(ob.causal_attention_bwd(q, pos, K, V, dO, 0.6),
+                    ob.causal_attention_bwd(q, pos, K, V, dO, 0.6, O=o)):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-12)
+
+
 def test_attention_gradients_match_library_autograd():
     """Standard causal attention (one row per position) against torch autograd
     through scaled_dot_product_attention in float64."""
