@@ -290,6 +290,20 @@ def run_kernel(args):
             fn = lambda: gq.gqe_attn_prefill_bwd(dc, q, qs, K, V, o, os_, lse, dO, dOs, dq, dqs, dK, dV, ws)  # noqa
             # five products per (query tile, key tile) against the forward's two
             work = dict(flops=2.5 * attn_useful_flops(dims))
+        elif args.kernel in ("layer_bwd", "train_step"):
+            x = rn(B, T, D)
+            Wt = gi.layer_weights(dims)
+            lay = gq.GQELayer(dims, {kk: torch.from_numpy(v.view(np.int16)) for kk, v in Wt.items()},
+                              gi.router_bias(w), device=device)
+            dy = rn(B, T, D)
+            _, saved = lay.forward(x, keep=True)
+            if args.kernel == "layer_bwd":
+                fn = lambda: lay.backward(x, dy, saved)  # noqa: E731
+            else:
+                def fn():
+                    _, sv = lay.forward(x, keep=True)
+                    lay.backward(x, dy, sv)
+            work = dict(tokens=float(dims.N))
         elif args.kernel in ("router", "qproj", "kv", "linear", "combine", "combine_out"):
             x = rn(B, T, D)
             Wt = gi.layer_weights(dims)
@@ -335,6 +349,8 @@ def run_kernel(args):
         out["TFLOP/s"] = work["flops"] / ms / 1e9
     if "bytes" in work:
         out["GB/s"] = work["bytes"] / ms / 1e6
+    if "tokens" in work:
+        out["tokens/s"] = work["tokens"] / ms * 1e3
     print(json.dumps(out), flush=True)
     return 0
 

@@ -70,7 +70,8 @@ typedef struct {
   int output_mode;       /* 0 GQE, 1 hard concat only, 2 weighted concat */
 } gqe_dims;
 
-enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3, GQE_OP_ATTN_BWD = 4 };
+enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3, GQE_OP_ATTN_BWD = 4,
+       GQE_OP_BWD_PACK_WEIGHTS = 5 };
 
 /* Bytes of scratch the call `op` needs for these dims (L_max: the decode
  * cache length, used by GQE_OP_ATTN_DECODE only).  Returns
@@ -161,6 +162,61 @@ gqe_status gqe_attn_prefill_bwd(const gqe_dims* dims, const gqe_bf16* q_routed, 
                                 const gqe_bf16* o_sh, const float* lse, const gqe_bf16* do_routed,
                                 const gqe_bf16* do_sh, gqe_bf16* dq_routed, gqe_bf16* dq_sh, gqe_bf16* dK,
                                 gqe_bf16* dV, void* ws, size_t ws_bytes, gqe_stream stream);
+
+/* Backward of the output construction ("GQE" study note §3-2 3) hard slots,
+ * 4) weighted-sum slot, 5) shared head; §4-1: the weighted-sum slot is the
+ * router's gradient path).  Per token, for selected (g, j) with weight w:
+ *   output_mode 0: do = dh_hard + w dh_route,  dw = <dh_route, o>;
+ *   output_mode 1: do = dh_hard,               dw = 0;
+ *   output_mode 2: do = w dh_hard,             dw = <dh_hard, o>;
+ *   do_sh = the shared slot of dh.
+ *   o_routed [B, G, T, k, d], topk_w [B*T, G, k] fp32 (the forward's),
+ *   dh [B*T, slots*d] bf16 -> do_routed [B, G, T, k, d], do_sh [B, T, d] bf16,
+ *   dtopk_w [B*T, G, k] fp32.  o_sh is not read (may be NULL). */
+gqe_status gqe_combine_bwd(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe_bf16* o_sh,
+                           const float* topk_w, const gqe_bf16* dh, gqe_bf16* do_routed, gqe_bf16* do_sh,
+                           float* dtopk_w, gqe_stream stream);
+
+/* Backward of the router ("GQE" study note §3-2 2) in-group softmax, 4)
+ * renormalisation; TopK is a selection and passes no gradient):
+ *   dp~ -> dp on the selected experts (dp_i = (dw_i - sum_j dw_j p~_j) / Z
+ *   over the renorm scope, or dw_i for scope 2) -> ds_e = p_e (dp_e -
+ *   sum_e' p_e' dp_e') per group.
+ *   probs [B*T, G, E], topk_idx, topk_w [B*T, G, k] as gqe_router_topk wrote
+ *   them; dtopk_w [B*T, G, k] -> dlogits [B*T, G*E] fp32; dbias [G*E] fp32 (the
+ *   column sums of dlogits, accumulated with atomics in an order that may
+ *   differ between runs) or NULL. */
+gqe_status gqe_router_bwd(const gqe_dims* dims, const float* probs, const int32_t* topk_idx, const float* topk_w,
+                          const float* dtopk_w, float* dlogits, float* dbias, gqe_stream stream);
+
+/* Columns Kc of the packed projection-gradient matrix of gqe_bwd_pack:
+ * G*E*d + n_shared*d + 2*G*d + 64*ceil(G*E/64). */
+gqe_status gqe_bwd_pack_cols(const gqe_dims* dims, int* cols);
+
+/* The projection gradients as one bf16 matrix A [B*T, Kc], row = token:
+ * [dq scattered to its expert's d columns, block g*E+e, zeros for experts the
+ * token did not select | dq_sh | dK of groups 0..G-1 | dV | dlogits (bf16),
+ * zero padding].  With W_cat = [Wq; Wsh; Wk; Wv; Wr^T] stacked by rows,
+ * dx = A W_cat and dW_cat = A^T x ("GQE" study note §3-2 2): only selected
+ * experts receive query gradient).
+ *   dq_routed [B, G, T, k, d], dq_sh [B, T, d], dK, dV [B, G, T, d] bf16,
+ *   dlogits [B*T, G*E] fp32. */
+gqe_status gqe_bwd_pack(const gqe_dims* dims, const int32_t* topk_idx, const gqe_bf16* dq_routed,
+                        const gqe_bf16* dq_sh, const gqe_bf16* dK, const gqe_bf16* dV, const float* dlogits,
+                        gqe_bf16* A, gqe_stream stream);
+
+/* W_cat^T [d_model, Kc] bf16 from the layer's weights (Wr [d_model, G*E],
+ * Wq [G, E, d, d_model], Wsh [d, d_model], Wk, Wv [G*d, d_model]): the B
+ * operand of dx = A W_cat in gqe_linear's [N, K] layout.
+ * ws: gqe_workspace_size(GQE_OP_BWD_PACK_WEIGHTS) bytes. */
+gqe_status gqe_bwd_pack_weights(const gqe_dims* dims, const gqe_bf16* Wr, const gqe_bf16* Wq, const gqe_bf16* Wsh,
+                                const gqe_bf16* Wk, const gqe_bf16* Wv, gqe_bf16* WcatT, void* ws, size_t ws_bytes,
+                                gqe_stream stream);
+
+/* dst[c * ld_dst + r] = src[r * cols + c] for a row-major bf16 src [rows, cols];
+ * dst columns r in [rows, ld_dst) are zeroed (a K padded to a multiple of 64
+ * for gqe_linear). */
+gqe_status gqe_transpose(int rows, int cols, const gqe_bf16* src, gqe_bf16* dst, int ld_dst, gqe_stream stream);
 
 /* Decode attention: one new token per sequence (dims->T must be 1) against a
  * dense cache (freeguideonline GQA tutorial, "自回归推理中的内存带宽优势": a

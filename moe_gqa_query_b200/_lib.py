@@ -22,6 +22,7 @@ GQE_OP_ROUTED_QPROJ = 1
 GQE_OP_ATTN_DECODE = 2
 GQE_OP_COMBINE_OUT_PROJ = 3
 GQE_OP_ATTN_BWD = 4
+GQE_OP_BWD_PACK_WEIGHTS = 5
 STATUS_NAMES = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED",
                 3: "GQE_ERR_WORKSPACE", 4: "GQE_ERR_CUDA", 5: "GQE_ERR_DEVICE_CHECK"}
 
@@ -70,6 +71,12 @@ SIGNATURES = {
     "gqe_combine": [_D, _P, _P, _P, _P, _P],
     "gqe_combine_out_proj": [_D, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "gqe_linear": [_I, _I, _I, _P, _P, _P, _P],
+    "gqe_combine_bwd": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
+    "gqe_router_bwd": [_D, _P, _P, _P, _P, _P, _P, _P],
+    "gqe_bwd_pack_cols": [_D, ctypes.POINTER(_I)],
+    "gqe_bwd_pack": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
+    "gqe_bwd_pack_weights": [_D, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
+    "gqe_transpose": [_I, _I, _P, _P, _I, _P],
     "gqe_device_error": [ctypes.POINTER(_I), _P],
     "gqe_debug_exp2": [_P, _P, _P, _P, _I, _P],
     "gqe_status_string": [_I],
@@ -261,6 +268,56 @@ def gqe_linear(A, W, C, stream=None):
     N = W.shape[0]
     _check("gqe_linear", lib.gqe_linear(M, N, K, _ptr(A, "A", b), _ptr(W, "W", b), _ptr(C, "C", b),
                                         _stream(stream)))
+
+
+def gqe_combine_bwd(dims, o_routed, o_sh, topk_w, dh, do_routed, do_sh, dtopk_w, stream=None):
+    import torch
+    b = _bf16()
+    _check("gqe_combine_bwd", lib.gqe_combine_bwd(
+        ctypes.byref(dims), _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True),
+        _ptr(topk_w, "topk_w", torch.float32), _ptr(dh, "dh", b), _ptr(do_routed, "do_routed", b),
+        _ptr(do_sh, "do_sh", b, optional=True), _ptr(dtopk_w, "dtopk_w", torch.float32), _stream(stream)))
+
+
+def gqe_router_bwd(dims, probs, topk_idx, topk_w, dtopk_w, dlogits, dbias=None, stream=None):
+    import torch
+    f = torch.float32
+    _check("gqe_router_bwd", lib.gqe_router_bwd(
+        ctypes.byref(dims), _ptr(probs, "probs", f), _ptr(topk_idx, "topk_idx", torch.int32),
+        _ptr(topk_w, "topk_w", f), _ptr(dtopk_w, "dtopk_w", f), _ptr(dlogits, "dlogits", f),
+        _ptr(dbias, "dbias", f, optional=True), _stream(stream)))
+
+
+def gqe_bwd_pack_cols(dims) -> int:
+    n = _I(0)
+    _check("gqe_bwd_pack_cols", lib.gqe_bwd_pack_cols(ctypes.byref(dims), ctypes.byref(n)))
+    return int(n.value)
+
+
+def gqe_bwd_pack(dims, topk_idx, dq_routed, dq_sh, dK, dV, dlogits, A, stream=None):
+    import torch
+    b = _bf16()
+    _check("gqe_bwd_pack", lib.gqe_bwd_pack(
+        ctypes.byref(dims), _ptr(topk_idx, "topk_idx", torch.int32), _ptr(dq_routed, "dq_routed", b),
+        _ptr(dq_sh, "dq_sh", b, optional=True), _ptr(dK, "dK", b), _ptr(dV, "dV", b),
+        _ptr(dlogits, "dlogits", torch.float32), _ptr(A, "A", b), _stream(stream)))
+
+
+def gqe_bwd_pack_weights(dims, Wr, Wq, Wsh, Wk, Wv, WcatT, ws, stream=None):
+    b = _bf16()
+    ws_bytes = ws.numel() * ws.element_size()
+    _check("gqe_bwd_pack_weights", lib.gqe_bwd_pack_weights(
+        ctypes.byref(dims), _ptr(Wr, "Wr", b), _ptr(Wq, "Wq", b), _ptr(Wsh, "Wsh", b, optional=True),
+        _ptr(Wk, "Wk", b), _ptr(Wv, "Wv", b), _ptr(WcatT, "WcatT", b), _ptr(ws, "ws"), ws_bytes, _stream(stream)))
+
+
+def gqe_transpose(src, dst, ld_dst=None, stream=None):
+    """dst [cols, ld_dst] <- src [rows, cols]^T (columns past rows zeroed)."""
+    b = _bf16()
+    rows, cols = src.shape[0], src.numel() // src.shape[0]
+    ld = rows if ld_dst is None else int(ld_dst)
+    _check("gqe_transpose", lib.gqe_transpose(rows, cols, _ptr(src, "src", b), _ptr(dst, "dst", b), ld,
+                                              _stream(stream)))
 
 
 def gqe_device_error(stream=None) -> int:

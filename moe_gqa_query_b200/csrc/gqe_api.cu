@@ -8,6 +8,7 @@
 
 #include "../../include/gqe.h"
 #include "attn.cuh"
+#include "bwd.cuh"
 #include "gemm.cuh"
 #include "route.cuh"
 
@@ -242,6 +243,10 @@ gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* b
   if (op == GQE_OP_COMBINE_OUT_PROJ) {
     const size_t slots = (size_t)dims->k * dims->G + (dims->output_mode == 0 ? 1 : 0) + dims->n_shared;
     *bytes = (size_t)N * slots * dims->d_head * 2;
+    return GQE_OK;
+  }
+  if (op == GQE_OP_BWD_PACK_WEIGHTS) {
+    *bytes = (size_t)bwd_pack_cols(dims->G, dims->E, dims->d_head, dims->n_shared) * dims->d_model * 2;
     return GQE_OK;
   }
   if (op == GQE_OP_ATTN_BWD) {
@@ -647,6 +652,121 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
     return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0, 0}, mW, mW, mO, mO, ep, M, K, nt,
                                               nt, pbn, S(stream)));
   return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, K, nt, nt, bn, S(stream)));
+}
+
+gqe_status gqe_combine_bwd(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe_bf16* o_sh,
+                           const float* topk_w, const gqe_bf16* dh, gqe_bf16* do_routed, gqe_bf16* do_sh,
+                           float* dtopk_w, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  (void)o_sh;
+  GQE_REQUIRE(o_routed && topk_w && dh && do_routed && dtopk_w, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || do_sh, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(o_routed) && aligned16(dh) && aligned16(do_routed), GQE_ERR_INVALID_ARG);
+  CombineBwdParams p{};
+  p.o_routed = o_routed;
+  p.w = topk_w;
+  p.dh = dh;
+  p.do_routed = do_routed;
+  p.do_sh = do_sh;
+  p.dw = dtopk_w;
+  p.B = dims->B;
+  p.T = dims->T;
+  p.G = dims->G;
+  p.k = dims->k;
+  p.d = dims->d_head;
+  p.n_shared = dims->n_shared;
+  p.output_mode = dims->output_mode;
+  p.slots = dims->k * dims->G + (dims->output_mode == 0 ? 1 : 0) + dims->n_shared;
+  return cuda_status(launch_combine_bwd(p, S(stream)));
+}
+
+gqe_status gqe_router_bwd(const gqe_dims* dims, const float* probs, const int32_t* topk_idx, const float* topk_w,
+                          const float* dtopk_w, float* dlogits, float* dbias, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(probs && topk_idx && topk_w && dtopk_w && dlogits, GQE_ERR_INVALID_ARG);
+  RouterBwdParams p{};
+  p.probs = probs;
+  p.idx = topk_idx;
+  p.w = topk_w;
+  p.dw = dtopk_w;
+  p.dlogits = dlogits;
+  p.dbias = dbias;
+  p.N = dims->B * dims->T;
+  p.G = dims->G;
+  p.E = dims->E;
+  p.k = dims->k;
+  p.scope = dims->renorm_scope;
+  return cuda_status(launch_router_bwd(p, S(stream)));
+}
+
+gqe_status gqe_bwd_pack_cols(const gqe_dims* dims, int* cols) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(cols, GQE_ERR_INVALID_ARG);
+  *cols = bwd_pack_cols(dims->G, dims->E, dims->d_head, dims->n_shared);
+  return GQE_OK;
+}
+
+gqe_status gqe_bwd_pack(const gqe_dims* dims, const int32_t* topk_idx, const gqe_bf16* dq_routed,
+                        const gqe_bf16* dq_sh, const gqe_bf16* dK, const gqe_bf16* dV, const float* dlogits,
+                        gqe_bf16* A, gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(topk_idx && dq_routed && dK && dV && dlogits && A, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || dq_sh, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(aligned16(dq_routed) && aligned16(dK) && aligned16(dV) && aligned16(A), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || aligned16(dq_sh), GQE_ERR_INVALID_ARG);
+  PackParams p{};
+  p.idx = topk_idx;
+  p.dq = dq_routed;
+  p.dq_sh = dq_sh;
+  p.dK = dK;
+  p.dV = dV;
+  p.dlogits = dlogits;
+  p.A = A;
+  p.B = dims->B;
+  p.T = dims->T;
+  p.G = dims->G;
+  p.E = dims->E;
+  p.k = dims->k;
+  p.d = dims->d_head;
+  p.n_shared = dims->n_shared;
+  p.Kc = bwd_pack_cols(dims->G, dims->E, dims->d_head, dims->n_shared);
+  return cuda_status(launch_bwd_pack(p, S(stream)));
+}
+
+gqe_status gqe_transpose(int rows, int cols, const gqe_bf16* src, gqe_bf16* dst, int ld_dst, gqe_stream stream) {
+  GQE_REQUIRE(rows >= 1 && cols >= 1 && ld_dst >= rows, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(src && dst, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE((long long)rows * cols < (1ll << 31) && (long long)cols * ld_dst < (1ll << 31), GQE_ERR_UNSUPPORTED);
+  return cuda_status(launch_transpose(src, dst, rows, cols, ld_dst, S(stream)));
+}
+
+gqe_status gqe_bwd_pack_weights(const gqe_dims* dims, const gqe_bf16* Wr, const gqe_bf16* Wq, const gqe_bf16* Wsh,
+                                const gqe_bf16* Wk, const gqe_bf16* Wv, gqe_bf16* WcatT, void* ws, size_t ws_bytes,
+                                gqe_stream stream) {
+  GQE_CHECK(check_dims(dims));
+  GQE_REQUIRE(Wr && Wq && Wk && Wv && WcatT, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(!dims->n_shared || Wsh, GQE_ERR_INVALID_ARG);
+  const int D = dims->d_model, G = dims->G, E = dims->E, d = dims->d_head, GE = G * E;
+  const int Kc = bwd_pack_cols(G, E, d, dims->n_shared);
+  GQE_REQUIRE(ws && ws_bytes >= (size_t)Kc * D * 2, GQE_ERR_WORKSPACE);
+  // W_cat [Kc, D] = [Wq (G*E*d rows); Wsh; Wk; Wv; Wr^T; zero rows], then transposed
+  uint16_t* Wcat = static_cast<uint16_t*>(ws);
+  cudaStream_t st = S(stream);
+  size_t row = 0;
+  auto put = [&](const gqe_bf16* src, size_t rows) {
+    const cudaError_t e = cudaMemcpyAsync(Wcat + row * D, src, rows * D * 2, cudaMemcpyDeviceToDevice, st);
+    row += rows;
+    return e;
+  };
+  GQE_REQUIRE(put(Wq, (size_t)GE * d) == cudaSuccess, GQE_ERR_CUDA);
+  if (dims->n_shared) GQE_REQUIRE(put(Wsh, d) == cudaSuccess, GQE_ERR_CUDA);
+  GQE_REQUIRE(put(Wk, (size_t)G * d) == cudaSuccess, GQE_ERR_CUDA);
+  GQE_REQUIRE(put(Wv, (size_t)G * d) == cudaSuccess, GQE_ERR_CUDA);
+  GQE_REQUIRE(launch_transpose(Wr, Wcat + row * D, D, GE, D, st) == cudaSuccess, GQE_ERR_CUDA);
+  row += GE;
+  if ((int)row < Kc)
+    GQE_REQUIRE(cudaMemsetAsync(Wcat + row * D, 0, ((size_t)Kc - row) * D * 2, st) == cudaSuccess, GQE_ERR_CUDA);
+  return cuda_status(launch_transpose(Wcat, WcatT, Kc, D, Kc, st));
 }
 
 gqe_status gqe_device_error(int* code, gqe_stream stream) {

@@ -8,6 +8,9 @@ stream; every step of the forward runs in libgqe.so's kernels:
            projection, without materialising h where the shape allows)
   decode   gqe_router_topk -> gqe_routed_qproj -> gqe_kv_append ->
            gqe_attn_decode -> gqe_combine -> gqe_linear
+  backward gqe_linear (dh) -> gqe_combine_bwd -> gqe_attn_prefill_bwd ->
+           gqe_router_bwd -> gqe_bwd_pack -> gqe_linear (dx) and, through
+           gqe_transpose, gqe_linear for the weight gradients
 
 Weight layouts (bf16): Wr [D, G*E]; Wq [G, E, d, D]; Wk, Wv [G*d, D];
 Wsh [n_shared*d, D]; Wo [D, slots*d] with slots = k*G + 1 + n_shared (GQE's
@@ -108,6 +111,8 @@ class GQELayer:
         o = self._buf("o", (B, c.G, T, c.k, c.d))
         os_ = self._buf("os", (B, T, c.d)) if c.n_shared else None
         y = self._buf("y", (B, T, c.D)) if out is None else out
+        probs = self._buf("probs", (N, c.G, c.E), torch.float32) if keep else None
+        lse = self._buf("lse", (N * c.G * c.k + N * c.n_shared,), torch.float32) if keep else None
         ws = self._ws("ws_q", L.gqe_workspace_size(dims, L.GQE_OP_ROUTED_QPROJ))
         ws_o = self._ws("ws_o", L.gqe_workspace_size(dims, L.GQE_OP_COMBINE_OUT_PROJ))
         if stream is None and self.concurrent_kv:
@@ -124,20 +129,94 @@ class GQELayer:
                 L.gqe_kv_proj(dims, x, self.Wk, self.Wv, K, V)
                 join = torch.cuda.Event()
                 join.record(self._side)
-            L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, None)
+            L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, probs)
             L.gqe_routed_qproj(dims, x, self.Wq, self.Wsh, idx, q, qs, ws, None)
             main.wait_event(join)
         else:
-            L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, None, stream)
+            L.gqe_router_topk(dims, x, self.Wr, self.bias, idx, w, probs, stream)
             L.gqe_routed_qproj(dims, x, self.Wq, self.Wsh, idx, q, qs, ws, None, stream)
             L.gqe_kv_proj(dims, x, self.Wk, self.Wv, K, V, stream)
-        L.gqe_attn_prefill(dims, q, qs, K, V, o, os_, None, stream)
+        L.gqe_attn_prefill(dims, q, qs, K, V, o, os_, lse, stream)
         L.gqe_combine_out_proj(dims, o, os_, w, self.Wo, y, ws_o, stream)
         if keep:
             h = self._buf("h", (N, c.slots * c.d))
-            L.gqe_combine(dims, o, os_, w, h, stream)     # h itself, for inspection only
-            return y, dict(idx=idx, w=w, q=q, q_sh=qs, K=K, V=V, o=o, o_sh=os_, h=h)
+            L.gqe_combine(dims, o, os_, w, h, stream)     # h itself, for the backward and inspection
+            return y, dict(idx=idx, w=w, probs=probs, q=q, q_sh=qs, K=K, V=V, o=o, o_sh=os_, lse=lse, h=h)
         return y
+
+    # ------------------------------------------------------------------ backward
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, saved: dict, stream=None) -> dict:
+        """Gradients of <y, dy> for the forward(x, keep=True) that returned
+        `saved`: dx [B, T, D] and dWr, dbias (fp32), dWq, dWk, dWv, dWsh, dWo,
+        in the weights' layouts.  TopK passes no gradient; the router learns
+        through the weighted-sum slot (output_mode 0) or the weighted hard
+        slots (mode 2).  The returned tensors are the layer's own buffers,
+        overwritten by the next backward.
+
+        The projection gradients go through one packed matrix A (gqe_bwd_pack):
+        dx = A W_cat and dW_cat = A^T x with W_cat = [Wq; Wsh; Wk; Wv; Wr^T],
+        where dq is scattered to its expert's columns (zeros for unselected
+        experts, so the query part of these two GEMMs runs dense over all E
+        experts of a group)."""
+        c = self.cfg
+        B, T = x.shape[0], x.shape[1]
+        dims = L.make_dims(c, B=B, T=T)
+        N, D, d, S = B * T, c.D, c.d, c.slots * c.d
+        Np = (N + 63) // 64 * 64
+        GE = c.G * c.E
+        buf = self._buf
+        # weight-side operands
+        WoT = buf("WoT", (S, D))
+        L.gqe_transpose(self.Wo, WoT, None, stream)
+        Kc = L.gqe_bwd_pack_cols(dims)
+        WcatT = buf("WcatT", (D, Kc))
+        ws_w = self._ws("ws_w", L.gqe_workspace_size(dims, L.GQE_OP_BWD_PACK_WEIGHTS))
+        L.gqe_bwd_pack_weights(dims, self.Wr, self.Wq, self.Wsh, self.Wk, self.Wv, WcatT, ws_w, stream)
+        # output projection: dh = dy Wo, dWo = dy^T h
+        dy2 = dy.reshape(N, D)
+        dh = buf("dh", (N, S))
+        L.gqe_linear(dy2, WoT, dh, stream)
+        dyT = buf("dyT", (D, Np))
+        L.gqe_transpose(dy2, dyT, Np, stream)
+        hT = buf("hT", (S, Np))
+        L.gqe_transpose(saved["h"], hT, Np, stream)
+        dWo = buf("dWo", (D, S))
+        L.gqe_linear(dyT, hT, dWo, stream)
+        # output construction, attention, router
+        do = buf("do", (B, c.G, T, c.k, d))
+        do_sh = buf("do_sh", (B, T, d)) if c.n_shared else None
+        dw = buf("dw", (N, c.G, c.k), torch.float32)
+        L.gqe_combine_bwd(dims, saved["o"], saved["o_sh"], saved["w"], dh, do, do_sh, dw, stream)
+        dq = buf("dq", (B, c.G, T, c.k, d))
+        dq_sh = buf("dq_sh", (B, T, d)) if c.n_shared else None
+        dK = buf("dK", (B, c.G, T, d))
+        dV = buf("dV", (B, c.G, T, d))
+        ws_a = self._ws("ws_a", L.gqe_workspace_size(dims, L.GQE_OP_ATTN_BWD))
+        L.gqe_attn_prefill_bwd(dims, saved["q"], saved["q_sh"], saved["K"], saved["V"], saved["o"], saved["o_sh"],
+                               saved["lse"], do, do_sh, dq, dq_sh, dK, dV, ws_a, stream)
+        dlogits = buf("dlogits", (N, GE), torch.float32)
+        dbias = buf("dbias", (GE,), torch.float32)
+        L.gqe_router_bwd(dims, saved["probs"], saved["idx"], saved["w"], dw, dlogits, dbias, stream)
+        # projections: dx = A W_cat, dW_cat = A^T x
+        A = buf("A", (N, Kc))
+        L.gqe_bwd_pack(dims, saved["idx"], dq, dq_sh, dK, dV, dlogits, A, stream)
+        dx = buf("dx", (B, T, D))
+        L.gqe_linear(A, WcatT, dx, stream)
+        AT = buf("AT", (Kc, Np))
+        L.gqe_transpose(A, AT, Np, stream)
+        xT = buf("xT", (D, Np))
+        L.gqe_transpose(x.reshape(N, D), xT, Np, stream)
+        dWcat = buf("dWcat", (Kc, D))
+        L.gqe_linear(AT, xT, dWcat, stream)
+        r0 = GE * d
+        r1 = r0 + c.n_shared * d
+        r2 = r1 + c.G * d
+        r3 = r2 + c.G * d
+        dWr = buf("dWr", (D, GE))
+        L.gqe_transpose(dWcat[r3:r3 + GE], dWr, None, stream)
+        return dict(dx=dx, dWr=dWr, dbias=dbias, dWq=dWcat[:r0].view(c.G, c.E, d, D),
+                    dWsh=dWcat[r0:r1] if c.n_shared else None, dWk=dWcat[r1:r2], dWv=dWcat[r2:r3], dWo=dWo,
+                    dh=dh, do=do, do_sh=do_sh, dw=dw, dq=dq, dq_sh=dq_sh, dK=dK, dV=dV, dlogits=dlogits)
 
     def forward_graph(self, x: torch.Tensor, out=None) -> torch.Tensor:
         """forward() replayed from a CUDA graph captured on first use for this
