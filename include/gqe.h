@@ -70,8 +70,7 @@ typedef struct {
   int output_mode;       /* 0 GQE, 1 hard concat only, 2 weighted concat */
 } gqe_dims;
 
-enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3, GQE_OP_ATTN_BWD = 4,
-       GQE_OP_BWD_PACK_WEIGHTS = 5 };
+enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3, GQE_OP_ATTN_BWD = 4 };
 
 /* Bytes of scratch the call `op` needs for these dims (L_max: the decode
  * cache length, used by GQE_OP_ATTN_DECODE only).  Returns
@@ -163,6 +162,17 @@ gqe_status gqe_attn_prefill_bwd(const gqe_dims* dims, const gqe_bf16* q_routed, 
                                 const gqe_bf16* do_sh, gqe_bf16* dq_routed, gqe_bf16* dq_sh, gqe_bf16* dK,
                                 gqe_bf16* dV, void* ws, size_t ws_bytes, gqe_stream stream);
 
+/* C [M, N] = sum_k A(m, k) B(n, k), bf16 in and out, fp32 accumulation on
+ * tcgen05 (the projections of the backward pass).  Operand layouts:
+ *   a_kn = 0: A stored [M, K] row-major;  a_kn = 1: A stored [K, M] (A^T).
+ *   b_kn = 0: B stored [N, K] (nn.Linear weight); b_kn = 1: B stored [K, N].
+ * C row-major [M, N].  N % 64 == 0; the contiguous dimension of each operand
+ * a multiple of 8 elements; any K (the tail is zero-filled).  Errors:
+ * GQE_ERR_UNSUPPORTED for other shapes, GQE_ERR_INVALID_ARG for null or
+ * misaligned pointers. */
+gqe_status gqe_gemm(int M, int N, int K, const gqe_bf16* A, int a_kn, const gqe_bf16* B, int b_kn, gqe_bf16* C,
+                    gqe_stream stream);
+
 /* Backward of the output construction ("GQE" study note §3-2 3) hard slots,
  * 4) weighted-sum slot, 5) shared head; §4-1: the weighted-sum slot is the
  * router's gradient path).  Per token, for selected (g, j) with weight w:
@@ -205,13 +215,12 @@ gqe_status gqe_bwd_pack(const gqe_dims* dims, const int32_t* topk_idx, const gqe
                         const gqe_bf16* dq_sh, const gqe_bf16* dK, const gqe_bf16* dV, const float* dlogits,
                         gqe_bf16* A, gqe_stream stream);
 
-/* W_cat^T [d_model, Kc] bf16 from the layer's weights (Wr [d_model, G*E],
- * Wq [G, E, d, d_model], Wsh [d, d_model], Wk, Wv [G*d, d_model]): the B
- * operand of dx = A W_cat in gqe_linear's [N, K] layout.
- * ws: gqe_workspace_size(GQE_OP_BWD_PACK_WEIGHTS) bytes. */
+/* W_cat [Kc, d_model] bf16 = [Wq; Wsh; Wk; Wv; Wr^T; zero rows] stacked by rows
+ * from the layer's weights (Wr [d_model, G*E], Wq [G, E, d, d_model],
+ * Wsh [d, d_model], Wk, Wv [G*d, d_model]): the B operand (stored [K, N]) of
+ * dx = A W_cat in gqe_gemm. */
 gqe_status gqe_bwd_pack_weights(const gqe_dims* dims, const gqe_bf16* Wr, const gqe_bf16* Wq, const gqe_bf16* Wsh,
-                                const gqe_bf16* Wk, const gqe_bf16* Wv, gqe_bf16* WcatT, void* ws, size_t ws_bytes,
-                                gqe_stream stream);
+                                const gqe_bf16* Wk, const gqe_bf16* Wv, gqe_bf16* Wcat, gqe_stream stream);
 
 /* dst[c * ld_dst + r] = src[r * cols + c] for a row-major bf16 src [rows, cols];
  * dst columns r in [rows, ld_dst) are zeroed (a K padded to a multiple of 64

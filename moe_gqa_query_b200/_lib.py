@@ -22,7 +22,6 @@ GQE_OP_ROUTED_QPROJ = 1
 GQE_OP_ATTN_DECODE = 2
 GQE_OP_COMBINE_OUT_PROJ = 3
 GQE_OP_ATTN_BWD = 4
-GQE_OP_BWD_PACK_WEIGHTS = 5
 STATUS_NAMES = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED",
                 3: "GQE_ERR_WORKSPACE", 4: "GQE_ERR_CUDA", 5: "GQE_ERR_DEVICE_CHECK"}
 
@@ -71,11 +70,12 @@ SIGNATURES = {
     "gqe_combine": [_D, _P, _P, _P, _P, _P],
     "gqe_combine_out_proj": [_D, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "gqe_linear": [_I, _I, _I, _P, _P, _P, _P],
+    "gqe_gemm": [_I, _I, _I, _P, _I, _P, _I, _P, _P],
     "gqe_combine_bwd": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
     "gqe_router_bwd": [_D, _P, _P, _P, _P, _P, _P, _P],
     "gqe_bwd_pack_cols": [_D, ctypes.POINTER(_I)],
     "gqe_bwd_pack": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
-    "gqe_bwd_pack_weights": [_D, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
+    "gqe_bwd_pack_weights": [_D, _P, _P, _P, _P, _P, _P, _P],
     "gqe_transpose": [_I, _I, _P, _P, _I, _P],
     "gqe_device_error": [ctypes.POINTER(_I), _P],
     "gqe_debug_exp2": [_P, _P, _P, _P, _I, _P],
@@ -270,6 +270,22 @@ def gqe_linear(A, W, C, stream=None):
                                         _stream(stream)))
 
 
+def gqe_gemm(A, a_kn, B, b_kn, C, stream=None):
+    """C [M, N] = A B^T over K, with A stored [M, K] (a_kn=0) or [K, M] (a_kn=1)
+    and B stored [N, K] (b_kn=0) or [K, N] (b_kn=1)."""
+    b = _bf16()
+    A2 = A.reshape(-1, A.shape[-1])
+    B2 = B.reshape(-1, B.shape[-1])
+    M, K = (A2.shape[1], A2.shape[0]) if a_kn else (A2.shape[0], A2.shape[1])
+    N, Kb = (B2.shape[1], B2.shape[0]) if b_kn else (B2.shape[0], B2.shape[1])
+    if K != Kb:
+        raise ValueError(f"K mismatch: {K} vs {Kb}")
+    if C.numel() != M * N:
+        raise ValueError(f"C has {C.numel()} elements, expected {M}x{N}")
+    _check("gqe_gemm", lib.gqe_gemm(M, N, K, _ptr(A, "A", b), int(a_kn), _ptr(B, "B", b), int(b_kn),
+                                    _ptr(C, "C", b), _stream(stream)))
+
+
 def gqe_combine_bwd(dims, o_routed, o_sh, topk_w, dh, do_routed, do_sh, dtopk_w, stream=None):
     import torch
     b = _bf16()
@@ -303,12 +319,11 @@ def gqe_bwd_pack(dims, topk_idx, dq_routed, dq_sh, dK, dV, dlogits, A, stream=No
         _ptr(dlogits, "dlogits", torch.float32), _ptr(A, "A", b), _stream(stream)))
 
 
-def gqe_bwd_pack_weights(dims, Wr, Wq, Wsh, Wk, Wv, WcatT, ws, stream=None):
+def gqe_bwd_pack_weights(dims, Wr, Wq, Wsh, Wk, Wv, Wcat, stream=None):
     b = _bf16()
-    ws_bytes = ws.numel() * ws.element_size()
     _check("gqe_bwd_pack_weights", lib.gqe_bwd_pack_weights(
         ctypes.byref(dims), _ptr(Wr, "Wr", b), _ptr(Wq, "Wq", b), _ptr(Wsh, "Wsh", b, optional=True),
-        _ptr(Wk, "Wk", b), _ptr(Wv, "Wv", b), _ptr(WcatT, "WcatT", b), _ptr(ws, "ws"), ws_bytes, _stream(stream)))
+        _ptr(Wk, "Wk", b), _ptr(Wv, "Wv", b), _ptr(Wcat, "Wcat", b), _stream(stream)))
 
 
 def gqe_transpose(src, dst, ld_dst=None, stream=None):

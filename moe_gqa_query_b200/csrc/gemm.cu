@@ -135,13 +135,26 @@ __device__ __forceinline__ void epilogue_tile_tma(const EpiParams& ep, const CUt
 }
 
 // ---------------------------------------------------------------------------
+// Operand majorness.  K-major (the default): a tile of rows x 64 k, one 128-byte
+// row per M (N) index.  MN-major (kMnA / kMnB): the operand is stored [K, M]
+// ([K, N]) and comes in as 64-column boxes of 64 k rows, 8 KB each, so a
+// 16-deep k-step is 16 rows (2 KB) further on and the 64-wide M (N) atoms are
+// kMnBox apart.
+constexpr int kMnA = 1, kMnB = 2;
+constexpr int kMnBox = 64 * 64 * 2;
+
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk, int mn_major) {
+  return mn_major ? sdesc_sw128(base + kk * 2048, kMnBox, 1024) : sdesc_sw128(base + kk * 32, 16, 1024);
+}
+
+// ---------------------------------------------------------------------------
 // dense: A [M, K] and W [N, K] by TMA; persistent over (m-tile, n-tile)
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
 gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                   const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapO0,
                   const __grid_constant__ CUtensorMap mapO1, EpiParams ep, int M, int K, int n_tiles_b0,
-                  int n_tiles_total) {
+                  int n_tiles_total, int mn) {
   constexpr int kBTileBytes = BN * kBK * 2;
   constexpr uint32_t kTmemCols = 2 * BN;
   extern __shared__ uint8_t smem_raw[];
@@ -193,14 +206,24 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
           if (it >= STAGES && !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, ep.err, kErrTimeoutGemm))
             break;
           mbar_arrive_expect_tx(&bar->full[s], kATileBytes + kBTileBytes);
-          tma_load_2d(sA + s * kATileBytes, &mapA, &bar->full[s], kb * kBK, mt * kBM);
-          tma_load_2d(sB + s * kBTileBytes, mB, &bar->full[s], kb * kBK, n0);
+          if (mn & kMnA) {
+            for (int h = 0; h < kBM / 64; ++h)
+              tma_load_2d(sA + s * kATileBytes + h * kMnBox, &mapA, &bar->full[s], mt * kBM + h * 64, kb * kBK);
+          } else {
+            tma_load_2d(sA + s * kATileBytes, &mapA, &bar->full[s], kb * kBK, mt * kBM);
+          }
+          if (mn & kMnB) {
+            for (int h = 0; h < BN / 64; ++h)
+              tma_load_2d(sB + s * kBTileBytes + h * kMnBox, mB, &bar->full[s], n0 + h * 64, kb * kBK);
+          } else {
+            tma_load_2d(sB + s * kBTileBytes, mB, &bar->full[s], kb * kBK, n0);
+          }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
+      const uint32_t idesc = idesc_bf16_f32(kBM, BN, (mn & kMnA) != 0, (mn & kMnB) != 0);
       int it = 0, tc = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tc) {
         const int ab = tc & 1, use = tc >> 1;
@@ -215,8 +238,7 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
           const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_ss(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
-                    (kb | kk) != 0);
+            umma_ss(acc, operand_desc(a0, kk, mn & kMnA), operand_desc(b0, kk, mn & kMnB), idesc, (kb | kk) != 0);
           umma_commit(&bar->empty[s]);
         }
         umma_commit(&bar->acc_full[ab]);
@@ -270,7 +292,7 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
                        const __grid_constant__ CUtensorMap mapB0,
                        const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapO0,
                        const __grid_constant__ CUtensorMap mapO1, EpiParams ep, int M, int K, int n_tiles_b0,
-                       int n_tiles_total) {
+                       int n_tiles_total, int mn) {
   constexpr int kPM = 2 * kBM;                       // pair tile rows
   constexpr int kHalfB = (BN / 2) * kBK * 2;         // this CTA's half of the W k-block
   constexpr uint32_t kTmemCols = 2 * BN;
@@ -333,7 +355,10 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             break;
           if (rank == 0) mbar_arrive_expect_tx(&bar->full[s], 2 * (kATileBytes + kHalfB));
           const uint32_t fb = full0 + (uint32_t)(s * sizeof(uint64_t));
-          if (as.mode == kASingle) {
+          if (as.mode == kASingle && (mn & kMnA)) {
+            for (int h = 0; h < kBM / 64; ++h)
+              tma_load_2d_pair(sA + s * kATileBytes + h * kMnBox, &mapA, fb, m0 + h * 64, kb * kBK);
+          } else if (as.mode == kASingle) {
             tma_load_2d_pair(sA + s * kATileBytes, &mapA, fb, kb * kBK, m0);
           } else {
             const int col = kb * kBK, slot = col / as.d, sub = col - slot * as.d;
@@ -347,13 +372,18 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
               tma_load_2d_pair(sA + s * kATileBytes, (slot == kG && as.route) ? &mapR : &mapS, fb, sub, m0);
             }
           }
-          tma_load_2d_pair(sB + s * kHalfB, mB, fb, kb * kBK, n0);
+          if (mn & kMnB) {
+            for (int h = 0; h < BN / 128; ++h)
+              tma_load_2d_pair(sB + s * kHalfB + h * kMnBox, mB, fb, n0 + h * 64, kb * kBK);
+          } else {
+            tma_load_2d_pair(sB + s * kHalfB, mB, fb, kb * kBK, n0);
+          }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kPM, BN, false, false);
+      const uint32_t idesc = idesc_bf16_f32(kPM, BN, (mn & kMnA) != 0, (mn & kMnB) != 0);
       const uint32_t empty_peer0 = cluster_addr(&bar->empty[0], peer);
       const uint32_t accf_peer0 = cluster_addr(&bar->acc_full[0], peer);
       int it = 0, tc = 0;
@@ -370,7 +400,7 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
           const uint32_t b0 = smem_u32(sB + s * kHalfB);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_ss_pair(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
+            umma_ss_pair(acc, operand_desc(a0, kk, mn & kMnA), operand_desc(b0, kk, mn & kMnB), idesc,
                          (kb | kk) != 0);
           umma_commit_pair(smem_u32(&bar->empty[s]));
           umma_commit_pair(empty_peer0 + (uint32_t)(s * sizeof(uint64_t)));
@@ -621,7 +651,7 @@ gemm_routed_kernel(const __grid_constant__ CUtensorMap mapWq, const __grid_const
 template <int BN, int STAGES>
 static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                                    const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M,
-                                   int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream) {
+                                   int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream, int mn) {
   const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
   auto kern = gemm_dense_kernel<BN, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
@@ -629,14 +659,15 @@ static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& m
   const int tiles = ((M + kBM - 1) / kBM) * n_tiles_total;
   const int grid = tiles < num_sms() ? tiles : num_sms();
   return launch_kernel(kern, dim3(grid), dim3(192), smem, stream, 1, mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K,
-                       n_tiles_b0, n_tiles_total);
+                       n_tiles_b0, n_tiles_total, mn);
 }
 
 template <int BN, int STAGES>
 static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorMap& mapR, const CUtensorMap& mapS,
                                         const ASource& as, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                                         const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep,
-                                        int M, int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream) {
+                                        int M, int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream,
+                                        int mn) {
   const size_t smem = 1024 + STAGES * (kATileBytes + (BN / 2) * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
   auto kern = gemm_dense_pair_kernel<BN, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
@@ -669,26 +700,26 @@ static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorM
   const int total = ((M + 255) / 256) * n_tiles_total;
   const int pairs = total < mp ? total : mp;
   return launch_kernel(kern, dim3(2 * pairs), dim3(192), smem, stream, 2, mapA, mapR, mapS, as, mapB0, mapB1,
-                       mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total);
+                       mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, mn);
 }
 
 cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapR, const CUtensorMap& mapS,
                                    const ASource& as, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                                    const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M,
-                                   int K, int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream) {
+                                   int K, int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream, int mn) {
   if (bn != 256) return cudaErrorInvalidValue;
   return launch_dense_pair_st<256, 6>(mapA, mapR, mapS, as, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0,
-                                      n_tiles_total, stream);
+                                      n_tiles_total, stream, mn);
 }
 
 int dense_tile_n(int n_per_weight) { return (n_per_weight % 256 == 0) ? 256 : 128; }
 
 cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                               const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
-                              int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream) {
+                              int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream, int mn) {
   if (bn == 256)
-    return launch_dense_bn<256, 4>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
-  return launch_dense_bn<128, 6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream);
+    return launch_dense_bn<256, 4>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream, mn);
+  return launch_dense_bn<128, 6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream, mn);
 }
 
 template <int BN, int STAGES, int CPS>

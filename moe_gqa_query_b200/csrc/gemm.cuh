@@ -53,10 +53,13 @@ struct RoutedParams {
 int dense_tile_n(int n_per_weight);
 
 // mapO0 / mapO1: output maps for ep.store_mode != kStorePerThread.
+// mn: bit 0 -> A is stored [K, M] (map over [K rows, M cols], box 64 x 64),
+// bit 1 -> B is stored [K, N] (same); otherwise [M, K] / [N, K].  K may then
+// be rounded up to a multiple of 64 (the maps' zero fill covers the tail).
 cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0,
                               const CUtensorMap& mapB1, const CUtensorMap& mapO0,
                               const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
-                              int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream);
+                              int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream, int mn = 0);
 
 // Where the pair GEMM's A operand comes from.  kASingle: one map over A [M, K]
 // (box 64 x 128).  kASlots: the output projection's h = [hard slots, weighted
@@ -78,7 +81,7 @@ cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& m
                                    const ASource& as, const CUtensorMap& mapB0,
                                    const CUtensorMap& mapB1, const CUtensorMap& mapO0,
                                    const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
-                                   int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream);
+                                   int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream, int mn = 0);
 
 cudaError_t launch_gemm_routed(const CUtensorMap& mapWq, const CUtensorMap& mapWsh,
                                const gqe_bf16_t* x, const RoutedParams& rp, const EpiParams& epr,

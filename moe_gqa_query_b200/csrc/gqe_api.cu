@@ -245,10 +245,6 @@ gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* b
     *bytes = (size_t)N * slots * dims->d_head * 2;
     return GQE_OK;
   }
-  if (op == GQE_OP_BWD_PACK_WEIGHTS) {
-    *bytes = (size_t)bwd_pack_cols(dims->G, dims->E, dims->d_head, dims->n_shared) * dims->d_model * 2;
-    return GQE_OK;
-  }
   if (op == GQE_OP_ATTN_BWD) {
     AttnBwdLayout L;
     attn_bwd_layout(dims->B, dims->T, dims->G, dims->k, dims->n_shared, dims->d_head, &L);
@@ -741,20 +737,18 @@ gqe_status gqe_transpose(int rows, int cols, const gqe_bf16* src, gqe_bf16* dst,
 }
 
 gqe_status gqe_bwd_pack_weights(const gqe_dims* dims, const gqe_bf16* Wr, const gqe_bf16* Wq, const gqe_bf16* Wsh,
-                                const gqe_bf16* Wk, const gqe_bf16* Wv, gqe_bf16* WcatT, void* ws, size_t ws_bytes,
-                                gqe_stream stream) {
+                                const gqe_bf16* Wk, const gqe_bf16* Wv, gqe_bf16* Wcat, gqe_stream stream) {
   GQE_CHECK(check_dims(dims));
-  GQE_REQUIRE(Wr && Wq && Wk && Wv && WcatT, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(Wr && Wq && Wk && Wv && Wcat, GQE_ERR_INVALID_ARG);
   GQE_REQUIRE(!dims->n_shared || Wsh, GQE_ERR_INVALID_ARG);
   const int D = dims->d_model, G = dims->G, E = dims->E, d = dims->d_head, GE = G * E;
   const int Kc = bwd_pack_cols(G, E, d, dims->n_shared);
-  GQE_REQUIRE(ws && ws_bytes >= (size_t)Kc * D * 2, GQE_ERR_WORKSPACE);
-  // W_cat [Kc, D] = [Wq (G*E*d rows); Wsh; Wk; Wv; Wr^T; zero rows], then transposed
-  uint16_t* Wcat = static_cast<uint16_t*>(ws);
+  // W_cat [Kc, D] = [Wq (G*E*d rows); Wsh; Wk; Wv; Wr^T; zero rows]
+  uint16_t* W = Wcat;
   cudaStream_t st = S(stream);
   size_t row = 0;
   auto put = [&](const gqe_bf16* src, size_t rows) {
-    const cudaError_t e = cudaMemcpyAsync(Wcat + row * D, src, rows * D * 2, cudaMemcpyDeviceToDevice, st);
+    const cudaError_t e = cudaMemcpyAsync(W + row * D, src, rows * D * 2, cudaMemcpyDeviceToDevice, st);
     row += rows;
     return e;
   };
@@ -762,11 +756,47 @@ gqe_status gqe_bwd_pack_weights(const gqe_dims* dims, const gqe_bf16* Wr, const 
   if (dims->n_shared) GQE_REQUIRE(put(Wsh, d) == cudaSuccess, GQE_ERR_CUDA);
   GQE_REQUIRE(put(Wk, (size_t)G * d) == cudaSuccess, GQE_ERR_CUDA);
   GQE_REQUIRE(put(Wv, (size_t)G * d) == cudaSuccess, GQE_ERR_CUDA);
-  GQE_REQUIRE(launch_transpose(Wr, Wcat + row * D, D, GE, D, st) == cudaSuccess, GQE_ERR_CUDA);
+  GQE_REQUIRE(launch_transpose(Wr, W + row * D, D, GE, D, st) == cudaSuccess, GQE_ERR_CUDA);
   row += GE;
   if ((int)row < Kc)
-    GQE_REQUIRE(cudaMemsetAsync(Wcat + row * D, 0, ((size_t)Kc - row) * D * 2, st) == cudaSuccess, GQE_ERR_CUDA);
-  return cuda_status(launch_transpose(Wcat, WcatT, Kc, D, Kc, st));
+    GQE_REQUIRE(cudaMemsetAsync(W + row * D, 0, ((size_t)Kc - row) * D * 2, st) == cudaSuccess, GQE_ERR_CUDA);
+  return GQE_OK;
+}
+
+gqe_status gqe_gemm(int M, int N, int K, const gqe_bf16* A, int a_kn, const gqe_bf16* B, int b_kn, gqe_bf16* C,
+                    gqe_stream stream) {
+  GQE_REQUIRE(M >= 1 && N >= 1 && K >= 1, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(A && B && C && (a_kn == 0 || a_kn == 1) && (b_kn == 0 || b_kn == 1), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(N % 64 == 0, GQE_ERR_UNSUPPORTED);
+  // TMA row pitches are multiples of 16 bytes
+  GQE_REQUIRE((a_kn ? M : K) % 8 == 0 && (b_kn ? N : K) % 8 == 0, GQE_ERR_UNSUPPORTED);
+  GQE_REQUIRE((long long)M * N < (1ll << 31) && (long long)M * K < (1ll << 31) && (long long)N * K < (1ll << 31),
+              GQE_ERR_UNSUPPORTED);
+  GQE_REQUIRE(aligned16(A) && aligned16(B) && aligned16(C), GQE_ERR_INVALID_ARG);
+  const int Kp = (K + 63) / 64 * 64;
+  const int pbn = pair_tile_n(M, N);
+  const int bn = pbn ? pbn : dense_tile_n(N);
+  CUtensorMap mA, mW;
+  if (a_kn) GQE_REQUIRE(map2d(&mA, A, M, K, 64), GQE_ERR_CUDA);
+  else GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
+  if (b_kn) GQE_REQUIRE(map2d(&mW, B, N, K, 64), GQE_ERR_CUDA);
+  else GQE_REQUIRE(map2d(&mW, B, K, N, pbn ? pbn / 2 : bn), GQE_ERR_CUDA);
+  EpiParams ep{};
+  ep.out0 = C;
+  ep.out1 = C;
+  ep.mode = kEpiRowMajor;
+  ep.ldo = N;
+  ep.n_limit = N;
+  ep.err = error_word();
+  CUtensorMap mO;
+  GQE_REQUIRE(map2d(&mO, C, N, M, 32), GQE_ERR_CUDA);
+  ep.store_mode = kStoreTma2d;
+  const int nt = (N + bn - 1) / bn;
+  const int mn = (a_kn ? 1 : 0) | (b_kn ? 2 : 0);
+  if (pbn)
+    return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0, 0}, mW, mW, mO, mO, ep, M, Kp,
+                                              nt, nt, pbn, S(stream), mn));
+  return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, Kp, nt, nt, bn, S(stream), mn));
 }
 
 gqe_status gqe_device_error(int* code, gqe_stream stream) {

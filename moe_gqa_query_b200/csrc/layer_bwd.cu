@@ -83,57 +83,53 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(CombineBwdParams p) {
 }
 
 // ---------------------------------------------------------------- router backward
-// One thread per token: d p~ -> dp (renormalisation) -> ds (in-group softmax).
-constexpr int kRouterBwdThreads = 128;
+// One thread per (token, group): d p~ -> dp (renormalisation) -> ds (in-group
+// softmax).  Token-scope sums are recomputed by each of the token's G threads.
+constexpr int kRouterBwdThreads = 256;
 
 __global__ void __launch_bounds__(kRouterBwdThreads) router_bwd_kernel(RouterBwdParams p) {
   __shared__ float sbias[kMaxBwdRouterCols];
   pdl_launch_dependents();
   pdl_wait();
   const int GE = p.G * p.E;
-  for (int i = threadIdx.x; i < GE; i += blockDim.x) sbias[i] = 0.f;
-  __syncthreads();
-  const int n = (int)(blockIdx.x * blockDim.x + threadIdx.x);
-  if (n < p.N) {
+  if (p.dbias) {
+    for (int i = threadIdx.x; i < GE; i += blockDim.x) sbias[i] = 0.f;
+    __syncthreads();
+  }
+  const long long tg = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tg < (long long)p.N * p.G) {
+    const int n = (int)(tg / p.G), g = (int)(tg % p.G);
     const float* pr = p.probs + (size_t)n * GE;
     const int* idx = p.idx + (size_t)n * p.G * p.k;
     const float* dw = p.dw + (size_t)n * p.G * p.k;
     const float* wt = p.w + (size_t)n * p.G * p.k;
-    // token-scope sums (scope 0)
-    float z_tok = 0.f, s_tok = 0.f;
-    if (p.scope == 0) {
-      for (int i = 0; i < p.G * p.k; ++i) {
-        z_tok += pr[(i / p.k) * p.E + idx[i]];
-        s_tok += dw[i] * wt[i];
+    // the renormalisation's sums: over all selections of the token (scope 0)
+    // or of this group (scope 1)
+    const int i0 = p.scope == 0 ? 0 : g * p.k;
+    const int i1 = p.scope == 0 ? p.G * p.k : (g + 1) * p.k;
+    float z = 0.f, sdw = 0.f;
+    if (p.scope != 2) {
+      for (int i = i0; i < i1; ++i) {
+        z += pr[(i / p.k) * p.E + idx[i]];
+        sdw += dw[i] * wt[i];
       }
     }
-    float* out = p.dlogits + (size_t)n * GE;
-    for (int g = 0; g < p.G; ++g) {
-      float z = z_tok, sdw = s_tok;
-      if (p.scope == 1) {
-        z = 0.f;
-        sdw = 0.f;
-        for (int j = 0; j < p.k; ++j) {
-          z += pr[g * p.E + idx[g * p.k + j]];
-          sdw += dw[g * p.k + j] * wt[g * p.k + j];
-        }
-      }
-      // dp on the selected experts, and sum_e p_e dp_e over the group
-      float pdp = 0.f;
-      float dsel[8];
-      for (int j = 0; j < p.k; ++j) {
-        const float dwj = dw[g * p.k + j];
-        dsel[j] = (p.scope == 2) ? dwj : (dwj - sdw) / z;
-        pdp += pr[g * p.E + idx[g * p.k + j]] * dsel[j];
-      }
-      for (int e = 0; e < p.E; ++e) {
-        float dp = 0.f;
-        for (int j = 0; j < p.k; ++j)
-          if (idx[g * p.k + j] == e) dp = dsel[j];
-        const float ds = pr[g * p.E + e] * (dp - pdp);
-        out[g * p.E + e] = ds;
-        if (p.dbias) atomicAdd(&sbias[g * p.E + e], ds);
-      }
+    // dp on the selected experts, and sum_e p_e dp_e over the group
+    float pdp = 0.f;
+    float dsel[8];
+    for (int j = 0; j < p.k; ++j) {
+      const float dwj = dw[g * p.k + j];
+      dsel[j] = (p.scope == 2) ? dwj : (dwj - sdw) / z;
+      pdp += pr[g * p.E + idx[g * p.k + j]] * dsel[j];
+    }
+    float* out = p.dlogits + (size_t)n * GE + g * p.E;
+    for (int e = 0; e < p.E; ++e) {
+      float dp = 0.f;
+      for (int j = 0; j < p.k; ++j)
+        if (idx[g * p.k + j] == e) dp = dsel[j];
+      const float ds = pr[g * p.E + e] * (dp - pdp);
+      out[e] = ds;
+      if (p.dbias) atomicAdd(&sbias[g * p.E + e], ds);
     }
   }
   if (p.dbias) {
@@ -232,7 +228,8 @@ cudaError_t launch_router_bwd(const RouterBwdParams& p, cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(p.dbias, 0, sizeof(float) * p.G * p.E, stream);
     if (e != cudaSuccess) return e;
   }
-  return launch_kernel(router_bwd_kernel, dim3((p.N + kRouterBwdThreads - 1) / kRouterBwdThreads),
+  const long long threads = (long long)p.N * p.G;
+  return launch_kernel(router_bwd_kernel, dim3((unsigned)((threads + kRouterBwdThreads - 1) / kRouterBwdThreads)),
                        dim3(kRouterBwdThreads), 0, stream, 1, p);
 }
 

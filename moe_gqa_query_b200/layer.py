@@ -8,9 +8,8 @@ stream; every step of the forward runs in libgqe.so's kernels:
            projection, without materialising h where the shape allows)
   decode   gqe_router_topk -> gqe_routed_qproj -> gqe_kv_append ->
            gqe_attn_decode -> gqe_combine -> gqe_linear
-  backward gqe_linear (dh) -> gqe_combine_bwd -> gqe_attn_prefill_bwd ->
-           gqe_router_bwd -> gqe_bwd_pack -> gqe_linear (dx) and, through
-           gqe_transpose, gqe_linear for the weight gradients
+  backward gqe_gemm (dh, dWo) -> gqe_combine_bwd -> gqe_attn_prefill_bwd ->
+           gqe_router_bwd -> gqe_bwd_pack -> gqe_gemm (dx, dW_cat)
 
 Weight layouts (bf16): Wr [D, G*E]; Wq [G, E, d, D]; Wk, Wv [G*d, D];
 Wsh [n_shared*d, D]; Wo [D, slots*d] with slots = k*G + 1 + n_shared (GQE's
@@ -162,26 +161,15 @@ class GQELayer:
         B, T = x.shape[0], x.shape[1]
         dims = L.make_dims(c, B=B, T=T)
         N, D, d, S = B * T, c.D, c.d, c.slots * c.d
-        Np = (N + 63) // 64 * 64
         GE = c.G * c.E
         buf = self._buf
-        # weight-side operands
-        WoT = buf("WoT", (S, D))
-        L.gqe_transpose(self.Wo, WoT, None, stream)
-        Kc = L.gqe_bwd_pack_cols(dims)
-        WcatT = buf("WcatT", (D, Kc))
-        ws_w = self._ws("ws_w", L.gqe_workspace_size(dims, L.GQE_OP_BWD_PACK_WEIGHTS))
-        L.gqe_bwd_pack_weights(dims, self.Wr, self.Wq, self.Wsh, self.Wk, self.Wv, WcatT, ws_w, stream)
-        # output projection: dh = dy Wo, dWo = dy^T h
+        # output projection: dh = dy Wo, dWo = dy^T h (operands read in place,
+        # [K, M] / [K, N] layouts straight from memory)
         dy2 = dy.reshape(N, D)
         dh = buf("dh", (N, S))
-        L.gqe_linear(dy2, WoT, dh, stream)
-        dyT = buf("dyT", (D, Np))
-        L.gqe_transpose(dy2, dyT, Np, stream)
-        hT = buf("hT", (S, Np))
-        L.gqe_transpose(saved["h"], hT, Np, stream)
+        L.gqe_gemm(dy2, 0, self.Wo, 1, dh, stream)
         dWo = buf("dWo", (D, S))
-        L.gqe_linear(dyT, hT, dWo, stream)
+        L.gqe_gemm(dy2, 1, saved["h"], 1, dWo, stream)
         # output construction, attention, router
         do = buf("do", (B, c.G, T, c.k, d))
         do_sh = buf("do_sh", (B, T, d)) if c.n_shared else None
@@ -198,16 +186,15 @@ class GQELayer:
         dbias = buf("dbias", (GE,), torch.float32)
         L.gqe_router_bwd(dims, saved["probs"], saved["idx"], saved["w"], dw, dlogits, dbias, stream)
         # projections: dx = A W_cat, dW_cat = A^T x
+        Kc = L.gqe_bwd_pack_cols(dims)
+        Wcat = buf("Wcat", (Kc, D))
+        L.gqe_bwd_pack_weights(dims, self.Wr, self.Wq, self.Wsh, self.Wk, self.Wv, Wcat, stream)
         A = buf("A", (N, Kc))
         L.gqe_bwd_pack(dims, saved["idx"], dq, dq_sh, dK, dV, dlogits, A, stream)
         dx = buf("dx", (B, T, D))
-        L.gqe_linear(A, WcatT, dx, stream)
-        AT = buf("AT", (Kc, Np))
-        L.gqe_transpose(A, AT, Np, stream)
-        xT = buf("xT", (D, Np))
-        L.gqe_transpose(x.reshape(N, D), xT, Np, stream)
+        L.gqe_gemm(A, 0, Wcat, 1, dx, stream)
         dWcat = buf("dWcat", (Kc, D))
-        L.gqe_linear(AT, xT, dWcat, stream)
+        L.gqe_gemm(A, 1, x.reshape(N, D), 1, dWcat, stream)
         r0 = GE * d
         r1 = r0 + c.n_shared * d
         r2 = r1 + c.G * d

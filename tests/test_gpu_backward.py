@@ -242,3 +242,47 @@ def test_transpose(rows, cols, ld):
     got = dst.cpu().view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(got[:, :rows], src.T)
     assert not got[:, rows:].any()
+
+
+@pytest.mark.parametrize("a_kn,b_kn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("M,N,K", [(200, 192, 104), (2304, 512, 1000), (64, 64, 16384), (4096, 256, 72)],
+                         ids=["small_ragged_k", "pair_tiles", "long_k", "pair_short_k"])
+def test_gemm_operand_layouts(M, N, K, a_kn, b_kn):
+    """C = A B^T with each operand stored either way round; the ragged K tail
+    (K not a multiple of 64) is zero-filled by the loads.  Projection
+    tolerance: 2^-8 |ref| + 1e-3 (bf16 output of an fp32 accumulation), inputs
+    scaled to unit-size outputs."""
+    A = gi.normal_bf16(10, "x", (M, K), std=K ** -0.5)
+    Bm = gi.normal_bf16(11, "x", (N, K))
+    tA = bf16_dev(np.ascontiguousarray(A.T) if a_kn else A)
+    tB = bf16_dev(np.ascontiguousarray(Bm.T) if b_kn else Bm)
+    C = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gq.gqe_gemm(tA, a_kn, tB, b_kn, C)
+    torch.cuda.synchronize()
+    ref = orc.f64(A) @ orc.f64(Bm).T
+    got = to_f64(C)
+    bad = np.abs(got - ref) > 2.0 ** -8 * np.abs(ref) + 1e-3
+    assert not bad.any(), (int(bad.sum()), float(np.abs(got - ref).max()))
+
+
+@pytest.mark.parametrize("K", [70, 1, 16389])
+def test_gemm_any_k_when_k_is_strided(K):
+    """With both operands stored [K, *] the contiguous dimensions are M and N,
+    so any K works (the token count of a weight gradient)."""
+    M, N = 320, 128
+    A = gi.normal_bf16(12, "x", (K, M), std=K ** -0.5)
+    Bm = gi.normal_bf16(13, "x", (K, N))
+    C = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gq.gqe_gemm(bf16_dev(A), 1, bf16_dev(Bm), 1, C)
+    torch.cuda.synchronize()
+    ref = orc.f64(A).T @ orc.f64(Bm)
+    got = to_f64(C)
+    assert not (np.abs(got - ref) > 2.0 ** -8 * np.abs(ref) + 1e-3).any()
+
+
+def test_gemm_rejects_unaligned_contiguous_k():
+    A = torch.zeros((64, 70), dtype=torch.bfloat16, device="cuda")
+    Bm = torch.zeros((64, 70), dtype=torch.bfloat16, device="cuda")
+    C = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(gq.GQEError):
+        gq.gqe_gemm(A, 0, Bm, 0, C)
