@@ -155,7 +155,7 @@ gqe_status gqe_attn_prefill(const gqe_dims* dims, const gqe_bf16* q_routed,
  *   overwritten.  fp32 accumulation; dq is summed over key tiles in an fp32
  *   workspace, in an order that may differ between runs.
  *   ws: scratch of gqe_workspace_size(GQE_OP_ATTN_BWD) bytes, 256-byte
- *   aligned.  d_head 64 only (GQE_ERR_UNSUPPORTED otherwise). */
+ *   aligned. */
 gqe_status gqe_attn_prefill_bwd(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh,
                                 const gqe_bf16* K, const gqe_bf16* V, const gqe_bf16* o_routed,
                                 const gqe_bf16* o_sh, const float* lse, const gqe_bf16* do_routed,

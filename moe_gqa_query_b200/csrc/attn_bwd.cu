@@ -32,6 +32,12 @@
 // Warpgroup w writes its bf16 P^T (dS^T) into the first half of its own
 // S^T (dP^T) columns, so the two warpgroups never touch each other's columns;
 // the MMAs read the K = 128 query operand as two 64-query halves.
+// Tensor memory (d = 128): S^T 0 | dP^T 128 | dV 256 | dK 384, all 512 columns.
+// P^T goes to S^T's columns 0-63 and dS^T to its columns 64-127 (the two
+// warpgroups meet at a named barrier once both hold their S^T in registers);
+// dQ_i accumulates over dP^T's columns once the warpgroups have read them, so
+// dP^T(i+1) waits for dQ_i to be drained and S^T(i+1) for dK_i.  dO has a
+// one-stage ring here (shared memory holds K, V, two Q stages, dO and dS).
 #include "attn.cuh"
 #include "launch.cuh"
 
@@ -45,7 +51,7 @@ constexpr int kBoxB = 128 * 64 * 2;   // one 128-row x 64-column bf16 TMA box
 
 struct __align__(8) BwdBarriers {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2], q_empty[2], o_full[2], o_empty[2];
   uint64_t s_full, p_full, pv_done, dp_full, ds_full, dk_done;
   uint64_t dq_full[2], dq_free[2];
   uint32_t tmem_base;
@@ -56,15 +62,19 @@ template <int D>
 struct BwdCfg {
   static constexpr int NB = D / 64;
   static constexpr int TileBytes = NB * kBoxB;        // one 128-row tile of Q, dO, K or V
-  static constexpr uint32_t kS = 0, kDP = 128, kDV = 256, kDK = 256 + D, kDQ = 256 + 2 * D;
+  static constexpr bool kWide = D == 128;
+  static constexpr int OST = kWide ? 1 : 2;           // dO ring depth
+  static constexpr int EpiCh = kWide ? 1 : D / 32;    // 32-column dQ chunks staged per warp at once
+  static constexpr uint32_t kS = 0, kDP = 128, kDV = 256, kDK = 256 + D;
+  static constexpr uint32_t kDQ = kWide ? 128 : 256 + 2 * D;
   // shared memory, every operand region 1024-byte aligned
   static constexpr int OffK = 0;
   static constexpr int OffV = OffK + TileBytes;
   static constexpr int OffQ = OffV + TileBytes;                 // [2] stages
-  static constexpr int OffDO = OffQ + 2 * TileBytes;            // [2]
-  static constexpr int OffDS = OffDO + 2 * TileBytes;           // 128 x 128 bf16, MN-major
-  static constexpr int OffEpi = OffDS + 2 * kBoxB;              // 4 warps x D/32 chunks x 4 KB
-  static constexpr int OffLse = OffEpi + 4 * (D / 32) * 4096;   // [2][128] f32
+  static constexpr int OffDO = OffQ + 2 * TileBytes;            // [OST]
+  static constexpr int OffDS = OffDO + OST * TileBytes;         // 128 x 128 bf16, MN-major
+  static constexpr int OffEpi = OffDS + 2 * kBoxB;              // 4 warps x EpiCh x 4 KB
+  static constexpr int OffLse = OffEpi + 4 * EpiCh * 4096;      // [2][128] f32
   static constexpr int OffDelta = OffLse + 2 * 512;             // [2][128] f32
   static constexpr int OffBar = OffDelta + 2 * 512;
   static constexpr size_t Smem = 1024 + OffBar + sizeof(BwdBarriers);
@@ -101,10 +111,29 @@ __device__ __forceinline__ QTile qtile(const AttnBwdParams& p, int s, int jt, in
   return q;
 }
 
-// Tensor-memory column of the bf16 query operand's k-step ks (16 queries):
-// queries [0, 64) packed at base + [0, 32), [64, 128) at base + 64 + [0, 32).
+// Tensor-memory column of the bf16 query operand's k-step ks (16 queries).
+// d = 64: queries [0, 64) packed at base + [0, 32), [64, 128) at
+// base + 64 + [0, 32) (each warpgroup inside its own fp32 columns).
+// d = 128: P^T contiguous at S^T's columns 0-63, dS^T at 64-127.
 __device__ __forceinline__ uint32_t half_col(uint32_t base, int ks) {
   return base + (ks >> 2) * 64 + (ks & 3) * 8;
+}
+template <int D>
+__device__ __forceinline__ uint32_t pt_col(int ks) {
+  return D == 64 ? half_col(BwdCfg<D>::kS, ks) : BwdCfg<D>::kS + ks * 8;
+}
+template <int D>
+__device__ __forceinline__ uint32_t dst_col(int ks) {
+  return D == 64 ? half_col(BwdCfg<D>::kDP, ks) : BwdCfg<D>::kS + 64 + ks * 8;
+}
+// Where warpgroup w writes its 32 packed columns of P^T and dS^T.
+template <int D>
+__device__ __forceinline__ uint32_t pt_wcol(int w) {
+  return D == 64 ? BwdCfg<D>::kS + 64 * w : BwdCfg<D>::kS + 32 * w;
+}
+template <int D>
+__device__ __forceinline__ uint32_t dst_wcol(int w) {
+  return D == 64 ? BwdCfg<D>::kDP + 64 * w : BwdCfg<D>::kS + 64 + 32 * w;
 }
 
 template <int D>
@@ -142,6 +171,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
     for (int st = 0; st < 2; ++st) {
       mbar_init(&bar->q_full[st], 1);
       mbar_init(&bar->q_empty[st], 2 + 256);
+      mbar_init(&bar->o_full[st], 1);
+      mbar_init(&bar->o_empty[st], 1);
       mbar_init(&bar->dq_full[st], 1);
       mbar_init(&bar->dq_free[st], 128);
     }
@@ -182,15 +213,20 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
         const CUtensorMap* mq = q.shared ? &mapQs : &mapQ;
         const CUtensorMap* mo = q.shared ? &mapdOs : &mapdO;
         const int seq = q.shared ? s / p.G : s;
-        mbar_arrive_expect_tx(&bar->q_full[st], 2 * C::TileBytes + 2 * 512);
-        for (int bx = 0; bx < C::NB; ++bx) {
+        mbar_arrive_expect_tx(&bar->q_full[st], C::TileBytes + 2 * 512);
+        for (int bx = 0; bx < C::NB; ++bx)
           tma_load_3d(smem + C::OffQ + st * C::TileBytes + bx * kBoxB, mq, &bar->q_full[st], bx * 64,
                       q.i * kTileB, seq);
-          tma_load_3d(smem + C::OffDO + st * C::TileBytes + bx * kBoxB, mo, &bar->q_full[st], bx * 64,
-                      q.i * kTileB, seq);
-        }
         bulk_load(sLse + st * 128, p.lse2 + q.row_pad, 512, &bar->q_full[st]);
         bulk_load(sDelta + st * 128, p.delta + q.row_pad, 512, &bar->q_full[st]);
+        const int so = n % C::OST;
+        if (n >= C::OST &&
+            !mbar_wait(&bar->o_empty[so], ((n / C::OST) - 1) & 1, abort, p.err, kErrTimeoutAttnBwd))
+          break;
+        mbar_arrive_expect_tx(&bar->o_full[so], C::TileBytes);
+        for (int bx = 0; bx < C::NB; ++bx)
+          tma_load_3d(smem + C::OffDO + so * C::TileBytes + bx * kBoxB, mo, &bar->o_full[so], bx * 64,
+                      q.i * kTileB, seq);
       }
     }
   } else if (warp == 1) {
@@ -213,36 +249,47 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
         return true;
       };
       auto issue_dp = [&](int n) {
-        const uint32_t o0 = smem_u32(smem + C::OffDO + (n & 1) * C::TileBytes);
+        const int so = n % C::OST;
+        if (!mbar_wait(&bar->o_full[so], (n / C::OST) & 1, abort, p.err, kErrTimeoutAttnBwd)) return false;
+        tc_fence_after();
+        const uint32_t o0 = smem_u32(smem + C::OffDO + so * C::TileBytes);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * kBoxB + (ks & 3) * 32;
           umma_ss(tmem + C::kDP, sdesc_sw128(v0 + off, 16, 1024), sdesc_sw128(o0 + off, 16, 1024), idesc_s, ks > 0);
         }
         umma_commit(&bar->dp_full);
+        return true;
       };
       bool ok = mbar_wait(&bar->kv_full, 0, abort, p.err, kErrTimeoutAttnBwd);
       if (ok) ok = issue_s(0);
-      if (ok) issue_dp(0);
+      if (ok) ok = issue_dp(0);
       for (int n = 0; ok && n < cnt; ++n) {
         // dV += P^T dO_i once P^T is in tensor memory
         if (!mbar_wait(&bar->p_full, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
         tc_fence_after();
-        const uint32_t o0 = smem_u32(smem + C::OffDO + (n & 1) * C::TileBytes);
+        const uint32_t o0 = smem_u32(smem + C::OffDO + (n % C::OST) * C::TileBytes);
 #pragma unroll
         for (int ks = 0; ks < kTileB / 16; ++ks)
-          umma_ts(tmem + C::kDV, tmem + half_col(C::kS, ks), sdesc_sw128(o0 + ks * 2048, kBoxB, 1024), idesc_v,
+          umma_ts(tmem + C::kDV, tmem + pt_col<D>(ks), sdesc_sw128(o0 + ks * 2048, kBoxB, 1024), idesc_v,
                   (n > 0 || ks > 0));
         umma_commit(&bar->pv_done);
         umma_commit(&bar->q_empty[n & 1]);
+        umma_commit(&bar->o_empty[n % C::OST]);
         if (n + 1 < cnt) {
-          // S^T(n+1) overwrites P^T(n): wait for dV to have read it
+          // S^T(n+1) overwrites P^T(n) (and, at d = 128, dS^T(n)): wait for
+          // dV (and dK) to have read them
           if (!mbar_wait(&bar->pv_done, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
+          if (C::kWide && !mbar_wait(&bar->dk_done, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
           if (!issue_s(n + 1)) break;
-          // dP^T(n+1) overwrites dS^T(n): wait for dK(n) to have read it
-          if (!mbar_wait(&bar->dk_done, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
+          // dP^T(n+1) overwrites dS^T(n) (d = 64) or dQ(n) (d = 128)
+          if (C::kWide) {
+            if (!mbar_wait(&bar->dq_free[0], n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
+          } else {
+            if (!mbar_wait(&bar->dk_done, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
+          }
           tc_fence_after();
-          issue_dp(n + 1);
+          if (!issue_dp(n + 1)) break;
         }
       }
     }
@@ -259,17 +306,22 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
         const uint32_t q0 = smem_u32(smem + C::OffQ + (n & 1) * C::TileBytes);
 #pragma unroll
         for (int ks = 0; ks < kTileB / 16; ++ks)
-          umma_ts(tmem + C::kDK, tmem + half_col(C::kDP, ks), sdesc_sw128(q0 + ks * 2048, kBoxB, 1024), idesc_k,
+          umma_ts(tmem + C::kDK, tmem + dst_col<D>(ks), sdesc_sw128(q0 + ks * 2048, kBoxB, 1024), idesc_k,
                   (n > 0 || ks > 0));
         umma_commit(&bar->q_empty[n & 1]);
-        if (n >= 2 && !mbar_wait(&bar->dq_free[b], ((n >> 1) - 1) & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
+        // d = 64: dQ double-buffered in its own columns.  d = 128: dQ over
+        // dP^T's columns, which the warpgroups have read (ds_full).
+        if (!C::kWide && n >= 2 &&
+            !mbar_wait(&bar->dq_free[b], ((n >> 1) - 1) & 1, abort, p.err, kErrTimeoutAttnBwd))
+          break;
         tc_fence_after();
+        const uint32_t dq_col = C::kWide ? C::kDQ : C::kDQ + b * D;
 #pragma unroll
         for (int ks = 0; ks < kTileB / 16; ++ks)
-          umma_ss(tmem + C::kDQ + b * D, sdesc_sw128(ds0 + ks * 2048, kBoxB, 1024),
+          umma_ss(tmem + dq_col, sdesc_sw128(ds0 + ks * 2048, kBoxB, 1024),
                   sdesc_sw128(k0 + ks * 2048, kBoxB, 1024), idesc_q, ks > 0);
         umma_commit(&bar->dk_done);
-        umma_commit(&bar->dq_full[b]);
+        umma_commit(&bar->dq_full[C::kWide ? 0 : b]);
       }
     }
   } else if (warp >= 4 && warp < 12) {
@@ -287,7 +339,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
       const QTile q = qtile(p, s, jt, n_r, n);
       ok = mbar_wait(&bar->q_full[st], (n >> 1) & 1, abort, p.err, kErrTimeoutAttnBwd);
       ok = ok && mbar_wait(&bar->s_full, n & 1, abort, p.err, kErrTimeoutAttnBwd);
-      if (!ok) break;
+      if (!C::kWide && !ok) break;
       tc_fence_after();
       const float* lse2 = sLse + st * 128 + col0;
       const float* dlt = sDelta + st * 128 + col0;
@@ -295,7 +347,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
       const int cmin = kv_pos * q.kk - q.i * kTileB - (int)col0;
       float pf[64];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < 2 && ok; ++h) {
         uint32_t sv[32];
         tmem_ld32(tmem + lane_off + C::kS + col0 + h * 32, sv);
 #pragma unroll
@@ -313,11 +365,24 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
         for (int c = 0; c < 64; ++c)
           if (c < cmin) pf[c] = 0.f;
       }
+      if (C::kWide) {
+        // both warpgroups hold their S^T columns in registers before warpgroup 1
+        // writes P^T over warpgroup 0's; every thread of the two warpgroups
+        // passes here each tile and they leave together if any wait failed
+        int any_fail;
+        asm volatile(
+            "{\n\t.reg .pred q, r;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+            "bar.red.or.pred r, 1, 256, q;\n\tselp.b32 %0, 1, 0, r;\n\t}"
+            : "=r"(any_fail)
+            : "r"((int)!ok)
+            : "memory");
+        if (any_fail) break;
+      }
       {
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
-        tmem_st32(tmem + lane_off + C::kS + col0, pk);
+        tmem_st32(tmem + lane_off + pt_wcol<D>(wg), pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -344,7 +409,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
         }
         // dS^T row r: into the first half of this warpgroup's dP^T columns (the
         // dK operand) ...
-        tmem_st8(tmem + lane_off + C::kDP + col0 + ch * 8, dsk);
+        tmem_st8(tmem + lane_off + dst_wcol<D>(wg) + ch * 8, dsk);
         // ... and into the MN-major smem operand of dQ: the 64-query atom of
         // this warpgroup, [128 keys x 128 B], 16-byte pieces swizzled by key row
         uint8_t* atom = sDS + wg * kBoxB + r * 128;
@@ -365,36 +430,43 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
     // ---------------- dQ drain (TMA reduce-add into fp32), then dK, dV
     const int qd = warp & 3;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    uint8_t* stage = smem + C::OffEpi + qd * (D / 32) * 4096;
+    uint8_t* stage = smem + C::OffEpi + qd * C::EpiCh * 4096;
     bool ok = true;
     for (int n = 0; n < cnt && ok; ++n) {
-      const int b = n & 1;
+      const int b = C::kWide ? 0 : (n & 1);
+      const int ph = C::kWide ? (n & 1) : ((n >> 1) & 1);
       const QTile q = qtile(p, s, jt, n_r, n);
-      ok = mbar_wait(&bar->dq_full[b], (n >> 1) & 1, abort, p.err, kErrTimeoutAttnBwd);
+      ok = mbar_wait(&bar->dq_full[b], ph, abort, p.err, kErrTimeoutAttnBwd);
       if (!ok) break;
       tc_fence_after();
-      if (lane == 0) bulk_wait_read<0>();   // the previous tile's reduce has read the staging
-      __syncwarp();
+      const uint32_t dq_col = C::kWide ? C::kDQ : C::kDQ + b * D;
 #pragma unroll
-      for (int c0 = 0; c0 < D / 32; ++c0) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::kDQ + b * D + c0 * 32, v);
-        if (c0 == D / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(&bar->dq_free[b]);
+      for (int g0 = 0; g0 < D / 32; g0 += C::EpiCh) {
+        // staging free: every earlier reduce of this warp has read it
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < C::EpiCh; ++c) {
+          const int c0 = g0 + c;
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + dq_col + c0 * 32, v);
+          if (c0 == D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&bar->dq_free[b]);
+          }
+          uint8_t* rowp = stage + c * 4096 + lane * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(rowp + ((j ^ (lane & 7)) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         }
-        uint8_t* rowp = stage + c0 * 4096 + lane * 128;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(rowp + ((j ^ (lane & 7)) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-#pragma unroll
-        for (int c0 = 0; c0 < D / 32; ++c0)
-          tma_reduce_add_2d(&mapdQ, stage + c0 * 4096, c0 * 32, q.row_pad + qd * 32);
-        bulk_commit();
+          for (int c = 0; c < C::EpiCh; ++c)
+            tma_reduce_add_2d(&mapdQ, stage + c * 4096, (g0 + c) * 32, q.row_pad + qd * 32);
+          bulk_commit();
+        }
       }
     }
     // dK, dV of the key tile
@@ -526,13 +598,13 @@ void attn_bwd_layout(int B, int T, int G, int k, int n_shared, int d, AttnBwdLay
 cudaError_t launch_attn_bwd(const CUtensorMap& mQ, const CUtensorMap& mQs, const CUtensorMap& mdO,
                             const CUtensorMap& mdOs, const CUtensorMap& mK, const CUtensorMap& mV,
                             const CUtensorMap& mdQ, const AttnBwdParams& p, cudaStream_t stream) {
-  if (p.d != 64) return cudaErrorNotSupported;
+  if (p.d != 64 && p.d != 128) return cudaErrorNotSupported;
   const long long threads = p.n_rows_pad * (p.d / 8);
   const int blocks = (int)((threads + 255) / 256);
   cudaError_t e = launch_kernel(attn_bwd_prep_kernel, dim3(blocks), dim3(256), 0, stream, 1, p);
   if (e != cudaSuccess) return e;
-  auto kern = attn_bwd_kernel<64>;
-  const size_t smem = BwdCfg<64>::Smem;
+  auto kern = p.d == 64 ? attn_bwd_kernel<64> : attn_bwd_kernel<128>;
+  const size_t smem = p.d == 64 ? BwdCfg<64>::Smem : BwdCfg<128>::Smem;
   e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int n_kvt = (p.T + kTileB - 1) / kTileB;

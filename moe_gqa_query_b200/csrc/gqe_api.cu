@@ -446,7 +446,6 @@ gqe_status gqe_attn_prefill_bwd(const gqe_dims* dims, const gqe_bf16* q_routed, 
                                 const gqe_bf16* do_sh, gqe_bf16* dq_routed, gqe_bf16* dq_sh, gqe_bf16* dK,
                                 gqe_bf16* dV, void* ws, size_t ws_bytes, gqe_stream stream) {
   GQE_CHECK(check_dims(dims));
-  if (dims->d_head != 64) return GQE_ERR_UNSUPPORTED;
   GQE_REQUIRE(q_routed && K && V && o_routed && lse && do_routed && dq_routed && dK && dV, GQE_ERR_INVALID_ARG);
   GQE_REQUIRE(!dims->n_shared || (q_sh && o_sh && do_sh && dq_sh), GQE_ERR_INVALID_ARG);
   const void* ptrs[] = {q_routed, K, V, o_routed, do_routed, dq_routed, dK, dV, lse};

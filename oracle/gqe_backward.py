@@ -35,7 +35,7 @@ from .gqe_oracle import (
 # ----------------------------------------------------------------------------
 # attention: [SN] §1-1, o = softmax(q K^T * scale) V, causal
 
-def causal_attention_bwd(q, pos, K, V, dO, scale, O=None):
+def causal_attention_bwd(q, pos, K, V, dO, scale, O=None, lse=None):
     """Gradients of o_r = sum_{j <= pos_r} P_rj V_j, P = softmax_j(q_r . K_j * scale).
 
     With S = q K^T * scale (masked to j <= pos_r) and P its row softmax:
@@ -44,15 +44,13 @@ def causal_attention_bwd(q, pos, K, V, dO, scale, O=None):
       Delta_r = sum_i P_ri dP_ri = dO_r . o_r,
       dq = scale * dS K,   dK = scale * dS^T q.
     Delta is the first sum unless the forward output O is given, then the
-    second (identical for the exact O; a call that receives a rounded O
-    computes it from that O).
+    second; P is the softmax unless the forward's log-sum-exp is given, then
+    exp(S - lse) (both identical for the exact O and lse; a call that
+    receives rounded ones computes from those).
     q, dO [R, d]; pos [R]; K, V [L, d].  Returns dq [R, d], dK, dV [L, d].
     """
     q, K, V, dO = f64(q), f64(K), f64(V), f64(dO)
-    s = (q @ K.T) * scale
-    s[np.arange(K.shape[0])[None, :] > np.asarray(pos)[:, None]] = -np.inf
-    z = np.exp(s - s.max(axis=1, keepdims=True))
-    P = z / z.sum(axis=1, keepdims=True)
+    P = _probs(q, pos, K, scale, lse)
     dV = P.T @ dO
     dP = dO @ V.T
     if O is None:
@@ -63,37 +61,67 @@ def causal_attention_bwd(q, pos, K, V, dO, scale, O=None):
     return scale * (dS @ K), scale * (dS.T @ q), dV
 
 
-def causal_attention_bwd_magnitudes(q, pos, K, V, dO, scale, O=None):
-    """The absolute-value sums behind the rounding bound of causal_attention_bwd
-    computed with bf16 MMA operands: a sum of products whose factors are rounded
-    to bf16 (relative error <= 2^-8) errs by at most 2^-8 times the sum of the
-    products' magnitudes.  Returns |dS*scale| |K|, |dS*scale|^T |q|, |P|^T |dO|
-    (the magnitudes for dq, dK, dV)."""
-    q, K, V, dO = f64(q), f64(K), f64(V), f64(dO)
+def _probs(q, pos, K, scale, lse=None):
     s = (q @ K.T) * scale
     s[np.arange(K.shape[0])[None, :] > np.asarray(pos)[:, None]] = -np.inf
+    if lse is not None:
+        return np.exp(s - np.asarray(lse, dtype=np.float64)[:, None])
     z = np.exp(s - s.max(axis=1, keepdims=True))
-    P = z / z.sum(axis=1, keepdims=True)
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def causal_attention_bwd_error_bound(q, pos, K, V, dO, scale, O=None, lse=None):
+    """Worst-case error of causal_attention_bwd's outputs when computed as a
+    tensor-core kernel does it: S, dP, Delta and the three gradient products
+    accumulated in fp32, the MMA operands P and dS rounded to bf16.  Before
+    the final bf16 rounding of the results (which adds 2^-8 |result|).
+
+    With u = 2^-8 (bf16 rounding) and g_n = n 2^-24 (an fp32 sum of n
+    products errs by at most g_n times the sum of their magnitudes):
+      err P    <= P scale g_d sum|q||K|                      (S in fp32)
+      err dS   <= scale (|dP - Delta| err P + P g_d (sum|dO||V| + sum|dO||O|))
+      dq: sum_j ((u + g_L) |scale dS| + err dS) |K_j|,  dK likewise with |q_r|,
+      dV: sum_r ((u + g_R) P + err P) |dO_r|.
+    Returns (bound_dq, bound_dK, bound_dV), absolute, shaped like the outputs.
+    """
+    q, K, V, dO = f64(q), f64(K), f64(V), f64(dO)
+    R, d = q.shape
+    L = K.shape[0]
+    P = _probs(q, pos, K, scale, lse)
     dP = dO @ V.T
-    delta = np.sum(P * dP, axis=1, keepdims=True) if O is None else np.sum(dO * f64(O), axis=1, keepdims=True)
+    Of = f64(O) if O is not None else P @ V
+    delta = np.sum(dO * Of, axis=1, keepdims=True)
+    gd, gL, gR = d * 2.0 ** -24, L * 2.0 ** -24, R * 2.0 ** -24
+    u = 2.0 ** -8
+    aq, aK, aV, adO = np.abs(q), np.abs(K), np.abs(V), np.abs(dO)
+    eP = P * scale * gd * (aq @ aK.T)
+    edS = scale * (np.abs(dP - delta) * eP + P * gd * (adO @ aV.T + np.sum(adO * np.abs(Of), axis=1, keepdims=True)))
     aS = np.abs(scale * P * (dP - delta))
-    return aS @ np.abs(K), aS.T @ np.abs(q), P.T @ np.abs(dO)
+    b_dq = ((u + gL) * aS + edS) @ aK
+    b_dK = ((u + gR) * aS + edS).T @ aq
+    b_dV = ((u + gR) * P + eP).T @ adO
+    return b_dq, b_dK, b_dV
 
 
-def attn_prefill_bwd_magnitudes(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_routed=None, o_sh=None):
-    """causal_attention_bwd_magnitudes laid out like attn_prefill_bwd's outputs."""
+def attn_prefill_bwd_error_bound(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_routed=None, o_sh=None,
+                                 lse=None):
+    """causal_attention_bwd_error_bound laid out like attn_prefill_bwd's
+    outputs.  lse: the forward's fp32 log-sum-exp in gqe_attn_prefill's layout
+    (routed rows, then shared rows), or None."""
     B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
     sc = dims.sm_scale
+    R = T * k
     pos = np.repeat(np.arange(T), k)
     mq = np.empty((B, G, T, k, d))
     mK = np.zeros((B, G, T, d))
     mV = np.zeros((B, G, T, d))
     for b in range(B):
         for g in range(G):
-            o_rows = None if o_routed is None else np.asarray(o_routed[b, g]).reshape(T * k, d)
-            a, bk, bv = causal_attention_bwd_magnitudes(np.asarray(q_routed[b, g]).reshape(T * k, d), pos, K[b, g],
-                                                        V[b, g], np.asarray(do_routed[b, g]).reshape(T * k, d), sc,
-                                                        o_rows)
+            o_rows = None if o_routed is None else np.asarray(o_routed[b, g]).reshape(R, d)
+            l_rows = None if lse is None else np.asarray(lse)[(b * G + g) * R:(b * G + g + 1) * R]
+            a, bk, bv = causal_attention_bwd_error_bound(np.asarray(q_routed[b, g]).reshape(R, d), pos, K[b, g],
+                                                         V[b, g], np.asarray(do_routed[b, g]).reshape(R, d), sc,
+                                                         o_rows, l_rows)
             mq[b, g] = a.reshape(T, k, d)
             mK[b, g] += bk
             mV[b, g] += bv
@@ -101,33 +129,37 @@ def attn_prefill_bwd_magnitudes(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_
     if dims.n_shared:
         mqs = np.empty((B, T, d))
         for b in range(B):
-            a, bk, bv = causal_attention_bwd_magnitudes(q_sh[b], np.arange(T), K[b, dims.sg], V[b, dims.sg],
-                                                        do_sh[b], sc, None if o_sh is None else o_sh[b])
+            l_rows = None if lse is None else np.asarray(lse)[B * G * R + b * T:B * G * R + (b + 1) * T]
+            a, bk, bv = causal_attention_bwd_error_bound(q_sh[b], np.arange(T), K[b, dims.sg], V[b, dims.sg],
+                                                         do_sh[b], sc, None if o_sh is None else o_sh[b], l_rows)
             mqs[b] = a
             mK[b, dims.sg] += bk
             mV[b, dims.sg] += bv
     return mq, mqs, mK, mV
 
 
-def attn_prefill_bwd(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_routed=None, o_sh=None):
+def attn_prefill_bwd(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_routed=None, o_sh=None, lse=None):
     """Backward of attn_prefill: every selected expert's rows and the shared
     head's rows send their dK/dV into the KV group they read ([SN] §3-2 2), 5)).
 
     q_routed, do_routed [B, G, T, k, d]; q_sh, do_sh [B, T, d] or None;
-    K, V [B, G, T, d]; o_routed, o_sh: the forward output to take Delta from
-    (see causal_attention_bwd), or None.  Returns dq_routed, dq_sh, dK, dV.
+    K, V [B, G, T, d]; o_routed, o_sh: the forward output to take Delta from,
+    lse: the forward's log-sum-exp in gqe_attn_prefill's layout to take P
+    from (see causal_attention_bwd), or None.  Returns dq_routed, dq_sh, dK, dV.
     """
     B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
     sc = dims.sm_scale
+    R = T * k
     pos = np.repeat(np.arange(T), k)
     dq = np.empty((B, G, T, k, d))
     dK = np.zeros((B, G, T, d))
     dV = np.zeros((B, G, T, d))
     for b in range(B):
         for g in range(G):
-            o_rows = None if o_routed is None else np.asarray(o_routed[b, g]).reshape(T * k, d)
-            a, bk, bv = causal_attention_bwd(np.asarray(q_routed[b, g]).reshape(T * k, d), pos, K[b, g], V[b, g],
-                                             np.asarray(do_routed[b, g]).reshape(T * k, d), sc, o_rows)
+            o_rows = None if o_routed is None else np.asarray(o_routed[b, g]).reshape(R, d)
+            l_rows = None if lse is None else np.asarray(lse)[(b * G + g) * R:(b * G + g + 1) * R]
+            a, bk, bv = causal_attention_bwd(np.asarray(q_routed[b, g]).reshape(R, d), pos, K[b, g], V[b, g],
+                                             np.asarray(do_routed[b, g]).reshape(R, d), sc, o_rows, l_rows)
             dq[b, g] = a.reshape(T, k, d)
             dK[b, g] += bk
             dV[b, g] += bv
@@ -135,8 +167,9 @@ def attn_prefill_bwd(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_routed=None
     if dims.n_shared:
         dq_sh = np.empty((B, T, d))
         for b in range(B):
+            l_rows = None if lse is None else np.asarray(lse)[B * G * R + b * T:B * G * R + (b + 1) * T]
             a, bk, bv = causal_attention_bwd(q_sh[b], np.arange(T), K[b, dims.sg], V[b, dims.sg], do_sh[b], sc,
-                                             None if o_sh is None else o_sh[b])
+                                             None if o_sh is None else o_sh[b], l_rows)
             dq_sh[b] = a
             dK[b, dims.sg] += bk
             dV[b, dims.sg] += bv

@@ -44,22 +44,20 @@ BF16_U = 2.0 ** -8      # relative half-ulp of bf16 (8 significant bits)
 GRAD_MEAN_REL = 2e-3    # gradients: mean-abs error <= 2e-3 rms(ref)
 
 
-def assert_close_grad(got, ref, mag, what="", floor=1e-6):
-    """Gradients computed with bf16 MMA operands and stored as bf16.
-
-    Per element |err| <= 2^-8 (|ref| + mag) + floor: ``mag`` is the sum of the
-    magnitudes of the products that make up the element (the oracle's
-    *_magnitudes functions), so 2^-8 mag bounds the effect of rounding each
-    bf16 operand by at most half an ulp, and 2^-8 |ref| the bf16 rounding of
-    the result.  On top, mean-abs <= 2e-3 rms(ref)."""
+def assert_close_grad(got, ref, bound, what="", floor=1e-6):
+    """Gradients computed with bf16 MMA operands and fp32 accumulation, stored
+    as bf16.  Per element |err| <= 2^-8 |ref| + bound + floor, where ``bound``
+    is the worst-case error of the arithmetic before the final rounding (the
+    oracle's *_error_bound functions) and 2^-8 |ref| that rounding; on top,
+    mean-abs <= 2e-3 rms(ref)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
-    mag = np.asarray(mag, dtype=np.float64)
-    assert got.shape == ref.shape == mag.shape, (what, got.shape, ref.shape, mag.shape)
+    bound = np.asarray(bound, dtype=np.float64)
+    assert got.shape == ref.shape == bound.shape, (what, got.shape, ref.shape, bound.shape)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     err = np.abs(got - ref)
-    bound = BF16_U * (np.abs(ref) + mag) + floor
-    worst = float((err / bound).max())
+    tol = BF16_U * np.abs(ref) + bound + floor
+    worst = float((err / tol).max())
     s = max(float(np.sqrt(np.mean(ref * ref))), 1e-3)
     mean = float(err.mean()) / s
     assert worst <= 1.0 and mean <= GRAD_MEAN_REL, f"{what}: worst err/bound {worst:.3f}, mean-abs/rms {mean:.3e}"

@@ -54,17 +54,39 @@ def test_attention_gradients_match_finite_differences(k):
     _check(lambda a: L(q, K, a), V, dV, rng)
 
 
-def test_delta_from_the_forward_output_is_the_same_sum():
-    """Delta_r = sum_j P_rj dP_rj equals dO_r . o_r for the exact forward output."""
+def test_delta_and_p_from_the_forward_outputs_are_the_same():
+    """Delta_r = sum_j P_rj dP_rj equals dO_r . o_r, and exp(S - lse) equals the
+    softmax, for the exact forward output and log-sum-exp."""
     rng = np.random.default_rng(6)
     T, d, k = 7, 4, 2
     pos = np.repeat(np.arange(T), k)
     q, dO = rng.standard_normal((T * k, d)), rng.standard_normal((T * k, d))
     K, V = rng.standard_normal((T, d)), rng.standard_normal((T, d))
-    o = orc.causal_attention(q, pos, K, V, 0.6)
+    o, lse = orc.causal_attention(q, pos, K, V, 0.6, want_lse=True)
     for a, b in zip(ob.causal_attention_bwd(q, pos, K, V, dO, 0.6),
-                    ob.causal_attention_bwd(q, pos, K, V, dO, 0.6, O=o)):
+                    ob.causal_attention_bwd(q, pos, K, V, dO, 0.6, O=o, lse=lse)):
         np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-12)
+
+
+def test_backward_error_bound_covers_an_emulated_bf16_kernel():
+    """The error bound holds for an emulation of the kernel's arithmetic
+    (P and dS rounded to bf16 before the products, results rounded to bf16)."""
+    rng = np.random.default_rng(7)
+    T, d, k = 40, 16, 2
+    pos = np.repeat(np.arange(T), k)
+    bf = lambda a: gi.bf16_bits_to_f32(gi.f32_to_bf16_bits(np.asarray(a, np.float32))).astype(np.float64)
+    q, dO = bf(rng.standard_normal((T * k, d))), bf(rng.standard_normal((T * k, d)))
+    K, V = bf(rng.standard_normal((T, d))), bf(rng.standard_normal((T, d)))
+    sc = d ** -0.5
+    o, lse = orc.causal_attention(q, pos, K, V, sc, want_lse=True)
+    o = bf(o)
+    ref = ob.causal_attention_bwd(q, pos, K, V, dO, sc, O=o, lse=lse)
+    bound = ob.causal_attention_bwd_error_bound(q, pos, K, V, dO, sc, O=o, lse=lse)
+    P = np.exp(np.where(np.arange(T)[None, :] > pos[:, None], -np.inf, q @ K.T * sc) - lse[:, None])
+    dS = bf(sc * P * (dO @ V.T - np.sum(dO * o, axis=1, keepdims=True)))
+    emu = (bf(dS @ K), bf(dS.T @ q), bf(bf(P).T @ dO))
+    for e, r, b in zip(emu, ref, bound):
+        assert np.all(np.abs(e - r) <= 2.0 ** -8 * np.abs(r) + b + 1e-12)
 
 
 def test_attention_gradients_match_library_autograd():
