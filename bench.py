@@ -431,8 +431,10 @@ def main():
     ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-train", action="store_true")
     ap.add_argument("--kernel", default=None,
-                    help="time one call alone: attn | decode | router | qproj | kv | combine | linear | combine_out")
+                    help="time one call alone: attn | attn_bwd | layer_bwd | train_step | decode | router | qproj | kv | "
+                         "combine | linear | combine_out")
     ap.add_argument("--workload", default=WORKLOAD, choices=[k for k, v in gi.WORKLOADS.items() if not v.decode])
     ap.add_argument("--sweep", default=None, choices=["gqa"],
                     help="gqa: GQE against dense GQA, prefill T from 2K to 128K (one JSON line per T)")
@@ -630,6 +632,52 @@ def main():
         del Kc, Vc
         torch.cuda.empty_cache()
 
+    # ---------------- training sub-measurement: forward (keeping what the
+    # backward reads) + backward of the same layer on the same batch
+    training = None
+    if not args.no_train:
+        dy = torch.randn((dims.B, dims.T, dims.D), device=device).to(torch.bfloat16)
+        _, saved = layer.forward(x, keep=True)
+        for _ in range(3):
+            layer.backward(x, dy, saved)
+        torch.cuda.synchronize()
+        nt = max(3, min(args.steps, 20))
+        t0, t1, t2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        t0.record(stream)
+        for _ in range(nt):
+            layer.backward(x, dy, saved)
+        t1.record(stream)
+        for _ in range(nt):
+            _, saved = layer.forward(x, keep=True)
+            layer.backward(x, dy, saved)
+        t2.record(stream)
+        torch.cuda.synchronize()
+        bwd_ms = max_over_ranks(t0.elapsed_time(t1) / nt, dist, device)
+        step_ms = max_over_ranks(t1.elapsed_time(t2) / nt, dist, device)
+        # the attention backward alone (five products per query/key tile pair)
+        dc = gq.make_dims(dims)
+        ws_a = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_ATTN_BWD),), dtype=torch.uint8, device=device)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        bufs = [torch.empty_like(saved[n]) for n in ("q", "q_sh", "K", "V")]
+        call = lambda: gq.gqe_attn_prefill_bwd(dc, saved["q"], saved["q_sh"], saved["K"], saved["V"], saved["o"],  # noqa
+                                               saved["o_sh"], saved["lse"], saved["o"], saved["o_sh"], *bufs, ws_a)
+        call()
+        torch.cuda.synchronize()
+        a0.record(stream)
+        for _ in range(nt):
+            call()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ab_ms = a0.elapsed_time(a1) / nt
+        ab_tf = 2.5 * attn_useful_flops(dims) / ab_ms / 1e9
+        training = {"workload": f"{WORKLOAD}: forward(keep) + backward of the layer, dy ~ N(0,1)",
+                    "ms_per_step": step_ms, "backward_ms": bwd_ms,
+                    "tokens_per_s": world * dims.N / (step_ms / 1e3),
+                    "attn_bwd": {"ms": ab_ms, "tflops": ab_tf, "frac": ab_tf / peaks["bf16_tflops"],
+                                 "flops_note": "2.5 x the forward's useful causal FLOPs (five products per tile pair)"}}
+        del saved, bufs, ws_a
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline()
@@ -645,7 +693,7 @@ def main():
             "segments_ms": {n: float(seg_ms[:, i].mean()) for i, n in enumerate(seg_names)},
             "segments_note": "per-call CUDA events in separate L2-flushed steps; their sum exceeds "
                              "ms_per_step by the overlap of each kernel's launch with its predecessor",
-            "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "decode": decode,
+            "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "decode": decode, "training": training,
             "clocks": clocks.summary(), "gpu_launches": launches_per_step * args.steps,
             "device_error": err_code,
         }

@@ -391,10 +391,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
       ok = mbar_wait(&bar->dp_full, n & 1, abort, p.err, kErrTimeoutAttnBwd);
       if (!ok) break;
       tc_fence_after();
+      // dP^T chunks of 16 columns.  d = 128: the next chunk's load in flight
+      // while this one is used (measured faster there, slower at d = 64)
+      constexpr bool kPipe = C::kWide;
+      uint32_t dpb[2][16];
+      if (kPipe) {
+        tmem_ld16_async(tmem + lane_off + C::kDP + col0, dpb[0]);
+        tmem_wait_ld16(dpb[0]);
+      }
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
-        uint32_t dp[16];
-        tmem_ld16(tmem + lane_off + C::kDP + col0 + ch * 16, dp);
+        uint32_t* dp = dpb[ch & 1];
+        if (!kPipe)
+          tmem_ld16(tmem + lane_off + C::kDP + col0 + ch * 16, dp);
+        else if (ch < 3)
+          tmem_ld16_async(tmem + lane_off + C::kDP + col0 + (ch + 1) * 16, dpb[(ch + 1) & 1]);
         uint32_t dsk[8];
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
@@ -419,6 +430,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
           st_shared_v4(atom + ((piece ^ (r & 7)) << 4), dsk[j2 * 4], dsk[j2 * 4 + 1], dsk[j2 * 4 + 2],
                        dsk[j2 * 4 + 3]);
         }
+        if (kPipe && ch < 3) tmem_wait_ld16(dpb[(ch + 1) & 1]);
       }
       tmem_wait_st();
       fence_proxy_async_smem();
