@@ -173,6 +173,15 @@ gqe_status gqe_attn_prefill_bwd(const gqe_dims* dims, const gqe_bf16* q_routed, 
 gqe_status gqe_gemm(int M, int N, int K, const gqe_bf16* A, int a_kn, const gqe_bf16* B, int b_kn, gqe_bf16* C,
                     gqe_stream stream);
 
+/* C [M, N] (fp32) = (accumulate ? C : 0) + sum_k A(m, k) B(n, k): gqe_gemm's
+ * operand layouts with an fp32 result added into C by reduce-add (weight
+ * gradients; accumulate = 1 sums over micro-batches).  The K range is split
+ * over several CTAs when the output alone has too few tiles to fill the GPU,
+ * so the fp32 sums are taken in an order that may differ between runs.  Same
+ * shape rules as gqe_gemm. */
+gqe_status gqe_gemm_acc(int M, int N, int K, const gqe_bf16* A, int a_kn, const gqe_bf16* B, int b_kn, float* C,
+                        int accumulate, gqe_stream stream);
+
 /* Backward of the output construction ("GQE" study note §3-2 3) hard slots,
  * 4) weighted-sum slot, 5) shared head; §4-1: the weighted-sum slot is the
  * router's gradient path).  Per token, for selected (g, j) with weight w:
@@ -226,6 +235,9 @@ gqe_status gqe_bwd_pack_weights(const gqe_dims* dims, const gqe_bf16* Wr, const 
  * dst columns r in [rows, ld_dst) are zeroed (a K padded to a multiple of 64
  * for gqe_linear). */
 gqe_status gqe_transpose(int rows, int cols, const gqe_bf16* src, gqe_bf16* dst, int ld_dst, gqe_stream stream);
+
+/* gqe_transpose for fp32 (e.g. a weight gradient into its weight's layout). */
+gqe_status gqe_transpose_f32(int rows, int cols, const float* src, float* dst, int ld_dst, gqe_stream stream);
 
 /* Decode attention: one new token per sequence (dims->T must be 1) against a
  * dense cache (freeguideonline GQA tutorial, "自回归推理中的内存带宽优势": a

@@ -71,6 +71,8 @@ SIGNATURES = {
     "gqe_combine_out_proj": [_D, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "gqe_linear": [_I, _I, _I, _P, _P, _P, _P],
     "gqe_gemm": [_I, _I, _I, _P, _I, _P, _I, _P, _P],
+    "gqe_gemm_acc": [_I, _I, _I, _P, _I, _P, _I, _P, _I, _P],
+    "gqe_transpose_f32": [_I, _I, _P, _P, _I, _P],
     "gqe_combine_bwd": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
     "gqe_router_bwd": [_D, _P, _P, _P, _P, _P, _P, _P],
     "gqe_bwd_pack_cols": [_D, ctypes.POINTER(_I)],
@@ -286,6 +288,22 @@ def gqe_gemm(A, a_kn, B, b_kn, C, stream=None):
                                     _ptr(C, "C", b), _stream(stream)))
 
 
+def gqe_gemm_acc(A, a_kn, B, b_kn, C, accumulate=False, stream=None):
+    """C [M, N] fp32 = (C if accumulate else 0) + A B^T over K (layouts as gqe_gemm)."""
+    import torch
+    b = _bf16()
+    A2 = A.reshape(-1, A.shape[-1])
+    B2 = B.reshape(-1, B.shape[-1])
+    M, K = (A2.shape[1], A2.shape[0]) if a_kn else (A2.shape[0], A2.shape[1])
+    N, Kb = (B2.shape[1], B2.shape[0]) if b_kn else (B2.shape[0], B2.shape[1])
+    if K != Kb:
+        raise ValueError(f"K mismatch: {K} vs {Kb}")
+    if C.numel() != M * N:
+        raise ValueError(f"C has {C.numel()} elements, expected {M}x{N}")
+    _check("gqe_gemm_acc", lib.gqe_gemm_acc(M, N, K, _ptr(A, "A", b), int(a_kn), _ptr(B, "B", b), int(b_kn),
+                                            _ptr(C, "C", torch.float32), int(bool(accumulate)), _stream(stream)))
+
+
 def gqe_combine_bwd(dims, o_routed, o_sh, topk_w, dh, do_routed, do_sh, dtopk_w, stream=None):
     import torch
     b = _bf16()
@@ -333,6 +351,15 @@ def gqe_transpose(src, dst, ld_dst=None, stream=None):
     ld = rows if ld_dst is None else int(ld_dst)
     _check("gqe_transpose", lib.gqe_transpose(rows, cols, _ptr(src, "src", b), _ptr(dst, "dst", b), ld,
                                               _stream(stream)))
+
+
+def gqe_transpose_f32(src, dst, ld_dst=None, stream=None):
+    """dst [cols, ld_dst] <- src [rows, cols]^T, fp32."""
+    import torch
+    rows, cols = src.shape[0], src.numel() // src.shape[0]
+    ld = rows if ld_dst is None else int(ld_dst)
+    _check("gqe_transpose_f32", lib.gqe_transpose_f32(rows, cols, _ptr(src, "src", torch.float32),
+                                                      _ptr(dst, "dst", torch.float32), ld, _stream(stream)))
 
 
 def gqe_device_error(stream=None) -> int:

@@ -80,13 +80,6 @@ struct BwdCfg {
   static constexpr size_t Smem = 1024 + OffBar + sizeof(BwdBarriers);
 };
 
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
-  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(smem_u32(src)), "r"(c0), "r"(c1)
-               : "memory");
-}
-
 // One query tile of the item's walk.
 struct QTile {
   bool shared;

@@ -50,5 +50,6 @@ cudaError_t launch_router_bwd(const RouterBwdParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_pack(const PackParams& p, cudaStream_t stream);
 cudaError_t launch_transpose(const uint16_t* src, uint16_t* dst, int rows, int cols, int ld_dst,
                              cudaStream_t stream);
+cudaError_t launch_transpose_f32(const float* src, float* dst, int rows, int cols, int ld_dst, cudaStream_t stream);
 
 }  // namespace gqe

@@ -40,16 +40,6 @@ struct __align__(8) GemmBarriers {
   int abort;
 };
 
-int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  }
-  return n;
-}
-
 // One 32-column chunk of an output row: fp32 from tensor memory -> bf16 -> global.
 __device__ __forceinline__ void store_chunk(const EpiParams& ep, int map_sel, int row_dst, int n,
                                             const uint32_t* v) {
@@ -97,9 +87,43 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, int map_sel, 
 constexpr int kStageOutBytes = 32 * 64 * 2;
 constexpr int kEpiStagingBytes = 4 * 2 * kStageOutBytes;   // four epilogue warps
 
+// fp32 partial tiles (one K slice each) reduce-added into an fp32 [M, N]
+// tensor: 32 columns of the warp's 32 rows per 4 KB staging buffer.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile_reduce(const EpiParams& ep, const CUtensorMap* mo, int row0, int n0,
+                                                     uint32_t tmem_row, uint8_t* stg, int& chunk, bool ok) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    if (n0 + c0 >= ep.n_limit) break;
+    uint32_t v[32];
+    tmem_ld32(tmem_row + c0, v);
+    if (!ok) continue;
+    uint8_t* buf = stg + (chunk & 1) * kStageOutBytes;
+    if (chunk >= 2) {
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      st_shared_v4(buf + lane * 128 + ((j ^ (lane & 7)) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_reduce_add_2d(mo, buf, n0 + c0, row0);
+      bulk_commit();
+    }
+    ++chunk;
+  }
+}
+
 template <int BN>
 __device__ __forceinline__ void epilogue_tile_tma(const EpiParams& ep, const CUtensorMap* mo, int row0, int n0,
                                                   uint32_t tmem_row, uint8_t* stg, int& chunk, bool ok) {
+  if (ep.store_mode == kStoreReduceF32) {
+    epilogue_tile_reduce<BN>(ep, mo, row0, n0, tmem_row, stg, chunk, ok);
+    return;
+  }
   const int lane = threadIdx.x & 31;
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 64) {
@@ -168,7 +192,8 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = K / kBK;
   const int m_tiles = (M + kBM - 1) / kBM;
-  const int total = m_tiles * n_tiles_total;
+  const int ks_n = ep.ksplit > 1 ? ep.ksplit : 1;   // K split (fp32 reduce-add epilogue)
+  const int total = m_tiles * n_tiles_total * ks_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -197,11 +222,13 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
     if (lane == 0) {
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        const int mt = t / n_tiles_total, nt = t % n_tiles_total;
+        const int ks = t % ks_n, tt = t / ks_n;
+        const int mt = tt / n_tiles_total, nt = tt % n_tiles_total;
+        const int kb0 = (int)((long long)nk * ks / ks_n), kb1 = (int)((long long)nk * (ks + 1) / ks_n);
         const int sel = nt >= n_tiles_b0;
         const CUtensorMap* mB = sel ? &mapB1 : &mapB0;
         const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           if (it >= STAGES && !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, ep.err, kErrTimeoutGemm))
             break;
@@ -227,10 +254,12 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
       int it = 0, tc = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tc) {
         const int ab = tc & 1, use = tc >> 1;
+        const int ks = t % ks_n;
+        const int kb0 = (int)((long long)nk * ks / ks_n), kb1 = (int)((long long)nk * (ks + 1) / ks_n);
         if (tc >= 2 && !mbar_wait(&bar->acc_empty[ab], (use & 1) ^ 1, abort, ep.err, kErrTimeoutGemm)) break;
         tc_fence_after();
         const uint32_t acc = tmem + (uint32_t)(ab * BN);
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&bar->full[s], (it / STAGES) & 1, abort, ep.err, kErrTimeoutGemm)) break;
           tc_fence_after();
@@ -238,7 +267,7 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
           const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_ss(acc, operand_desc(a0, kk, mn & kMnA), operand_desc(b0, kk, mn & kMnB), idesc, (kb | kk) != 0);
+            umma_ss(acc, operand_desc(a0, kk, mn & kMnA), operand_desc(b0, kk, mn & kMnB), idesc, (kb != kb0 || kk != 0));
           umma_commit(&bar->empty[s]);
         }
         umma_commit(&bar->acc_full[ab]);
@@ -253,7 +282,8 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
       const int ab = tc & 1, use = tc >> 1;
       const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, ep.err, kErrTimeoutGemm);
       tc_fence_after();
-      const int mt = t / n_tiles_total, nt = t % n_tiles_total;
+      const int ks = t % ks_n, tt = t / ks_n;
+      const int mt = tt / n_tiles_total, nt = tt % n_tiles_total;
       const int sel = nt >= n_tiles_b0;
       const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
       const int row = mt * kBM + lg * 32 + lane;
@@ -310,7 +340,8 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   const int nk = K / kBK;
   const int m_tiles = (M + kPM - 1) / kPM;
-  const int total = m_tiles * n_tiles_total;
+  const int ks_n = ep.ksplit > 1 ? ep.ksplit : 1;   // K split (fp32 reduce-add epilogue)
+  const int total = m_tiles * n_tiles_total * ks_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -344,12 +375,14 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
       const uint32_t full0 = cluster_addr(&bar->full[0], 0);
       int it = 0;
       for (int t = pair; t < total && !*abort; t += n_pairs) {
-        const int mt = t / n_tiles_total, nt = t % n_tiles_total;
+        const int ks = t % ks_n, tt = t / ks_n;
+        const int mt = tt / n_tiles_total, nt = tt % n_tiles_total;
+        const int kb0 = (int)((long long)nk * ks / ks_n), kb1 = (int)((long long)nk * (ks + 1) / ks_n);
         const int sel = nt >= n_tiles_b0;
         const CUtensorMap* mB = sel ? &mapB1 : &mapB0;
         const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN + (int)rank * (BN / 2);
         const int m0 = mt * kPM + (int)rank * kBM;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           if (it >= STAGES && !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, ep.err, kErrTimeoutGemm))
             break;
@@ -389,10 +422,12 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
       int it = 0, tc = 0;
       for (int t = pair; t < total && !*abort; t += n_pairs, ++tc) {
         const int ab = tc & 1, use = tc >> 1;
+        const int ks = t % ks_n;
+        const int kb0 = (int)((long long)nk * ks / ks_n), kb1 = (int)((long long)nk * (ks + 1) / ks_n);
         if (tc >= 2 && !mbar_wait(&bar->acc_empty[ab], (use & 1) ^ 1, abort, ep.err, kErrTimeoutGemm)) break;
         tc_fence_after();
         const uint32_t acc = tmem + (uint32_t)(ab * BN);
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&bar->full[s], (it / STAGES) & 1, abort, ep.err, kErrTimeoutGemm)) break;
           tc_fence_after();
@@ -401,7 +436,7 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             umma_ss_pair(acc, operand_desc(a0, kk, mn & kMnA), operand_desc(b0, kk, mn & kMnB), idesc,
-                         (kb | kk) != 0);
+                         (kb != kb0 || kk != 0));
           umma_commit_pair(smem_u32(&bar->empty[s]));
           umma_commit_pair(empty_peer0 + (uint32_t)(s * sizeof(uint64_t)));
         }
@@ -419,7 +454,8 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
       const int ab = tc & 1, use = tc >> 1;
       const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, ep.err, kErrTimeoutGemm);
       tc_fence_after();
-      const int mt = t / n_tiles_total, nt = t % n_tiles_total;
+      const int ks = t % ks_n, tt = t / ks_n;
+      const int mt = tt / n_tiles_total, nt = tt % n_tiles_total;
       const int sel = nt >= n_tiles_b0;
       const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
       const int row0 = mt * kPM + (int)rank * kBM + lg * 32;
@@ -656,7 +692,7 @@ static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& m
   auto kern = gemm_dense_kernel<BN, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  const int tiles = ((M + kBM - 1) / kBM) * n_tiles_total;
+  const int tiles = ((M + kBM - 1) / kBM) * n_tiles_total * (ep.ksplit > 1 ? ep.ksplit : 1);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   return launch_kernel(kern, dim3(grid), dim3(192), smem, stream, 1, mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K,
                        n_tiles_b0, n_tiles_total, mn);
@@ -697,7 +733,7 @@ static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorM
     }
     mp = n;
   }
-  const int total = ((M + 255) / 256) * n_tiles_total;
+  const int total = ((M + 255) / 256) * n_tiles_total * (ep.ksplit > 1 ? ep.ksplit : 1);
   const int pairs = total < mp ? total : mp;
   return launch_kernel(kern, dim3(2 * pairs), dim3(192), smem, stream, 2, mapA, mapR, mapS, as, mapB0, mapB1,
                        mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, mn);
@@ -710,6 +746,16 @@ cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& m
   if (bn != 256) return cudaErrorInvalidValue;
   return launch_dense_pair_st<256, 6>(mapA, mapR, mapS, as, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0,
                                       n_tiles_total, stream, mn);
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
 }
 
 int dense_tile_n(int n_per_weight) { return (n_per_weight % 256 == 0) ? 256 : 128; }

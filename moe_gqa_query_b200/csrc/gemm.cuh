@@ -24,6 +24,7 @@ struct EpiParams {
   int T, G, d, L_max;
   unsigned* err;         // device error word
   int store_mode;        // dense kernels: kStorePerThread or a TMA store layout
+  int ksplit;            // kStoreReduceF32: K split into this many slices (<= 1: none)
 };
 
 // How the dense kernels write their output.
@@ -31,6 +32,7 @@ enum StoreMode : int {
   kStorePerThread = 0,   // each thread stores its row (any EpiMode)
   kStoreTma2d = 1,       // kEpiRowMajor through maps over [M, N], box 64 cols x 32 rows
   kStoreTmaHeads = 2,    // kEpiHeads through maps over [B*G, T, d], box 64 x 32 x 1 (T % 32 == 0)
+  kStoreReduceF32 = 3,   // fp32 tiles reduce-added into an fp32 [M, N] map, box 32 cols x 32 rows
 };
 
 // Token-to-expert permutation produced by perm.cu, consumed by the routed GEMM.
@@ -51,6 +53,7 @@ struct RoutedParams {
 
 // Output tile width for a weight with n_per_weight rows: 256 when it divides, else 128.
 int dense_tile_n(int n_per_weight);
+int num_sms();
 
 // mapO0 / mapO1: output maps for ep.store_mode != kStorePerThread.
 // mn: bit 0 -> A is stored [K, M] (map over [K rows, M cols], box 64 x 64),

@@ -649,6 +649,47 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, K, nt, nt, bn, S(stream)));
 }
 
+gqe_status gqe_gemm_acc(int M, int N, int K, const gqe_bf16* A, int a_kn, const gqe_bf16* B, int b_kn, float* C,
+                        int accumulate, gqe_stream stream) {
+  GQE_REQUIRE(M >= 1 && N >= 1 && K >= 1, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(A && B && C && (a_kn == 0 || a_kn == 1) && (b_kn == 0 || b_kn == 1), GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(N % 64 == 0, GQE_ERR_UNSUPPORTED);
+  GQE_REQUIRE((a_kn ? M : K) % 8 == 0 && (b_kn ? N : K) % 8 == 0, GQE_ERR_UNSUPPORTED);
+  GQE_REQUIRE((long long)M * N < (1ll << 31) && (long long)M * K < (1ll << 31) && (long long)N * K < (1ll << 31),
+              GQE_ERR_UNSUPPORTED);
+  GQE_REQUIRE(aligned16(A) && aligned16(B) && aligned16(C), GQE_ERR_INVALID_ARG);
+  const int Kp = (K + 63) / 64 * 64;
+  const int pbn = pair_tile_n(M, N);
+  const int bn = pbn ? pbn : dense_tile_n(N);
+  CUtensorMap mA, mW, mO;
+  if (a_kn) GQE_REQUIRE(map2d(&mA, A, M, K, 64), GQE_ERR_CUDA);
+  else GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
+  if (b_kn) GQE_REQUIRE(map2d(&mW, B, N, K, 64), GQE_ERR_CUDA);
+  else GQE_REQUIRE(map2d(&mW, B, K, N, pbn ? pbn / 2 : bn), GQE_ERR_CUDA);
+  GQE_REQUIRE(map2d_f32(&mO, C, N, M, 32), GQE_ERR_CUDA);
+  const int nt = (N + bn - 1) / bn;
+  // split K so that the output tiles times the slices fill the SMs once
+  const int tiles = pbn ? ((M + 255) / 256) * nt : ((M + 127) / 128) * nt;
+  const int slots = pbn ? num_sms() / 2 : num_sms();
+  int ksplit = tiles >= slots ? 1 : slots / tiles;
+  if (ksplit > Kp / 64) ksplit = Kp / 64;
+  if (ksplit > 16) ksplit = 16;
+  EpiParams ep{};
+  ep.mode = kEpiRowMajor;
+  ep.ldo = N;
+  ep.n_limit = N;
+  ep.err = error_word();
+  ep.store_mode = kStoreReduceF32;
+  ep.ksplit = ksplit;
+  if (!accumulate && cudaMemsetAsync(C, 0, (size_t)M * N * sizeof(float), S(stream)) != cudaSuccess)
+    return GQE_ERR_CUDA;
+  const int mn = (a_kn ? 1 : 0) | (b_kn ? 2 : 0);
+  if (pbn)
+    return cuda_status(launch_gemm_dense_pair(mA, mA, mA, ASource{kASingle, 0, 0, 0, 0, 0}, mW, mW, mO, mO, ep, M, Kp,
+                                              nt, nt, pbn, S(stream), mn));
+  return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, Kp, nt, nt, bn, S(stream), mn));
+}
+
 gqe_status gqe_combine_bwd(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe_bf16* o_sh,
                            const float* topk_w, const gqe_bf16* dh, gqe_bf16* do_routed, gqe_bf16* do_sh,
                            float* dtopk_w, gqe_stream stream) {
@@ -733,6 +774,13 @@ gqe_status gqe_transpose(int rows, int cols, const gqe_bf16* src, gqe_bf16* dst,
   GQE_REQUIRE(src && dst, GQE_ERR_INVALID_ARG);
   GQE_REQUIRE((long long)rows * cols < (1ll << 31) && (long long)cols * ld_dst < (1ll << 31), GQE_ERR_UNSUPPORTED);
   return cuda_status(launch_transpose(src, dst, rows, cols, ld_dst, S(stream)));
+}
+
+gqe_status gqe_transpose_f32(int rows, int cols, const float* src, float* dst, int ld_dst, gqe_stream stream) {
+  GQE_REQUIRE(rows >= 1 && cols >= 1 && ld_dst >= rows, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE(src && dst, GQE_ERR_INVALID_ARG);
+  GQE_REQUIRE((long long)rows * cols < (1ll << 31) && (long long)cols * ld_dst < (1ll << 31), GQE_ERR_UNSUPPORTED);
+  return cuda_status(launch_transpose_f32(src, dst, rows, cols, ld_dst, S(stream)));
 }
 
 gqe_status gqe_bwd_pack_weights(const gqe_dims* dims, const gqe_bf16* Wr, const gqe_bf16* Wq, const gqe_bf16* Wsh,

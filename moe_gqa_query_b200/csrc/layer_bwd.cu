@@ -187,9 +187,10 @@ __global__ void __launch_bounds__(256) bwd_pack_kernel(PackParams p) {
 // are zeroed.  64 x 64 tiles through shared memory.
 constexpr int kTr = 64;
 
-__global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst,
+template <typename Elem>
+__global__ void __launch_bounds__(256) transpose_kernel(const Elem* __restrict__ src, Elem* __restrict__ dst,
                                                         int rows, int cols, int ld_dst) {
-  __shared__ uint16_t tile[kTr][kTr + 2];
+  __shared__ Elem tile[kTr][kTr + 2];
   pdl_launch_dependents();
   pdl_wait();
   const int r0 = blockIdx.y * kTr, c0 = blockIdx.x * kTr;
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int c = c0 + tx * 2 + h;
-      tile[i][tx * 2 + h] = (r < rows && c < cols) ? src[(size_t)r * cols + c] : (uint16_t)0;
+      tile[i][tx * 2 + h] = (r < rows && c < cols) ? src[(size_t)r * cols + c] : Elem(0);
     }
   }
   __syncthreads();
@@ -241,7 +242,12 @@ cudaError_t launch_bwd_pack(const PackParams& p, cudaStream_t stream) {
 cudaError_t launch_transpose(const uint16_t* src, uint16_t* dst, int rows, int cols, int ld_dst,
                              cudaStream_t stream) {
   const dim3 grid((cols + kTr - 1) / kTr, (ld_dst + kTr - 1) / kTr);
-  return launch_kernel(transpose_kernel, grid, dim3(256), 0, stream, 1, src, dst, rows, cols, ld_dst);
+  return launch_kernel(transpose_kernel<uint16_t>, grid, dim3(256), 0, stream, 1, src, dst, rows, cols, ld_dst);
+}
+
+cudaError_t launch_transpose_f32(const float* src, float* dst, int rows, int cols, int ld_dst, cudaStream_t stream) {
+  const dim3 grid((cols + kTr - 1) / kTr, (ld_dst + kTr - 1) / kTr);
+  return launch_kernel(transpose_kernel<float>, grid, dim3(256), 0, stream, 1, src, dst, rows, cols, ld_dst);
 }
 
 }  // namespace gqe

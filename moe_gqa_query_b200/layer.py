@@ -146,8 +146,9 @@ class GQELayer:
     # ------------------------------------------------------------------ backward
     def backward(self, x: torch.Tensor, dy: torch.Tensor, saved: dict, stream=None) -> dict:
         """Gradients of <y, dy> for the forward(x, keep=True) that returned
-        `saved`: dx [B, T, D] and dWr, dbias (fp32), dWq, dWk, dWv, dWsh, dWo,
-        in the weights' layouts.  TopK passes no gradient; the router learns
+        `saved`: dx [B, T, D] (bf16) and the fp32 weight gradients dWr, dbias,
+        dWq, dWk, dWv, dWsh, dWo in the weights' layouts (summed over the
+        tokens by split-K GEMMs with fp32 reduce-add).  TopK passes no gradient; the router learns
         through the weighted-sum slot (output_mode 0) or the weighted hard
         slots (mode 2).  The returned tensors are the layer's own buffers,
         overwritten by the next backward.
@@ -168,8 +169,8 @@ class GQELayer:
         dy2 = dy.reshape(N, D)
         dh = buf("dh", (N, S))
         L.gqe_gemm(dy2, 0, self.Wo, 1, dh, stream)
-        dWo = buf("dWo", (D, S))
-        L.gqe_gemm(dy2, 1, saved["h"], 1, dWo, stream)
+        dWo = buf("dWo", (D, S), torch.float32)
+        L.gqe_gemm_acc(dy2, 1, saved["h"], 1, dWo, False, stream)
         # output construction, attention, router
         do = buf("do", (B, c.G, T, c.k, d))
         do_sh = buf("do_sh", (B, T, d)) if c.n_shared else None
@@ -193,14 +194,14 @@ class GQELayer:
         L.gqe_bwd_pack(dims, saved["idx"], dq, dq_sh, dK, dV, dlogits, A, stream)
         dx = buf("dx", (B, T, D))
         L.gqe_gemm(A, 0, Wcat, 1, dx, stream)
-        dWcat = buf("dWcat", (Kc, D))
-        L.gqe_gemm(A, 1, x.reshape(N, D), 1, dWcat, stream)
+        dWcat = buf("dWcat", (Kc, D), torch.float32)
+        L.gqe_gemm_acc(A, 1, x.reshape(N, D), 1, dWcat, False, stream)
         r0 = GE * d
         r1 = r0 + c.n_shared * d
         r2 = r1 + c.G * d
         r3 = r2 + c.G * d
-        dWr = buf("dWr", (D, GE))
-        L.gqe_transpose(dWcat[r3:r3 + GE], dWr, None, stream)
+        dWr = buf("dWr", (D, GE), torch.float32)
+        L.gqe_transpose_f32(dWcat[r3:r3 + GE], dWr, None, stream)
         return dict(dx=dx, dWr=dWr, dbias=dbias, dWq=dWcat[:r0].view(c.G, c.E, d, D),
                     dWsh=dWcat[r0:r1] if c.n_shared else None, dWk=dWcat[r1:r2], dWv=dWcat[r2:r3], dWo=dWo,
                     dh=dh, do=do, do_sh=do_sh, dw=dw, dq=dq, dq_sh=dq_sh, dK=dK, dV=dV, dlogits=dlogits)

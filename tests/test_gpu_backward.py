@@ -294,3 +294,34 @@ def test_gemm_rejects_unaligned_contiguous_k():
     C = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(gq.GQEError):
         gq.gqe_gemm(A, 0, Bm, 0, C)
+
+
+@pytest.mark.parametrize("a_kn,b_kn", [(1, 1), (0, 1), (0, 0)])
+@pytest.mark.parametrize("M,N,K", [(1024, 640, 16384), (2176, 1024, 4104), (200, 64, 72)],
+                         ids=["dWo_shape", "pair_split", "small"])
+def test_gemm_acc_fp32_split_k(M, N, K, a_kn, b_kn):
+    """C (fp32) += A B^T with K split over CTAs and fp32 reduce-add: added onto
+    the values already in C; error within fp32 accumulation of bf16 products."""
+    A = gi.normal_bf16(14, "x", (M, K), std=K ** -0.5)
+    Bm = gi.normal_bf16(15, "x", (N, K))
+    tA = bf16_dev(np.ascontiguousarray(A.T) if a_kn else A)
+    tB = bf16_dev(np.ascontiguousarray(Bm.T) if b_kn else Bm)
+    C0 = np.random.default_rng(3).standard_normal((M, N)).astype(np.float32)
+    C = torch.from_numpy(C0).cuda()
+    gq.gqe_gemm_acc(tA, a_kn, tB, b_kn, C, accumulate=True)
+    torch.cuda.synchronize()
+    Af, Bf = orc.f64(A), orc.f64(Bm)
+    ref = C0.astype(np.float64) + Af @ Bf.T
+    bound = K * 2.0 ** -24 * (np.abs(Af) @ np.abs(Bf).T) + 2.0 ** -23 * np.abs(ref) + 1e-6
+    got = C.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) <= bound), float((np.abs(got - ref) / bound).max())
+
+
+def test_gemm_acc_overwrites_without_accumulate():
+    A = gi.normal_bf16(16, "x", (300, 128), std=128 ** -0.5)
+    Bm = gi.normal_bf16(17, "x", (192, 128))
+    C = torch.full((300, 192), float("nan"), dtype=torch.float32, device="cuda")
+    gq.gqe_gemm_acc(bf16_dev(A), 0, bf16_dev(Bm), 0, C)
+    torch.cuda.synchronize()
+    ref = orc.f64(A) @ orc.f64(Bm).T
+    np.testing.assert_allclose(C.cpu().numpy(), ref, rtol=1e-4, atol=1e-4)
