@@ -28,10 +28,12 @@
 // two warpgroups computing P and dS, one key row per thread, warpgroup w on
 // query columns [64 w, 64 w + 64) (two warps per SM sub-partition hide each
 // other's latency); warps 12-15 drain dQ and write dK, dV at the end.
-// Tensor memory (d = 64): S^T 0 | dP^T 128 | dV 256 | dK 320 | dQ[2] 384, 448.
-// Warpgroup w writes its bf16 P^T (dS^T) into the first half of its own
-// S^T (dP^T) columns, so the two warpgroups never touch each other's columns;
-// the MMAs read the K = 128 query operand as two 64-query halves.
+// Tensor memory (d = 64): S^T 0 | dP^T 128 | dV 256 | dK 320 | dQ 384 | P^T 448.
+// P^T has columns of its own, so S^T(i+1) is issued as soon as both
+// warpgroups hold S^T(i) in registers (s_free), before dV(i) has read P^T(i);
+// warpgroup w writes its dS^T into the first half of its own dP^T columns (the
+// MMAs read that K = 128 query operand as two 64-query halves).  dK(i)
+// signals as soon as it has read dS^T(i), ahead of dQ(i), so dP^T(i+1) follows.
 // Tensor memory (d = 128): S^T 0 | dP^T 128 | dV 256 | dK 384, all 512 columns.
 // P^T goes to S^T's columns 0-63 and dS^T to its columns 64-127 (the two
 // warpgroups meet at a named barrier once both hold their S^T in registers);
@@ -52,7 +54,7 @@ constexpr int kBoxB = 128 * 64 * 2;   // one 128-row x 64-column bf16 TMA box
 struct __align__(8) BwdBarriers {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2], o_full[2], o_empty[2];
-  uint64_t s_full, p_full, pv_done, dp_full, ds_full, dk_done;
+  uint64_t s_full, s_free, p_full, pv_done, dp_full, ds_full, dk_done;
   uint64_t dq_full[2], dq_free[2];
   uint32_t tmem_base;
   int abort;
@@ -66,7 +68,8 @@ struct BwdCfg {
   static constexpr int OST = kWide ? 1 : 2;           // dO ring depth
   static constexpr int EpiCh = kWide ? 1 : D / 32;    // 32-column dQ chunks staged per warp at once
   static constexpr uint32_t kS = 0, kDP = 128, kDV = 256, kDK = 256 + D;
-  static constexpr uint32_t kDQ = kWide ? 128 : 256 + 2 * D;
+  static constexpr uint32_t kDQ = kWide ? 128 : 384;
+  static constexpr uint32_t kPT = 448;                // d = 64: P^T
   // shared memory, every operand region 1024-byte aligned
   static constexpr int OffK = 0;
   static constexpr int OffV = OffK + TileBytes;
@@ -113,7 +116,7 @@ __device__ __forceinline__ uint32_t half_col(uint32_t base, int ks) {
 }
 template <int D>
 __device__ __forceinline__ uint32_t pt_col(int ks) {
-  return D == 64 ? half_col(BwdCfg<D>::kS, ks) : BwdCfg<D>::kS + ks * 8;
+  return D == 64 ? BwdCfg<D>::kPT + ks * 8 : BwdCfg<D>::kS + ks * 8;
 }
 template <int D>
 __device__ __forceinline__ uint32_t dst_col(int ks) {
@@ -122,7 +125,7 @@ __device__ __forceinline__ uint32_t dst_col(int ks) {
 // Where warpgroup w writes its 32 packed columns of P^T and dS^T.
 template <int D>
 __device__ __forceinline__ uint32_t pt_wcol(int w) {
-  return D == 64 ? BwdCfg<D>::kS + 64 * w : BwdCfg<D>::kS + 32 * w;
+  return D == 64 ? BwdCfg<D>::kPT + 32 * w : BwdCfg<D>::kS + 32 * w;
 }
 template <int D>
 __device__ __forceinline__ uint32_t dst_wcol(int w) {
@@ -170,6 +173,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
       mbar_init(&bar->dq_free[st], 128);
     }
     mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->s_free, 256);
     mbar_init(&bar->p_full, 256);
     mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->dp_full, 1);
@@ -258,6 +262,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
       if (ok) ok = issue_s(0);
       if (ok) ok = issue_dp(0);
       for (int n = 0; ok && n < cnt; ++n) {
+        // d = 64: S^T(n+1) as soon as the warpgroups hold S^T(n) in registers
+        if (!C::kWide && n + 1 < cnt) {
+          if (!mbar_wait(&bar->s_free, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
+          if (!issue_s(n + 1)) break;
+        }
         // dV += P^T dO_i once P^T is in tensor memory
         if (!mbar_wait(&bar->p_full, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
         tc_fence_after();
@@ -270,11 +279,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
         umma_commit(&bar->q_empty[n & 1]);
         umma_commit(&bar->o_empty[n % C::OST]);
         if (n + 1 < cnt) {
-          // S^T(n+1) overwrites P^T(n) (and, at d = 128, dS^T(n)): wait for
-          // dV (and dK) to have read them
-          if (!mbar_wait(&bar->pv_done, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
-          if (C::kWide && !mbar_wait(&bar->dk_done, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
-          if (!issue_s(n + 1)) break;
+          // d = 128: S^T(n+1) overwrites P^T(n) and dS^T(n): wait for dV and dK
+          // to have read them
+          if (C::kWide) {
+            if (!mbar_wait(&bar->pv_done, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
+            if (!mbar_wait(&bar->dk_done, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
+            if (!issue_s(n + 1)) break;
+          }
           // dP^T(n+1) overwrites dS^T(n) (d = 64) or dQ(n) (d = 128)
           if (C::kWide) {
             if (!mbar_wait(&bar->dq_free[0], n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
@@ -302,19 +313,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
           umma_ts(tmem + C::kDK, tmem + dst_col<D>(ks), sdesc_sw128(q0 + ks * 2048, kBoxB, 1024), idesc_k,
                   (n > 0 || ks > 0));
         umma_commit(&bar->q_empty[n & 1]);
-        // d = 64: dQ double-buffered in its own columns.  d = 128: dQ over
-        // dP^T's columns, which the warpgroups have read (ds_full).
-        if (!C::kWide && n >= 2 &&
-            !mbar_wait(&bar->dq_free[b], ((n >> 1) - 1) & 1, abort, p.err, kErrTimeoutAttnBwd))
+        // d = 64: dK(n) has read dS^T(n) from dP^T's columns
+        if (!C::kWide) umma_commit(&bar->dk_done);
+        // dQ(n) over dQ(n-1): wait for the drain (d = 128: dQ sits over dP^T's
+        // columns, which the warpgroups have read, ds_full)
+        if (!C::kWide && n >= 1 &&
+            !mbar_wait(&bar->dq_free[0], (n - 1) & 1, abort, p.err, kErrTimeoutAttnBwd))
           break;
         tc_fence_after();
-        const uint32_t dq_col = C::kWide ? C::kDQ : C::kDQ + b * D;
+        const uint32_t dq_col = C::kDQ;
 #pragma unroll
         for (int ks = 0; ks < kTileB / 16; ++ks)
           umma_ss(tmem + dq_col, sdesc_sw128(ds0 + ks * 2048, kBoxB, 1024),
                   sdesc_sw128(k0 + ks * 2048, kBoxB, 1024), idesc_q, ks > 0);
-        umma_commit(&bar->dk_done);
-        umma_commit(&bar->dq_full[C::kWide ? 0 : b]);
+        if (C::kWide) umma_commit(&bar->dk_done);
+        umma_commit(&bar->dq_full[0]);
       }
     }
   } else if (warp >= 4 && warp < 12) {
@@ -343,6 +356,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
       for (int h = 0; h < 2 && ok; ++h) {
         uint32_t sv[32];
         tmem_ld32(tmem + lane_off + C::kS + col0 + h * 32, sv);
+        if (!C::kWide && h == 1) {
+          // S^T(n) is in registers: S^T(n+1) may be computed into its columns
+          tc_fence_before();
+          mbar_arrive(&bar->s_free);
+        }
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2 + h * 32 + c4 * 4);
@@ -357,6 +375,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
 #pragma unroll
         for (int c = 0; c < 64; ++c)
           if (c < cmin) pf[c] = 0.f;
+      }
+      if (!C::kWide) {
+        // P^T(n-1) must have been read by dV(n-1) before P^T(n) replaces it
+        if (n > 0) ok = mbar_wait(&bar->pv_done, (n - 1) & 1, abort, p.err, kErrTimeoutAttnBwd);
+        if (!ok) break;
+        tc_fence_after();
       }
       if (C::kWide) {
         // both warpgroups hold their S^T columns in registers before warpgroup 1
@@ -416,6 +440,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
         tmem_st8(tmem + lane_off + dst_wcol<D>(wg) + ch * 8, dsk);
         // ... and into the MN-major smem operand of dQ: the 64-query atom of
         // this warpgroup, [128 keys x 128 B], 16-byte pieces swizzled by key row
+        // (d = 64: once dQ(n-1) has read the previous tile's)
+        if (!C::kWide && ch == 0 && n > 0) {
+          ok = mbar_wait(&bar->dq_full[0], (n - 1) & 1, abort, p.err, kErrTimeoutAttnBwd);
+          if (!ok) break;
+        }
         uint8_t* atom = sDS + wg * kBoxB + r * 128;
 #pragma unroll
         for (int j2 = 0; j2 < 2; ++j2) {
@@ -438,13 +467,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
     uint8_t* stage = smem + C::OffEpi + qd * C::EpiCh * 4096;
     bool ok = true;
     for (int n = 0; n < cnt && ok; ++n) {
-      const int b = C::kWide ? 0 : (n & 1);
-      const int ph = C::kWide ? (n & 1) : ((n >> 1) & 1);
+      const int b = 0;
+      const int ph = n & 1;
       const QTile q = qtile(p, s, jt, n_r, n);
       ok = mbar_wait(&bar->dq_full[b], ph, abort, p.err, kErrTimeoutAttnBwd);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t dq_col = C::kWide ? C::kDQ : C::kDQ + b * D;
+      const uint32_t dq_col = C::kDQ;
 #pragma unroll
       for (int g0 = 0; g0 < D / 32; g0 += C::EpiCh) {
         // staging free: every earlier reduce of this warp has read it
