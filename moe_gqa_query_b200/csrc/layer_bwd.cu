@@ -18,67 +18,67 @@ namespace gqe {
 
 namespace {
 
-__device__ __forceinline__ float bf16_to_f(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
-__device__ __forceinline__ uint16_t f_to_bf16(float f) {
-  return (uint16_t)(pack_bf16x2(f, 0.f) & 0xFFFFu);
+// ---------------------------------------------------------------- combine backward
+// One thread per 8 elements (16 bytes) of a selected head row: d/8 threads
+// per (token, g, j), the p~ gradient summed over them by shuffles; the shared
+// slot is copied by the threads of (token, g = 0, j = 0).
+__device__ __forceinline__ void unpack8(uint4 v, float* f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = bf16_lo(w[e]);
+    f[2 * e + 1] = bf16_hi(w[e]);
+  }
 }
 
-// ---------------------------------------------------------------- combine backward
-// One warp per token; each lane holds d/32 consecutive elements of a head row.
-template <int VEC>
 __global__ void __launch_bounds__(256) combine_bwd_kernel(CombineBwdParams p) {
   pdl_launch_dependents();
   pdl_wait();
-  const int warp = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
-  const int lane = threadIdx.x & 31;
-  const int N = p.B * p.T;
-  if (warp >= N) return;
-  const int n = warp, b = n / p.T, t = n % p.T;
-  const int d = p.d, Gk = p.G * p.k;
+  const int tpr = p.d / 8;                     // threads per head row
+  const int Gk = p.G * p.k;
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = gt / tpr;              // (token, g, j)
+  const int part = (int)(gt % tpr);
+  const bool live = row < (long long)p.B * p.T * Gk;
+  const long long rr = live ? row : 0;
+  const int n = (int)(rr / Gk), gj = (int)(rr % Gk);
+  const int g = gj / p.k, j = gj % p.k;
+  const int b = n / p.T, t = n % p.T;
+  const int d = p.d, e0 = part * 8;
   const gqe_bf16_t* dh = p.dh + (size_t)n * p.slots * d;
-  const int e0 = lane * VEC;
-  float route[VEC];
+  const size_t orow = ((((size_t)b * p.G + g) * p.T + t) * p.k + j) * d;
+  float hard[8], o[8], dov[8];
+  unpack8(*reinterpret_cast<const uint4*>(dh + gj * d + e0), hard);
+  unpack8(*reinterpret_cast<const uint4*>(p.o_routed + orow + e0), o);
+  const float w = p.w[(size_t)n * Gk + gj];
+  float dot = 0.f;
   if (p.output_mode == 0) {
+    float route[8];
+    unpack8(*reinterpret_cast<const uint4*>(dh + Gk * d + e0), route);
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) route[v] = bf16_to_f(dh[Gk * d + e0 + v]);
-  }
-  for (int gj = 0; gj < Gk; ++gj) {
-    const int g = gj / p.k, j = gj % p.k;
-    const size_t orow = ((((size_t)b * p.G + g) * p.T + t) * p.k + j) * d;
-    const float w = p.w[(size_t)n * Gk + gj];
-    float hard[VEC], o[VEC], dov[VEC];
-    float dot = 0.f;
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-      hard[v] = bf16_to_f(dh[gj * d + e0 + v]);
-      o[v] = bf16_to_f(p.o_routed[orow + e0 + v]);
+    for (int v = 0; v < 8; ++v) {
+      dov[v] = hard[v] + w * route[v];
+      dot += route[v] * o[v];
     }
-    if (p.output_mode == 0) {
+  } else if (p.output_mode == 1) {
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) {
-        dov[v] = hard[v] + w * route[v];
-        dot += route[v] * o[v];
-      }
-    } else if (p.output_mode == 1) {
+    for (int v = 0; v < 8; ++v) dov[v] = hard[v];
+  } else {
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) dov[v] = hard[v];
-    } else {
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) {
-        dov[v] = w * hard[v];
-        dot += hard[v] * o[v];
-      }
+    for (int v = 0; v < 8; ++v) {
+      dov[v] = w * hard[v];
+      dot += hard[v] * o[v];
     }
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) p.do_routed[orow + e0 + v] = f_to_bf16(dov[v]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-    if (lane == 0) p.dw[(size_t)n * Gk + gj] = dot;
   }
-  if (p.n_shared) {
+  if (live)
+    *reinterpret_cast<uint4*>(p.do_routed + orow + e0) =
+        make_uint4(pack_bf16x2(dov[0], dov[1]), pack_bf16x2(dov[2], dov[3]), pack_bf16x2(dov[4], dov[5]),
+                   pack_bf16x2(dov[6], dov[7]));
+  for (int off = tpr >> 1; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+  if (live && part == 0) p.dw[(size_t)n * Gk + gj] = dot;
+  if (live && p.n_shared && gj == 0) {
     const int col = Gk * d + (p.output_mode == 0 ? d : 0);
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) p.do_sh[(size_t)n * d + e0 + v] = dh[col + e0 + v];
+    *reinterpret_cast<uint4*>(p.do_sh + (size_t)n * d + e0) = *reinterpret_cast<const uint4*>(dh + col + e0);
   }
 }
 
@@ -139,47 +139,48 @@ __global__ void __launch_bounds__(kRouterBwdThreads) router_bwd_kernel(RouterBwd
 }
 
 // ---------------------------------------------------------------- pack
-// One warp per token row of A [N, Kc]; 8-byte (4 x bf16) pieces per lane.
+// One thread per 16 bytes (8 columns) of A [N, Kc]: consecutive threads write
+// consecutive chunks of a row.
 __global__ void __launch_bounds__(256) bwd_pack_kernel(PackParams p) {
   pdl_launch_dependents();
   pdl_wait();
-  const int warp = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
-  const int lane = threadIdx.x & 31;
-  const int N = p.B * p.T;
-  if (warp >= N) return;
-  const int n = warp, b = n / p.T, t = n % p.T;
+  const int cpr = p.Kc / 8;                    // chunks per row
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gt >= (long long)p.B * p.T * cpr) return;
+  const int n = (int)(gt / cpr), c = (int)(gt % cpr) * 8;
+  const int b = n / p.T, t = n % p.T;
   const int d = p.d;
-  uint16_t* row = p.A + (size_t)n * p.Kc;
-  const int* idx = p.idx + (size_t)n * p.G * p.k;
-  // dq scattered into the expert columns: block (g, e) of d columns
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
   const int n_q = p.G * p.E * d;
-  for (int c = lane * 4; c < n_q; c += 128) {
+  const int c_sh = n_q, c_k = c_sh + p.n_shared * d, c_v = c_k + p.G * d, c_l = c_v + p.G * d;
+  if (c < n_q) {
+    // dq scattered into the expert columns: block (g, e) of d columns
     const int blk = c / d, e_in = c % d;
     const int g = blk / p.E, e = blk % p.E;
-    uint2 v = make_uint2(0u, 0u);
+    const int* idx = p.idx + (size_t)n * p.G * p.k + g * p.k;
     for (int j = 0; j < p.k; ++j)
-      if (idx[g * p.k + j] == e)
-        v = *reinterpret_cast<const uint2*>(p.dq + ((((size_t)b * p.G + g) * p.T + t) * p.k + j) * d + e_in);
-    *reinterpret_cast<uint2*>(row + c) = v;
-  }
-  int col = n_q;
-  if (p.n_shared) {
-    for (int c = lane * 4; c < d; c += 128)
-      *reinterpret_cast<uint2*>(row + col + c) = *reinterpret_cast<const uint2*>(p.dq_sh + (size_t)n * d + c);
-    col += d;
-  }
-  for (int which = 0; which < 2; ++which) {
-    const uint16_t* src = which ? p.dV : p.dK;
-    for (int c = lane * 4; c < p.G * d; c += 128) {
-      const int g = c / d, e_in = c % d;
-      *reinterpret_cast<uint2*>(row + col + c) =
-          *reinterpret_cast<const uint2*>(src + (((size_t)b * p.G + g) * p.T + t) * d + e_in);
+      if (idx[j] == e)
+        v = *reinterpret_cast<const uint4*>(p.dq + ((((size_t)b * p.G + g) * p.T + t) * p.k + j) * d + e_in);
+  } else if (c < c_k) {
+    v = *reinterpret_cast<const uint4*>(p.dq_sh + (size_t)n * d + (c - c_sh));
+  } else if (c < c_l) {
+    const uint16_t* src = c < c_v ? p.dK : p.dV;
+    const int cc = c < c_v ? c - c_k : c - c_v;
+    const int g = cc / d, e_in = cc % d;
+    v = *reinterpret_cast<const uint4*>(src + (((size_t)b * p.G + g) * p.T + t) * d + e_in);
+  } else {
+    const int GE = p.G * p.E;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c0 = c - c_l + 2 * e;
+      const float lo = c0 < GE ? p.dlogits[(size_t)n * GE + c0] : 0.f;
+      const float hi = c0 + 1 < GE ? p.dlogits[(size_t)n * GE + c0 + 1] : 0.f;
+      w[e] = pack_bf16x2(lo, hi);
     }
-    col += p.G * d;
+    v = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  const int GE = p.G * p.E;
-  for (int c = lane; c < p.Kc - col; c += 32)
-    row[col + c] = c < GE ? f_to_bf16(p.dlogits[(size_t)n * GE + c]) : (uint16_t)0;
+  *reinterpret_cast<uint4*>(p.A + (size_t)n * p.Kc + c) = v;
 }
 
 // ---------------------------------------------------------------- transpose
@@ -218,10 +219,8 @@ __global__ void __launch_bounds__(256) transpose_kernel(const Elem* __restrict__
 }  // namespace
 
 cudaError_t launch_combine_bwd(const CombineBwdParams& p, cudaStream_t stream) {
-  const int N = p.B * p.T;
-  const dim3 grid((N + 7) / 8);
-  if (p.d == 64) return launch_kernel(combine_bwd_kernel<2>, grid, dim3(256), 0, stream, 1, p);
-  return launch_kernel(combine_bwd_kernel<4>, grid, dim3(256), 0, stream, 1, p);
+  const long long threads = (long long)p.B * p.T * p.G * p.k * (p.d / 8);
+  return launch_kernel(combine_bwd_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, stream, 1, p);
 }
 
 cudaError_t launch_router_bwd(const RouterBwdParams& p, cudaStream_t stream) {
@@ -235,8 +234,8 @@ cudaError_t launch_router_bwd(const RouterBwdParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_pack(const PackParams& p, cudaStream_t stream) {
-  const int N = p.B * p.T;
-  return launch_kernel(bwd_pack_kernel, dim3((N + 7) / 8), dim3(256), 0, stream, 1, p);
+  const long long threads = (long long)p.B * p.T * (p.Kc / 8);
+  return launch_kernel(bwd_pack_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, stream, 1, p);
 }
 
 cudaError_t launch_transpose(const uint16_t* src, uint16_t* dst, int rows, int cols, int ld_dst,
