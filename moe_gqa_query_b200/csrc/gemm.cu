@@ -173,12 +173,12 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk, int mn_m
 
 // ---------------------------------------------------------------------------
 // dense: A [M, K] and W [N, K] by TMA; persistent over (m-tile, n-tile)
-template <int BN, int STAGES>
+template <int BN, int STAGES, int mn>
 __global__ void __launch_bounds__(192, 1)
 gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                   const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapO0,
                   const __grid_constant__ CUtensorMap mapO1, EpiParams ep, int M, int K, int n_tiles_b0,
-                  int n_tiles_total, int mn) {
+                  int n_tiles_total) {
   constexpr int kBTileBytes = BN * kBK * 2;
   constexpr uint32_t kTmemCols = 2 * BN;
   extern __shared__ uint8_t smem_raw[];
@@ -233,13 +233,13 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
           if (it >= STAGES && !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, ep.err, kErrTimeoutGemm))
             break;
           mbar_arrive_expect_tx(&bar->full[s], kATileBytes + kBTileBytes);
-          if (mn & kMnA) {
+          if constexpr ((mn & kMnA) != 0) {
             for (int h = 0; h < kBM / 64; ++h)
               tma_load_2d(sA + s * kATileBytes + h * kMnBox, &mapA, &bar->full[s], mt * kBM + h * 64, kb * kBK);
           } else {
             tma_load_2d(sA + s * kATileBytes, &mapA, &bar->full[s], kb * kBK, mt * kBM);
           }
-          if (mn & kMnB) {
+          if constexpr ((mn & kMnB) != 0) {
             for (int h = 0; h < BN / 64; ++h)
               tma_load_2d(sB + s * kBTileBytes + h * kMnBox, mB, &bar->full[s], n0 + h * 64, kb * kBK);
           } else {
@@ -250,7 +250,7 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, BN, (mn & kMnA) != 0, (mn & kMnB) != 0);
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, (mn & kMnA) != 0, (mn & kMnB) != 0);
       int it = 0, tc = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tc) {
         const int ab = tc & 1, use = tc >> 1;
@@ -315,14 +315,14 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
 // 16 + 32 KB for the same MMA work: a third fewer bytes through L2 per FLOP.
 // Both CTAs' loads count on the even CTA's `full` barrier; the even CTA's MMA
 // thread releases stages and accumulators in both CTAs with one commit each.
-template <int BN, int STAGES>
+template <int BN, int STAGES, int mn>
 __global__ void __launch_bounds__(192, 1)
 gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapR,
                        const __grid_constant__ CUtensorMap mapS, ASource as,
                        const __grid_constant__ CUtensorMap mapB0,
                        const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapO0,
                        const __grid_constant__ CUtensorMap mapO1, EpiParams ep, int M, int K, int n_tiles_b0,
-                       int n_tiles_total, int mn) {
+                       int n_tiles_total) {
   constexpr int kPM = 2 * kBM;                       // pair tile rows
   constexpr int kHalfB = (BN / 2) * kBK * 2;         // this CTA's half of the W k-block
   constexpr uint32_t kTmemCols = 2 * BN;
@@ -388,7 +388,7 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             break;
           if (rank == 0) mbar_arrive_expect_tx(&bar->full[s], 2 * (kATileBytes + kHalfB));
           const uint32_t fb = full0 + (uint32_t)(s * sizeof(uint64_t));
-          if (as.mode == kASingle && (mn & kMnA)) {
+          if ((mn & kMnA) != 0 && as.mode == kASingle) {
             for (int h = 0; h < kBM / 64; ++h)
               tma_load_2d_pair(sA + s * kATileBytes + h * kMnBox, &mapA, fb, m0 + h * 64, kb * kBK);
           } else if (as.mode == kASingle) {
@@ -405,7 +405,7 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
               tma_load_2d_pair(sA + s * kATileBytes, (slot == kG && as.route) ? &mapR : &mapS, fb, sub, m0);
             }
           }
-          if (mn & kMnB) {
+          if constexpr ((mn & kMnB) != 0) {
             for (int h = 0; h < BN / 128; ++h)
               tma_load_2d_pair(sB + s * kHalfB + h * kMnBox, mB, fb, n0 + h * 64, kb * kBK);
           } else {
@@ -416,7 +416,7 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kPM, BN, (mn & kMnA) != 0, (mn & kMnB) != 0);
+      constexpr uint32_t idesc = idesc_bf16_f32(kPM, BN, (mn & kMnA) != 0, (mn & kMnB) != 0);
       const uint32_t empty_peer0 = cluster_addr(&bar->empty[0], peer);
       const uint32_t accf_peer0 = cluster_addr(&bar->acc_full[0], peer);
       int it = 0, tc = 0;
@@ -689,13 +689,16 @@ static cudaError_t launch_dense_bn(const CUtensorMap& mapA, const CUtensorMap& m
                                    const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M,
                                    int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream, int mn) {
   const size_t smem = 1024 + STAGES * (kATileBytes + BN * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
-  auto kern = gemm_dense_kernel<BN, STAGES>;
+  auto kern = mn == 3   ? gemm_dense_kernel<BN, STAGES, 3>
+              : mn == 2 ? gemm_dense_kernel<BN, STAGES, 2>
+              : mn == 1 ? gemm_dense_kernel<BN, STAGES, 1>
+                        : gemm_dense_kernel<BN, STAGES, 0>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int tiles = ((M + kBM - 1) / kBM) * n_tiles_total * (ep.ksplit > 1 ? ep.ksplit : 1);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   return launch_kernel(kern, dim3(grid), dim3(192), smem, stream, 1, mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K,
-                       n_tiles_b0, n_tiles_total, mn);
+                       n_tiles_b0, n_tiles_total);
 }
 
 template <int BN, int STAGES>
@@ -705,7 +708,10 @@ static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorM
                                         int M, int K, int n_tiles_b0, int n_tiles_total, cudaStream_t stream,
                                         int mn) {
   const size_t smem = 1024 + STAGES * (kATileBytes + (BN / 2) * kBK * 2) + kEpiStagingBytes + sizeof(GemmBarriers);
-  auto kern = gemm_dense_pair_kernel<BN, STAGES>;
+  auto kern = mn == 3   ? gemm_dense_pair_kernel<BN, STAGES, 3>
+              : mn == 2 ? gemm_dense_pair_kernel<BN, STAGES, 2>
+              : mn == 1 ? gemm_dense_pair_kernel<BN, STAGES, 1>
+                        : gemm_dense_pair_kernel<BN, STAGES, 0>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
@@ -736,7 +742,7 @@ static cudaError_t launch_dense_pair_st(const CUtensorMap& mapA, const CUtensorM
   const int total = ((M + 255) / 256) * n_tiles_total * (ep.ksplit > 1 ? ep.ksplit : 1);
   const int pairs = total < mp ? total : mp;
   return launch_kernel(kern, dim3(2 * pairs), dim3(192), smem, stream, 2, mapA, mapR, mapS, as, mapB0, mapB1,
-                       mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, mn);
+                       mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total);
 }
 
 cudaError_t launch_gemm_dense_pair(const CUtensorMap& mapA, const CUtensorMap& mapR, const CUtensorMap& mapS,
