@@ -313,6 +313,13 @@ gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, 
  * internal waits runs out of time (0 = none).  Synchronises `stream`. */
 gqe_status gqe_device_error(int* code, gqe_stream stream);
 
+/* Failure-path check: launches one thread that waits, through the kernels'
+ * own bounded wait (about one second of GPU time), on a barrier nothing ever
+ * completes.  When the limit passes it records code 0x7F1 in the device error
+ * word (read and cleared by gqe_device_error) and returns: the context stays
+ * usable.  No fault, no trap. */
+gqe_status gqe_debug_wait_timeout(gqe_stream stream);
+
 /* Diagnostics.  Evaluates the attention kernel's exponential helpers on n
  * fp32 inputs (device arrays): y_poly the polynomial exp2 used on the FMA
  * pipe, y_pair its packed two-lane form, y_hw the hardware exp2 (MUFU).  For

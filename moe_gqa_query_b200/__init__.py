@@ -12,6 +12,6 @@ from ._lib import (  # noqa: F401
     gqe_attn_prefill, gqe_attn_prefill_bwd, gqe_attn_decode, gqe_attn_decode_noalloc, DECODE_NOALLOC_MAX_BYTES, gqe_combine,
     gqe_combine_out_proj, gqe_linear, gqe_device_error, gqe_gemm, gqe_gemm_acc, gqe_combine_bwd, gqe_router_bwd, gqe_bwd_pack_cols,
     gqe_bwd_pack, gqe_bwd_pack_weights, gqe_transpose, gqe_transpose_f32,
-    gqe_status_string, gqe_debug_exp2,
+    gqe_status_string, gqe_debug_exp2, gqe_debug_wait_timeout,
 )
 from .layer import GQEConfig, GQELayer  # noqa: F401

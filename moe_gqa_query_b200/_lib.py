@@ -81,6 +81,7 @@ SIGNATURES = {
     "gqe_transpose": [_I, _I, _P, _P, _I, _P],
     "gqe_device_error": [ctypes.POINTER(_I), _P],
     "gqe_debug_exp2": [_P, _P, _P, _P, _I, _P],
+    "gqe_debug_wait_timeout": [_P],
     "gqe_status_string": [_I],
 }
 
@@ -366,6 +367,10 @@ def gqe_device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     _check("gqe_device_error", lib.gqe_device_error(ctypes.byref(code), _stream(stream)))
     return int(code.value)
+
+
+def gqe_debug_wait_timeout(stream=None):
+    _check("gqe_debug_wait_timeout", lib.gqe_debug_wait_timeout(_stream(stream)))
 
 
 def gqe_debug_exp2(x, y_poly, y_pair, y_hw, stream=None):

@@ -16,6 +16,9 @@ struct AttnParams {
   unsigned* err;          // device error word
 };
 
+// diag.cu: a bounded wait that runs out (failure-path test)
+cudaError_t launch_debug_wait(unsigned* err, cudaStream_t stream);
+
 cudaError_t launch_attn_prefill(const CUtensorMap& mQ, const CUtensorMap& mQs, const CUtensorMap& mK,
                                 const CUtensorMap& mV, const AttnParams& p, int d,
                                 cudaStream_t stream);

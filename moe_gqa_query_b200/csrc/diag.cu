@@ -17,7 +17,28 @@ __global__ void exp2_diag_kernel(const float* __restrict__ x, float* y_poly, flo
   y_hw[i] = ex2(v);
 }
 
+// One thread waits, through the kernels' own bounded wait, on an mbarrier that
+// nothing ever arrives at: after the wait limit it records kErrTimeoutDebug in
+// the error word and the kernel returns normally.
+__global__ void debug_wait_kernel(unsigned* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    volatile int* abort = &abort_flag;
+    mbar_wait(&bar, 0, abort, err, kErrTimeoutDebug);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_debug_wait(unsigned* err, cudaStream_t stream) {
+  debug_wait_kernel<<<1, 32, 0, stream>>>(err);
+  return cudaGetLastError();
+}
+
 }  // namespace gqe
 
 extern "C" gqe_status gqe_debug_exp2(const float* x, float* y_poly, float* y_pair, float* y_hw, int n,

@@ -846,6 +846,12 @@ gqe_status gqe_gemm(int M, int N, int K, const gqe_bf16* A, int a_kn, const gqe_
   return cuda_status(launch_gemm_dense(mA, mW, mW, mO, mO, ep, M, Kp, nt, nt, bn, S(stream), mn));
 }
 
+gqe_status gqe_debug_wait_timeout(gqe_stream stream) {
+  unsigned* err = error_word();
+  GQE_REQUIRE(err, GQE_ERR_CUDA);
+  return cuda_status(launch_debug_wait(err, S(stream)));
+}
+
 gqe_status gqe_device_error(int* code, gqe_stream stream) {
   GQE_REQUIRE(code, GQE_ERR_INVALID_ARG);
   unsigned v = 0;

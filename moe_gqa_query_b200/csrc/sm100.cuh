@@ -20,6 +20,7 @@ enum DeviceErrorCode : unsigned {
   kErrTimeoutAttnBwd = 0x202,
   kErrTimeoutDecode = 0x301,
   kErrTimeoutRouter = 0x401,
+  kErrTimeoutDebug = 0x7F1,   // gqe_debug_wait_timeout: a wait that nothing completes
 };
 
 // A wait gives up after this long (the longest legitimate wait is a few ms).
