@@ -107,10 +107,11 @@ __device__ __forceinline__ QTile qtile(const AttnBwdParams& p, int s, int jt, in
   return q;
 }
 
-// Tensor-memory column of the bf16 query operand's k-step ks (16 queries).
-// d = 64: queries [0, 64) packed at base + [0, 32), [64, 128) at
-// base + 64 + [0, 32) (each warpgroup inside its own fp32 columns).
-// d = 128: P^T contiguous at S^T's columns 0-63, dS^T at 64-127.
+// Tensor-memory column of a bf16 query operand's k-step ks (16 queries).
+// P^T: contiguous, in columns of its own (d = 64) or S^T's columns 0-63
+// (d = 128).  dS^T: d = 64, queries [0, 64) packed at dP^T + [0, 32) and
+// [64, 128) at dP^T + 64 + [0, 32) (each warpgroup inside its own fp32
+// columns); d = 128, contiguous at S^T's columns 64-127.
 __device__ __forceinline__ uint32_t half_col(uint32_t base, int ks) {
   return base + (ks >> 2) * 64 + (ks & 3) * 8;
 }
@@ -304,7 +305,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
       constexpr uint32_t idesc_q = idesc_bf16_f32(kTileB, D, true, true);
       const uint32_t k0 = smem_u32(sK), ds0 = smem_u32(sDS);
       for (int n = 0; n < cnt; ++n) {
-        const int b = n & 1;
         if (!mbar_wait(&bar->ds_full, n & 1, abort, p.err, kErrTimeoutAttnBwd)) break;
         tc_fence_after();
         const uint32_t q0 = smem_u32(smem + C::OffQ + (n & 1) * C::TileBytes);

@@ -282,7 +282,7 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
       const int ab = tc & 1, use = tc >> 1;
       const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, ep.err, kErrTimeoutGemm);
       tc_fence_after();
-      const int ks = t % ks_n, tt = t / ks_n;
+      const int tt = t / ks_n;   // the K slice (t % ks_n) does not change where the tile goes
       const int mt = tt / n_tiles_total, nt = tt % n_tiles_total;
       const int sel = nt >= n_tiles_b0;
       const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
@@ -454,7 +454,7 @@ gemm_dense_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
       const int ab = tc & 1, use = tc >> 1;
       const bool ok = mbar_wait(&bar->acc_full[ab], use & 1, abort, ep.err, kErrTimeoutGemm);
       tc_fence_after();
-      const int ks = t % ks_n, tt = t / ks_n;
+      const int tt = t / ks_n;   // the K slice (t % ks_n) does not change where the tile goes
       const int mt = tt / n_tiles_total, nt = tt % n_tiles_total;
       const int sel = nt >= n_tiles_b0;
       const int n0 = (sel ? nt - n_tiles_b0 : nt) * BN;
