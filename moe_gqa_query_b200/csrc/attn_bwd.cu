@@ -313,8 +313,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
           umma_ts(tmem + C::kDK, tmem + dst_col<D>(ks), sdesc_sw128(q0 + ks * 2048, kBoxB, 1024), idesc_k,
                   (n > 0 || ks > 0));
         umma_commit(&bar->q_empty[n & 1]);
-        // d = 64: dK(n) has read dS^T(n) from dP^T's columns
-        if (!C::kWide) umma_commit(&bar->dk_done);
+        // dK(n) has read dS^T(n) (d = 64: from dP^T's columns, d = 128: from
+        // S^T's): signal before dQ(n), so dP^T(n+1) / S^T(n+1) may follow
+        umma_commit(&bar->dk_done);
         // dQ(n) over dQ(n-1): wait for the drain (d = 128: dQ sits over dP^T's
         // columns, which the warpgroups have read, ds_full)
         if (!C::kWide && n >= 1 &&
@@ -326,7 +327,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant_
         for (int ks = 0; ks < kTileB / 16; ++ks)
           umma_ss(tmem + dq_col, sdesc_sw128(ds0 + ks * 2048, kBoxB, 1024),
                   sdesc_sw128(k0 + ks * 2048, kBoxB, 1024), idesc_q, ks > 0);
-        if (C::kWide) umma_commit(&bar->dk_done);
         umma_commit(&bar->dq_full[0]);
       }
     }
