@@ -132,3 +132,61 @@ def test_package_fails_loudly_without_library(tmp_path, monkeypatch):
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
     sys.modules.pop("gqe_lib_probe", None)
+
+
+# ---------------------------------------------------------------------------
+# backward calls: sizes and argument checks (host side only)
+
+def test_attention_backward_workspace_size():
+    """LSE2 and Delta per padded query row (routed rows of each (b, g) padded to
+    128, then the shared head's), 256-byte aligned, then the fp32 dQ accumulator."""
+    for cfg in (_cfg(B=8, T=2048, D=1024, G=8, E=2, k=1), _cfg(B=2, T=300, D=256, G=3, E=4, k=3, d=128),
+                _cfg(B=1, T=70, D=128, G=2, E=2, k=2)):
+        for n_shared in (0, 1):
+            d = gq.make_dims(cfg, n_shared=n_shared)
+            rows_pad = -(-cfg.T * cfg.k // 128) * 128
+            rows_pad_sh = -(-cfg.T // 128) * 128
+            n = cfg.B * cfg.G * rows_pad + n_shared * cfg.B * rows_pad_sh
+            a256 = lambda b: -(-b // 256) * 256
+            assert gq.gqe_workspace_size(d, gq.GQE_OP_ATTN_BWD) == 2 * a256(4 * n) + 4 * n * cfg.d
+
+
+def test_backward_pack_columns():
+    """Kc = G*E*d (dq per expert) + n_shared*d + 2*G*d (dK, dV) + d logits padded to 64."""
+    for cfg, n_shared in ((_cfg(B=8, T=2048, D=1024, G=8, E=2, k=1), 1), (_cfg(G=4, E=8, k=4, d=128), 1),
+                          (_cfg(G=3, E=3, k=2), 0), (_cfg(G=8, E=8, k=1), 1)):
+        d = gq.make_dims(cfg, n_shared=n_shared)
+        GE = cfg.G * cfg.E
+        want = GE * cfg.d + n_shared * cfg.d + 2 * cfg.G * cfg.d + 64 * (-(-GE // 64))
+        assert gq.gqe_bwd_pack_cols(d) == want
+    assert gq.gqe_bwd_pack_cols(gq.make_dims(_cfg(B=8, T=2048, D=1024, G=8, E=2, k=1))) == 2176
+
+
+def test_backward_calls_reject_bad_arguments_before_launch():
+    d = gq.make_dims(_cfg())
+    lib = _lib.lib
+    assert lib.gqe_attn_prefill_bwd(ctypes.byref(d), *([None] * 14), 0, None) == 1
+    assert lib.gqe_combine_bwd(ctypes.byref(d), None, None, None, None, None, None, None, None) == 1
+    assert lib.gqe_router_bwd(ctypes.byref(d), None, None, None, None, None, None, None) == 1
+    assert lib.gqe_bwd_pack(ctypes.byref(d), None, None, None, None, None, None, None, None) == 1
+    assert lib.gqe_bwd_pack_weights(ctypes.byref(d), None, None, None, None, None, None, None) == 1
+    # a short attention-backward workspace
+    assert lib.gqe_attn_prefill_bwd(ctypes.byref(d), *([256] * 13), 256, 16, None) == 3
+    # transposes: empty or a destination narrower than the source's rows
+    assert lib.gqe_transpose(0, 64, 16, 16, 64, None) == 1
+    assert lib.gqe_transpose(100, 64, 16, 16, 64, None) == 1
+    assert lib.gqe_transpose_f32(100, 64, 16, 16, 64, None) == 1
+
+
+@pytest.mark.parametrize("fn", ["gqe_gemm", "gqe_gemm_acc"])
+def test_gemm_argument_checks(fn):
+    lib = _lib.lib
+    call = (lambda M, N, K, A, ak, B, bk, C: lib.gqe_gemm(M, N, K, A, ak, B, bk, C, None)) if fn == "gqe_gemm" \
+        else (lambda M, N, K, A, ak, B, bk, C: lib.gqe_gemm_acc(M, N, K, A, ak, B, bk, C, 0, None))
+    assert call(0, 64, 64, 16, 0, 16, 0, 16) == 1          # empty
+    assert call(64, 64, 64, None, 0, 16, 0, 16) == 1       # null operand
+    assert call(64, 64, 64, 16, 2, 16, 0, 16) == 1         # layout flag not 0/1
+    assert call(64, 96, 64, 16, 0, 16, 0, 16) == 2         # N not a multiple of 64
+    assert call(64, 64, 70, 16, 0, 16, 0, 16) == 2         # contiguous K not a multiple of 8
+    assert call(60, 64, 70, 16, 1, 16, 1, 16) == 2         # contiguous M not a multiple of 8
+    assert call(64, 64, 64, 18, 0, 16, 0, 16) == 1         # misaligned A
