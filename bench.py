@@ -188,14 +188,18 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle on a bounded sample
 
-def cpu_baseline(seconds_budget=20.0):
-    import oracle as orc
-    cores = os.cpu_count()
+def oracle_threads():
+    """Threads the oracle's BLAS actually uses (os.cpu_count() when unknown)."""
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 0) for i in threadpool_info()] + [1])
+        return max([i.get("num_threads", 0) for i in threadpool_info()] + [1])
     except Exception:
-        pass
+        return os.cpu_count()
+
+
+def cpu_baseline(seconds_budget=20.0):
+    import oracle as orc
+    cores = oracle_threads()
     w = gi.WORKLOADS[WORKLOAD]
     dims = w.dims.replace(B=1)           # one 2048-token sequence of the workload
     x = gi.layer_input(w.dims, rows=[0])
@@ -224,14 +228,15 @@ def run_reference(args):
     dims = w.dims.replace(B=1)
     x = gi.layer_input(w.dims, rows=[0])
     Wt = gi.layer_weights(dims)
+    bias = gi.router_bias(w)
     for _ in range(min(args.warmup, 1)):
-        orc.gqe_forward(x, Wt, dims)
+        orc.gqe_forward(x, Wt, dims, bias)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        orc.gqe_forward(x, Wt, dims)
+        orc.gqe_forward(x, Wt, dims, bias)
     dt = time.perf_counter() - t0
     value = args.steps * dims.N / dt
-    cores = os.cpu_count()
+    cores = oracle_threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

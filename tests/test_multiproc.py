@@ -4,8 +4,11 @@ The GQE path does not shard across GPUs here: each rank runs its own replica.
 The only cross-rank steps are the barrier around the timed region and the max
 over ranks of the measured time; these run as world_size-2 gloo ranks.
 """
+import json
 import os
 import socket
+import subprocess
+import sys
 
 import pytest
 import torch
@@ -56,3 +59,35 @@ def test_work_counts():
     assert bench.attn_useful_flops(main) == pytest.approx(3.867e10, rel=1e-3)
     dec = gi.WORKLOADS["decode"]
     assert bench.decode_attn_bytes(dec.dims, dec.L) == pytest.approx(4.295e9, rel=1e-3)
+
+
+def _bench(args, env_extra):
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **env_extra)
+    return subprocess.run([sys.executable, "bench.py", *args], cwd=root, env=env, capture_output=True,
+                          text=True, timeout=600)
+
+
+def test_reference_arm_json_line():
+    """`bench.py --impl reference`: the oracle timed on the host cores, one JSON
+    line with the main arm's metric, unit and direction, a cpu_baseline that
+    describes the run and an e2e object with no host-device bytes."""
+    r = _bench(["--impl", "reference", "--steps", "1", "--warmup", "0"], {})
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    import bench
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["steps"] == 1 and line["n_gpus"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    """Under torchrun only rank 0 runs and prints the reference arm."""
+    r = _bench(["--impl", "reference", "--steps", "1", "--warmup", "0", "--gpus", "2"],
+               {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
