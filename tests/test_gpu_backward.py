@@ -325,3 +325,53 @@ def test_gemm_acc_overwrites_without_accumulate():
     torch.cuda.synchronize()
     ref = orc.f64(A) @ orc.f64(Bm).T
     np.testing.assert_allclose(C.cpu().numpy(), ref, rtol=1e-4, atol=1e-4)
+
+
+# ----------------------------------------------------------------------------
+# the packed projection-gradient matrix (layout only: bit-exact)
+
+PACK_CASES = {
+    "main_like": D(B=2, T=300, D=128, G=8, E=2, k=1, d=64),
+    "wide_k4_d128": D(B=1, T=130, D=128, G=4, E=8, k=4, d=128),
+    "E3_k2_no_shared": D(B=2, T=77, D=128, G=3, E=3, k=2, d=64, n_shared=0),
+    "GE64": D(B=1, T=70, D=128, G=16, E=4, k=1, d=64),
+}
+
+
+@pytest.mark.parametrize("case", list(PACK_CASES))
+def test_bwd_pack_bit_exact(case):
+    """A = [dq in its expert's columns (zeros elsewhere) | dq_sh | dK | dV |
+    dlogits as bf16 (round to nearest even), zero padding], compared bit for
+    bit with the same packing done on the host."""
+    dims = PACK_CASES[case]
+    B, T, G, E, k, d, N = dims.B, dims.T, dims.G, dims.E, dims.k, dims.d, dims.N
+    idx = gi.random_routing(dims, 2)
+    rng = np.random.default_rng(9)
+    bits = lambda *shape: gi.f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))  # noqa: E731
+    dq, dK, dV = bits(B, G, T, k, d), bits(B, G, T, d), bits(B, G, T, d)
+    dqs = bits(B, T, d) if dims.n_shared else None
+    dl = rng.standard_normal((N, G * E), dtype=np.float32)
+    dc = gq.make_dims(dims)
+    Kc = gq.gqe_bwd_pack_cols(dc)
+    A = torch.full((N, Kc), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gq.gqe_bwd_pack(dc, torch.from_numpy(idx).cuda(), bf16_dev(dq), None if dqs is None else bf16_dev(dqs),
+                    bf16_dev(dK), bf16_dev(dV), torch.from_numpy(dl).cuda(), A)
+    torch.cuda.synchronize()
+    want = np.zeros((N, Kc), dtype=np.uint16)
+    n = np.arange(N)
+    b, t = n // T, n % T
+    for g in range(G):
+        for j in range(k):
+            cols = (g * E + idx[:, g, j])[:, None] * d + np.arange(d)[None, :]
+            want[n[:, None], cols] = dq[b, g, t, j]
+    c = G * E * d
+    if dqs is not None:
+        want[:, c:c + d] = dqs.reshape(N, d)
+        c += d
+    for src in (dK, dV):
+        for g in range(G):
+            want[:, c + g * d:c + (g + 1) * d] = src[b, g, t]
+        c += G * d
+    want[:, c:c + G * E] = gi.f32_to_bf16_bits(dl)
+    got = A.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, want)
