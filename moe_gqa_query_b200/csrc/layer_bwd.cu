@@ -139,55 +139,48 @@ __global__ void __launch_bounds__(kRouterBwdThreads) router_bwd_kernel(RouterBwd
 }
 
 // ---------------------------------------------------------------- pack
-// Threads (x, y) of a 64 x 4 block: x walks the 16-byte chunks (8 columns) of
-// a row of A [N, Kc], consecutive threads writing consecutive chunks; y picks
-// one of four rows, and the grid strides over rows.  No 64-bit division: the
-// head width d (64 or 128) is a power of two.
-constexpr int kPackX = 64, kPackY = 4;
-
-__global__ void __launch_bounds__(kPackX * kPackY) bwd_pack_kernel(PackParams p) {
+// One thread per 16 bytes (8 columns) of A [N, Kc]: consecutive threads write
+// consecutive chunks of a row.
+__global__ void __launch_bounds__(256) bwd_pack_kernel(PackParams p) {
   pdl_launch_dependents();
   pdl_wait();
   const int cpr = p.Kc / 8;                    // chunks per row
-  const int chunk = blockIdx.x * kPackX + threadIdx.x;
-  if (chunk >= cpr) return;
-  const int c = chunk * 8;
-  const int N = p.B * p.T;
-  const int d = p.d, dsh = 31 - __clz(d);
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gt >= (long long)p.B * p.T * cpr) return;
+  const int n = (int)(gt / cpr), c = (int)(gt % cpr) * 8;
+  const int b = n / p.T, t = n % p.T;
+  const int d = p.d;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
   const int n_q = p.G * p.E * d;
   const int c_sh = n_q, c_k = c_sh + p.n_shared * d, c_v = c_k + p.G * d, c_l = c_v + p.G * d;
-  for (int n = blockIdx.y * kPackY + threadIdx.y; n < N; n += gridDim.y * kPackY) {
-    const int b = n / p.T, t = n - b * p.T;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (c < n_q) {
-      // dq scattered into the expert columns: block (g, e) of d columns
-      const int blk = c >> dsh, e_in = c & (d - 1);
-      const int g = blk / p.E, e = blk - g * p.E;
-      const int* idx = p.idx + ((size_t)n * p.G + g) * p.k;
-      for (int j = 0; j < p.k; ++j)
-        if (idx[j] == e)
-          v = *reinterpret_cast<const uint4*>(p.dq + ((((size_t)b * p.G + g) * p.T + t) * p.k + j) * d + e_in);
-    } else if (c < c_k) {
-      v = *reinterpret_cast<const uint4*>(p.dq_sh + (size_t)n * d + (c - c_sh));
-    } else if (c < c_l) {
-      const uint16_t* src = c < c_v ? p.dK : p.dV;
-      const int cc = c < c_v ? c - c_k : c - c_v;
-      const int g = cc >> dsh, e_in = cc & (d - 1);
-      v = *reinterpret_cast<const uint4*>(src + (((size_t)b * p.G + g) * p.T + t) * d + e_in);
-    } else {
-      const int GE = p.G * p.E;
-      uint32_t w[4];
+  if (c < n_q) {
+    // dq scattered into the expert columns: block (g, e) of d columns
+    const int blk = c / d, e_in = c % d;
+    const int g = blk / p.E, e = blk % p.E;
+    const int* idx = p.idx + (size_t)n * p.G * p.k + g * p.k;
+    for (int j = 0; j < p.k; ++j)
+      if (idx[j] == e)
+        v = *reinterpret_cast<const uint4*>(p.dq + ((((size_t)b * p.G + g) * p.T + t) * p.k + j) * d + e_in);
+  } else if (c < c_k) {
+    v = *reinterpret_cast<const uint4*>(p.dq_sh + (size_t)n * d + (c - c_sh));
+  } else if (c < c_l) {
+    const uint16_t* src = c < c_v ? p.dK : p.dV;
+    const int cc = c < c_v ? c - c_k : c - c_v;
+    const int g = cc / d, e_in = cc % d;
+    v = *reinterpret_cast<const uint4*>(src + (((size_t)b * p.G + g) * p.T + t) * d + e_in);
+  } else {
+    const int GE = p.G * p.E;
+    uint32_t w[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c0 = c - c_l + 2 * e;
-        const float lo = c0 < GE ? p.dlogits[(size_t)n * GE + c0] : 0.f;
-        const float hi = c0 + 1 < GE ? p.dlogits[(size_t)n * GE + c0 + 1] : 0.f;
-        w[e] = pack_bf16x2(lo, hi);
-      }
-      v = make_uint4(w[0], w[1], w[2], w[3]);
+    for (int e = 0; e < 4; ++e) {
+      const int c0 = c - c_l + 2 * e;
+      const float lo = c0 < GE ? p.dlogits[(size_t)n * GE + c0] : 0.f;
+      const float hi = c0 + 1 < GE ? p.dlogits[(size_t)n * GE + c0 + 1] : 0.f;
+      w[e] = pack_bf16x2(lo, hi);
     }
-    *reinterpret_cast<uint4*>(p.A + (size_t)n * p.Kc + c) = v;
+    v = make_uint4(w[0], w[1], w[2], w[3]);
   }
+  *reinterpret_cast<uint4*>(p.A + (size_t)n * p.Kc + c) = v;
 }
 
 // ---------------------------------------------------------------- transpose
@@ -241,12 +234,8 @@ cudaError_t launch_router_bwd(const RouterBwdParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_pack(const PackParams& p, cudaStream_t stream) {
-  if ((p.d & (p.d - 1)) != 0) return cudaErrorInvalidValue;   // d is 64 or 128
-  const int N = p.B * p.T;
-  const int gx = (p.Kc / 8 + kPackX - 1) / kPackX;
-  const int rows = (N + kPackY - 1) / kPackY;
-  const int gy = rows < 65535 ? rows : 65535;
-  return launch_kernel(bwd_pack_kernel, dim3(gx, gy), dim3(kPackX, kPackY), 0, stream, 1, p);
+  const long long threads = (long long)p.B * p.T * (p.Kc / 8);
+  return launch_kernel(bwd_pack_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, stream, 1, p);
 }
 
 cudaError_t launch_transpose(const uint16_t* src, uint16_t* dst, int rows, int cols, int ld_dst,
