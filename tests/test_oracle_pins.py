@@ -98,6 +98,30 @@ def test_margin_definition():
     assert np.isinf(orc.selection_margin(s, 4)).all()
 
 
+def test_near_tie_alternatives_sets():
+    """The near-tie helper the router parity tests use: for a (token, group)
+    whose k-th/(k+1)-th logit margin is under 1e-4, the experts within 1e-4 of
+    the k-th logit are undecided and those clearly above it are sure; clear
+    groups and k = E give no entry."""
+    s = np.array([[[1.0, 1.00005, 0.2, -0.3],      # k=1: a two-way tie on top
+                   [3.0, 0.0, -1.0, 0.5]],         # clear
+                  [[2.0, 1.0, 1.00003, 0.0],       # k=2: expert 0 sure, 1 and 2 tied for 2nd
+                   [0.1, 0.1, 0.1, 0.1]]])         # four-way tie
+    r1 = {"logits": s, "margin": orc.selection_margin(s, 1)}
+    alt1 = orc.near_tie_alternatives(r1, 1)
+    assert set(alt1) == {(0, 0), (1, 1)}
+    sure, und = alt1[(0, 0)]
+    assert sure.tolist() == [] and und.tolist() == [0, 1]
+    sure, und = alt1[(1, 1)]
+    assert sure.tolist() == [] and und.tolist() == [0, 1, 2, 3]
+    r2 = {"logits": s, "margin": orc.selection_margin(s, 2)}
+    alt2 = orc.near_tie_alternatives(r2, 2)
+    assert set(alt2) == {(1, 0), (1, 1)}
+    sure, und = alt2[(1, 0)]
+    assert sure.tolist() == [0] and und.tolist() == [1, 2]
+    assert orc.near_tie_alternatives({"logits": s, "margin": orc.selection_margin(s, 4)}, 4) == {}
+
+
 def test_router_bias_is_added_per_expert():
     rng = np.random.default_rng(3)
     x = _rand(rng, 10, 6)
