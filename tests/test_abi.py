@@ -21,6 +21,39 @@ def test_library_exports_every_header_function():
         assert n in names
 
 
+def _header_prototypes():
+    """name -> list of parameter declarations, from include/gqe.h."""
+    import re
+    with open(_lib.HEADER_PATH) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*(?:const\s+)?\w+\*?\s+\*?(gqe_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.M):
+        params = [p.strip() for p in m.group(2).replace("\n", " ").split(",") if p.strip()]
+        out[m.group(1)] = [] if params == ["void"] else params
+    return out
+
+
+def test_bindings_match_header_prototypes():
+    """Every declared function has a ctypes signature with the same number of
+    parameters, and each parameter's kind agrees: pointers (and the stream
+    handle) as pointers, size_t as size_t, int (and the status enum) as int."""
+    protos = _header_prototypes()
+    assert set(protos) == set(gq.header_functions())
+    for name, params in protos.items():
+        sig = _lib.SIGNATURES.get(name)
+        assert sig is not None, f"{name} has no binding"
+        assert len(sig) == len(params), f"{name}: header {len(params)} parameters, binding {len(sig)}"
+        for decl, t in zip(params, sig):
+            if "*" in decl or decl.startswith("gqe_stream"):
+                assert t is ctypes.c_void_p or issubclass(t, ctypes._Pointer), f"{name}: {decl}"
+            elif decl.startswith("size_t"):
+                assert t is ctypes.c_size_t, f"{name}: {decl}"
+            elif decl.startswith("int") or decl.startswith("gqe_status"):   # the status enum is an int
+                assert t is ctypes.c_int, f"{name}: {decl}"
+            else:
+                raise AssertionError(f"{name}: unexpected parameter {decl}")
+
+
 def test_library_is_built_for_sm100a():
     with open(gq.LIB_PATH, "rb") as f:
         blob = f.read()
