@@ -95,7 +95,10 @@ class GQELayer:
     def forward(self, x: torch.Tensor, stream=None, keep=False, out=None) -> torch.Tensor:
         """x [B, T, D] bf16 on the device -> y [B, T, D] bf16 (into `out` when given).
 
-        keep=True also returns the intermediates (router outputs, q, K, V, o, h).
+        keep=True also returns the intermediates (router outputs and probabilities,
+        q, K, V, o, the log-sum-exp, h) that backward() reads.  They are the
+        layer's own buffers: the next forward overwrites them, so run the
+        backward of a step before the next step's forward.
         """
         c = self.cfg
         B, T = x.shape[0], x.shape[1]
