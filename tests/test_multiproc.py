@@ -1,8 +1,10 @@
-"""Host logic of the N-GPU benchmark (independent replicas) on CPU ranks.
+"""Host logic of the benchmark, on CPU.
 
 The GQE path does not shard across GPUs here: each rank runs its own replica.
 The only cross-rank steps are the barrier around the timed region and the max
-over ranks of the measured time; these run as world_size-2 gloo ranks.
+over ranks of the measured time; these run as world_size-2 gloo ranks.  Also:
+the work counts behind the roofline, the reference arm's JSON line, the
+traffic lookup that follows the captured kernel source, and the peak fallback.
 """
 import json
 import os
@@ -91,3 +93,36 @@ def test_reference_arm_other_ranks_exit_quietly():
                {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_roofline_traffic_follows_the_captured_source(tmp_path, monkeypatch):
+    """The bench reports a kernel's ncu DRAM traffic only while the kernel's
+    source file still hashes to the captured version; a label without a
+    capture gives null."""
+    import shutil
+    import bench
+    label = "attn_prefill_single_kernel (d=64)"
+    got = bench.profiled_traffic(label)
+    assert got == 52472064 + 1871104
+    assert bench.profiled_traffic("no such kernel") is None
+    # the same capture against an edited copy of the source
+    (tmp_path / "profiles").mkdir()
+    shutil.copy(os.path.join(bench.ROOT, "profiles", "traffic.json"), tmp_path / "profiles" / "traffic.json")
+    src = tmp_path / "moe_gqa_query_b200" / "csrc" / "attn_prefill.cu"
+    src.parent.mkdir(parents=True)
+    shutil.copy(os.path.join(bench.ROOT, "moe_gqa_query_b200", "csrc", "attn_prefill.cu"), src)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic(label) == got
+    src.write_text(src.read_text() + "\n// edited\n")
+    assert bench.profiled_traffic(label) is None
+
+
+def test_peaks_fall_back_without_the_measured_file(tmp_path, monkeypatch):
+    import bench
+    p = bench.load_peaks()
+    if os.path.exists(os.path.join(bench.ROOT, "MEASURED_PEAKS.json")):
+        assert p["source"] == "measured" and p["bf16_tflops"] > 0 and p["hbm_gbs"] > 0
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f = bench.load_peaks()
+    assert f["source"] == "fallback"
+    assert (f["hbm_gbs"], f["bf16_tflops"]) == (6650.0, 1590.0)
