@@ -19,8 +19,6 @@ context, a wide 8-expert group with skewed routing, and a decode step against a
 from __future__ import annotations
 
 import dataclasses
-import math
-
 import numpy as np
 
 # tensor ids for the seeded streams
@@ -69,10 +67,6 @@ class GQEDims:
     def h_active(self) -> int:
         """Query heads whose attention is computed per token: k*G + n_shared."""
         return self.k * self.G + self.n_shared
-
-    @property
-    def sm_scale(self) -> float:
-        return self.scale if self.scale else 1.0 / math.sqrt(self.d)
 
     def replace(self, **kw) -> "GQEDims":
         return dataclasses.replace(self, **kw)

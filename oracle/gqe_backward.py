@@ -28,7 +28,7 @@ import numpy as np
 
 from .gqe_oracle import (
     f64, router_logits, group_softmax, topk_select, renormalise, routed_qproj,
-    kv_proj, attn_prefill, combine,
+    kv_proj, attn_prefill, attention_scale, combine,
 )
 
 
@@ -109,7 +109,7 @@ def attn_prefill_bwd_error_bound(q_routed, q_sh, K, V, do_routed, do_sh, dims, o
     outputs.  lse: the forward's fp32 log-sum-exp in gqe_attn_prefill's layout
     (routed rows, then shared rows), or None."""
     B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
-    sc = dims.sm_scale
+    sc = attention_scale(dims)
     R = T * k
     pos = np.repeat(np.arange(T), k)
     mq = np.empty((B, G, T, k, d))
@@ -148,7 +148,7 @@ def attn_prefill_bwd(q_routed, q_sh, K, V, do_routed, do_sh, dims, o_routed=None
     from (see causal_attention_bwd), or None.  Returns dq_routed, dq_sh, dK, dV.
     """
     B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
-    sc = dims.sm_scale
+    sc = attention_scale(dims)
     R = T * k
     pos = np.repeat(np.arange(T), k)
     dq = np.empty((B, G, T, k, d))

@@ -44,6 +44,8 @@ float64; everything is computed in float64.
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 
@@ -190,6 +192,12 @@ def kv_proj(x, Wk, Wv, dims):
 # ----------------------------------------------------------------------------
 # attention: [SN] §1-1 (softmax(QK^T/sqrt(d))V), causal
 
+def attention_scale(dims) -> float:
+    """Factor applied to q.K before the softmax: the layer's explicit scale
+    when it sets one, else 1/sqrt(d) ([SN] §1-1, the attention equation)."""
+    return float(dims.scale) if dims.scale else 1.0 / math.sqrt(dims.d)
+
+
 def causal_attention(q, pos, K, V, scale, chunk=2048, want_lse=False):
     """o_r = sum_{j <= pos_r} softmax_j(q_r . K_j * scale) V_j.
 
@@ -226,7 +234,7 @@ def attn_prefill(q_routed, q_sh, K, V, dims, chunk=2048):
     Returns o_routed [B, G, T, k, d], o_sh [B, T, d] or None, and the LSEs.
     """
     B, T, G, k, d = dims.B, dims.T, dims.G, dims.k, dims.d
-    sc = dims.sm_scale
+    sc = attention_scale(dims)
     o = np.empty((B, G, T, k, d))
     lse = np.empty((B, G, T, k))
     pos = np.repeat(np.arange(T), k)
@@ -254,7 +262,7 @@ def attn_decode(q_routed, q_sh, Kc, Vc, cache_len, dims):
     cache_len-1).  Returns o_routed [B, G, k, d], o_sh [B, d] or None.
     """
     B, G, k, d = q_routed.shape
-    sc = dims.sm_scale
+    sc = attention_scale(dims)
     o = np.empty((B, G, k, d))
     o_sh = np.empty((B, d)) if dims.n_shared else None
     for b in range(B):

@@ -117,13 +117,13 @@ def test_attn_bwd_full_size_sampled(wname):
     pos = np.repeat(np.arange(T), k)
     R = T * k
     for b, g in [(0, dims.sg), (B - 1, G - 1)]:
-        args = (q[b, g].reshape(R, d), pos, K[b, g], V[b, g], dO[b, g].reshape(R, d), dims.sm_scale,
+        args = (q[b, g].reshape(R, d), pos, K[b, g], V[b, g], dO[b, g].reshape(R, d), orc.attention_scale(dims),
                 o[b, g].reshape(R, d), lse[(b * G + g) * R:(b * G + g + 1) * R])
         a, bk, bv = ob.causal_attention_bwd(*args)
         ma, mk, mv = ob.causal_attention_bwd_error_bound(*args)
         if g == dims.sg:
             ls = lse[B * G * R + b * T:B * G * R + (b + 1) * T]
-            args2 = (qs[b], np.arange(T), K[b, g], V[b, g], dOs[b], dims.sm_scale, os_[b], ls)
+            args2 = (qs[b], np.arange(T), K[b, g], V[b, g], dOs[b], orc.attention_scale(dims), os_[b], ls)
             a2, bk2, bv2 = ob.causal_attention_bwd(*args2)
             ma2, mk2, mv2 = ob.causal_attention_bwd_error_bound(*args2)
             bk, bv, mk, mv = bk + bk2, bv + bv2, mk + mk2, mv + mv2

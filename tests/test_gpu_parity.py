@@ -288,12 +288,12 @@ def test_attn_prefill_full_size_sampled(wname):
              list(rng.integers(0, T, 24)) + [0, T - 1, 127, 128]]
     got = to_f64(o)
     for b, g, t in picks:
-        ref = orc.causal_attention(q[b, g, t], np.full(k, t), K[b, g], V[b, g], dims.sm_scale)
+        ref = orc.causal_attention(q[b, g, t], np.full(k, t), K[b, g], V[b, g], orc.attention_scale(dims))
         err = np.abs(got[b, g, t] - ref).max()
         assert err <= ATTN_MAX_ABS, (b, g, t, err)
     gsh = to_f64(os_)
     for b, _, t in picks:
-        ref = orc.causal_attention(qs[b, t][None], np.array([t]), K[b, dims.sg], V[b, dims.sg], dims.sm_scale)[0]
+        ref = orc.causal_attention(qs[b, t][None], np.array([t]), K[b, dims.sg], V[b, dims.sg], orc.attention_scale(dims))[0]
         assert np.abs(gsh[b, t] - ref).max() <= ATTN_MAX_ABS
     assert torch.isfinite(o.float()).all() and torch.isfinite(os_.float()).all()
 
@@ -345,11 +345,11 @@ def test_attn_decode_small(case):
         n = lens[b]
         Kb, Vb = host[b]
         for g in range(dims.G):
-            ref = orc.causal_attention(q[b, g], np.full(dims.k, n - 1), Kb[g, :n], Vb[g, :n], dims.sm_scale)
+            ref = orc.causal_attention(q[b, g], np.full(dims.k, n - 1), Kb[g, :n], Vb[g, :n], orc.attention_scale(dims))
             assert_close_attn(o[b, g], ref, f"decode b{b} g{g}")
         if dims.n_shared:
             ref = orc.causal_attention(qs[b][None], np.array([n - 1]), Kb[dims.sg, :n], Vb[dims.sg, :n],
-                                       dims.sm_scale)[0]
+                                       orc.attention_scale(dims))[0]
             assert_close_attn(os_[b], ref, f"decode shared b{b}")
 
 
@@ -362,9 +362,9 @@ def test_attn_decode_full_size_sampled():
     for b in rows:
         Kb, Vb = host[b]
         for g in range(dims.G):
-            ref = orc.causal_attention(q[b, g], np.full(dims.k, L_max - 1), Kb[g], Vb[g], dims.sm_scale)
+            ref = orc.causal_attention(q[b, g], np.full(dims.k, L_max - 1), Kb[g], Vb[g], orc.attention_scale(dims))
             assert_close_attn(o[b, g], ref, f"decode b{b} g{g}")
-        ref = orc.causal_attention(qs[b][None], np.array([L_max - 1]), Kb[dims.sg], Vb[dims.sg], dims.sm_scale)[0]
+        ref = orc.causal_attention(qs[b][None], np.array([L_max - 1]), Kb[dims.sg], Vb[dims.sg], orc.attention_scale(dims))[0]
         assert_close_attn(os_[b], ref, f"decode shared b{b}")
     assert np.isfinite(o).all()
 

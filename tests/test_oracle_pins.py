@@ -197,9 +197,9 @@ def test_packed_rows_each_use_their_own_token_position():
     for t in range(5):
         for j in range(3):
             ref = _scalar_attention(q[0, 0, t, j].tolist(), K[0, 0].tolist(), V[0, 0].tolist(),
-                                    t, dims.sm_scale)
+                                    t, 1.0 / math.sqrt(dims.d))
             np.testing.assert_allclose(o[0, 0, t, j], ref, rtol=1e-12)
-            s = [float(q[0, 0, t, j] @ K[0, 0, i]) * dims.sm_scale for i in range(t + 1)]
+            s = [float(q[0, 0, t, j] @ K[0, 0, i]) * 1.0 / math.sqrt(dims.d) for i in range(t + 1)]
             np.testing.assert_allclose(lse[0, 0, t, j], math.log(sum(math.exp(v) for v in s)),
                                        rtol=1e-12)
 
