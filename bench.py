@@ -197,23 +197,46 @@ def oracle_threads():
         return os.cpu_count()
 
 
-def cpu_baseline(seconds_budget=20.0):
+def cpu_baseline(wname=WORKLOAD, seconds_budget=20.0):
+    """The fp64 oracle's throughput on a bounded sample of a workload.
+
+    Sequences of up to 8192 tokens: whole sequences of the workload through
+    oracle.gqe_forward (up to 3, or until the budget is spent).  Longer
+    sequences: oracle.gqe_forward over the sequence's first T/4 and first T/2
+    tokens; the oracle's time for the whole sequence is extrapolated from
+    those two runs as a T + b T^2 (projections linear in T, causal attention
+    quadratic).
+    """
     import oracle as orc
     cores = oracle_threads()
-    w = gi.WORKLOADS[WORKLOAD]
-    dims = w.dims.replace(B=1)           # one 2048-token sequence of the workload
+    w = gi.WORKLOADS[wname]
+    dims = w.dims.replace(B=1)
     x = gi.layer_input(w.dims, rows=[0])
-    Wt = gi.layer_weights(dims)
-    n, t0 = 0, time.perf_counter()
-    while True:
-        orc.gqe_forward(x, Wt, dims, gi.router_bias(w))
-        n += 1
-        if time.perf_counter() - t0 > seconds_budget or n >= 3:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": n * dims.N / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} x one sequence (T={dims.T}) of the {WORKLOAD} workload, fp64 numpy, "
-                      f"{dt:.1f} s"}
+    Wt = gi.layer_weights(w.dims)
+    bias = gi.router_bias(w)
+    if dims.T <= 8192:
+        n, t0 = 0, time.perf_counter()
+        while True:
+            orc.gqe_forward(x, Wt, dims, bias)
+            n += 1
+            if time.perf_counter() - t0 > seconds_budget or n >= 3:
+                break
+        dt = time.perf_counter() - t0
+        return {"value": n * dims.N / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                "sample": f"{n} x one sequence (T={dims.T}) of the {wname} workload, fp64 numpy, {dt:.1f} s"}
+    T1 = dims.T // 4
+    times = []
+    for Tp in (T1, 2 * T1):
+        t0 = time.perf_counter()
+        orc.gqe_forward(x[:, :Tp], Wt, dims.replace(T=Tp), bias)
+        times.append(time.perf_counter() - t0)
+    b = max((times[1] - 2 * times[0]) / (2.0 * T1 * T1), 0.0)
+    a = (times[0] - b * T1 * T1) / T1
+    est = a * dims.T + b * dims.T ** 2
+    return {"value": dims.T / est, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{wname}: the first {T1} and {2 * T1} tokens of one sequence through the whole-layer "
+                      f"oracle ({times[0]:.1f} s, {times[1]:.1f} s); time for its T={dims.T} extrapolated as "
+                      f"a T + b T^2 = {est:.0f} s, fp64 numpy"}
 
 
 # ----------------------------------------------------------------------------
@@ -428,6 +451,113 @@ def run_sweep_gqa(args):
     return 0
 
 
+LAUNCHES_PER_STEP = 7   # router, permutation, routed GEMM, K/V GEMM, attention, combine, Wo GEMM (+ one memset)
+CONFIG_WORKLOADS = ("tiny_prefill", "main_prefill", "long_prefill", "wide_skewed_prefill")
+SEG_NAMES = ("router", "routed_qproj", "kv_proj", "attn_prefill", "combine_out_proj")
+
+
+def attn_kernel_label(dims) -> str:
+    return "attn_prefill_single_kernel (d=64)" if dims.d == 64 else f"attn_prefill_kernel<{dims.d}>"
+
+
+def measure_prefill(gq, wname, device, dist, peaks, steps, warmup, flush, rank, world, keep_layer=False):
+    """Times the prefill layer forward of one workload on this GPU.
+
+    Timed steps: GQELayer.forward (the K/V projection on a side stream), one
+    event pair around each step, the L2 flushed between steps outside the
+    events.  Per-call split: separate steps with an event between every call.
+    Returns tokens/s (all ranks), ms per step (max over ranks), the per-call
+    split and the attention kernel's roofline against the measured peak.
+    """
+    import torch
+    w = gi.WORKLOADS[wname]
+    dims = w.dims
+    Wt = gi.layer_weights(dims, seed=0)
+    layer = gq.GQELayer(dims, {k: torch.from_numpy(v.view(np.int16)) for k, v in Wt.items()},
+                        gi.router_bias(w), device=device)
+    x_host = torch.from_numpy(gi.layer_input(dims, seed=rank).view(np.int16)).view(torch.bfloat16)
+    x = x_host.to(device)
+    stream = torch.cuda.current_stream(device)
+    c = layer.cfg
+    B, T, N = dims.B, dims.T, dims.N
+    d_ = gq.make_dims(c, B=B, T=T)
+
+    def step(evs):
+        idx = layer._buf("idx", (N, c.G, c.k), torch.int32)
+        wt = layer._buf("w", (N, c.G, c.k), torch.float32)
+        q = layer._buf("q", (B, c.G, T, c.k, c.d))
+        qs = layer._buf("qs", (B, T, c.d))
+        K = layer._buf("K", (B, c.G, T, c.d))
+        V = layer._buf("V", (B, c.G, T, c.d))
+        o = layer._buf("o", (B, c.G, T, c.k, c.d))
+        os_ = layer._buf("os", (B, T, c.d))
+        y = layer._buf("y", (B, T, c.D))
+        ws = layer._ws("ws_q", gq.gqe_workspace_size(d_, gq.GQE_OP_ROUTED_QPROJ))
+        ws_o = layer._ws("ws_o", gq.gqe_workspace_size(d_, gq.GQE_OP_COMBINE_OUT_PROJ))
+        evs[0].record(stream)
+        gq.gqe_router_topk(d_, x, layer.Wr, layer.bias, idx, wt, None)
+        evs[1].record(stream)
+        gq.gqe_routed_qproj(d_, x, layer.Wq, layer.Wsh, idx, q, qs, ws)
+        evs[2].record(stream)
+        gq.gqe_kv_proj(d_, x, layer.Wk, layer.Wv, K, V)
+        evs[3].record(stream)
+        gq.gqe_attn_prefill(d_, q, qs, K, V, o, os_, None)
+        evs[4].record(stream)
+        gq.gqe_combine_out_proj(d_, o, os_, wt, layer.Wo, y, ws_o)
+        evs[5].record(stream)
+
+    y_step = torch.empty((B, T, dims.D), dtype=torch.bfloat16, device=device)
+    warm_evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(warmup):
+        step(warm_evs)
+        layer.forward(x, out=y_step)
+        flush.zero_()
+    torch.cuda.synchronize()
+    assert gq.gqe_device_error() == 0
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    for s_ in range(steps):
+        flush.zero_()                       # L2 flushed between timed steps (outside the events)
+        # a GPU-side pause (outside the events) lets the host enqueue the whole
+        # step before the GPU reaches it, so the events time device work only
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
+        events[s_][0].record(stream)
+        layer.forward(x, out=y_step)        # the layer's own call sequence (K/V on a side stream)
+        events[s_][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    local_total_ms = float(sum(a.elapsed_time(b) for a, b in events))
+    n_seg = min(steps, 10)
+    seg_events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(SEG_NAMES) + 1)] for _ in range(n_seg)]
+    for s_ in range(n_seg):
+        flush.zero_()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
+        step(seg_events[s_])
+    torch.cuda.synchronize()
+    seg_ms = np.array([[seg_events[s_][i].elapsed_time(seg_events[s_][i + 1]) for i in range(len(SEG_NAMES))]
+                       for s_ in range(n_seg)])
+    total_ms = max_over_ranks(local_total_ms, dist, device)
+    attn_ms = float(seg_ms[:, 3].mean())
+    flops = attn_useful_flops(dims)
+    achieved_tf = flops / (attn_ms / 1e3) / 1e12
+    label = attn_kernel_label(dims)
+    out = {"workload": f"{wname}: {w.desc}", "B": B, "T": T, "d_model": dims.D, "G": dims.G, "E": dims.E,
+           "k": dims.k, "d_head": dims.d, "n_shared": dims.n_shared, "steps": steps,
+           "tokens_per_s": world * N * steps / (total_ms / 1e3), "ms_per_step": total_ms / steps,
+           "segments_ms": {n: float(seg_ms[:, i].mean()) for i, n in enumerate(SEG_NAMES)},
+           "roofline": {"bound": "tensor", "kernel": label, "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
+                        "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
+                        "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": profiled_traffic(label),
+                        "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_ms},
+           "gpu_launches": LAUNCHES_PER_STEP * steps, "device_error": gq.gqe_device_error()}
+    if keep_layer:
+        out.update(_layer=layer, _x=x, _x_host=x_host)
+    else:
+        del layer, x
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -437,6 +567,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-train", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="measure the headline workload only")
     ap.add_argument("--kernel", default=None,
                     help="time one call alone: attn | attn_bwd | layer_bwd | train_step | decode | router | qproj | kv | "
                          "combine | linear | combine_out")
@@ -462,108 +593,31 @@ def main():
     dist = init_dist(world, "nccl")
     peaks = load_peaks()
 
-    # ---------------- prefill workload
+    # ---------------- prefill: the headline workload, timed under the clock sampler
     w = gi.WORKLOADS[WORKLOAD]
     dims = w.dims
-    Wt = gi.layer_weights(dims, seed=0)
-    layer = gq.GQELayer(dims, {k: torch.from_numpy(v.view(np.int16)) for k, v in Wt.items()},
-                        gi.router_bias(w), device=device)
-    x_host = torch.from_numpy(gi.layer_input(dims, seed=rank).view(np.int16)).view(torch.bfloat16)
-    x = x_host.to(device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
-
-    # per-call events inside every timed step (router, q-proj, kv-proj, attention, combine, out-proj)
-    seg_names = ["router", "routed_qproj", "kv_proj", "attn_prefill", "combine_out_proj"]
-
-    def step(evs=None):
-        c = layer.cfg
-        B, T, N = dims.B, dims.T, dims.N
-        d_ = gq.make_dims(c, B=B, T=T)
-        L = gq
-        idx = layer._buf("idx", (N, c.G, c.k), torch.int32)
-        wt = layer._buf("w", (N, c.G, c.k), torch.float32)
-        q = layer._buf("q", (B, c.G, T, c.k, c.d))
-        qs = layer._buf("qs", (B, T, c.d))
-        K = layer._buf("K", (B, c.G, T, c.d))
-        V = layer._buf("V", (B, c.G, T, c.d))
-        o = layer._buf("o", (B, c.G, T, c.k, c.d))
-        os_ = layer._buf("os", (B, T, c.d))
-        y = layer._buf("y", (B, T, c.D))
-        ws = layer._ws("ws_q", L.gqe_workspace_size(d_, L.GQE_OP_ROUTED_QPROJ))
-        ws_o = layer._ws("ws_o", L.gqe_workspace_size(d_, L.GQE_OP_COMBINE_OUT_PROJ))
-        if evs is None:
-            rec = lambda i: None
-        elif len(evs) == 2:                     # whole step: start and end only
-            rec = lambda i: evs[min(i, 1)].record(stream) if i in (0, 5) else None
-        else:                                   # per call
-            rec = lambda i: evs[i].record(stream)
-        rec(0)
-        L.gqe_router_topk(d_, x, layer.Wr, layer.bias, idx, wt, None)
-        rec(1)
-        L.gqe_routed_qproj(d_, x, layer.Wq, layer.Wsh, idx, q, qs, ws)
-        rec(2)
-        L.gqe_kv_proj(d_, x, layer.Wk, layer.Wv, K, V)
-        rec(3)
-        L.gqe_attn_prefill(d_, q, qs, K, V, o, os_, None)
-        rec(4)
-        L.gqe_combine_out_proj(d_, o, os_, wt, layer.Wo, y, ws_o)
-        rec(5)
-        return y
-
-    launches_per_step = 7   # router, permutation, routed GEMM, K/V GEMM, attention, combine, Wo GEMM (+ one memset)
-
-    y_step = torch.empty((dims.B, dims.T, dims.D), dtype=torch.bfloat16, device=device)
-    for _ in range(args.warmup):
-        step()
-        layer.forward(x, out=y_step)
-        flush.zero_()
-    torch.cuda.synchronize()
-    assert gq.gqe_device_error() == 0
-
-    # timed steps: GQELayer.forward (the K/V projection on a side stream) with
-    # one event pair around it (events between the calls would stop each kernel
-    # from launching while its predecessor drains)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    barrier(dist, device)
-    torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        for s in range(args.steps):
-            flush.zero_()                       # L2 flushed between timed steps (outside the events)
-            # a GPU-side pause (outside the events) lets the host enqueue the whole
-            # step before the GPU reaches it, so the events time device work only
-            torch.cuda._sleep(HOST_LEAD_CYCLES)
-            events[s][0].record(stream)
-            layer.forward(x, out=y_step)        # the layer's own call sequence (K/V on a side stream)
-            events[s][1].record(stream)
-        torch.cuda.synchronize()
-    barrier(dist, device)
-    step_ms = np.array([events[s][0].elapsed_time(events[s][1]) for s in range(args.steps)])
-    local_total_ms = float(step_ms.sum())
-    # per-call split, from separate steps with an event between every call
-    n_seg = min(args.steps, 10)
-    seg_events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(seg_names) + 1)] for _ in range(n_seg)]
-    for s in range(n_seg):
-        flush.zero_()
-        torch.cuda._sleep(HOST_LEAD_CYCLES)
-        step(seg_events[s])
-    torch.cuda.synchronize()
-    seg_ms = np.array([[seg_events[s][i].elapsed_time(seg_events[s][i + 1]) for i in range(len(seg_names))]
-                       for s in range(n_seg)])
-    total_ms = max_over_ranks(local_total_ms, dist, device)
-    tokens = world * dims.N * args.steps
-    value = tokens / (total_ms / 1e3)
+        head = measure_prefill(gq, WORKLOAD, device, dist, peaks, args.steps, args.warmup, flush, rank, world,
+                               keep_layer=True)
+    layer, x, x_host = head.pop("_layer"), head.pop("_x"), head.pop("_x_host")
+    total_ms = head["ms_per_step"] * args.steps
+    value = head["tokens_per_s"]
+    roofline = head["roofline"]
+    seg_ms_mean = head["segments_ms"]
     err_code = gq.gqe_device_error()
+    launches_per_step = LAUNCHES_PER_STEP
 
-    # attention kernel roofline (tensor bound)
-    attn_ms = float(seg_ms[:, 3].mean())
-    flops = attn_useful_flops(dims)
-    achieved_tf = flops / (attn_ms / 1e3) / 1e12
-    attn_kernel = "attn_prefill_single_kernel (d=64)" if dims.d == 64 else f"attn_prefill_kernel<{dims.d}>"
-    roofline = {"bound": "tensor", "kernel": attn_kernel, "achieved": achieved_tf,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
-                "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": profiled_traffic(attn_kernel),
-                "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_ms}
+    # ---------------- the other prefill workloads: same measurement, fewer steps
+    configs = {WORKLOAD: {k_: v for k_, v in head.items()}}
+    if not args.no_configs:
+        for wn in CONFIG_WORKLOADS:
+            if wn == WORKLOAD:
+                continue
+            configs[wn] = measure_prefill(gq, wn, device, dist, peaks, min(args.steps, 10), args.warmup, flush,
+                                          rank, world)
+            torch.cuda.empty_cache()
 
     # ---------------- end to end through host buffers (pinned), on the same step
     # each step copies its input batch in and its output batch out; the copies
@@ -685,7 +739,11 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline()
+        cpu = cpu_baseline(WORKLOAD)
+        configs[WORKLOAD]["cpu_baseline"] = cpu
+        for wn in configs:
+            if wn != WORKLOAD:
+                configs[wn]["cpu_baseline"] = cpu_baseline(wn)
 
     if rank == 0:
         line = {
@@ -695,12 +753,16 @@ def main():
             "config": {"workload": f"{WORKLOAD}: {w.desc}", "B": dims.B, "T": dims.T, "d_model": dims.D,
                        "G": dims.G, "E": dims.E, "k": dims.k, "d_head": dims.d, "n_shared": dims.n_shared,
                        "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MB write)"},
-            "segments_ms": {n: float(seg_ms[:, i].mean()) for i, n in enumerate(seg_names)},
+            "segments_ms": seg_ms_mean,
             "segments_note": "per-call CUDA events in separate L2-flushed steps; their sum exceeds "
                              "ms_per_step by the overlap of each kernel's launch with its predecessor",
             "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "decode": decode, "training": training,
             "clocks": clocks.summary(), "gpu_launches": launches_per_step * args.steps,
             "device_error": err_code,
+            "configs": configs,
+            "configs_note": "every prefill workload measured the same way as the headline (layer forward, "
+                            "L2 flushed between steps, attention roofline from per-call events); the headline "
+                            "is the main layer, the workload the metric is quoted on",
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

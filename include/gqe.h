@@ -23,8 +23,9 @@
  *   - Argument errors return GQE_ERR_INVALID_ARG / GQE_ERR_UNSUPPORTED /
  *     GQE_ERR_WORKSPACE before anything is launched; a failed launch returns
  *     GQE_ERR_CUDA.  Errors inside a kernel surface at the caller's next
- *     synchronisation; a kernel whose internal wait runs out of time records a
- *     code that gqe_device_error() returns.
+ *     synchronisation; a kernel whose internal wait runs out of time, or a
+ *     decode that meets a cache length outside its range, records a code
+ *     that gqe_device_error() returns.
  *   - Supported shapes: d_head in {64, 128}; 1 <= k <= E <= 8; G*E <= 64;
  *     d_model a multiple of 64; n_shared in {0, 1}; 0 <= shared_kv_group < G.
  */
@@ -243,7 +244,11 @@ gqe_status gqe_transpose_f32(int rows, int cols, const float* src, float* dst, i
  * dense cache (freeguideonline GQA tutorial, "自回归推理中的内存带宽优势": a
  * decode step reads the whole KV cache).
  *   q_routed [B, G, k, d], q_sh [B, d]; Kc, Vc [B, G, L_max, d];
- *   cache_len [B] int32 device array: rows [0, cache_len[b]) are attended.
+ *   cache_len [B] int32 device array, each value in [1, L_max]: rows
+ *   [0, cache_len[b]) are attended.  A value outside that range is a caller
+ *   error the device detects: the kernel records code 0x302 in the device
+ *   error word (gqe_device_error) and clamps the value to [0, L_max]; a
+ *   sequence clamped to 0 gets zero outputs.
  *   o_routed [B, G, k, d], o_sh [B, d].
  *   ws: scratch of gqe_workspace_size(GQE_OP_ATTN_DECODE) bytes (split-L
  *   partial softmax states). */
@@ -266,8 +271,11 @@ gqe_status gqe_attn_decode(const gqe_dims* dims, const gqe_bf16* q_routed,
  *   partial states need more (gqe_workspace_size(GQE_OP_ATTN_DECODE) larger
  *   than the maximum) are rejected with GQE_ERR_WORKSPACE before anything is
  *   launched.  The 64-sequence, 8-group, 32768-key main-layer decode needs 4.3 MB.
- *   The first call on a device looks up the array's device address with that
- *   device current; make that first call before any stream capture.
+ *   A call looks up the array's device address with the current device,
+ *   and a call made under stream capture reuses the address that the last
+ *   uncaptured call on that device found: make the first call on a device
+ *   before any stream capture, and again after a reset of the device's
+ *   primary context (cudaDeviceReset), which reloads the array elsewhere.
  *   Every call shares the array and it keeps the last call's contents (each
  *   slot a call reads is written earlier in the same call, so nothing needs
  *   clearing).  Calls that can overlap on the GPU, e.g. on two streams with no
@@ -309,8 +317,12 @@ gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, 
                                 const float* topk_w, const gqe_bf16* Wo, gqe_bf16* y, void* ws,
                                 size_t ws_bytes, gqe_stream stream);
 
-/* Reads and clears the device error word that kernels set when one of their
- * internal waits runs out of time (0 = none).  Synchronises `stream`. */
+/* Reads and clears the device error word (0 = none).  Kernels set it when one
+ * of their internal waits runs out of time (0x101 GEMM, 0x201 attention,
+ * 0x202 attention backward, 0x301 decode, 0x401 router, 0x7F1 the failure
+ * check below) and when gqe_attn_decode meets a cache_len outside
+ * [1, L_max] (0x302).  The first code recorded is kept.  Synchronises
+ * `stream`. */
 gqe_status gqe_device_error(int* code, gqe_stream stream);
 
 /* Failure-path check: launches one thread that waits, through the kernels'

@@ -59,7 +59,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_const
   const int rr = tid >> 1, half = tid & 1;
   pdl_launch_dependents();
   pdl_wait();
-  const int len = p.cache_len[b];
+  int len = p.cache_len[b];
+  if (len < 1 || len > p.L_max) {
+    // outside the documented range: flag it once per sequence and clamp, so
+    // no key past the cache is counted and the merge stays finite
+    if (tid == 0 && c == 0 && g == 0 && p.err) atomicCAS(p.err, 0u, (unsigned)kErrDecodeCacheLen);
+    len = min(max(len, 0), p.L_max);
+  }
   const int start = c * p.chunk;
   const int end = min(start + p.chunk, len);
   const int nq = p.k + ((p.n_shared && g == p.sg) ? 1 : 0);
@@ -261,7 +267,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeParams p) {
       L += s[1] * f;
       A += s[2 + dim] * f;
     }
-    const float o = A / L;
+    const float o = L > 0.f ? A / L : 0.f;   // L == 0 only for a flagged empty cache
     const uint32_t pk = pack_bf16x2(o, 0.f);
     gqe_bf16_t* dst = (qi < p.k) ? p.o_routed + (((size_t)b * p.G + g) * p.k + qi) * D + dim
                                  : p.o_sh + (size_t)b * D + dim;
@@ -329,15 +335,20 @@ constexpr size_t kNoAllocScratchBytes = GQE_DECODE_NOALLOC_MAX_BYTES;
 static __device__ __align__(256) float g_decode_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 // Device address of the array on the current device.  Host code only sees a
-// host-side stand-in under the array's name, so the address is looked up once
-// per device, with that device current, and cached.
-float* noalloc_scratch() {
+// host-side stand-in under the array's name, so the address is looked up with
+// the device current.  It is looked up again on every call made outside
+// stream capture (a reset primary context reloads the module at another
+// address); a call under capture uses the address the last uncaptured call
+// on that device found, and fails when there is none.
+float* noalloc_scratch(cudaStream_t stream) {
   static std::mutex mu;
   static float* cache[64] = {nullptr};
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!cache[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch) != cudaSuccess) return nullptr;
     cache[dev] = static_cast<float*>(ptr);
@@ -362,7 +373,7 @@ extern "C" gqe_status gqe_attn_decode_noalloc(const gqe_dims* dims, const gqe_bf
   // cache_len writes its empty state), so nothing is cleared beforehand.
   if (decode_workspace_bytes(p.B, p.G, p.k, p.d, p.n_shared, L_max) > kNoAllocScratchBytes)
     return GQE_ERR_WORKSPACE;
-  float* scratch = noalloc_scratch();
+  float* scratch = noalloc_scratch(reinterpret_cast<cudaStream_t>(stream));
   if (!scratch) return GQE_ERR_CUDA;
   p.part = scratch;
   return launch_attn_decode_maps(mK, mV, p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? GQE_OK

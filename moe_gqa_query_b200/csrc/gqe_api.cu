@@ -180,8 +180,10 @@ inline gqe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GQE_OK 
 
 namespace gqe {
 
-// Argument checks and tensor maps of a decode call whose partial-state scratch
-// the callee provides (used by gqe_attn_decode_noalloc in attn_decode.cu).
+// Argument checks, tensor maps and parameters of a decode call, all but the
+// partial-state scratch, which the caller attaches (gqe_attn_decode: the
+// caller's workspace; gqe_attn_decode_noalloc in attn_decode.cu: the
+// library's fixed array).
 gqe_status decode_setup(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh, const gqe_bf16* Kc,
                         const gqe_bf16* Vc, int L_max, const int32_t* cache_len, gqe_bf16* o_routed,
                         gqe_bf16* o_sh, CUtensorMap* mK, CUtensorMap* mV, DecodeParams* p) {
@@ -505,38 +507,12 @@ gqe_status gqe_attn_prefill_bwd(const gqe_dims* dims, const gqe_bf16* q_routed, 
 gqe_status gqe_attn_decode(const gqe_dims* dims, const gqe_bf16* q_routed, const gqe_bf16* q_sh, const gqe_bf16* Kc,
                            const gqe_bf16* Vc, int L_max, const int32_t* cache_len, gqe_bf16* o_routed,
                            gqe_bf16* o_sh, void* ws, size_t ws_bytes, gqe_stream stream) {
-  GQE_CHECK(check_dims(dims));
-  GQE_REQUIRE(dims->T == 1 && L_max >= 1, GQE_ERR_INVALID_ARG);
-  GQE_REQUIRE(q_routed && Kc && Vc && cache_len && o_routed, GQE_ERR_INVALID_ARG);
-  GQE_REQUIRE(!dims->n_shared || (q_sh && o_sh), GQE_ERR_INVALID_ARG);
-  GQE_REQUIRE(aligned16(q_routed) && aligned16(Kc) && aligned16(Vc), GQE_ERR_INVALID_ARG);
-  GQE_REQUIRE(!dims->n_shared || aligned16(q_sh), GQE_ERR_INVALID_ARG);
-  const int B = dims->B, G = dims->G, d = dims->d_head;
-  const size_t need = decode_workspace_bytes(B, G, dims->k, d, dims->n_shared, L_max);
-  GQE_REQUIRE(ws && aligned16(ws) && ws_bytes >= need, GQE_ERR_WORKSPACE);
   CUtensorMap mK, mV;
-  GQE_REQUIRE(map3d(&mK, Kc, d, L_max, (uint64_t)B * G, 64), GQE_ERR_CUDA);
-  GQE_REQUIRE(map3d(&mV, Vc, d, L_max, (uint64_t)B * G, 64), GQE_ERR_CUDA);
-  DecodeParams p{};
-  p.q_routed = q_routed;
-  p.q_sh = q_sh;
-  p.Kc = Kc;
-  p.Vc = Vc;
-  p.cache_len = cache_len;
-  p.o_routed = o_routed;
-  p.o_sh = o_sh;
+  DecodeParams p;
+  GQE_CHECK(decode_setup(dims, q_routed, q_sh, Kc, Vc, L_max, cache_len, o_routed, o_sh, &mK, &mV, &p));
+  const size_t need = decode_workspace_bytes(p.B, p.G, p.k, p.d, p.n_shared, L_max);
+  GQE_REQUIRE(ws && aligned16(ws) && ws_bytes >= need, GQE_ERR_WORKSPACE);
   p.part = static_cast<float*>(ws);
-  p.B = B;
-  p.G = G;
-  p.k = dims->k;
-  p.d = d;
-  p.n_shared = dims->n_shared;
-  p.sg = dims->shared_kv_group;
-  p.L_max = L_max;
-  decode_split_plan(L_max, &p.chunk, &p.n_chunks);
-  p.nq_max = dims->k + dims->n_shared;
-  p.scale_log2 = scale_log2(dims);
-  p.err = error_word();
   return cuda_status(launch_attn_decode_maps(mK, mV, p, S(stream)));
 }
 

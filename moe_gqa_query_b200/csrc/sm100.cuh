@@ -19,6 +19,7 @@ enum DeviceErrorCode : unsigned {
   kErrTimeoutAttn = 0x201,
   kErrTimeoutAttnBwd = 0x202,
   kErrTimeoutDecode = 0x301,
+  kErrDecodeCacheLen = 0x302,  // a cache_len outside [1, L_max] (clamped; see gqe_attn_decode)
   kErrTimeoutRouter = 0x401,
   kErrTimeoutDebug = 0x7F1,   // gqe_debug_wait_timeout: a wait that nothing completes
 };

@@ -331,6 +331,57 @@ def gqe_forward(x, Wt, dims, bias=None):
     return dict(router=r, q_routed=q_routed, q_sh=q_sh, K=K, V=V, o=o, o_sh=o_sh, h=h, y=y)
 
 
+def gqe_forward_rows(x, Wt, dims, rows, bias=None, chunk=2048):
+    """The prefill layer at chosen token rows only, in fp64.
+
+    A token's row of h and y is made of its own router decision, its own
+    query projections, and attention of those queries over the keys and
+    values of tokens 0..t of its own sequence; K and V are the dense GQA
+    projections of that prefix ([SN] §1-2 3), KV unchanged).  Nothing else of
+    the batch enters the row, so each requested row is the full layer's row,
+    computed from x[b, :t+1] alone.  This is the full-layer definition
+    restricted to those rows; used where gqe_forward over a whole workload
+    would take too long.
+
+    x [B, T, D]; rows: iterable of (b, t).  Returns dict(router over the rows,
+    h [R, slots*d], y [R, D]) in the order of ``rows``.
+    """
+    rows = [(int(b), int(t)) for b, t in rows]
+    R = len(rows)
+    G, E, k, d = dims.G, dims.E, dims.k, dims.d
+    x = np.asarray(x)
+    xr = np.stack([f64(x[b, t]) for b, t in rows])
+    r = router_topk(xr, Wt["Wr"], G, E, k, bias, dims.renorm_scope)
+    one = _Shape(B=R, T=1, G=G, k=k, d=d, n_shared=dims.n_shared, output_mode=getattr(dims, "output_mode", 0))
+    q_routed, q_sh = routed_qproj(xr, Wt["Wq"], Wt["Wsh"], r["idx"], one)     # [R, G, 1, k, d], [R, 1, d]
+    sc = attention_scale(dims)
+    o = np.empty((R, G, 1, k, d))
+    o_sh = np.empty((R, 1, d)) if dims.n_shared else None
+    for b in sorted({b for b, _ in rows}):
+        mine = [i for i, (bb, _) in enumerate(rows) if bb == b]
+        t_end = max(rows[i][1] for i in mine) + 1
+        pre = _Shape(B=1, T=t_end, G=G, d=d)
+        K, V = kv_proj(x[b, :t_end], Wt["Wk"], Wt["Wv"], pre)                 # [1, G, t_end, d]
+        for i in mine:
+            t = rows[i][1]
+            for g in range(G):
+                o[i, g, 0] = causal_attention(q_routed[i, g, 0], np.full(k, t), K[0, g, :t + 1],
+                                              V[0, g, :t + 1], sc, chunk)
+            if dims.n_shared:
+                o_sh[i] = causal_attention(q_sh[i], np.array([t]), K[0, dims.sg, :t + 1],
+                                           V[0, dims.sg, :t + 1], sc, chunk)
+    h = combine(o, o_sh, r["w"], one)
+    y = out_proj(h, Wt["Wo"])
+    return dict(router=r, h=h, y=y)
+
+
+class _Shape:
+    """The shape fields the helpers above read, for a sub-batch of rows."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
 def decode_step(x_new, Wt, Kc, Vc, cache_len, dims, bias=None):
     """One decode step for B sequences (T = 1).
 

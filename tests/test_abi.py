@@ -54,10 +54,26 @@ def test_bindings_match_header_prototypes():
                 raise AssertionError(f"{name}: unexpected parameter {decl}")
 
 
-def test_library_is_built_for_sm100a():
-    with open(gq.LIB_PATH, "rb") as f:
-        blob = f.read()
-    assert b"sm_100a" in blob
+def test_library_build_targets_sm100a_only():
+    """The build compiles every source for sm_100a and for nothing else (read
+    from the build script's flags, not from the built binary)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("gqe_build", os.path.join(os.path.dirname(gq.LIB_PATH), "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    flags = mod.NVCC_FLAGS
+    archs = [flags[i + 1] for i, f in enumerate(flags) if f == "-gencode"]
+    assert archs == ["arch=compute_100a,code=sm_100a"]
+    assert not any(f.startswith("-arch") for f in flags)
+
+
+def test_noalloc_limit_matches_header():
+    """The binding's size limit of gqe_attn_decode_noalloc is the header's."""
+    import re
+    with open(_lib.HEADER_PATH) as f:
+        m = re.search(r"#define\s+GQE_DECODE_NOALLOC_MAX_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", f.read())
+    assert m, "GQE_DECODE_NOALLOC_MAX_BYTES not found in the header"
+    assert gq.DECODE_NOALLOC_MAX_BYTES == int(m.group(1)) << int(m.group(2))
 
 
 def _cfg(**kw):

@@ -514,3 +514,34 @@ def test_router_stats_closed_forms_and_brute_force():
             for e in r["idx"][t, g]:
                 loop[g * E + int(e)] += 1
     np.testing.assert_array_equal(counts, loop)
+
+
+# ----------------------------------------------------------------------------
+# the layer at chosen rows equals the whole layer at those rows
+
+@pytest.mark.parametrize("kw", [
+    dict(B=2, T=19, D=24, G=3, E=4, k=2, d=4, sg=1),
+    dict(B=1, T=33, D=16, G=2, E=2, k=1, d=8),
+    dict(B=3, T=7, D=16, G=2, E=3, k=3, d=4, n_shared=0),
+    dict(B=2, T=12, D=16, G=2, E=4, k=2, d=4, renorm_scope=1, output_mode=2),
+    dict(B=1, T=10, D=16, G=4, E=2, k=1, d=4, output_mode=1),
+])
+def test_forward_rows_equals_full_layer(kw):
+    """gqe_forward_rows (used for sampled rows of the large workloads) gives
+    the full oracle layer's router decision, h and y at every requested row,
+    in the requested order, repeated rows included."""
+    dims = gi.GQEDims(**kw)
+    rng = np.random.default_rng(sum(kw.values()))
+    x = gi.f32_to_bf16_bits(rng.standard_normal((dims.B, dims.T, dims.D)).astype(np.float32))
+    Wt = {n: gi.f32_to_bf16_bits((rng.standard_normal(v.shape) * 0.3).astype(np.float32))
+          for n, v in gi.layer_weights(dims).items()}
+    bias = rng.standard_normal(dims.G * dims.E).astype(np.float32)
+    full = orc.gqe_forward(x, Wt, dims, bias)
+    rows = [(b, t) for b in range(dims.B) for t in range(dims.T)]
+    rows = rows[::-1] + rows[:3]
+    part = orc.gqe_forward_rows(x, Wt, dims, rows, bias)
+    flat = [b * dims.T + t for b, t in rows]
+    assert np.array_equal(part["router"]["idx"], full["router"]["idx"][flat])
+    np.testing.assert_allclose(part["router"]["w"], full["router"]["w"][flat], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(part["h"], full["h"][flat], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(part["y"], full["y"][flat], rtol=1e-11, atol=1e-13)

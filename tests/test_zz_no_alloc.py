@@ -7,9 +7,11 @@ library offers gqe_attn_decode_noalloc, which keeps the split-L partial states
 in one fixed device array inside the library instead of a caller workspace.
 
 These tests call it through the C ABI and compare it with gqe_attn_decode
-(caller workspace) within the attention tolerance, on two calls in a row: the
-second call has other inputs and shorter caches, so state left in the shared
-array by the first call would show.  Shapes whose partial states exceed the
+(caller workspace) and with the fp64 oracle, within the attention tolerance,
+on two calls in a row: the second call has other inputs and shorter caches,
+so state left in the shared array by the first call would show.  One call
+runs the main-layer decode shape (64 sequences, 8 groups, 32768 keys) and is
+checked on sampled sequences.  Shapes whose partial states exceed the
 array are refused before anything is launched.  The file sorts last so that a
 run stopping at the first failure has run every other test first.
 """
@@ -18,7 +20,8 @@ import pytest
 import torch
 
 import gqe_inputs as gi
-from helpers import assert_close_attn, to_f64
+import oracle as orc
+from helpers import assert_close_attn, bf16_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -85,3 +88,68 @@ def test_noalloc_decode_rejects_oversize_before_launch():
     with pytest.raises(gq.GQEError) as ei:
         gq.gqe_attn_decode_noalloc(dc, buf, buf, buf, buf, L_max, cl, buf, buf)
     assert ei.value.status == 3     # GQE_ERR_WORKSPACE
+
+
+def _noalloc(dims, q, qs, Kc, Vc, L_max, lens):
+    dc = gq.make_dims(dims, T=1)
+    o = torch.full((dims.B, dims.G, dims.k, dims.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    os_ = torch.full((dims.B, dims.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    cl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    gq.gqe_attn_decode_noalloc(dc, q, qs, Kc, Vc, L_max, cl, o, os_)
+    torch.cuda.synchronize()
+    return to_f64(o), to_f64(os_)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_noalloc_decode_against_oracle_two_calls(d):
+    """Seeded inputs, both calls checked against the oracle's decode attention."""
+    dims = gi.GQEDims(B=3, T=1, D=256, G=2, E=4, k=2, d=d, sg=1)
+    L_max = 3000
+    for seed, lens in ((41, [3000, 1, 1234]), (42, [77, 2999, 640])):
+        q = gi.normal_bf16(seed, "q", (dims.B, dims.G, dims.k, d))
+        qs = gi.normal_bf16(seed, "qsh", (dims.B, d))
+        Kc = gi.normal_bf16(seed, "Kc", (dims.B, dims.G, L_max, d))
+        Vc = gi.normal_bf16(seed, "Vc", (dims.B, dims.G, L_max, d))
+        o, os_ = _noalloc(dims, bf16_dev(q), bf16_dev(qs), bf16_dev(Kc), bf16_dev(Vc), L_max, lens)
+        o_ref, os_ref = orc.attn_decode(q, qs, Kc, Vc, np.array(lens), dims)
+        assert_close_attn(o, o_ref, f"noalloc routed rows vs oracle (seed {seed})")
+        assert_close_attn(os_, os_ref, f"noalloc shared row vs oracle (seed {seed})")
+
+
+def test_noalloc_decode_main_layer_sampled():
+    """The main-layer decode (64 x 8 x 32768 x 64 cache, 4.3 MB of partial
+    states in the array): three sequences regenerated on the host and checked
+    against the oracle, the whole output against gqe_attn_decode."""
+    w = gi.WORKLOADS["decode"]
+    dims, L_max = w.dims, w.L
+    B, G, k, d = dims.B, dims.G, dims.k, dims.d
+    seed, rows = 51, [0, 29, 63]
+    q = gi.normal_bf16(seed, "q", (B, G, k, d))
+    qs = gi.normal_bf16(seed, "qsh", (B, d))
+    gen = torch.Generator(device="cuda").manual_seed(seed)
+    Kc = torch.empty((B, G, L_max, d), dtype=torch.bfloat16, device="cuda").normal_(generator=gen)
+    Vc = torch.empty_like(Kc).normal_(generator=gen)
+    host = {}
+    for b in rows:
+        Kb = gi.normal_bf16(seed, "Kc", (B, G, L_max, d), rows=[b])
+        Vb = gi.normal_bf16(seed, "Vc", (B, G, L_max, d), rows=[b])
+        Kc[b] = bf16_dev(Kb[0])
+        Vc[b] = bf16_dev(Vb[0])
+        host[b] = (Kb, Vb)
+    lens = [L_max] * B
+    o, os_ = _noalloc(dims, bf16_dev(q), bf16_dev(qs), Kc, Vc, L_max, lens)
+    sub = dims.replace(B=1)
+    for b in rows:
+        Kb, Vb = host[b]
+        o_ref, os_ref = orc.attn_decode(q[b:b + 1], qs[b:b + 1], Kb, Vb, np.array([L_max]), sub)
+        assert_close_attn(o[b], o_ref[0], f"noalloc main-layer decode b{b}")
+        assert_close_attn(os_[b], os_ref[0], f"noalloc main-layer decode shared b{b}")
+    dc = gq.make_dims(dims, T=1)
+    ws = torch.empty((gq.gqe_workspace_size(dc, gq.GQE_OP_ATTN_DECODE, L_max),), dtype=torch.uint8, device="cuda")
+    o2 = torch.empty((B, G, k, d), dtype=torch.bfloat16, device="cuda")
+    os2 = torch.empty((B, d), dtype=torch.bfloat16, device="cuda")
+    gq.gqe_attn_decode(dc, bf16_dev(q), bf16_dev(qs), Kc, Vc, L_max, torch.tensor(lens, dtype=torch.int32,
+                       device="cuda"), o2, os2, ws)
+    torch.cuda.synchronize()
+    assert_close_attn(o, to_f64(o2), "noalloc vs workspace decode, all sequences")
+    assert_close_attn(os_, to_f64(os2), "noalloc vs workspace decode shared, all sequences")
