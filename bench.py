@@ -46,12 +46,14 @@ L2_FLUSH_BYTES = 256 << 20
 HOST_LEAD_CYCLES = 600_000      # ~0.3 ms at B200 clocks: longer than the host needs to enqueue a step
 
 
-def profiled_traffic(kernel_label):
-    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
-    or None when there is none or the kernel's source changed since the capture."""
+def profiled_traffic(kernel_label, workload=WORKLOAD):
+    """DRAM bytes per launch of a kernel on a workload from the committed ncu
+    summaries (profiles/traffic.json), or None when there is no capture for
+    that kernel and workload or the kernel's source changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            entry = json.load(f).get(kernel_label)
+            caps = json.load(f)["captures"]
+        entry = next((c for c in caps if c["kernel"] == kernel_label and c["workload"] == workload), None)
         if not entry:
             return None
         with open(os.path.join(ROOT, entry["source"]), "rb") as f:
@@ -548,7 +550,7 @@ def measure_prefill(gq, wname, device, dist, peaks, steps, warmup, flush, rank, 
            "segments_ms": {n: float(seg_ms[:, i].mean()) for i, n in enumerate(SEG_NAMES)},
            "roofline": {"bound": "tensor", "kernel": label, "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
                         "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
-                        "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": profiled_traffic(label),
+                        "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": profiled_traffic(label, wname),
                         "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_ms},
            "gpu_launches": LAUNCHES_PER_STEP * steps, "device_error": gq.gqe_device_error()}
     if keep_layer:
@@ -685,7 +687,8 @@ def main():
                   "ms_per_step": step_dec_ms,
                   "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<64> + merge", "achieved": gbs,
                                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                               "peak_source": f"{peaks['source']} HBM copy", "traffic": None,
+                               "peak_source": f"{peaks['source']} HBM copy",
+                               "traffic": profiled_traffic("decode_split_kernel<64> + merge", DECODE_WORKLOAD),
                                "algorithmic_bytes_per_launch": bytes_, "avg_launch_ms": attn_dec_ms},
                   "data": "synthetic: cache ~N(0,1) from a seeded torch generator on the device"}
         del Kc, Vc

@@ -105,6 +105,7 @@ def test_roofline_traffic_follows_the_captured_source(tmp_path, monkeypatch):
     got = bench.profiled_traffic(label)
     assert got == 52472064 + 1871104
     assert bench.profiled_traffic("no such kernel") is None
+    assert bench.profiled_traffic(label, "long_prefill") is None       # captured on the main layer only
     # the same capture against an edited copy of the source
     (tmp_path / "profiles").mkdir()
     shutil.copy(os.path.join(bench.ROOT, "profiles", "traffic.json"), tmp_path / "profiles" / "traffic.json")
