@@ -281,9 +281,23 @@ def run_kernel(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
-    if args.kernel == "decode":
+    if args.kernel == "decode_step":
+        # the whole decode step of the layer (router, query projection, K/V
+        # append, attention, output construction and projection)
         w = gi.WORKLOADS[DECODE_WORKLOAD]
-        dd, Lc = w.dims, w.L
+        dd, Lc = w.dims, (args.decode_L or w.L)
+        gen = torch.Generator(device=device).manual_seed(7)
+        Kc = torch.empty((dd.B, dd.G, Lc, dd.d), dtype=torch.bfloat16, device=device).normal_(generator=gen)
+        Vc = torch.empty_like(Kc).normal_(generator=gen)
+        lay = gq.GQELayer(dd, {kk: torch.from_numpy(v.view(np.int16)) for kk, v in gi.layer_weights(dd).items()},
+                          device=device)
+        xn = torch.randn((dd.B, dd.D), device=device, generator=gen).to(torch.bfloat16)
+        cl = torch.full((dd.B,), Lc, dtype=torch.int32, device=device)
+        fn = lambda: lay.decode_step(xn, Kc, Vc, cl)  # noqa: E731
+        work = dict(bytes=decode_attn_bytes(dd, Lc), tokens=float(dd.B))
+    elif args.kernel == "decode":
+        w = gi.WORKLOADS[DECODE_WORKLOAD]
+        dd, Lc = w.dims, (args.decode_L or w.L)
         gen = torch.Generator(device=device).manual_seed(7)
         Kc = torch.empty((dd.B, dd.G, Lc, dd.d), dtype=torch.bfloat16, device=device).normal_(generator=gen)
         Vc = torch.empty_like(Kc).normal_(generator=gen)
@@ -373,7 +387,7 @@ def run_kernel(args):
         b.record(stream)
     torch.cuda.synchronize()
     ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    out = {"kernel": args.kernel, "workload": DECODE_WORKLOAD if args.kernel == "decode" else args.workload,
+    out = {"kernel": args.kernel, "workload": DECODE_WORKLOAD if args.kernel.startswith("decode") else args.workload,
            "ms": ms, "device_error": gq.gqe_device_error()}
     if "flops" in work:
         out["TFLOP/s"] = work["flops"] / ms / 1e9
@@ -571,8 +585,10 @@ def main():
     ap.add_argument("--no-train", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="measure the headline workload only")
     ap.add_argument("--kernel", default=None,
-                    help="time one call alone: attn | attn_bwd | layer_bwd | train_step | decode | router | qproj | kv | "
+                    help="time one call alone: attn | attn_bwd | layer_bwd | train_step | decode | decode_step | router | qproj | kv | "
                          "combine | linear | combine_out")
+    ap.add_argument("--decode-L", type=int, default=0,
+                    help="cache length for --kernel decode / decode_step (default: the decode workload's 32768)")
     ap.add_argument("--workload", default=WORKLOAD, choices=[k for k, v in gi.WORKLOADS.items() if not v.decode])
     ap.add_argument("--sweep", default=None, choices=["gqa"],
                     help="gqa: GQE against dense GQA, prefill T from 2K to 128K (one JSON line per T)")

@@ -14,7 +14,9 @@ import os
 import re
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libgqe.so")
+# GQE_LIB_PATH selects another build of the library (the traced diagnostic
+# build, libgqe_trace.so); by default the package's own libgqe.so.
+LIB_PATH = os.environ.get("GQE_LIB_PATH") or os.path.join(_PKG, "libgqe.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "gqe.h")
 
 GQE_OK = 0

@@ -14,6 +14,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgqe.so")
+# diagnostic build: the same sources with the attention kernel's CTA timeline
+# recorded (include/gqe_trace.h)
+TRACE_LIB = os.path.join(PKG, "libgqe_trace.so")
+TRACE_FLAGS = ["-DGQE_ATTN_TRACE"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -34,12 +38,15 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def build_library(verbose: bool = False, extra=()) -> str:
-    """Compile every CUDA source into moe_gqa_query_b200/libgqe.so."""
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "gqe.h")]
-    if os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(d) for d in deps) and not extra:
-        return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *sources()]
+def build_library(verbose: bool = False, extra=(), trace: bool = False) -> str:
+    """Compile every CUDA source into moe_gqa_query_b200/libgqe.so (or, with
+    trace=True, the diagnostic libgqe_trace.so)."""
+    out = TRACE_LIB if trace else LIB
+    extra = tuple(extra) + (tuple(TRACE_FLAGS) if trace else ())
+    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
+    if os.path.exists(out) and all(os.path.getmtime(out) >= os.path.getmtime(d) for d in deps) and not extra:
+        return out
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-o", out + ".tmp", *sources()]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -48,9 +55,11 @@ def build_library(verbose: bool = False, extra=()) -> str:
         raise RuntimeError("nvcc failed building libgqe.so")
     if verbose and (r.stdout or r.stderr):
         sys.stderr.write(r.stdout + r.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build_library(verbose=True, extra=tuple(sys.argv[1:])))
+    args = sys.argv[1:]
+    trace = "--trace" in args
+    print(build_library(verbose=True, extra=tuple(a for a in args if a != "--trace"), trace=trace))

@@ -36,6 +36,17 @@
 
 namespace gqe {
 
+// Per-CTA timeline of the d = 64 kernel, built only into the diagnostic
+// library (GQE_ATTN_TRACE; read by gqe_debug_attn_trace, include/gqe_trace.h):
+// 12 values per CTA, globaltimer nanoseconds unless noted.
+#ifdef GQE_ATTN_TRACE
+constexpr int kTraceCtas = 16384;
+__device__ unsigned long long g_attn_trace[kTraceCtas * 12];
+#define ATTN_TRACE(...) __VA_ARGS__
+#else
+#define ATTN_TRACE(...)
+#endif
+
 namespace {
 
 constexpr int kThreads = 320;
@@ -416,6 +427,9 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
                            const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                            AttnParams p) {
   constexpr int D = 64;
+  ATTN_TRACE(const unsigned long long tr_entry = globaltimer();
+             unsigned long long* TR = blockIdx.x < kTraceCtas ? g_attn_trace + (size_t)blockIdx.x * 12 : nullptr;
+             unsigned long long tr_ws = 0, tr_wpv = 0;)
   constexpr int ST = kSingleST;
   constexpr uint32_t kS = 0, kP = 128, kO = 192;
   extern __shared__ uint8_t smem_raw[];
@@ -480,6 +494,13 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
   const uint32_t tmem = bar->tmem_base;
   pdl_launch_dependents();
   pdl_wait();
+  ATTN_TRACE(if (TR && threadIdx.x == 0) {
+    unsigned sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    TR[0] = sm | ((unsigned long long)n_kv << 16) | ((unsigned long long)routed << 31);
+    TR[1] = tr_entry;
+    TR[2] = globaltimer();
+  })
 
   if (warp == 4) {
     if (lane == 0) {
@@ -495,6 +516,7 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       }
       const uint32_t q0 = smem_u32(sQ);
       bool ok = mbar_wait(&bar->q_full, 0, abort, p.err, kErrTimeoutAttn);
+      ATTN_TRACE(if (TR) TR[3] = globaltimer();)
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % ST;
         if (j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, abort, p.err, kErrTimeoutAttn);
@@ -564,7 +586,13 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
+      ATTN_TRACE(const unsigned long long tw0 = globaltimer();)
       ok = mbar_wait(&bar->s_full, j & 1, abort, p.err, kErrTimeoutAttn);
+      ATTN_TRACE(if (TR && threadIdx.x == 0) {
+        const unsigned long long tw1 = globaltimer();
+        if (j == 0) TR[4] = tw1;
+        else tr_ws += tw1 - tw0;
+      })
       tc_fence_after();
       const bool diag = j * kTile + kTile - 1 > ti.t_first;
       const int lim = t_r - j * kTile;
@@ -636,7 +664,9 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
         }
         // P(j-1) V must be done before P is overwritten (and O rescaled)
         if (h == 0 && j > 0) {
+          ATTN_TRACE(const unsigned long long tp0 = globaltimer();)
           ok = mbar_wait(&bar->pv_done, (j - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
+          ATTN_TRACE(if (threadIdx.x == 0) tr_wpv += globaltimer() - tp0;)
           tc_fence_after();
         }
         tmem_st32(p_base + h * 32, pk);
@@ -664,9 +694,16 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar->p_full);
+      ATTN_TRACE(if (TR && threadIdx.x == 0 && j == 0) TR[5] = globaltimer();)
     }
+    ATTN_TRACE(if (TR && threadIdx.x == 0) {
+      TR[6] = globaltimer();
+      TR[10] = tr_ws;
+      TR[11] = tr_wpv;
+    })
     // ---------------- epilogue: O / l -> bf16
     ok = mbar_wait(&bar->pv_done, (n_kv - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
+    ATTN_TRACE(if (TR && threadIdx.x == 0) TR[7] = globaltimer();)
     tc_fence_after();
     const float inv_l = 1.f / l_run;
     gqe_bf16_t* orow = routed ? p.o_routed + ((size_t)seq * rows_total + prow) * D
@@ -690,9 +727,11 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
                                : (size_t)BG * p.T * p.k + (size_t)seq * p.T + prow;
       p.lse[li] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
+    ATTN_TRACE(if (TR && threadIdx.x == 0) TR[8] = globaltimer();)
   }
   tc_fence_before();
   __syncthreads();
+  ATTN_TRACE(if (TR && threadIdx.x == 0) TR[9] = globaltimer();)
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
@@ -734,3 +773,10 @@ cudaError_t launch_attn_prefill(const CUtensorMap& mQ, const CUtensorMap& mQs, c
 }
 
 }  // namespace gqe
+
+#ifdef GQE_ATTN_TRACE
+extern "C" int gqe_debug_attn_trace(void* host, size_t bytes) {
+  if (!host || bytes > sizeof(gqe::g_attn_trace)) return 1;
+  return cudaMemcpyFromSymbol(host, gqe::g_attn_trace, bytes) == cudaSuccess ? 0 : 4;
+}
+#endif

@@ -96,26 +96,37 @@ def test_reference_arm_other_ranks_exit_quietly():
 
 
 def test_roofline_traffic_follows_the_captured_source(tmp_path, monkeypatch):
-    """The bench reports a kernel's ncu DRAM traffic only while the kernel's
-    source file still hashes to the captured version; a label without a
-    capture gives null."""
+    """The bench reports a kernel's ncu DRAM traffic only for the captured
+    kernel and workload, and only while the kernel's source file still hashes
+    to the captured version; anything else gives null."""
+    import hashlib
     import shutil
     import bench
     label = "attn_prefill_single_kernel (d=64)"
-    got = bench.profiled_traffic(label)
-    assert got == 52472064 + 1871104
     assert bench.profiled_traffic("no such kernel") is None
-    assert bench.profiled_traffic(label, "long_prefill") is None       # captured on the main layer only
-    # the same capture against an edited copy of the source
-    (tmp_path / "profiles").mkdir()
-    shutil.copy(os.path.join(bench.ROOT, "profiles", "traffic.json"), tmp_path / "profiles" / "traffic.json")
     src = tmp_path / "moe_gqa_query_b200" / "csrc" / "attn_prefill.cu"
     src.parent.mkdir(parents=True)
     shutil.copy(os.path.join(bench.ROOT, "moe_gqa_query_b200", "csrc", "attn_prefill.cu"), src)
+    (tmp_path / "profiles").mkdir()
+    entry = {"kernel": label, "workload": "main_prefill", "source": "moe_gqa_query_b200/csrc/attn_prefill.cu",
+             "source_sha256_16": hashlib.sha256(src.read_bytes()).hexdigest()[:16],
+             "dram_read_bytes": 1000, "dram_write_bytes": 24}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"captures": [entry]}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.profiled_traffic(label) == got
+    assert bench.profiled_traffic(label, "main_prefill") == 1024
+    assert bench.profiled_traffic(label, "long_prefill") is None
     src.write_text(src.read_text() + "\n// edited\n")
-    assert bench.profiled_traffic(label) is None
+    assert bench.profiled_traffic(label, "main_prefill") is None
+
+
+def test_committed_traffic_entries_are_well_formed():
+    import bench
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        caps = json.load(f)["captures"]
+    for c in caps:
+        assert os.path.exists(os.path.join(bench.ROOT, c["source"]))
+        assert c["workload"] in bench.gi.WORKLOADS
+        assert int(c["dram_read_bytes"]) > 0 and int(c["dram_write_bytes"]) >= 0
 
 
 def test_peaks_fall_back_without_the_measured_file(tmp_path, monkeypatch):
