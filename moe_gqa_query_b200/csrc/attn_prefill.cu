@@ -586,7 +586,7 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
-      ATTN_TRACE(const unsigned long long tw0 = globaltimer();)
+      ATTN_TRACE(const unsigned long long tw0 = threadIdx.x == 0 ? globaltimer() : 0ull;)
       ok = mbar_wait(&bar->s_full, j & 1, abort, p.err, kErrTimeoutAttn);
       ATTN_TRACE(if (TR && threadIdx.x == 0) {
         const unsigned long long tw1 = globaltimer();
@@ -664,7 +664,7 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
         }
         // P(j-1) V must be done before P is overwritten (and O rescaled)
         if (h == 0 && j > 0) {
-          ATTN_TRACE(const unsigned long long tp0 = globaltimer();)
+          ATTN_TRACE(const unsigned long long tp0 = threadIdx.x == 0 ? globaltimer() : 0ull;)
           ok = mbar_wait(&bar->pv_done, (j - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
           ATTN_TRACE(if (threadIdx.x == 0) tr_wpv += globaltimer() - tp0;)
           tc_fence_after();

@@ -280,12 +280,16 @@ gqe_status gqe_router_topk(const gqe_dims* dims, const gqe_bf16* x, const gqe_bf
   p.k = dims->k;
   p.scope = dims->renorm_scope;
   p.err = error_word();
-  // tcgen05 router with TMA-streamed x for prefill-sized batches
-  if (p.N >= 1024 && p.D % 64 == 0) {
-    CUtensorMap mX;
-    GQE_REQUIRE(map2d(&mX, x, p.D, p.N, 128), GQE_ERR_CUDA);
-    const cudaError_t e = launch_router_tc(mX, p, S(stream));
-    if (e != cudaErrorNotSupported) return cuda_status(e);
+  // tcgen05 router with x and Wr streamed by TMA for prefill-sized batches
+  // (Wr rows must be 16-byte strided: G*E a multiple of 8)
+  const int GE = p.G * p.E;
+  if (p.N >= 1024 && p.D % 64 == 0 && GE % 8 == 0 && GE <= 64 && aligned16(Wr)) {
+    const int R = router_tc_tile_rows(p.N);
+    CUtensorMap mX, mW;
+    if (map2d(&mX, x, p.D, p.N, R) && map2d(&mW, Wr, GE, p.D, 64)) {
+      const cudaError_t e = launch_router_tc(mX, mW, p, R, S(stream));
+      if (e != cudaErrorNotSupported) return cuda_status(e);
+    }
   }
   return cuda_status(launch_router(p, S(stream)));
 }

@@ -17,9 +17,13 @@ struct RouterParams {
   unsigned* err;          // device error word (bounded waits of the tcgen05 router)
 };
 cudaError_t launch_router(const RouterParams& p, cudaStream_t stream);
-// tcgen05 router streaming x by TMA (map over x [N, D], box 64 x 128); returns
-// cudaErrorNotSupported for shapes it does not take (the caller falls back).
-cudaError_t launch_router_tc(const CUtensorMap& mapX, const RouterParams& p, cudaStream_t stream);
+// tcgen05 router streaming x and Wr by TMA: mapX over x [N, D] with a box of
+// 64 columns x R rows, R = router_tc_tile_rows(N); mapW over Wr [D, G*E] with
+// a box of 64 x 64 (G*E a multiple of 8).  Returns cudaErrorNotSupported for
+// shapes it does not take (the caller falls back to the CUDA-core routers).
+int router_tc_tile_rows(int N);
+cudaError_t launch_router_tc(const CUtensorMap& mapX, const CUtensorMap& mapW, const RouterParams& p, int R,
+                             cudaStream_t stream);
 
 // Token-to-expert permutation workspace (int32 arrays, see perm.cu): segment
 // counters, then per segment `cap` slots of source and destination rows.

@@ -422,28 +422,30 @@ cudaError_t launch_router_gep(const RouterParams& p, cudaStream_t stream) {
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// tcgen05 router: 128-token x tiles stream in by TMA (128-byte swizzle); Wr^T
-// sits in shared memory for the whole kernel as the MMA's B operand (GEP
-// expert rows, zero-padded, one 128-byte row per 64-column k-block); the
-// logits of a tile accumulate in fp32 in tensor memory (two accumulators, so
-// one tile's routing overlaps the next tile's MMAs), and the epilogue routes
-// one token per thread: per-group softmax and TopK on logit + bias, the
-// renormalised weights of the selected experts.
-//
-// CTA (192 threads): warp 0 TMA producer, warp 1 MMA issuer (and tensor-memory
-// owner), warps 2..5 routing epilogue.
+// tcgen05 router.  A CTA takes R consecutive tokens at a time (R <= 128, a
+// multiple of 8, chosen on the host so that the tiles spread evenly over the
+// SMs: the kernel streams x once and is HBM bound).  Every 64-dimension
+// k-block of a tile arrives by TMA in one ring stage together with the same
+// 64 rows of Wr, as Wr is stored ([D, G*E]): the MMA reads it as an MN-major B
+// operand of 64 columns, the columns past G*E zero-filled by the TMA, so Wr
+// is never rearranged in shared memory.  The logits accumulate in fp32 in
+// tensor memory (two buffers, so one tile's routing overlaps the next tile's
+// MMAs) and the epilogue routes one token per thread: per-group softmax and
+// TopK on logit + bias, the renormalised weights of the selected experts.
 namespace {
 
-constexpr int kRtBM = 128;
+constexpr int kRtBM = 128;                    // MMA rows; rows R..127 of a tile are not routed
 constexpr int kRtBK = 64;
-constexpr int kRtTile = kRtBM * kRtBK * 2;   // 16 KB x tile
+constexpr int kRtN = 64;                      // MMA columns: G*E zero-padded by the TMA
+constexpr int kRtX = kRtBM * kRtBK * 2;       // 16 KB of x rows per stage
+constexpr int kRtW = kRtN * kRtBK * 2;        // 8 KB of Wr rows per stage
+constexpr int kRtStage = kRtX + kRtW;
 
 struct __align__(8) RouterTcBarriers {
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
-  uint64_t w_full;           // Wr copied into shared memory (bulk copy)
   uint32_t tmem_base;
   int abort;
 };
@@ -557,27 +559,24 @@ __device__ __forceinline__ void route_token_e(const RouterParams& p, const float
 }
 
 // CTA (224 threads): warp 0 TMA producer; warps 1 and 6 issue the MMAs of the
-// even and odd k-blocks into two partial accumulators (an N <= 64 MMA keeps
-// the tensor pipe busy for less time than one thread needs to issue it);
-// warps 2..5 sum the partials and route, one token per thread.
+// even and odd k-blocks into two partial accumulators (a small-N MMA keeps the
+// tensor pipe busy for less time than one thread needs to issue it); warps
+// 2..5 sum the partials and route, one token per thread.
 template <int GEP, int STAGES>
-__global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant__ CUtensorMap mapX, RouterParams p,
-                                                           int wr_staged) {
-  constexpr int kWBlk = GEP * 128;                 // one k-block of Wr^T
-  constexpr uint32_t kTmemCols = 4 * GEP;          // 2 buffers x 2 partial accumulators
+__global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant__ CUtensorMap mapX,
+                                                           const __grid_constant__ CUtensorMap mapW, RouterParams p,
+                                                           int R) {
+  constexpr uint32_t kTmemCols = 4 * kRtN;          // 2 buffers x 2 partial accumulators
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int nk = p.D / kRtBK;
-  uint8_t* sW = smem;                                        // nk x [GEP rows x 128 B]
-  uint8_t* sX = sW + ((nk * kWBlk + 1023) & ~1023);          // STAGES x 16 KB
-  RouterTcBarriers* bar = reinterpret_cast<RouterTcBarriers*>(sX + STAGES * kRtTile);
+  uint8_t* sS = smem;                                        // STAGES x [x 16 KB | Wr 8 KB]
+  RouterTcBarriers* bar = reinterpret_cast<RouterTcBarriers*>(sS + STAGES * kRtStage);
   float* sBias = reinterpret_cast<float*>(bar + 1);          // GEP
-  // Wr as it is in memory ([D, GE]), when it is brought in by one bulk copy
-  uint8_t* sWr = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sBias + GEP) + 127) & ~uintptr_t(127));
   volatile int* abort = &bar->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int GE = p.G * p.E;
-  const int n_tiles = (p.N + kRtBM - 1) / kRtBM;
+  const int nk = p.D / kRtBK;
+  const int n_tiles = (p.N + R - 1) / R;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -588,92 +587,15 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
       mbar_init(&bar->acc_full[a], 2);     // one commit from each MMA thread
       mbar_init(&bar->acc_empty[a], 4);
     }
-    mbar_init(&bar->w_full, 1);
     bar->abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&mapX);
+    tma_prefetch_desc(&mapW);
   }
   if (warp == 1) tmem_alloc(&bar->tmem_base, kTmemCols);
   pdl_launch_dependents();
   pdl_wait();
-  __syncthreads();   // barriers initialised
-  // the first x tiles are requested before Wr^T is built (they do not need it)
-  const int first_tiles = min(STAGES, (blockIdx.x < n_tiles ? ((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0) * nk);
-  const uint32_t wr_bytes = (uint32_t)p.D * GE * 2;
-  if (threadIdx.x == 0) {
-    for (int it = 0; it < first_tiles; ++it) {
-      const int t = blockIdx.x + (it / nk) * gridDim.x, kb = it % nk;
-      mbar_arrive_expect_tx(&bar->full[it], kRtTile);
-      tma_load_2d(sX + it * kRtTile, &mapX, &bar->full[it], kb * kRtBK, t * kRtBM);
-    }
-    if (wr_staged) {
-      mbar_arrive_expect_tx(&bar->w_full, wr_bytes);
-      bulk_load(sWr, p.Wr, wr_bytes, &bar->w_full);
-    }
-  }
-  // Wr [D, GE] -> Wr^T in the swizzled K-major layout (rows GE..GEP-1 zero)
-  if (wr_staged) {
-    // from the bulk copy in shared memory: 16 bytes = 8 experts of one model dimension
-    mbar_wait(&bar->w_full, 0, abort, p.err, kErrTimeoutRouter);
-    const int per_row = GE / 8;
-    for (int e = threadIdx.x; e < p.D * per_row; e += blockDim.x) {
-      const int dd = e / per_row, n0 = (e % per_row) * 8;
-      const uint4 v = *reinterpret_cast<const uint4*>(sWr + ((size_t)dd * GE + n0) * 2);
-      const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
-      const int kb = dd >> 6, c = dd & 63;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int n = n0 + i;
-        *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) = h[i];
-      }
-    }
-    for (int e = threadIdx.x; e < p.D * (GEP - GE); e += blockDim.x) {
-      const int dd = e / (GEP - GE), n = GE + e % (GEP - GE);
-      const int kb = dd >> 6, c = dd & 63;
-      *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) = 0;
-    }
-  } else if ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0) {
-    // 16-byte loads of 8 consecutive experts of one model dimension
-    const int per_row = GE / 8;
-    const int total = p.D * per_row;
-    for (int e0 = threadIdx.x; e0 < total; e0 += 4 * blockDim.x) {
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * blockDim.x;
-        if (e < total)
-          v[u] = __ldg(reinterpret_cast<const uint4*>(p.Wr + (size_t)(e / per_row) * GE + (e % per_row) * 8));
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * blockDim.x;
-        if (e >= total) break;
-        const int dd = e / per_row, n0 = (e % per_row) * 8;
-        const uint16_t* h = reinterpret_cast<const uint16_t*>(&v[u]);
-        const int kb = dd >> 6, c = dd & 63;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int n = n0 + i;
-          *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) =
-              h[i];
-        }
-      }
-    }
-    for (int e = threadIdx.x; e < p.D * (GEP - GE); e += blockDim.x) {
-      const int dd = e / (GEP - GE), n = GE + e % (GEP - GE);
-      const int kb = dd >> 6, c = dd & 63;
-      *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) = 0;
-    }
-  } else {
-    for (int e = threadIdx.x; e < p.D * GEP; e += blockDim.x) {
-      const int dd = e / GEP, n = e % GEP;
-      const int kb = dd >> 6, c = dd & 63;
-      const uint16_t v = n < GE ? p.Wr[(size_t)dd * GE + n] : (uint16_t)0;
-      *reinterpret_cast<uint16_t*>(sW + kb * kWBlk + n * 128 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2) = v;
-    }
-  }
   for (int e = threadIdx.x; e < GEP; e += blockDim.x) sBias[e] = (p.bias && e < GE) ? p.bias[e] : 0.f;
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -681,16 +603,17 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
 
   if (warp == 0) {
     if (lane == 0) {
+      const uint32_t stage_tx = (uint32_t)R * kRtBK * 2 + kRtW;
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          if (it < first_tiles) continue;   // requested before Wr^T was built
           const int s = it % STAGES;
           if (it >= STAGES &&
               !mbar_wait(&bar->empty[s], ((it / STAGES) & 1) ^ 1, abort, p.err, kErrTimeoutRouter))
             break;
-          mbar_arrive_expect_tx(&bar->full[s], kRtTile);
-          tma_load_2d(sX + s * kRtTile, &mapX, &bar->full[s], kb * kRtBK, t * kRtBM);
+          mbar_arrive_expect_tx(&bar->full[s], stage_tx);
+          tma_load_2d(sS + s * kRtStage, &mapX, &bar->full[s], kb * kRtBK, t * R);
+          tma_load_2d(sS + s * kRtStage + kRtX, &mapW, &bar->full[s], 0, kb * kRtBK);
         }
       }
     }
@@ -698,14 +621,13 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
     if (lane == 0) {
       // warp 1: k-blocks 0, 2, 4, ... into partial 0; warp 6: 1, 3, 5, ... into partial 1
       const int half = warp == 6 ? 1 : 0;
-      constexpr uint32_t idesc = idesc_bf16_f32(kRtBM, GEP, false, false);
-      const uint32_t w0 = smem_u32(sW);
+      constexpr uint32_t idesc = idesc_bf16_f32(kRtBM, kRtN, false, true);
       int tc = 0;
       for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tc) {
         const int ab = tc & 1, use = tc >> 1;
         if (tc >= 2 && !mbar_wait(&bar->acc_empty[ab], (use & 1) ^ 1, abort, p.err, kErrTimeoutRouter)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)((2 * ab + half) * GEP);
+        const uint32_t acc = tmem + (uint32_t)((2 * ab + half) * kRtN);
         bool ok = true;
         for (int kb = half; kb < nk; kb += 2) {
           const int it = tc * nk + kb;
@@ -715,11 +637,12 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sX + s * kRtTile);
-          const uint32_t b0 = w0 + (uint32_t)(kb * kWBlk);
+          const uint32_t a0 = smem_u32(sS + s * kRtStage);
+          const uint32_t b0 = a0 + kRtX;
 #pragma unroll
           for (int kk = 0; kk < kRtBK / 16; ++kk)
-            umma_ss(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
+            // A: x rows, K-major; B: Wr rows, MN-major (a 16-deep k-step is 16 rows of 128 bytes)
+            umma_ss(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 2048, kRtW, 1024), idesc,
                     (kb != half) || kk != 0);
           umma_commit(&bar->empty[s]);
         }
@@ -730,6 +653,7 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
   } else {
     const int lg = warp & 3;
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    const int r = lg * 32 + lane;
     int tc = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
       const int ab = tc & 1, use = tc >> 1;
@@ -739,11 +663,11 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
 #pragma unroll
       for (int c0 = 0; c0 < GEP; c0 += 16) {
         uint32_t v[16];
-        tmem_ld16(tmem + lane_off + (uint32_t)(2 * ab * GEP + c0), v);
+        tmem_ld16(tmem + lane_off + (uint32_t)(2 * ab * kRtN + c0), v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) logit[c0 + i] = __uint_as_float(v[i]);
         if (nk > 1) {   // the odd k-blocks' partial
-          tmem_ld16(tmem + lane_off + (uint32_t)((2 * ab + 1) * GEP + c0), v);
+          tmem_ld16(tmem + lane_off + (uint32_t)((2 * ab + 1) * kRtN + c0), v);
 #pragma unroll
           for (int i = 0; i < 16; ++i) logit[c0 + i] += __uint_as_float(v[i]);
         }
@@ -751,8 +675,8 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->acc_empty[ab]);
-      const int n = t * kRtBM + lg * 32 + lane;
-      if (ok && n < p.N) {
+      const int n = t * R + r;
+      if (ok && r < R && n < p.N) {
         if (p.E == 2 && GEP <= 32) route_token_e<GEP, 2>(p, logit, sBias, n);
         else if (p.E == 4) route_token_e<GEP, 4>(p, logit, sBias, n);
         else if (p.E == 8) route_token_e<GEP, 8>(p, logit, sBias, n);
@@ -771,38 +695,38 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
 }
 
 template <int GEP>
-size_t router_tc_smem(int D, int stages, size_t staging) {
-  return 1024 + (((size_t)(D / kRtBK) * GEP * 128 + 1023) & ~size_t(1023)) + (size_t)stages * kRtTile +
-         sizeof(RouterTcBarriers) + GEP * sizeof(float) + 128 + staging;
-}
-
-template <int GEP>
-cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const RouterParams& p, cudaStream_t stream) {
-  constexpr int STAGES = 6;
-  // Wr by one bulk copy when it and its staging fit (16-byte aligned, whole 16-byte rows of 8 experts)
-  const int GE = p.G * p.E;
-  const size_t wr_bytes = (size_t)p.D * GE * 2;
-  int staged = ((GE & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Wr) & 15) == 0 && wr_bytes % 16 == 0) ? 1 : 0;
-  if (staged && router_tc_smem<GEP>(p.D, STAGES, wr_bytes) > 220 * 1024) staged = 0;
-  const size_t smem = router_tc_smem<GEP>(p.D, STAGES, staged ? wr_bytes : 0);
-  if (smem > 220 * 1024) return cudaErrorNotSupported;
+cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const CUtensorMap& mapW, const RouterParams& p, int R,
+                                 cudaStream_t stream) {
+  constexpr int STAGES = 8;
+  const size_t smem = 1024 + (size_t)STAGES * kRtStage + sizeof(RouterTcBarriers) + GEP * sizeof(float);
   auto kern = router_tc_kernel<GEP, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  const int n_tiles = (p.N + kRtBM - 1) / kRtBM;
+  const int n_tiles = (p.N + R - 1) / R;
   const int sms = router_num_sms();
   const int grid = n_tiles < sms ? n_tiles : sms;
-  return launch_kernel(kern, dim3(grid), dim3(224), smem, stream, 1, mapX, p, staged);
+  return launch_kernel(kern, dim3(grid), dim3(224), smem, stream, 1, mapX, mapW, p, R);
 }
 
 }  // namespace
 
-cudaError_t launch_router_tc(const CUtensorMap& mapX, const RouterParams& p, cudaStream_t stream) {
+int router_tc_tile_rows(int N) {
+  const int sms = router_num_sms();
+  const long long per_cta = (N + (long long)kRtBM * sms - 1) / ((long long)kRtBM * sms);   // tiles per CTA
+  long long R = (N + sms * per_cta - 1) / (sms * per_cta);
+  R = (R + 7) / 8 * 8;
+  // below 64 rows a tile's x is smaller than its share of Wr (8 KB per k-block)
+  return (int)(R < kRtBM ? (R < 64 ? 64 : R) : kRtBM);
+}
+
+cudaError_t launch_router_tc(const CUtensorMap& mapX, const CUtensorMap& mapW, const RouterParams& p, int R,
+                             cudaStream_t stream) {
   const int GE = p.G * p.E;
-  if (p.D % kRtBK != 0 || p.E > 8) return cudaErrorNotSupported;
-  if (GE <= 16) return launch_router_tc_gep<16>(mapX, p, stream);
-  if (GE <= 32) return launch_router_tc_gep<32>(mapX, p, stream);
-  return launch_router_tc_gep<64>(mapX, p, stream);
+  if (p.D % kRtBK != 0 || p.E > 8 || GE > kRtN || GE % 8 != 0 || R < 8 || R > kRtBM || R % 8 != 0)
+    return cudaErrorNotSupported;
+  if (GE <= 16) return launch_router_tc_gep<16>(mapX, mapW, p, R, stream);
+  if (GE <= 32) return launch_router_tc_gep<32>(mapX, mapW, p, R, stream);
+  return launch_router_tc_gep<64>(mapX, mapW, p, R, stream);
 }
 
 // ---------------------------------------------------------------------------
