@@ -469,7 +469,10 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
   const int n_kv = ti.n_kv;
   const CUtensorMap* mq = routed ? &mapQ : &mapQs;
 
-  if (threadIdx.x == 0) {
+  // The K-side thread sets up the barriers and puts Q and the first K and V
+  // tiles in flight before the CTA-wide barrier, so they load while tensor
+  // memory is allocated.
+  if (warp == 4 && lane == 0) {
     mbar_init(&bar->q_full, 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(&bar->k_full[s], 1);
@@ -483,9 +486,15 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     mbar_init(&bar->pv_done, 1);
     bar->abort = 0;
     fence_mbar_init();
-    tma_prefetch_desc(mq);
-    tma_prefetch_desc(&mapK);
-    tma_prefetch_desc(&mapV);
+    pdl_wait();
+    mbar_arrive_expect_tx(&bar->q_full, kBox);
+    tma_load_3d(sQ, mq, &bar->q_full, 0, ti.row0, seq);
+    for (int j = 0; j < ST && j < n_kv; ++j) {
+      mbar_arrive_expect_tx(&bar->k_full[j], kBox);
+      tma_load_3d(sK + j * kBox, &mapK, &bar->k_full[j], 0, j * kTile, kvseq);
+      mbar_arrive_expect_tx(&bar->v_full[j], kBox);
+      tma_load_3d(sV + j * kBox, &mapV, &bar->v_full[j], 0, j * kTile, kvseq);
+    }
   }
   if (warp == 5) tmem_alloc(&bar->tmem_base, 256);
   tc_fence_before();
@@ -508,12 +517,6 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       // is issued as soon as the softmax holds S(j) in registers (s_free), so
       // it runs while the exponentials of tile j do.
       constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
-      mbar_arrive_expect_tx(&bar->q_full, kBox);
-      tma_load_3d(sQ, mq, &bar->q_full, 0, ti.row0, seq);
-      for (int j = 0; j < ST && j < n_kv; ++j) {
-        mbar_arrive_expect_tx(&bar->k_full[j], kBox);
-        tma_load_3d(sK + j * kBox, &mapK, &bar->k_full[j], 0, j * kTile, kvseq);
-      }
       const uint32_t q0 = smem_u32(sQ);
       bool ok = mbar_wait(&bar->q_full, 0, abort, p.err, kErrTimeoutAttn);
       ATTN_TRACE(if (TR) TR[3] = globaltimer();)
@@ -545,10 +548,6 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       // tensor memory (a second issuing thread: an MMA of N = 64 takes the
       // tensor pipe for less time than one thread needs to issue it)
       constexpr uint32_t idesc_o = idesc_bf16_f32(kTile, D, false, true);
-      for (int j = 0; j < ST && j < n_kv; ++j) {
-        mbar_arrive_expect_tx(&bar->v_full[j], kBox);
-        tma_load_3d(sV + j * kBox, &mapV, &bar->v_full[j], 0, j * kTile, kvseq);
-      }
       bool ok = true;
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % ST;
@@ -708,18 +707,19 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     const float inv_l = 1.f / l_run;
     gqe_bf16_t* orow = routed ? p.o_routed + ((size_t)seq * rows_total + prow) * D
                               : p.o_sh + ((size_t)seq * p.T + prow) * D;
-#pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      tmem_ld32(o_base + c0, o);
+    {
+      uint32_t o[64];
+      tmem_ld64(o_base, o);
       if (valid && ok) {
-        uint32_t pk[16];
+        uint4* d4 = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-        uint4* d4 = reinterpret_cast<uint4*>(orow + c0);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t pk[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int e = 0; e < 4; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(o[8 * c + 2 * e]) * inv_l, __uint_as_float(o[8 * c + 2 * e + 1]) * inv_l);
+          d4[c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
       }
     }
     if (p.lse && valid && ok) {
