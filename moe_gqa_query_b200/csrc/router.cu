@@ -422,9 +422,9 @@ cudaError_t launch_router_gep(const RouterParams& p, cudaStream_t stream) {
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// tcgen05 router.  A CTA takes R consecutive tokens at a time (R <= 128, a
-// multiple of 8, chosen on the host so that the tiles spread evenly over the
-// SMs: the kernel streams x once and is HBM bound).  Every 64-dimension
+// tcgen05 router.  A CTA takes R consecutive tokens at a time (R <= 128 and a
+// multiple of 8, given by router_tc_tile_rows; the kernel streams x once and
+// is HBM bound).  Every 64-dimension
 // k-block of a tile arrives by TMA in one ring stage together with the same
 // 64 rows of Wr, as Wr is stored ([D, G*E]): the MMA reads it as an MN-major B
 // operand of 64 columns, the columns past G*E zero-filled by the TMA, so Wr
@@ -440,6 +440,12 @@ constexpr int kRtN = 64;                      // MMA columns: G*E zero-padded by
 constexpr int kRtX = kRtBM * kRtBK * 2;       // 16 KB of x rows per stage
 constexpr int kRtW = kRtN * kRtBK * 2;        // 8 KB of Wr rows per stage
 constexpr int kRtStage = kRtX + kRtW;
+// Ring depth of the tcgen05 router.  Deeper rings make the router alone faster
+// but slow the layer, whose K/V projection reads x beside it (main layer step:
+// 4 stages 196.5 us, 6 stages 197.4 us, 8 stages 198.4 us).
+#ifndef GQE_ROUTER_TC_STAGES
+#define GQE_ROUTER_TC_STAGES 4
+#endif
 
 struct __align__(8) RouterTcBarriers {
   uint64_t full[8];
@@ -697,7 +703,7 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
 template <int GEP>
 cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const CUtensorMap& mapW, const RouterParams& p, int R,
                                  cudaStream_t stream) {
-  constexpr int STAGES = 8;
+  constexpr int STAGES = GQE_ROUTER_TC_STAGES;
   const size_t smem = 1024 + (size_t)STAGES * kRtStage + sizeof(RouterTcBarriers) + GEP * sizeof(float);
   auto kern = router_tc_kernel<GEP, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
@@ -711,12 +717,12 @@ cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const CUtensorMap& map
 }  // namespace
 
 int router_tc_tile_rows(int N) {
-  const int sms = router_num_sms();
-  const long long per_cta = (N + (long long)kRtBM * sms - 1) / ((long long)kRtBM * sms);   // tiles per CTA
-  long long R = (N + sms * per_cta - 1) / (sms * per_cta);
-  R = (R + 7) / 8 * 8;
-  // below 64 rows a tile's x is smaller than its share of Wr (8 KB per k-block)
-  return (int)(R < kRtBM ? (R < 64 ? 64 : R) : kRtBM);
+  // 128-row tiles: at 16384 tokens 128 CTAs stream x and the remaining SMs
+  // are free for the K/V projection the layer runs beside the router (tiles
+  // sized to cover every SM made the router alone faster but the layer's step
+  // slower, 202 against 195.5 us on the main layer)
+  (void)N;
+  return kRtBM;
 }
 
 cudaError_t launch_router_tc(const CUtensorMap& mapX, const CUtensorMap& mapW, const RouterParams& p, int R,
