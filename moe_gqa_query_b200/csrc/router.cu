@@ -440,12 +440,14 @@ constexpr int kRtN = 64;                      // MMA columns: G*E zero-padded by
 constexpr int kRtX = kRtBM * kRtBK * 2;       // 16 KB of x rows per stage
 constexpr int kRtW = kRtN * kRtBK * 2;        // 8 KB of Wr rows per stage
 constexpr int kRtStage = kRtX + kRtW;
-// Ring depth of the tcgen05 router.  Deeper rings make the router alone faster
-// but slow the layer, whose K/V projection reads x beside it (main layer step:
-// 4 stages 196.5 us, 6 stages 197.4 us, 8 stages 198.4 us).
-#ifndef GQE_ROUTER_TC_STAGES
-#define GQE_ROUTER_TC_STAGES 4
-#endif
+// Ring depth of the tcgen05 router.  With short x rows (d_model < 2048) a
+// deeper ring makes the router alone faster but slows the layer, whose K/V
+// projection reads x beside it (main layer step: 4 stages 196.5 us, 6 stages
+// 197.4 us, 8 stages 198.4 us); with long rows the router needs the deeper
+// ring to keep enough of x in flight (d_model 4096: 55 us at 4 stages, 42 us
+// at 8).
+constexpr int kRouterStagesShort = 4;
+constexpr int kRouterStagesLong = 8;
 
 struct __align__(8) RouterTcBarriers {
   uint64_t full[8];
@@ -700,10 +702,9 @@ __global__ void __launch_bounds__(224, 1) router_tc_kernel(const __grid_constant
   drain_after_abort(abort);
 }
 
-template <int GEP>
-cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const CUtensorMap& mapW, const RouterParams& p, int R,
-                                 cudaStream_t stream) {
-  constexpr int STAGES = GQE_ROUTER_TC_STAGES;
+template <int GEP, int STAGES>
+cudaError_t launch_router_tc_st(const CUtensorMap& mapX, const CUtensorMap& mapW, const RouterParams& p, int R,
+                                cudaStream_t stream) {
   const size_t smem = 1024 + (size_t)STAGES * kRtStage + sizeof(RouterTcBarriers) + GEP * sizeof(float);
   auto kern = router_tc_kernel<GEP, STAGES>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
@@ -712,6 +713,13 @@ cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const CUtensorMap& map
   const int sms = router_num_sms();
   const int grid = n_tiles < sms ? n_tiles : sms;
   return launch_kernel(kern, dim3(grid), dim3(224), smem, stream, 1, mapX, mapW, p, R);
+}
+
+template <int GEP>
+cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const CUtensorMap& mapW, const RouterParams& p, int R,
+                                 cudaStream_t stream) {
+  if (p.D / kRtBK >= 32) return launch_router_tc_st<GEP, kRouterStagesLong>(mapX, mapW, p, R, stream);
+  return launch_router_tc_st<GEP, kRouterStagesShort>(mapX, mapW, p, R, stream);
 }
 
 }  // namespace
