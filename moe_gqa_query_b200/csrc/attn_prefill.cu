@@ -54,16 +54,16 @@ constexpr int kTile = 128;          // query rows and keys per tile
 constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16, 16 KB
 constexpr float kRescaleLog2 = 8.0f;
 // Single-tile kernel (d = 64): GQE_ATTN1_F2 computes the scaled logits and the
-// row sums with packed f32x2 FMA/ADD (half the instructions), and
-// GQE_ATTN1_POLY column pairs of every 16 take the FMA-pipe polynomial 2^x
-// instead of MUFU ex2.  Measured on B200: 2 of 16 is 3-5 % faster than 0,
-// 4 of 16 no better (register pressure).
+// row sums with packed f32x2 FMA/ADD (half the instructions), and POLY column
+// pairs of every 16 (a template parameter) take the FMA-pipe polynomial 2^x
+// instead of MUFU ex2.  Measured on B200: 2 of 16 is 3-5 % faster than 0 at
+// T = 2048, where 3 of 16 is 2 % slower; at T = 32768, where the steady
+// per-tile loop dominates, 3 of 16 is 1 % faster than 2 and 4 of 16 slower
+// than both.  The launcher takes 3 from T = 16384 on.
 #ifndef GQE_ATTN1_F2
 #define GQE_ATTN1_F2 1
 #endif
-#ifndef GQE_ATTN1_POLY
-#define GQE_ATTN1_POLY 2
-#endif
+constexpr int kPolyShortT = 2, kPolyLongT = 3, kPolyLongFromT = 16384;
 #ifndef GQE_ATTN_POLY_PAIRS
 #define GQE_ATTN_POLY_PAIRS 0
 #endif
@@ -422,6 +422,7 @@ struct __align__(8) Attn1Barriers {
 constexpr int kSingleST = 2;   // two CTAs per SM must fit in 228 KB of shared memory
 constexpr size_t kSingleSmem = 1024 + kBox + 2 * kSingleST * kBox + sizeof(Attn1Barriers);
 
+template <int POLY>
 __global__ void __launch_bounds__(192, 2)
 attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapQs,
                            const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
@@ -643,7 +644,7 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
           const unsigned long long x =
               f2_fma(f2_pack(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), sl2x2, negm2);
           float p0, p1;
-          if ((c & 15) < GQE_ATTN1_POLY) {
+          if ((c & 15) < POLY) {
             exp2_poly2(x, p0, p1);
           } else {
             float x0, x1;
@@ -755,7 +756,7 @@ static cudaError_t launch_d(const CUtensorMap& mQ, const CUtensorMap& mQs, const
 
 static cudaError_t launch_single(const CUtensorMap& mQ, const CUtensorMap& mQs, const CUtensorMap& mK,
                                  const CUtensorMap& mV, const AttnParams& p, cudaStream_t stream) {
-  auto kern = attn_prefill_single_kernel;
+  auto kern = p.T >= kPolyLongFromT ? attn_prefill_single_kernel<kPolyLongT> : attn_prefill_single_kernel<kPolyShortT>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), kSingleSmem);
   if (e != cudaSuccess) return e;
   const int n_levels = (p.T + kTile - 1) / kTile;
