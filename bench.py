@@ -474,6 +474,18 @@ CONFIG_WORKLOADS = ("tiny_prefill", "main_prefill", "long_prefill", "wide_skewed
 SEG_NAMES = ("router", "routed_qproj", "kv_proj", "attn_prefill", "combine_out_proj")
 
 
+def router_near_ties(wname):
+    """The workload's router near-ties ((token, group) pairs whose k-th and
+    (k+1)-th logits differ by less than 1e-4, where either expert is a correct
+    choice), as the oracle counted them in tests/golden/near_ties.json."""
+    try:
+        with open(os.path.join(ROOT, "tests", "golden", "near_ties.json")) as f:
+            v = json.load(f)["workloads"][wname]
+        return {"pairs": v["near_ties"], "of": v["pairs"], "source": "tests/golden/near_ties.json (fp64 oracle)"}
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def attn_kernel_label(dims) -> str:
     return "attn_prefill_single_kernel (d=64)" if dims.d == 64 else f"attn_prefill_kernel<{dims.d}>"
 
@@ -568,7 +580,8 @@ def measure_prefill(gq, wname, device, dist, peaks, steps, warmup, flush, rank, 
                         "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
                         "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": profiled_traffic(label, wname),
                         "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_ms},
-           "gpu_launches": LAUNCHES_PER_STEP * steps, "device_error": gq.gqe_device_error()}
+           "gpu_launches": LAUNCHES_PER_STEP * steps, "router_near_ties": router_near_ties(wname),
+           "device_error": gq.gqe_device_error()}
     if keep_layer:
         out.update(_layer=layer, _x=x, _x_host=x_host)
     else:
