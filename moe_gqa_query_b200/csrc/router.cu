@@ -446,7 +446,22 @@ constexpr int kRtStage = kRtX + kRtW;
 // 197.4 us, 8 stages 198.4 us); with long rows the router needs the deeper
 // ring to keep enough of x in flight (d_model 4096: 55 us at 4 stages, 42 us
 // at 8).
-constexpr int kRouterStagesShort = 4;
+// Ring depth below d_model 2048, and 128-token tiles per CTA.  The layer runs
+// its K/V projection on a side stream beside the router, so the router is
+// sized for the step, not for its own time: with four tiles per CTA (32 CTAs
+// at 16384 tokens) each CTA's routing epilogue overlaps its next tile's x
+// stream and the other SMs start the K/V GEMM at once.  Measured on B200,
+// main-layer step 187.2 -> 178.9 us (one tile per CTA, 4 stages -> four, 8),
+// wide/skewed 1326 -> 1268 us, T = 32768 1666 -> 1650 us; the router call
+// alone 21.7 -> 28.6 us.  Two tiles per CTA, three and six or eight gave
+// steps in between or slower.
+#ifndef GQE_ROUTER_STAGES_SHORT
+#define GQE_ROUTER_STAGES_SHORT 8
+#endif
+#ifndef GQE_ROUTER_TILES_PER_CTA
+#define GQE_ROUTER_TILES_PER_CTA 4
+#endif
+constexpr int kRouterStagesShort = GQE_ROUTER_STAGES_SHORT;
 constexpr int kRouterStagesLong = 8;
 
 struct __align__(8) RouterTcBarriers {
@@ -711,7 +726,8 @@ cudaError_t launch_router_tc_st(const CUtensorMap& mapX, const CUtensorMap& mapW
   if (e != cudaSuccess) return e;
   const int n_tiles = (p.N + R - 1) / R;
   const int sms = router_num_sms();
-  const int grid = n_tiles < sms ? n_tiles : sms;
+  const int want = (n_tiles + GQE_ROUTER_TILES_PER_CTA - 1) / GQE_ROUTER_TILES_PER_CTA;
+  const int grid = want < sms ? want : sms;
   return launch_kernel(kern, dim3(grid), dim3(224), smem, stream, 1, mapX, mapW, p, R);
 }
 
@@ -725,10 +741,8 @@ cudaError_t launch_router_tc_gep(const CUtensorMap& mapX, const CUtensorMap& map
 }  // namespace
 
 int router_tc_tile_rows(int N) {
-  // 128-row tiles: at 16384 tokens 128 CTAs stream x and the remaining SMs
-  // are free for the K/V projection the layer runs beside the router (tiles
-  // sized to cover every SM made the router alone faster but the layer's step
-  // slower, 202 against 195.5 us on the main layer)
+  // 128-row tiles (tiles sized to cover every SM made the router alone faster
+  // but the layer's step slower, 202 against 195.5 us on the main layer)
   (void)N;
   return kRtBM;
 }
