@@ -764,13 +764,21 @@ int num_sms() {
   return n;
 }
 
-int dense_tile_n(int n_per_weight) { return (n_per_weight % 256 == 0) ? 256 : 128; }
+// Output tile width of the single-CTA dense GEMM.  With all rows in one
+// 128-row tile (the decode step's M = batch), 64-column tiles put four times
+// as many CTAs on the weight stream as 256-column ones.
+int dense_tile_n(int n_per_weight, int M) {
+  if (M <= kBM && n_per_weight % 64 == 0) return 64;
+  return (n_per_weight % 256 == 0) ? 256 : 128;
+}
 
 cudaError_t launch_gemm_dense(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                               const CUtensorMap& mapO0, const CUtensorMap& mapO1, const EpiParams& ep, int M, int K,
                               int n_tiles_b0, int n_tiles_total, int bn, cudaStream_t stream, int mn) {
   if (bn == 256)
     return launch_dense_bn<256, 4>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream, mn);
+  if (bn == 64)
+    return launch_dense_bn<64, 7>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream, mn);
   return launch_dense_bn<128, 6>(mapA, mapB0, mapB1, mapO0, mapO1, ep, M, K, n_tiles_b0, n_tiles_total, stream, mn);
 }
 

@@ -52,7 +52,7 @@ struct RoutedParams {
 };
 
 // Output tile width for a weight with n_per_weight rows: 256 when it divides, else 128.
-int dense_tile_n(int n_per_weight);
+int dense_tile_n(int n_per_weight, int M);
 int num_sms();
 
 // mapO0 / mapO1: output maps for ep.store_mode != kStorePerThread.

@@ -363,7 +363,7 @@ static gqe_status kv_common(const gqe_dims* dims, const gqe_bf16* x, const gqe_b
                             EpiParams& ep, int M, gqe_stream stream) {
   const int G = dims->G, d = dims->d_head, D = dims->d_model;
   const int pbn = pair_tile_n(M, G * d);
-  const int bn = pbn ? pbn : dense_tile_n(G * d);
+  const int bn = pbn ? pbn : dense_tile_n(G * d, M);
   CUtensorMap mA, mK, mV;
   GQE_REQUIRE(map2d(&mA, x, D, M, 128), GQE_ERR_CUDA);
   GQE_REQUIRE(map2d(&mK, Wk, D, (uint64_t)G * d, pbn ? pbn / 2 : bn), GQE_ERR_CUDA);
@@ -608,7 +608,7 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
   GQE_REQUIRE((long long)M * N < (1ll << 31) && (long long)M * K < (1ll << 31), GQE_ERR_UNSUPPORTED);
   GQE_REQUIRE(aligned16(A) && aligned16(W) && aligned16(C), GQE_ERR_INVALID_ARG);
   const int pbn = pair_tile_n(M, N);
-  const int bn = pbn ? pbn : dense_tile_n(N);
+  const int bn = pbn ? pbn : dense_tile_n(N, M);
   CUtensorMap mA, mW;
   GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
   GQE_REQUIRE(map2d(&mW, W, K, N, pbn ? pbn / 2 : bn), GQE_ERR_CUDA);
@@ -640,7 +640,7 @@ gqe_status gqe_gemm_acc(int M, int N, int K, const gqe_bf16* A, int a_kn, const 
   GQE_REQUIRE(aligned16(A) && aligned16(B) && aligned16(C), GQE_ERR_INVALID_ARG);
   const int Kp = (K + 63) / 64 * 64;
   const int pbn = pair_tile_n(M, N);
-  const int bn = pbn ? pbn : dense_tile_n(N);
+  const int bn = pbn ? pbn : dense_tile_n(N, M);
   CUtensorMap mA, mW, mO;
   if (a_kn) GQE_REQUIRE(map2d(&mA, A, M, K, 64), GQE_ERR_CUDA);
   else GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
@@ -802,7 +802,7 @@ gqe_status gqe_gemm(int M, int N, int K, const gqe_bf16* A, int a_kn, const gqe_
   GQE_REQUIRE(aligned16(A) && aligned16(B) && aligned16(C), GQE_ERR_INVALID_ARG);
   const int Kp = (K + 63) / 64 * 64;
   const int pbn = pair_tile_n(M, N);
-  const int bn = pbn ? pbn : dense_tile_n(N);
+  const int bn = pbn ? pbn : dense_tile_n(N, M);
   CUtensorMap mA, mW;
   if (a_kn) GQE_REQUIRE(map2d(&mA, A, M, K, 64), GQE_ERR_CUDA);
   else GQE_REQUIRE(map2d(&mA, A, K, M, 128), GQE_ERR_CUDA);
