@@ -559,6 +559,30 @@ __device__ __forceinline__ void route_token_e(const RouterParams& p, const float
       den_tok += sum;
     }
   }
+  if (k == 1 && G == GM && GM % 4 == 0 && !p.probs &&
+      ((reinterpret_cast<uintptr_t>(p.topk_idx) | reinterpret_cast<uintptr_t>(p.topk_w)) & 15u) == 0) {
+    // one selection per group: the token's index and weight rows (G entries
+    // each, 16-byte aligned) leave as 16-byte vectors
+    int ri[GM];
+    float rw[GM];
+#pragma unroll
+    for (int g = 0; g < GM; ++g) {
+      int e1 = 0;
+#pragma unroll
+      for (int e = 1; e < E; ++e)
+        if ((chosen[g] >> e) & 1u) e1 = e;
+      ri[g] = e1;
+      rw[g] = pr[g * E + e1] * (p.scope == 2 ? 1.f : 1.f / (p.scope == 0 ? den_tok : gsum[g]));
+    }
+    int4* di = reinterpret_cast<int4*>(p.topk_idx + (size_t)n * GM);
+    float4* dw = reinterpret_cast<float4*>(p.topk_w + (size_t)n * GM);
+#pragma unroll
+    for (int q = 0; q < GM / 4; ++q) {
+      di[q] = make_int4(ri[4 * q], ri[4 * q + 1], ri[4 * q + 2], ri[4 * q + 3]);
+      dw[q] = make_float4(rw[4 * q], rw[4 * q + 1], rw[4 * q + 2], rw[4 * q + 3]);
+    }
+    return;
+  }
 #pragma unroll
   for (int g = 0; g < GM; ++g) {
     if (g < G) {
