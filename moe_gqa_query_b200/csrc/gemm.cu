@@ -807,6 +807,8 @@ static cudaError_t launch_routed_bn(const CUtensorMap& mapWq, const CUtensorMap&
 #ifndef GQE_ROUTED64_CPS
 #define GQE_ROUTED64_CPS 3
 #endif
+// d = 128 (wide/skewed, routed call alone): 3 stages x 2 CTAs 341 us; 2 x 3
+// 484, 6 x 1 410, 4 x 1 444 us.
 #ifndef GQE_ROUTED128_ST
 #define GQE_ROUTED128_ST 3
 #endif
