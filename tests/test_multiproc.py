@@ -138,3 +138,15 @@ def test_peaks_fall_back_without_the_measured_file(tmp_path, monkeypatch):
     f = bench.load_peaks()
     assert f["source"] == "fallback"
     assert (f["hbm_gbs"], f["bf16_tflops"]) == (6650.0, 1590.0)
+
+
+def test_router_near_ties_come_from_the_oracle_file():
+    # the bench line's per-workload near-tie counts are those the oracle wrote
+    # into tests/golden/near_ties.json; an unknown workload reports none
+    import bench
+    with open(os.path.join(bench.ROOT, "tests", "golden", "near_ties.json")) as f:
+        golden = json.load(f)["workloads"]
+    for wname, v in golden.items():
+        got = bench.router_near_ties(wname)
+        assert got["pairs"] == v["near_ties"] and got["of"] == v["pairs"]
+    assert bench.router_near_ties("no_such_workload") is None
