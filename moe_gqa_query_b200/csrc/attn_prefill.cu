@@ -64,15 +64,6 @@ constexpr float kRescaleLog2 = 8.0f;
 #define GQE_ATTN1_F2 1
 #endif
 constexpr int kPolyShortT = 2, kPolyLongT = 3, kPolyLongFromT = 16384;
-// Single-tile kernel: the K-side thread issues the first GQE_ATTN_PV_SPLIT of
-// the eight 16-key steps of every P(j) V (after S(j+1)), the V-side thread the
-// rest, so P(j) V completes sooner and the softmax waits less before writing
-// P(j+1).  Measured on B200 (same box, interleaved): 0 -> 2 steps 75.8 -> 73.7
-// us at T = 2048 and 1.488 -> 1.447 ms at T = 32768; 3 and 4 steps in between.
-#ifndef GQE_ATTN_PV_SPLIT
-#define GQE_ATTN_PV_SPLIT 2
-#endif
-constexpr int kPvSplit = GQE_ATTN_PV_SPLIT;
 #ifndef GQE_ATTN_POLY_PAIRS
 #define GQE_ATTN_POLY_PAIRS 0
 #endif
@@ -488,12 +479,12 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       mbar_init(&bar->k_full[s], 1);
       mbar_init(&bar->k_empty[s], 1);
       mbar_init(&bar->v_full[s], 1);
-      mbar_init(&bar->v_empty[s], kPvSplit ? 2 : 1);
+      mbar_init(&bar->v_empty[s], 1);
     }
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->s_free, 128);
     mbar_init(&bar->p_full, 128);
-    mbar_init(&bar->pv_done, kPvSplit ? 2 : 1);
+    mbar_init(&bar->pv_done, 1);
     bar->abort = 0;
     fence_mbar_init();
     pdl_wait();
@@ -521,23 +512,6 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     TR[2] = globaltimer();
   })
 
-  // With kPvSplit > 0 the K-side thread also issues the first kPvSplit 16-key
-  // steps of every P(j) V (after S(j+1)), the V-side thread the rest; O starts
-  // from zeros the softmax writes, so neither part has to go first.
-  auto pv_part = [&](int j, int ks0, int ks1) -> bool {
-    const int s = j % ST;
-    constexpr uint32_t idesc_o = idesc_bf16_f32(kTile, D, false, true);
-    bool ok = mbar_wait(&bar->p_full, j & 1, abort, p.err, kErrTimeoutAttn);
-    ok = ok && mbar_wait(&bar->v_full[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn);
-    if (!ok) return false;
-    tc_fence_after();
-    const uint32_t v0 = smem_u32(sV + s * kBox);
-    for (int ks = ks0; ks < ks1; ++ks)
-      umma_ts(tmem + kO, tmem + kP + ks * 8, sdesc_sw128(v0 + ks * 2048, kBox, 1024), idesc_o, 1u);
-    umma_commit(&bar->pv_done);
-    umma_commit(&bar->v_empty[s]);
-    return true;
-  };
   if (warp == 4) {
     if (lane == 0) {
       // ---------------- K side: Q and K tiles by TMA, S(j) = Q K_j^T.  S(j+1)
@@ -560,10 +534,6 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
                   ks > 0);
         umma_commit(&bar->s_full);
         umma_commit(&bar->k_empty[s]);
-        if (kPvSplit && j > 0) {
-          ok = pv_part(j - 1, 0, kPvSplit);
-          if (!ok) break;
-        }
         if (j + ST < n_kv) {
           // refill this stage with K_{j+ST} once S(j) has read it
           ok = mbar_wait(&bar->k_empty[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn);
@@ -572,7 +542,6 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
           tma_load_3d(sK + s * kBox, &mapK, &bar->k_full[s], 0, (j + ST) * kTile, kvseq);
         }
       }
-      if (kPvSplit && ok) pv_part(n_kv - 1, 0, kPvSplit);
     }
   } else if (warp == 5) {
     if (lane == 0) {
@@ -589,9 +558,9 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
         tc_fence_after();
         const uint32_t v0 = smem_u32(sV + s * kBox);
 #pragma unroll
-        for (int ks = kPvSplit; ks < kTile / 16; ++ks)
+        for (int ks = 0; ks < kTile / 16; ++ks)
           umma_ts(tmem + kO, tmem + kP + ks * 8, sdesc_sw128(v0 + ks * 2048, kBox, 1024), idesc_o,
-                  kPvSplit ? 1 : (j > 0 || ks > 0));
+                  (j > 0 || ks > 0));
         umma_commit(&bar->pv_done);
         umma_commit(&bar->v_empty[s]);
         if (j + ST < n_kv) {
@@ -616,13 +585,6 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    if (kPvSplit) {
-      uint32_t z[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) z[c] = 0u;
-      tmem_st32(o_base, z);
-      tmem_st32(o_base + 32, z);
-    }
     for (int j = 0; j < n_kv && ok; ++j) {
       ATTN_TRACE(const unsigned long long tw0 = threadIdx.x == 0 ? globaltimer() : 0ull;)
       ok = mbar_wait(&bar->s_full, j & 1, abort, p.err, kErrTimeoutAttn);
