@@ -408,13 +408,18 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
 //
 // The softmax warps copy S(j) into registers and release its columns at once
 // (s_free), so the MMA warp computes S(j+1) = Q K_{j+1}^T while the
-// exponentials of tile j run; P(j) V follows when P(j) is in tensor memory.
-// Before writing P(j+1) (and rescaling O) the softmax waits for P(j) V to
-// finish (pv_done).
+// exponentials of tile j run.  Before writing P(j+1) (and rescaling O) the
+// softmax waits for P(j) V to finish (pv_done).  P(j) is announced in two
+// halves: the V-side thread issues the first four 16-key steps of P(j) V once
+// keys 0-63 of P(j) (and the rescaled O) are in tensor memory (p_half), while
+// the softmax computes keys 64-127, and the last four at p_full.  One thread
+// issues every P V step in order, so the result does not depend on timing.
+// Measured on B200 (same box, interleaved): 75.8 -> 73.7 us at T = 2048,
+// 1.487 -> 1.464 ms at T = 32768.
 struct __align__(8) Attn1Barriers {
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full, s_free, p_full, pv_done;
+  uint64_t s_full, s_free, p_half, p_full, pv_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -483,6 +488,7 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
     }
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->s_free, 128);
+    mbar_init(&bar->p_half, 128);
     mbar_init(&bar->p_full, 128);
     mbar_init(&bar->pv_done, 1);
     bar->abort = 0;
@@ -552,15 +558,23 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
       bool ok = true;
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % ST;
-        ok = mbar_wait(&bar->p_full, j & 1, abort, p.err, kErrTimeoutAttn);
+        // keys 0-63 of P(j) V as soon as the softmax has stored that half of
+        // P(j) (p_half), keys 64-127 once all of it is in (p_full)
+        ok = mbar_wait(&bar->p_half, j & 1, abort, p.err, kErrTimeoutAttn);
         ok = ok && mbar_wait(&bar->v_full[s], (j / ST) & 1, abort, p.err, kErrTimeoutAttn);
         if (!ok) break;
         tc_fence_after();
         const uint32_t v0 = smem_u32(sV + s * kBox);
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks)
+        for (int ks = 0; ks < kTile / 32; ++ks)
           umma_ts(tmem + kO, tmem + kP + ks * 8, sdesc_sw128(v0 + ks * 2048, kBox, 1024), idesc_o,
                   (j > 0 || ks > 0));
+        ok = mbar_wait(&bar->p_full, j & 1, abort, p.err, kErrTimeoutAttn);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = kTile / 32; ks < kTile / 16; ++ks)
+          umma_ts(tmem + kO, tmem + kP + ks * 8, sdesc_sw128(v0 + ks * 2048, kBox, 1024), idesc_o, 1u);
         umma_commit(&bar->pv_done);
         umma_commit(&bar->v_empty[s]);
         if (j + ST < n_kv) {
@@ -662,14 +676,30 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
 #endif
           pk[c] = pack_bf16x2(p0, p1);
         }
-        // P(j-1) V must be done before P is overwritten (and O rescaled)
+        // P(j-1) V must be done before P is overwritten and O rescaled; the
+        // rescaled O and the first half of P(j) are announced together
         if (h == 0 && j > 0) {
           ATTN_TRACE(const unsigned long long tp0 = threadIdx.x == 0 ? globaltimer() : 0ull;)
           ok = mbar_wait(&bar->pv_done, (j - 1) & 1, abort, p.err, kErrTimeoutAttn) && ok;
           ATTN_TRACE(if (threadIdx.x == 0) tr_wpv += globaltimer() - tp0;)
           tc_fence_after();
+          if (rescale) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(o_base + c0, o);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              tmem_st32(o_base + c0, o);
+            }
+          }
         }
         tmem_st32(p_base + h * 32, pk);
+        if (h == 0) {
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bar->p_half);
+        }
       }
 #if GQE_ATTN1_F2
       {
@@ -681,16 +711,6 @@ attn_prefill_single_kernel(const __grid_constant__ CUtensorMap mapQ, const __gri
 #else
       l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
 #endif
-      if (rescale) {
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(o_base + c0, o);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(o_base + c0, o);
-        }
-      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar->p_full);
