@@ -43,6 +43,7 @@ DECODE_WORKLOAD = "decode"
 METRIC = "GQE prefill tokens/s per layer"
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 L2_FLUSH_BYTES = 256 << 20
+E2E_CHUNK_SEQS = 2              # sequences per copy/compute chunk of the end-to-end leg
 HOST_LEAD_CYCLES = 600_000      # ~0.3 ms at B200 clocks: longer than the host needs to enqueue a step
 
 
@@ -653,27 +654,31 @@ def main():
             torch.cuda.empty_cache()
 
     # ---------------- end to end through host buffers (pinned), on the same step
-    # each step copies its input batch in and its output batch out; the copies
-    # of neighbouring steps overlap each other and the compute (three streams)
+    # one C-ABI call per step (gqe_layer_forward_host): the batch's input is
+    # copied in and its output copied back one sequence at a time, the copies
+    # overlapping each other and the compute on three streams; consecutive
+    # steps chain on the same streams
     e2e = None
     x_pin = x_host.pin_memory()
     y_pins = [torch.empty((dims.B, dims.T, dims.D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     n_e2e = max(3, min(args.steps, 20))
-    xs_h = [x_pin] * n_e2e
-    ys_h = [y_pins[i & 1] for i in range(n_e2e)]
-    layer.forward_host_pipelined(xs_h[:4], ys_h[:4])     # warm-up: graphs captured, streams created
+    for i in range(3):                                    # warm-up: streams, scratch, tensor maps
+        layer.forward_host_c(x_pin, y_pins[i & 1], chunk_seqs=E2E_CHUNK_SEQS)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dist, device)
     torch.cuda.synchronize()
     e0.record(stream)
-    layer.forward_host_pipelined(xs_h, ys_h)
+    for i in range(n_e2e):
+        done = layer.forward_host_c(x_pin, y_pins[i & 1], chunk_seqs=E2E_CHUNK_SEQS, join=False)
+    stream.wait_event(done)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     e2e = {"value": world * dims.N * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(y_pins[0].numel() * 2),
-           "steps": n_e2e, "api": "GQELayer.forward_host_pipelined (pinned host batches, graph replay)"}
+           "steps": n_e2e, "api": f"gqe_layer_forward_host via GQELayer.forward_host_c (pinned host batches, "
+                                  f"{E2E_CHUNK_SEQS}-sequence chunks)"}
 
     # ---------------- decode sub-measurement (64 sequences x 32768-entry cache)
     decode = None

@@ -71,7 +71,14 @@ typedef struct {
   int output_mode;       /* 0 GQE, 1 hard concat only, 2 weighted concat */
 } gqe_dims;
 
-enum { GQE_OP_ROUTED_QPROJ = 1, GQE_OP_ATTN_DECODE = 2, GQE_OP_COMBINE_OUT_PROJ = 3, GQE_OP_ATTN_BWD = 4 };
+enum {
+  GQE_OP_ROUTED_QPROJ = 1,
+  GQE_OP_ATTN_DECODE = 2,
+  GQE_OP_COMBINE_OUT_PROJ = 3,
+  GQE_OP_ATTN_BWD = 4,
+  GQE_OP_LAYER_FORWARD = 5,       /* gqe_layer_forward */
+  GQE_OP_LAYER_FORWARD_HOST = 6   /* gqe_layer_forward_host; dims->B = sequences per chunk */
+};
 
 /* Bytes of scratch the call `op` needs for these dims (L_max: the decode
  * cache length, used by GQE_OP_ATTN_DECODE only).  Returns
@@ -316,6 +323,62 @@ gqe_status gqe_linear(int M, int N, int K, const gqe_bf16* A, const gqe_bf16* W,
 gqe_status gqe_combine_out_proj(const gqe_dims* dims, const gqe_bf16* o_routed, const gqe_bf16* o_sh,
                                 const float* topk_w, const gqe_bf16* Wo, gqe_bf16* y, void* ws,
                                 size_t ws_bytes, gqe_stream stream);
+
+/* The weights of one layer, device pointers in the layouts the calls above
+ * take: Wr [d_model, G*E], bias [G*E] fp32 or NULL, Wq [G, E, d_head,
+ * d_model], Wsh [n_shared*d_head, d_model] (NULL when n_shared == 0), Wk and
+ * Wv [G*d_head, d_model], Wo [d_model, slots*d_head].  All but Wr and bias
+ * 16-byte aligned. */
+typedef struct {
+  const gqe_bf16* Wr;
+  const float* bias;
+  const gqe_bf16* Wq;
+  const gqe_bf16* Wsh;
+  const gqe_bf16* Wk;
+  const gqe_bf16* Wv;
+  const gqe_bf16* Wo;
+} gqe_layer_weights;
+
+/* Prefill forward of a whole GQE layer in one call ("GQE" study note §3-2
+ * 1)-7): router and renormalised weights, routed and shared query
+ * projection, dense K/V projection, routed causal attention, output
+ * construction and projection).  Enqueues on `stream`, in this order,
+ * gqe_router_topk, gqe_routed_qproj, gqe_kv_proj, gqe_attn_prefill and
+ * gqe_combine_out_proj, the same kernels as those calls; the intermediates
+ * (top-k indices and weights, q, K, V, the attention outputs and the calls'
+ * own scratch) live in `ws`.
+ *   x [B, T, d_model] bf16 -> y [B, T, d_model] bf16, device, 16-byte aligned.
+ *   ws: gqe_workspace_size(GQE_OP_LAYER_FORWARD) bytes, 16-byte aligned.
+ * Errors: GQE_ERR_INVALID_ARG (null or misaligned pointers, bad dims) and
+ * GQE_ERR_WORKSPACE are returned before anything is launched; a failed
+ * launch returns GQE_ERR_CUDA, possibly after earlier steps were enqueued. */
+gqe_status gqe_layer_forward(const gqe_dims* dims, const gqe_layer_weights* w, const gqe_bf16* x,
+                             gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream stream);
+
+/* The same forward on HOST buffers: x_host and y_host [B, T, d_model] bf16
+ * in host memory (page-locked, e.g. from cudaHostAlloc, for the copies to
+ * run asynchronously; pageable memory works but the copies then block the
+ * calling thread).  The batch is cut into chunks of chunk_seqs sequences
+ * (the last one may be shorter); chunk i is copied in on stream_in, run
+ * through the layer on stream_compute and copied back on stream_out, with
+ * two device buffers for each direction, so the copies of neighbouring
+ * chunks overlap each other and the compute.  The three streams may be the
+ * same stream (nothing overlaps then).  The call orders the streams with
+ * CUDA events that it creates and releases itself; it allocates no device
+ * memory and does not synchronise.  It returns once everything is enqueued;
+ * y_host is written when the work this call left on stream_compute (or on
+ * stream_out) has completed.  It also leaves stream_in behind its last
+ * compute step and stream_compute behind its last copy-back, so calls in a
+ * row on the same streams may reuse ws without further synchronisation.
+ *   chunk_seqs in [1, B].
+ *   ws: device, 16-byte aligned, gqe_workspace_size(GQE_OP_LAYER_FORWARD_HOST)
+ *   bytes for dims with B = chunk_seqs.
+ * Errors as gqe_layer_forward; GQE_ERR_INVALID_ARG also for a bad
+ * chunk_seqs or a null host pointer. */
+gqe_status gqe_layer_forward_host(const gqe_dims* dims, const gqe_layer_weights* w,
+                                  const gqe_bf16* x_host, gqe_bf16* y_host, int chunk_seqs, void* ws,
+                                  size_t ws_bytes, gqe_stream stream_in, gqe_stream stream_compute,
+                                  gqe_stream stream_out);
 
 /* Reads and clears the device error word (0 = none).  Kernels set it when one
  * of their internal waits runs out of time (0x101 GEMM, 0x201 attention,

@@ -24,6 +24,8 @@ GQE_OP_ROUTED_QPROJ = 1
 GQE_OP_ATTN_DECODE = 2
 GQE_OP_COMBINE_OUT_PROJ = 3
 GQE_OP_ATTN_BWD = 4
+GQE_OP_LAYER_FORWARD = 5
+GQE_OP_LAYER_FORWARD_HOST = 6
 STATUS_NAMES = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED",
                 3: "GQE_ERR_WORKSPACE", 4: "GQE_ERR_CUDA", 5: "GQE_ERR_DEVICE_CHECK"}
 
@@ -42,6 +44,12 @@ class gqe_dims(ctypes.Structure):
                 ("scale", ctypes.c_float), ("output_mode", ctypes.c_int)]
 
 
+class gqe_layer_weights(ctypes.Structure):
+    _fields_ = [("Wr", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("Wq", ctypes.c_void_p),
+                ("Wsh", ctypes.c_void_p), ("Wk", ctypes.c_void_p), ("Wv", ctypes.c_void_p),
+                ("Wo", ctypes.c_void_p)]
+
+
 def make_dims(cfg, **override) -> gqe_dims:
     """Shape struct from any object with B, T, D, G, E, k, d (+ n_shared, sg,
     renorm_scope, scale, output_mode) attributes."""
@@ -57,6 +65,7 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SZ = ctypes.c_size_t
 _D = ctypes.POINTER(gqe_dims)
+_LW = ctypes.POINTER(gqe_layer_weights)
 
 SIGNATURES = {
     "gqe_workspace_size": [_D, _I, _I, ctypes.POINTER(_SZ)],
@@ -71,6 +80,8 @@ SIGNATURES = {
     "gqe_attn_decode_noalloc": [_D, _P, _P, _P, _P, _I, _P, _P, _P, _P],
     "gqe_combine": [_D, _P, _P, _P, _P, _P],
     "gqe_combine_out_proj": [_D, _P, _P, _P, _P, _P, _P, _SZ, _P],
+    "gqe_layer_forward": [_D, _LW, _P, _P, _P, _SZ, _P],
+    "gqe_layer_forward_host": [_D, _LW, _P, _P, _I, _P, _SZ, _P, _P, _P],
     "gqe_linear": [_I, _I, _I, _P, _P, _P, _P],
     "gqe_gemm": [_I, _I, _I, _P, _I, _P, _I, _P, _P],
     "gqe_gemm_acc": [_I, _I, _I, _P, _I, _P, _I, _P, _I, _P],
@@ -264,6 +275,51 @@ def gqe_combine_out_proj(dims, o_routed, o_sh, topk_w, Wo, y, ws, stream=None):
         ctypes.byref(dims), _ptr(o_routed, "o_routed", b), _ptr(o_sh, "o_sh", b, optional=True),
         _ptr(topk_w, "topk_w", torch.float32), _ptr(Wo, "Wo", b), _ptr(y, "y", b),
         _ptr(ws, "ws"), ws_bytes, _stream(stream)))
+
+
+def layer_weights(src) -> gqe_layer_weights:
+    """The weight struct of gqe_layer_forward[_host] from an object (e.g. a
+    GQELayer) or dict holding the device tensors Wr, bias, Wq, Wsh, Wk, Wv, Wo
+    (bias and Wsh may be None).  The struct holds raw pointers: keep the
+    tensors alive while it is in use."""
+    import torch
+    get = src.get if isinstance(src, dict) else (lambda k: getattr(src, k, None))
+    b = _bf16()
+    return gqe_layer_weights(
+        Wr=_ptr(get("Wr"), "Wr", b), bias=_ptr(get("bias"), "bias", torch.float32, optional=True),
+        Wq=_ptr(get("Wq"), "Wq", b), Wsh=_ptr(get("Wsh"), "Wsh", b, optional=True),
+        Wk=_ptr(get("Wk"), "Wk", b), Wv=_ptr(get("Wv"), "Wv", b), Wo=_ptr(get("Wo"), "Wo", b))
+
+
+def _host_ptr(t, name):
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != _bf16():
+        raise ValueError(f"{name} must be {_bf16()}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def gqe_layer_forward(dims, weights, x, y, ws, stream=None):
+    """Whole prefill forward, device x [B, T, D] -> y; weights from layer_weights()."""
+    b = _bf16()
+    ws_bytes = ws.numel() * ws.element_size()
+    _check("gqe_layer_forward", lib.gqe_layer_forward(
+        ctypes.byref(dims), ctypes.byref(weights), _ptr(x, "x", b), _ptr(y, "y", b), _ptr(ws, "ws"), ws_bytes,
+        _stream(stream)))
+
+
+def gqe_layer_forward_host(dims, weights, x_host, y_host, chunk_seqs, ws, stream_in=None, stream_compute=None,
+                           stream_out=None):
+    """Whole prefill forward on host x_host [B, T, D] -> y_host (pinned for
+    overlap), chunk_seqs sequences per chunk; streams default to the current
+    one.  y_host is written once stream_compute reaches this point."""
+    ws_bytes = ws.numel() * ws.element_size()
+    _check("gqe_layer_forward_host", lib.gqe_layer_forward_host(
+        ctypes.byref(dims), ctypes.byref(weights), _host_ptr(x_host, "x_host"), _host_ptr(y_host, "y_host"),
+        int(chunk_seqs), _ptr(ws, "ws"), ws_bytes, _stream(stream_in), _stream(stream_compute),
+        _stream(stream_out)))
 
 
 def gqe_linear(A, W, C, stream=None):

@@ -180,6 +180,9 @@ inline gqe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GQE_OK 
 
 namespace gqe {
 
+// Scratch of the whole-layer forward (layer_fwd.cu).
+gqe_status layer_workspace_bytes(const gqe_dims* dims, bool host, size_t* bytes);
+
 // Argument checks, tensor maps and parameters of a decode call, all but the
 // partial-state scratch, which the caller attaches (gqe_attn_decode: the
 // caller's workspace; gqe_attn_decode_noalloc in attn_decode.cu: the
@@ -258,6 +261,8 @@ gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* b
     *bytes = decode_workspace_bytes(dims->B, dims->G, dims->k, dims->d_head, dims->n_shared, L_max);
     return GQE_OK;
   }
+  if (op == GQE_OP_LAYER_FORWARD || op == GQE_OP_LAYER_FORWARD_HOST)
+    return layer_workspace_bytes(dims, op == GQE_OP_LAYER_FORWARD_HOST, bytes);
   return GQE_ERR_INVALID_ARG;
 }
 

@@ -237,6 +237,38 @@ class GQELayer:
         y_host.copy_(y, non_blocking=True)
         return y_host
 
+    def forward_host_c(self, x_host: torch.Tensor, y_host: torch.Tensor, chunk_seqs: int = 1, join: bool = True):
+        """End to end in ONE C-ABI call, gqe_layer_forward_host: x_host [B, T, D]
+        (pinned) -> y_host, the batch cut into chunks of chunk_seqs sequences
+        whose copies in, forwards and copies back overlap on the layer's three
+        streams, behind the current stream's work so far.  Returns an event
+        that completes once y_host is written; with join=True the current
+        stream also waits for it.  Calls in a row with join=False chain on the
+        layer's streams, each call's copies overlapping the previous call's
+        last steps; join once after the last one."""
+        c = self.cfg
+        B, T = x_host.shape[0], x_host.shape[1]
+        chunk = max(1, min(int(chunk_seqs), B))
+        ws = self._ws("ws_host", L.gqe_workspace_size(L.make_dims(c, B=chunk, T=T), L.GQE_OP_LAYER_FORWARD_HOST))
+        if getattr(self, "_wstruct", None) is None:
+            self._wstruct = L.layer_weights(self)
+        cur = torch.cuda.current_stream(self.device)
+        if getattr(self, "_pipe_streams", None) is None:
+            self._pipe_streams = tuple(torch.cuda.Stream(self.device) for _ in range(3))
+        s_in, s_cmp, s_out = self._pipe_streams
+        start = torch.cuda.Event()
+        start.record(cur)
+        for s_ in (s_in, s_cmp, s_out):
+            s_.wait_event(start)
+            ws.record_stream(s_)
+        L.gqe_layer_forward_host(L.make_dims(c, B=B, T=T), self._wstruct, x_host, y_host, chunk, ws,
+                                 s_in, s_cmp, s_out)
+        done = torch.cuda.Event()
+        done.record(s_cmp)          # the call leaves s_cmp behind its last copy back
+        if join:
+            cur.wait_event(done)
+        return done
+
     def forward_host_pipelined(self, x_hosts, y_hosts):
         """End to end over a sequence of batches in (pinned) host memory:
         y_hosts[i] <- forward(x_hosts[i]).  The host->device copy of batch i,

@@ -239,3 +239,55 @@ def test_gemm_argument_checks(fn):
     assert call(64, 64, 70, 16, 0, 16, 0, 16) == 2         # contiguous K not a multiple of 8
     assert call(60, 64, 70, 16, 1, 16, 1, 16) == 2         # contiguous M not a multiple of 8
     assert call(64, 64, 64, 18, 0, 16, 0, 16) == 1         # misaligned A
+
+
+def _fake_weights(**override):
+    """Weight struct of made-up, 256-byte aligned addresses: only for calls
+    that must return an argument error before touching them."""
+    v = dict(Wr=0x10000, bias=None, Wq=0x20000, Wsh=0x30000, Wk=0x40000, Wv=0x50000, Wo=0x60000)
+    v.update(override)
+    return gq.gqe_layer_weights(**v)
+
+
+def test_layer_forward_workspace_sizes():
+    """The one-call forward's scratch holds every intermediate of the chained
+    calls, and its host form adds two x and two y chunk buffers."""
+    def up(n):
+        return (n + 255) // 256 * 256
+    for kw in (dict(B=8, T=2048, D=1024, G=8, E=2, k=1), dict(B=2, T=8192, D=4096, G=4, E=8, k=4, d=128),
+               dict(B=1, T=128, D=256, G=2, E=2, k=1)):
+        cfg = _cfg(**kw)
+        d = gq.make_dims(cfg)
+        N, G, k, dh, D = cfg.B * cfg.T, cfg.G, cfg.k, cfg.d, cfg.D
+        parts = [N * G * k * 4, N * G * k * 4, N * G * k * dh * 2, N * dh * 2, N * G * dh * 2, N * G * dh * 2,
+                 N * G * k * dh * 2, N * dh * 2, gq.gqe_workspace_size(d, gq.GQE_OP_ROUTED_QPROJ),
+                 gq.gqe_workspace_size(d, gq.GQE_OP_COMBINE_OUT_PROJ)]
+        whole = gq.gqe_workspace_size(d, gq.GQE_OP_LAYER_FORWARD)
+        assert whole == sum(up(p) for p in parts)
+        assert gq.gqe_workspace_size(d, gq.GQE_OP_LAYER_FORWARD_HOST) == whole + 4 * up(N * D * 2)
+
+
+def test_layer_forward_bad_arguments_rejected_before_launch():
+    lib = _lib.lib
+    d = gq.make_dims(_cfg(B=4, T=128))
+    w = _fake_weights()
+    xh = (ctypes.c_uint16 * 16)()
+    ws_ok = 1 << 30
+    host = lambda **kw: lib.gqe_layer_forward_host(   # noqa: E731
+        ctypes.byref(kw.get("d", d)), kw.get("w", ctypes.byref(w)), kw.get("x", ctypes.addressof(xh)),
+        kw.get("y", ctypes.addressof(xh)), kw.get("chunk", 1), kw.get("ws", 0x1000000), kw.get("ws_bytes", ws_ok),
+        None, None, None)
+    assert host(chunk=0) == 1
+    assert host(chunk=5) == 1                       # more than B sequences
+    assert host(x=None) == 1
+    assert host(w=None) == 1
+    assert host(w=ctypes.byref(_fake_weights(Wq=None))) == 1
+    assert host(w=ctypes.byref(_fake_weights(Wsh=None))) == 1      # the shared head needs Wsh
+    assert host(w=ctypes.byref(_fake_weights(Wo=0x60008))) == 1    # misaligned
+    assert host(ws=None) == 3
+    assert host(ws_bytes=16) == 3
+    assert host(d=gq.make_dims(_cfg(B=4, T=128, d=96))) == 2
+    dev = lib.gqe_layer_forward
+    assert dev(ctypes.byref(d), ctypes.byref(w), None, 0x1000000, 0x2000000, ws_ok, None) == 1
+    assert dev(ctypes.byref(d), ctypes.byref(w), 0x1000008, 0x1000000, 0x2000000, ws_ok, None) == 1
+    assert dev(ctypes.byref(d), ctypes.byref(w), 0x1000000, 0x1000000, 0x2000000, 100, None) == 3
