@@ -250,8 +250,7 @@ class GQELayer:
         B, T = x_host.shape[0], x_host.shape[1]
         chunk = max(1, min(int(chunk_seqs), B))
         ws = self._ws("ws_host", L.gqe_workspace_size(L.make_dims(c, B=chunk, T=T), L.GQE_OP_LAYER_FORWARD_HOST))
-        if getattr(self, "_wstruct", None) is None:
-            self._wstruct = L.layer_weights(self)
+        wstruct = L.layer_weights(self)     # read each call: the weight tensors may have been replaced
         cur = torch.cuda.current_stream(self.device)
         if getattr(self, "_pipe_streams", None) is None:
             self._pipe_streams = tuple(torch.cuda.Stream(self.device) for _ in range(3))
@@ -261,7 +260,7 @@ class GQELayer:
         for s_ in (s_in, s_cmp, s_out):
             s_.wait_event(start)
             ws.record_stream(s_)
-        L.gqe_layer_forward_host(L.make_dims(c, B=B, T=T), self._wstruct, x_host, y_host, chunk, ws,
+        L.gqe_layer_forward_host(L.make_dims(c, B=B, T=T), wstruct, x_host, y_host, chunk, ws,
                                  s_in, s_cmp, s_out)
         done = torch.cuda.Event()
         done.record(s_cmp)          # the call leaves s_cmp behind its last copy back
