@@ -56,9 +56,12 @@ ROUTER_CASES = {
     "tc_E3_group_scope": (gi.Workload("t3", D(B=2, T=640, D=256, G=5, E=3, k=2, renorm_scope=1)), None),
     "tc_E8_k4_ragged": (gi.Workload("t8", D(B=1, T=1100, D=192, G=4, E=8, k=4)), None),
     "tc_E4_GE64": (gi.Workload("t4", D(B=1, T=1536, D=128, G=16, E=4, k=1)), None),
-    # Wr^T too large for the tcgen05 router's shared memory: the streaming router
+    # the tcgen05 router with Wr read in place at larger d_model
     "tc_K_chunked_GE64": (gi.Workload("tk", D(B=1, T=1100, D=1024, G=8, E=8, k=2)), None),
     "tc_K_chunked_group_scope": (gi.Workload("tg", D(B=2, T=600, D=2048, G=4, E=8, k=3, renorm_scope=1)), None),
+    # Wr too large to keep in shared memory and fewer than 1024 tokens (no
+    # tcgen05 router): the streaming CUDA-core router, ragged last tile
+    "stream_D4096_N500": (gi.Workload("s1", D(B=1, T=500, D=4096, G=4, E=8, k=3)), None),
 }
 
 
