@@ -81,8 +81,9 @@ enum {
 };
 
 /* Bytes of scratch the call `op` needs for these dims (L_max: the decode
- * cache length, used by GQE_OP_ATTN_DECODE only).  Returns
- * GQE_ERR_INVALID_ARG for bad dims or op. */
+ * cache length, used by GQE_OP_ATTN_DECODE only).  For
+ * GQE_OP_LAYER_FORWARD_HOST, dims->B is the number of sequences per chunk,
+ * not the batch.  Returns GQE_ERR_INVALID_ARG for bad dims or op. */
 gqe_status gqe_workspace_size(const gqe_dims* dims, int op, int L_max, size_t* bytes);
 
 /* Router: "GQE" study note §3-2 2) (score, in-group softmax, TopK) and 4)
