@@ -295,6 +295,33 @@ def test_decode_equals_last_prefill_row():
     np.testing.assert_allclose(dec2["y"], dec["y"], atol=0)
 
 
+def test_decode_ragged_cache_lengths_match_scalar_loops():
+    """Decode attention with a different cache length per sequence: every
+    routed row of sequence b attends to rows 0..cache_len[b]-1 of its own
+    group's cache and the shared row to group sg's, written out as scalar
+    loops (GQA tutorial, decode with a KV cache; study note §3-2 5))."""
+    rng = np.random.default_rng(12)
+    B, G, k, d, L = 3, 3, 2, 4, 11
+    dims = gi.GQEDims(B=B, T=1, D=8, G=G, E=3, k=k, d=d, n_shared=1, sg=2)
+    q = _rand(rng, B, G, k, d)
+    qs = _rand(rng, B, d)
+    Kc = _rand(rng, B, G, L, d)
+    Vc = _rand(rng, B, G, L, d)
+    lens = np.array([L, 1, 6])
+    o, o_sh = orc.attn_decode(q, qs, Kc, Vc, lens, dims)
+    sc = 1.0 / math.sqrt(d)
+    for b in range(B):
+        n = int(lens[b])
+        for g in range(G):
+            for j in range(k):
+                ref = _scalar_attention(q[b, g, j].tolist(), Kc[b, g, :n].tolist(), Vc[b, g, :n].tolist(), n - 1, sc)
+                np.testing.assert_allclose(o[b, g, j], ref, rtol=1e-12, atol=1e-13)
+        ref = _scalar_attention(qs[b].tolist(), Kc[b, 2, :n].tolist(), Vc[b, 2, :n].tolist(), n - 1, sc)
+        np.testing.assert_allclose(o_sh[b], ref, rtol=1e-12, atol=1e-13)
+    # a cache of one row returns that row's value
+    np.testing.assert_allclose(o[1], np.broadcast_to(Vc[1, :, 0][:, None, :], (G, k, d)), atol=1e-15)
+
+
 # ----------------------------------------------------------------------------
 # output construction and locality: GQE study note §3-2 3)-5)
 
