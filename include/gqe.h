@@ -369,13 +369,16 @@ gqe_status gqe_layer_forward(const gqe_dims* dims, const gqe_layer_weights* w, c
  * memory and does not synchronise.  It returns once everything is enqueued;
  * y_host is written when the work this call left on stream_compute (or on
  * stream_out) has completed.  It also leaves stream_in behind its last
- * compute step and stream_compute behind its last copy-back, so calls in a
- * row on the same streams may reuse ws without further synchronisation.
- *   chunk_seqs in [1, B].
+ * compute step and stream_compute behind its last copy-back.  So calls in a
+ * row on the same streams may share ws without further synchronisation
+ * when their dims agree apart from B and they pass the same chunk_seqs (the
+ * layout of ws depends on those alone).  Before ws serves a call with other
+ * dims or another chunk_seqs, let stream_out's work complete.
+ *   chunk_seqs >= 1; a batch of fewer sequences runs as one chunk.
  *   ws: device, 16-byte aligned, gqe_workspace_size(GQE_OP_LAYER_FORWARD_HOST)
  *   bytes for dims with B = chunk_seqs.
- * Errors as gqe_layer_forward; GQE_ERR_INVALID_ARG also for a bad
- * chunk_seqs or a null host pointer. */
+ * Errors as gqe_layer_forward; GQE_ERR_INVALID_ARG also for chunk_seqs < 1
+ * or a null host pointer. */
 gqe_status gqe_layer_forward_host(const gqe_dims* dims, const gqe_layer_weights* w,
                                   const gqe_bf16* x_host, gqe_bf16* y_host, int chunk_seqs, void* ws,
                                   size_t ws_bytes, gqe_stream stream_in, gqe_stream stream_compute,

@@ -119,7 +119,7 @@ gqe_status gqe_layer_forward_host(const gqe_dims* dims, const gqe_layer_weights*
   size_t full = 0;
   GQE_TRY(gqe_workspace_size(dims, GQE_OP_LAYER_FORWARD, 0, &full));   // validates dims
   GQE_TRY(check_weights(dims, w));
-  if (!x_host || !y_host || chunk_seqs < 1 || chunk_seqs > dims->B) return GQE_ERR_INVALID_ARG;
+  if (!x_host || !y_host || chunk_seqs < 1) return GQE_ERR_INVALID_ARG;
   gqe_dims cd = *dims;
   cd.B = chunk_seqs;
   size_t need = 0;

@@ -248,7 +248,10 @@ class GQELayer:
         last steps; join once after the last one."""
         c = self.cfg
         B, T = x_host.shape[0], x_host.shape[1]
-        chunk = max(1, min(int(chunk_seqs), B))
+        chunk = max(1, int(chunk_seqs))
+        # the scratch's layout depends on T and chunk_seqs alone, so batches of
+        # any size chain on it; another layout gets another buffer (the old one
+        # is released only after the streams' work on it, record_stream below)
         ws = self._ws("ws_host", L.gqe_workspace_size(L.make_dims(c, B=chunk, T=T), L.GQE_OP_LAYER_FORWARD_HOST))
         wstruct = L.layer_weights(self)     # read each call: the weight tensors may have been replaced
         cur = torch.cuda.current_stream(self.device)

@@ -278,7 +278,7 @@ def test_layer_forward_bad_arguments_rejected_before_launch():
         kw.get("y", ctypes.addressof(xh)), kw.get("chunk", 1), kw.get("ws", 0x1000000), kw.get("ws_bytes", ws_ok),
         None, None, None)
     assert host(chunk=0) == 1
-    assert host(chunk=5) == 1                       # more than B sequences
+    assert host(chunk=-2) == 1
     assert host(x=None) == 1
     assert host(w=None) == 1
     assert host(w=ctypes.byref(_fake_weights(Wq=None))) == 1

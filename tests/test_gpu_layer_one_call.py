@@ -82,11 +82,13 @@ def test_layer_forward_one_call_tiny_against_oracle():
     assert torch.equal(y, y_layer), "one-call forward differs from the chained calls"
     ref = orc.gqe_forward(x, Wt, dims, bias)
     assert_close_attn(to_f64(y).reshape(dims.N, -1), ref["y"], "gqe_layer_forward y vs oracle")
-    # the host form on the same workload, one chunk per sequence
-    yh = _host_out(dims)
-    layer.forward_host_c(_pinned(x), yh, chunk_seqs=1)
-    torch.cuda.synchronize()
-    assert torch.equal(yh, y.cpu()), "host-buffer forward differs from the device one"
+    # the host form on the same workload, one chunk per sequence, and with a
+    # chunk size above the batch (the batch runs as one chunk)
+    for chunk in (1, 4):
+        yh = _host_out(dims)
+        layer.forward_host_c(_pinned(x), yh, chunk_seqs=chunk)
+        torch.cuda.synchronize()
+        assert torch.equal(yh, y.cpu()), f"host-buffer forward (chunk {chunk}) differs from the device one"
 
 
 @pytest.mark.parametrize("wname,chunks", [("main_prefill", (1, 2, 3, 8)), ("wide_skewed_prefill", (1,))])

@@ -19,7 +19,10 @@ stream wait with the byte ranges it reads and writes.  From that log:
     graph, each chunk's host output derives from that chunk's input (and the
     weights) alone;
   - the documented end state: the last work each call leaves on the compute
-    stream (and on the copy-back stream) comes after every copy back.
+    stream (and on the copy-back stream) comes after every copy back;
+  - calls in a row with batches of different sizes (one chunk_seqs) chain
+    race-free; with another chunk_seqs on the same workspace they would not,
+    which is why the header asks for a synchronisation there.
 
 A planted mistake, one of the waits taken out of the log, must be caught.
 """
@@ -80,21 +83,27 @@ W_BASE = 0x4000_0000_0000
 CALL_STRIDE = 1 << 36
 
 
-def _run(fake, B, chunk, calls, streams=(0x11, 0x22, 0x33), T=4, D=128):
-    """Issues `calls` host-buffer forwards in a row on the same streams and
-    workspace (each on its own host x and y) and returns the parsed log."""
-    dims = Dims(B=B, T=T, d_model=D, G=2, E=3, k=2, d_head=64, n_shared=1, shared_kv_group=1,
+def _dims(B, T, D):
+    return Dims(B=B, T=T, d_model=D, G=2, E=3, k=2, d_head=64, n_shared=1, shared_kv_group=1,
                 renorm_scope=0, scale=0.0, output_mode=0)
+
+
+def _run(fake, Bs, chunks, streams=(0x11, 0x22, 0x33), T=4, D=128):
+    """Issues one host-buffer forward per entry of Bs (batch sizes) and chunks
+    (chunk_seqs), in a row on the same streams and workspace, each on its own
+    host x and y; returns the parsed log."""
     w = Weights(**{n: W_BASE + i * 0x10000 for i, n in enumerate(("Wr", "bias", "Wq", "Wsh", "Wk", "Wv", "Wo"))})
     w.bias = None
-    cd = Dims.from_buffer_copy(dims)
-    cd.B = chunk
-    need = ctypes.c_size_t(0)
-    assert fake.gqe_workspace_size(ctypes.byref(cd), GQE_OP_LAYER_FORWARD_HOST, 0, ctypes.byref(need)) == 0
+    need = 0
+    for chunk in chunks:
+        n = ctypes.c_size_t(0)
+        assert fake.gqe_workspace_size(ctypes.byref(_dims(chunk, T, D)), GQE_OP_LAYER_FORWARD_HOST, 0,
+                                       ctypes.byref(n)) == 0
+        need = max(need, n.value)
     fake.fake_log_clear()
-    for c in range(calls):
-        st = fake.gqe_layer_forward_host(ctypes.byref(dims), ctypes.byref(w), X_HOST + c * CALL_STRIDE,
-                                         Y_HOST + c * CALL_STRIDE, chunk, WS, need.value, *streams)
+    for c, (B, chunk) in enumerate(zip(Bs, chunks)):
+        st = fake.gqe_layer_forward_host(ctypes.byref(_dims(B, T, D)), ctypes.byref(w), X_HOST + c * CALL_STRIDE,
+                                         Y_HOST + c * CALL_STRIDE, chunk, WS, need, *streams)
         assert st == 0
     lines = [fake.fake_log_line(i).decode() for i in range(fake.fake_log_size())]
     seq_bytes = T * D * 2
@@ -200,11 +209,11 @@ class _Memory:
         return labels
 
 
-def _simulate(nodes, preds, rng, B, chunk, calls, seq_bytes):
+def _simulate(nodes, preds, rng, Bs, chunk, seq_bytes):
     """Runs the nodes in one random order that respects the graph; returns,
-    per (call, chunk), the labels the host output derives from."""
+    per (call, sequence), the labels the host output derives from."""
     mem = _Memory()
-    for c in range(calls):
+    for c, B in enumerate(Bs):
         for b in range(B):
             base = X_HOST + c * CALL_STRIDE + b * seq_bytes
             mem.write(base, base + seq_bytes, frozenset({("x", c, b // chunk)}))
@@ -232,34 +241,36 @@ def _simulate(nodes, preds, rng, B, chunk, calls, seq_bytes):
                 ready.append(j)
     assert done == len(nodes)
     out = {}
-    for c in range(calls):
+    for c, B in enumerate(Bs):
         for b in range(B):
             base = Y_HOST + c * CALL_STRIDE + b * seq_bytes
             out[(c, b)] = mem.read(base, base + seq_bytes)
     return out
 
 
-CASES = [  # (B, chunk, calls)
-    (8, 1, 2), (8, 3, 2), (8, 8, 3), (5, 2, 3), (1, 1, 3), (6, 4, 2), (7, 7, 1),
+CASES = [  # (batch size of each call in the row, chunk_seqs)
+    ((8, 8), 1), ((8, 8), 3), ((8, 8, 8), 8), ((5, 5, 5), 2), ((1, 1, 1), 1), ((6, 6), 4), ((7,), 7),
+    ((8, 5, 3), 2),         # batches of different sizes chain on one layout
+    ((2, 9, 1), 4),         # chunk_seqs above the batch: one chunk
 ]
 
 
-@pytest.mark.parametrize("B,chunk,calls", CASES)
+@pytest.mark.parametrize("Bs,chunk", CASES)
 @pytest.mark.parametrize("one_stream", [False, True])
-def test_host_pipeline_is_race_free_and_keeps_chunks_apart(fake, B, chunk, calls, one_stream):
+def test_host_pipeline_is_race_free_and_keeps_chunks_apart(fake, Bs, chunk, one_stream):
     streams = (0x11, 0x11, 0x11) if one_stream else (0x11, 0x22, 0x33)
-    ops, seq_bytes = _run(fake, B, chunk, calls, streams)
-    n_chunks = -(-B // chunk)
-    assert sum(op["kind"] == "copy" for op in ops) == 2 * n_chunks * calls
-    assert sum(op["kind"] == "kernel" for op in ops) == 5 * n_chunks * calls
+    ops, seq_bytes = _run(fake, Bs, [chunk] * len(Bs), streams)
+    n_chunks = sum(-(-B // chunk) for B in Bs)
+    assert sum(op["kind"] == "copy" for op in ops) == 2 * n_chunks
+    assert sum(op["kind"] == "kernel" for op in ops) == 5 * n_chunks
     created = [op["event"] for op in ops if op["kind"] == "create"]
     destroyed = [op["event"] for op in ops if op["kind"] == "destroy"]
     assert sorted(created) == sorted(destroyed)         # every event released
     nodes, preds, anc = _graph(ops)
     assert _races(nodes, anc) == []
-    rng = random.Random(1234 + B * 31 + chunk)
+    rng = random.Random(1234 + sum(Bs) * 31 + chunk)
     for _ in range(20):
-        got = _simulate(nodes, preds, rng, B, chunk, calls, seq_bytes)
+        got = _simulate(nodes, preds, rng, Bs, chunk, seq_bytes)
         for (c, b), labels in got.items():
             assert labels == {("x", c, b // chunk), "W"}, (c, b, labels)
     # y_host is complete once the compute stream's (or the copy-back
@@ -274,7 +285,7 @@ def test_host_pipeline_is_race_free_and_keeps_chunks_apart(fake, B, chunk, calls
 def test_a_missing_wait_is_caught(fake, drop):
     """Planted mistakes: taking any one of the pipeline's waits out of the log
     leaves a race that the check finds."""
-    ops, _ = _run(fake, 8, 1, 2)
+    ops, _ = _run(fake, (8, 8), (1, 1))
     waits = [i for i, op in enumerate(ops) if op["kind"] == "wait"]
     s_in, s_cmp = 0x11, 0x22
     # the first call's waits, in issue order: on s_in for chunks >= 2 (x slot
@@ -293,3 +304,13 @@ def test_a_missing_wait_is_caught(fake, drop):
     broken = ops[:pick] + ops[pick + 1:]
     nodes, _, anc = _graph(broken)
     assert _races(nodes, anc), f"dropping the {drop} wait went unnoticed"
+
+
+def test_another_chunk_size_on_the_same_workspace_needs_a_synchronisation(fake):
+    """Why the header asks callers to let stream_out's work complete before
+    the workspace serves another chunk_seqs: the layout moves, and the next
+    call's copy in can land on a buffer the previous call is still copying
+    back from."""
+    ops, _ = _run(fake, (8, 8), (1, 4))
+    nodes, _, anc = _graph(ops)
+    assert ("d2h", "h2d") in _races(nodes, anc)
