@@ -25,6 +25,8 @@ stream wait with the byte ranges it reads and writes.  From that log:
     which is why the header asks for a synchronisation there.
 
 A planted mistake, one of the waits taken out of the log, must be caught.
+Errors injected on the host into one step or one copy come back as the
+call's status, and the call releases its events on that path too.
 """
 import ctypes
 import os
@@ -67,6 +69,7 @@ def fake(tmp_path_factory):
     assert r.returncode == 0, r.stderr
     lib = ctypes.CDLL(out)
     lib.fake_log_line.restype = ctypes.c_char_p
+    lib.fake_fail.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.gqe_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int, ctypes.c_int,
                                        ctypes.POINTER(ctypes.c_size_t)]
     lib.gqe_layer_forward_host.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(Weights), ctypes.c_void_p,
@@ -88,7 +91,7 @@ def _dims(B, T, D):
                 renorm_scope=0, scale=0.0, output_mode=0)
 
 
-def _run(fake, Bs, chunks, streams=(0x11, 0x22, 0x33), T=4, D=128):
+def _run(fake, Bs, chunks, streams=(0x11, 0x22, 0x33), T=4, D=128, expect=0):
     """Issues one host-buffer forward per entry of Bs (batch sizes) and chunks
     (chunk_seqs), in a row on the same streams and workspace, each on its own
     host x and y; returns the parsed log."""
@@ -104,7 +107,7 @@ def _run(fake, Bs, chunks, streams=(0x11, 0x22, 0x33), T=4, D=128):
     for c, (B, chunk) in enumerate(zip(Bs, chunks)):
         st = fake.gqe_layer_forward_host(ctypes.byref(_dims(B, T, D)), ctypes.byref(w), X_HOST + c * CALL_STRIDE,
                                          Y_HOST + c * CALL_STRIDE, chunk, WS, need, *streams)
-        assert st == 0
+        assert st == expect
     lines = [fake.fake_log_line(i).decode() for i in range(fake.fake_log_size())]
     seq_bytes = T * D * 2
     return [_parse(s) for s in lines], seq_bytes
@@ -314,3 +317,22 @@ def test_another_chunk_size_on_the_same_workspace_needs_a_synchronisation(fake):
     ops, _ = _run(fake, (8, 8), (1, 4))
     nodes, _, anc = _graph(ops)
     assert ("d2h", "h2d") in _races(nodes, anc)
+
+
+@pytest.mark.parametrize("step,copy", [(0, -1), (3, -1), (7, -1), (19, -1), (-1, 0), (-1, 5), (-1, 7)])
+def test_a_failing_step_or_copy_is_reported_and_releases_the_events(fake, step, copy):
+    """An error from one of the steps (injected on the host, GQE_ERR_CUDA from
+    the fifth step say) or from a copy comes back as the call's status, and
+    every event the call created is released on that path too (8 sequences in
+    chunks of 2: 20 steps, 8 copies)."""
+    fake.fake_fail(step, 4, copy)
+    try:
+        ops, _ = _run(fake, (8,), (2,), expect=4)
+    finally:
+        fake.fake_fail(-1, 0, -1)
+    created = sorted(op["event"] for op in ops if op["kind"] == "create")
+    destroyed = sorted(op["event"] for op in ops if op["kind"] == "destroy")
+    assert len(created) == 5 and created == destroyed
+    n_steps = sum(op["kind"] == "kernel" for op in ops)
+    if step >= 0:
+        assert n_steps == step          # nothing launched after the failing step
